@@ -1,0 +1,424 @@
+"""Benchmark of the Based attention path on B200.
+
+One step = one pass of the prefill hot path over one batch of the
+360M-layer-shape workload (B=8, L=2048, d_model=1024): causal Taylor linear
+attention over 16 heads (d=16 -> 273 features, d_v=64) with state export, plus
+sliding-window-64 softmax attention over 16 heads of d_head=64.  The metric is
+tokens/s (B*L per step).  The same run also measures the recurrent decode step
+(B=128 sequences x 16 + 16 heads, 273x64 fp32 states, 64-slot rings) and
+reports it under "decode".
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch with torchrun; each rank runs an independent replica (the
+path has no exchange step), and value = all ranks' tokens / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "Based attn prefill tokens/s (L=2048) & decode tokens/s; % of roofline"
+UNIT = "tokens/s"
+PREFILL = "layer_360m"
+DECODE = "decode_b128"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes / flops (per launch)
+# ---------------------------------------------------------------------------
+
+def linattn_bytes(w):
+    """q, k (d), v, out (d_v) in the input dtype per token-head, + exported states."""
+    es = 4 if w.dtype == "f32" else 2
+    per_tok = (2 * w.d + 2 * w.dv) * es
+    return w.B * w.H * w.L * per_tok + w.B * w.H * 273 * (w.dv + 1) * 4
+
+
+def window_bytes(w):
+    es = 4 if w.dtype == "f32" else 2
+    return w.B * w.Hw * w.L * 4 * w.dh * es
+
+
+def decode_bytes(w):
+    es = 2 if w.dtype == "bf16" else 4
+    lin = w.B * w.H * (2 * 273 * (w.dv + 1) * 4 + (2 * w.d + 2 * w.dv) * es)
+    win = w.B * w.Hw * (2 * w.window * w.dh * es + 2 * w.dh * es + 4 * w.dh * es)
+    return lin + win
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank, world, dev):
+    import linear_attention_lm_b200 as lab
+    from linear_attention_lm_b200 import build as lab_build
+    from linear_attention_lm_b200.inputs import WORKLOADS, decode_step_inputs, prefill_inputs
+
+    if rank == 0:
+        lab_build.build()
+    if world > 1:
+        torch.distributed.barrier()
+    lab.load_library()
+    peaks = load_peaks()
+    w = WORKLOADS[PREFILL]
+    # rotate input sets so that consecutive steps never find their data in L2
+    set_bytes = linattn_bytes(w) + window_bytes(w)
+    n_sets = max(2, int(np.ceil(3 * L2_BYTES / set_bytes)))
+    sets = []
+    for i in range(n_sets):
+        x = prefill_inputs(w, device=dev) if i == 0 else {k: t.clone() for k, t in sets[0][0].items()}
+        outs = {"y": torch.empty_like(x["v"]), "yw": torch.empty_like(x["wq"]),
+                "S": torch.empty((w.B, w.H, 273, w.dv), dtype=torch.float32, device=dev),
+                "z": torch.empty((w.B, w.H, 273), dtype=torch.float32, device=dev)}
+        sets.append((x, outs))
+    ws_bytes = lab.based_linattn_workspace_bytes(w.B, w.H, w.L, w.d, w.dv, lab.BASED_BF16)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+
+    def step(i, ev=None):
+        x, o = sets[i % n_sets]
+        if ev is not None:
+            ev[0].record()
+        lab.based_linattn_fwd(x["q"], x["k"], x["v"], o["y"], w.eps, o["S"], o["z"],
+                              workspace=ws[:ws_bytes] if ws_bytes else None)
+        if ev is not None:
+            ev[1].record()
+        lab.based_window_attn_fwd(x["wq"], x["wk"], x["wv"], o["yw"], w.window)
+        if ev is not None:
+            ev[2].record()
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        start.record()
+        for i in range(args.steps):
+            step(i, evs[i])
+        stop.record()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+    elapsed_ms = start.elapsed_time(stop)
+    t_lin = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    t_win = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    assert lab.based_get_device_error() == 0
+    elapsed_max = elapsed_ms
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed_max = float(t.item())
+    tokens = world * w.B * w.L * args.steps
+    value = tokens / (elapsed_max / 1e3)
+
+    # roofline of the dominant kernel (both are HBM-bound by algorithmic bytes)
+    kern = {"linattn_prefill": (linattn_bytes(w), t_lin), "window_attn": (window_bytes(w), t_win)}
+    dom = max(kern, key=lambda k: kern[k][1])
+    b, t_ms = kern[dom]
+    achieved = b / (t_ms / 1e3) / 1e9
+    roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                "peak_source": peaks["source"],
+                "per_kernel_ms": {k: round(v[1], 5) for k, v in kern.items()},
+                "per_kernel_frac": {k: round(v[0] / (v[1] / 1e3) / 1e9 / peaks["hbm_gbs"], 4)
+                                    for k, v in kern.items()}}
+
+    e2e = run_e2e(args, w, lab, dev, world, sets[0][0])
+    decode = run_decode(args, lab, dev, world, peaks)
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(elapsed_max / args.steps, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{PREFILL}: B=8 L=2048 d_model=1024; linear attn 16 heads "
+                               f"d=16->273 d_v=64 (+state export); window-64 attn 16 heads d_h=64",
+                   "global_batch": w.B * world, "seq_len": w.L,
+                   "parallelism": f"replicas{world}",
+                   "l2": f"inputs larger than L2: {n_sets} rotating input sets of "
+                         f"{set_bytes / 1e6:.0f} MB"},
+        "roofline": roofline,
+        "e2e": e2e,
+        "decode": decode,
+        "gpu_launches": 2 * args.steps,
+        "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+    }
+    if rank == 0 and world == 1:
+        line["cpu_baseline"] = cpu_baseline(w)
+    return line
+
+
+def run_e2e(args, w, lab, dev, world, x):
+    """Same metric through the public API with pinned host buffers: H2D of the
+    step's inputs, both kernels, D2H of both outputs, every step."""
+    n = max(1, min(args.steps, 30))
+    host_in = {k: t.to("cpu").pin_memory() for k, t in x.items()}
+    host_out = {"y": torch.empty(x["v"].shape, dtype=x["v"].dtype).pin_memory(),
+                "yw": torch.empty(x["wq"].shape, dtype=x["wq"].dtype).pin_memory()}
+    dev_in = {k: torch.empty_like(t, device=dev) for k, t in x.items()}
+    y = torch.empty_like(dev_in["v"])
+    yw = torch.empty_like(dev_in["wq"])
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+
+    def one():
+        for k in dev_in:
+            dev_in[k].copy_(host_in[k], non_blocking=True)
+        lab.based_linattn_fwd(dev_in["q"], dev_in["k"], dev_in["v"], y, w.eps)
+        lab.based_window_attn_fwd(dev_in["wq"], dev_in["wk"], dev_in["wv"], yw, w.window)
+        host_out["y"].copy_(y, non_blocking=True)
+        host_out["yw"].copy_(yw, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    s.record()
+    for _ in range(n):
+        one()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": round(world * w.B * w.L * n / (ms / 1e3), 1), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n}
+
+
+def run_decode(args, lab, dev, world, peaks):
+    """Recurrent decode: prefill 512 tokens (state export + ring fill), then
+    time decode steps; two independent batches alternate so the 176 MB of
+    state + ring per batch is never resident in L2 from the previous step."""
+    from linear_attention_lm_b200.inputs import WORKLOADS, decode_step_inputs, prefill_inputs
+    w = WORKLOADS[DECODE]
+    groups = []
+    for gi in range(2):
+        x = prefill_inputs(w, device=dev)
+        _, S, z = lab.linattn(x["q"], x["k"], x["v"], w.eps, return_state=True)
+        kr, vr = lab.window_ring_fill(x["wk"], x["wv"], w.window)
+        groups.append((S, z, kr, vr))
+        del x
+    step_in = [decode_step_inputs(w, s, device=dev) for s in range(8)]
+    out = torch.empty((w.B, w.H, w.dv), dtype=torch.bfloat16, device=dev)
+    wout = torch.empty((w.B, w.Hw, w.dh), dtype=torch.bfloat16, device=dev)
+    n = max(8, min(args.steps, 512))
+
+    def one(i):
+        S, z, kr, vr = groups[i % 2]
+        d = step_in[i % len(step_in)]
+        lab.based_decode_step(d["q"], d["k"], d["v"], S, z, out, d["wq"], d["wk"], d["wv"], kr,
+                              vr, wout, pos=w.L + i // 2, window=w.window, eps=w.eps)
+
+    for i in range(max(3, args.warmup)):
+        one(i)
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for i in range(n):
+        one(i)
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / n
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    b = decode_bytes(w)
+    ach = b / (ms / 1e3) / 1e9
+    return {"value": round(world * w.B / (ms / 1e3), 1), "unit": "tokens/s",
+            "ms_per_step": round(ms, 5), "steps": n, "batch": w.B, "heads": w.H,
+            "roofline": {"kernel": "decode_step", "bound": "hbm", "achieved": round(ach, 1),
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None,
+                         "algorithmic_bytes": int(b)}}
+
+
+# ---------------------------------------------------------------------------
+# CPU baselines (the fp64 oracle, as it stands)
+# ---------------------------------------------------------------------------
+
+def _oracle_step_sample(w, n_lin, n_win, n_tok, threads):
+    """Run the oracle on n_lin linear-attention and n_win window sequences of
+    the workload, each truncated to its first n_tok tokens; returns seconds."""
+    import oracle
+    from linear_attention_lm_b200.inputs import prefill_inputs, to_f64
+    x = prefill_inputs(w.with_(B=1), device="cpu")
+    q, k, v = (to_f64(x[n])[0, :, :n_tok] for n in ("q", "k", "v"))
+    wq, wk, wv = (to_f64(x[n])[0, :, :n_tok] for n in ("wq", "wk", "wv"))
+    reps_l = int(np.ceil(n_lin / w.H))
+    reps_w = int(np.ceil(n_win / w.Hw))
+    ql, kl, vl = (np.concatenate([a] * reps_l)[:n_lin] for a in (q, k, v))
+    qw, kw, vw = (np.concatenate([a] * reps_w)[:n_win] for a in (wq, wk, wv))
+    oracle.build()
+    t0 = time.perf_counter()
+    oracle.linattn_recurrent(ql, kl, vl, w.eps, threads=threads)
+    oracle.window_attn(qw, kw, vw, w.window, threads=threads)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w):
+    threads = os.cpu_count() or 1
+    n_seq = w.B * w.H  # one whole step of the workload
+    sec = _oracle_step_sample(w, n_seq, n_seq, w.L, threads)
+    tok_per_s = (n_seq * w.L / w.H) / sec  # tokens through all 16 + 16 heads
+    return {"value": round(tok_per_s, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{n_seq} linear-attention + {n_seq} window sequences of L={w.L} "
+                      f"(fp64 recurrent form and direct window softmax), "
+                      f"= {n_seq / w.H:.2f} batch rows of the {PREFILL} step"}
+
+
+def run_reference(args, rank, world):
+    """The fp64 oracle on host cores as the reference arm: each step is one
+    linear-attention + one window sequence of the workload, truncated to a
+    token count that keeps the whole run within a few minutes."""
+    from linear_attention_lm_b200.inputs import WORKLOADS
+    w = WORKLOADS[PREFILL]
+    threads = 1
+    budget_s = 150.0
+    n_tok = w.L
+    probe = _oracle_step_sample(w, 1, 1, 256, threads)
+    per_tok = probe / 256
+    n_tok = int(max(32, min(w.L, budget_s / max(1, args.steps + args.warmup) / per_tok)))
+    for _ in range(args.warmup):
+        _oracle_step_sample(w, 1, 1, n_tok, threads)
+    t = 0.0
+    for _ in range(args.steps):
+        t += _oracle_step_sample(w, 1, 1, n_tok, threads)
+    # one step pushes n_tok tokens through one head of each layer type; a token
+    # of the workload needs 16 + 16 heads
+    value = args.steps * n_tok / w.H / t
+    sample = (f"per step: 1 linear-attention + 1 window sequence of the {PREFILL} workload, "
+              f"first {n_tok} tokens; tokens/s counts a token once all 16+16 heads are done")
+    return {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * t / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": f"{PREFILL}: B=8 L=2048 d_model=1024; linear attn 16 heads "
+                                   f"d=16->273 d_v=64; window-64 attn 16 heads d_h=64",
+                       "global_batch": w.B, "seq_len": w.L, "parallelism": "host cores"},
+            "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": threads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    try:
+        line = run_ours(args, rank, world, dev)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,159 @@
+/*
+ * based.h -- C ABI of the B200 (sm_100a) Based attention library.
+ *
+ * The library computes the data-parallel attention path of the Based
+ * architecture ("Simple linear attention language models balance the
+ * recall-throughput tradeoff", HazyResearch/based):
+ *
+ *   - causal linear attention with the second-order Taylor feature map
+ *       phi(x) = [1, x / d^(1/4), vec(x x^T) / (sqrt(2) sqrt(d))],  d = 16,
+ *     i.e. 1 + 16 + 256 = 273 features ("Базированная модель, часть 2",
+ *     section "Что за линейное внимание?": the map cat(1, x, vec(xx^T)/sqrt 2)
+ *     whose dot product is the expansion 1 + qk + (qk)^2/2 of exp(qk), here
+ *     applied to x / d^(1/4) so it expands exp(q.k / sqrt(d))), and
+ *       y_t = phi(q_t)^T S_t / (phi(q_t) . z_t + eps),
+ *       S_t = sum_{s<=t} phi(k_s) v_s^T   (the KV state),
+ *       z_t = sum_{s<=t} phi(k_s)         (the K state, same post, paragraph
+ *                                          on the state size);
+ *   - exact softmax attention over a sliding window of the last `window`
+ *     tokens, current token included (Based README, introduction, item 1:
+ *     window size 64), scale 1/sqrt(d_head);
+ *   - the one-token recurrent decode step of both (the recurrent form of the
+ *     linear attention over the KV/K states, and a `window`-slot ring cache).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers, owned by the caller, C-contiguous
+ *     in the layouts given below, 16-byte aligned.  The library never keeps a
+ *     pointer after the call returns and never allocates device memory.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *     asynchronous on it; the caller synchronises before reading results.
+ *   - Argument errors are detected on the host, before any launch, and return
+ *     BASED_ERR_INVALID_ARG / BASED_ERR_UNSUPPORTED with nothing written.
+ *     A failed launch returns BASED_ERR_CUDA.  A kernel that gives up on a
+ *     bounded wait records BASED_ERR_TIMEOUT in a device status word, read
+ *     with based_get_device_error().
+ *   - dtype BASED_BF16: q/k/v/out are bfloat16, arithmetic accumulates in fp32.
+ *     dtype BASED_F32: everything is fp32 (fp32 CUDA-core arithmetic).
+ *     Recurrent states (state_kv, state_k) are always fp32.
+ *   - Feature order of the 273-row states: row 0 = constant 1; rows 1..16 =
+ *     x_i / 2; row 17 + 16 i + j = x_i x_j / (4 sqrt 2)   (d = 16).
+ *   - Thread safety: calls on different streams may run concurrently as long
+ *     as they do not share output buffers or workspace.
+ */
+#ifndef BASED_H
+#define BASED_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BASED_OK = 0,
+    BASED_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, negative size, ... */
+    BASED_ERR_UNSUPPORTED = 2,  /* valid but not implemented (d_feat != 16, ...) */
+    BASED_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+    BASED_ERR_TIMEOUT = 4,      /* a kernel gave up on a bounded wait */
+    BASED_ERR_WORKSPACE = 5     /* workspace missing or smaller than required */
+} based_status_t;
+
+typedef enum { BASED_F32 = 0, BASED_BF16 = 1 } based_dtype_t;
+
+typedef void* based_stream_t; /* a cudaStream_t */
+
+/* Version of this ABI (bumped on any incompatible change). */
+int based_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* based_status_string(based_status_t status);
+
+/*
+ * Bytes of device workspace based_linattn_fwd needs for this problem on the
+ * CURRENT device (it may split long sequences across CTAs and keep per-segment
+ * partial states there).  0 means the call needs none (workspace may be NULL).
+ * Returns (size_t)-1 for arguments based_linattn_fwd would reject.
+ */
+size_t based_linattn_workspace_bytes(int B, int H, int L, int d_feat, int d_v,
+                                     based_dtype_t dt);
+
+/*
+ * Causal linear attention with the Taylor feature map, one fused forward pass
+ * (the chunked "parallel" training view of the based/train README computed by
+ * one kernel: intra-chunk masked phi(Q)phi(K)^T [V|1], inter-chunk readout of
+ * the running KV/K states, state update, normaliser).
+ *
+ *   q, k      [B, H, L, d_feat]   dt          (d_feat must be 16)
+ *   v         [B, H, L, d_v]      dt          (d_v in {64, 128})
+ *   out       [B, H, L, d_v]      dt          (written)
+ *   eps       >= 0, added to the denominator only
+ *   state_kv  [B, H, 273, d_v] fp32 or NULL   final KV state S_L (written)
+ *   state_k   [B, H, 273]      fp32 or NULL   final K state z_L (written)
+ *   workspace device scratch of based_linattn_workspace_bytes(...) bytes, or
+ *             NULL when that is 0; contents need not be initialised and are
+ *             clobbered.
+ * L = 0 is valid: nothing is read, the states (if requested) are zeroed.
+ */
+based_status_t based_linattn_fwd(const void* q, const void* k, const void* v, void* out,
+                                 int B, int H, int L, int d_feat, int d_v,
+                                 based_dtype_t dt, float eps,
+                                 float* state_kv, float* state_k,
+                                 void* workspace, size_t workspace_bytes,
+                                 based_stream_t stream);
+
+/*
+ * Sliding-window causal softmax attention:
+ *   y_t = sum_{s = max(0, t-window+1)}^{t} softmax_s(q_t . k_s / sqrt(d_head)) v_s
+ *   q, k, v, out  [B, H, L, d_head]  dt   (d_head in {64, 128}; 1 <= window <= 64)
+ */
+based_status_t based_window_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                                     int B, int H, int L, int d_head, int window,
+                                     based_dtype_t dt, based_stream_t stream);
+
+/*
+ * Copy the last min(L, window) window keys/values of a prefill into the ring
+ * caches used by based_decode_step: position p (L-window <= p < L) goes to
+ * slot p mod window.  Other slots are left untouched.
+ *   k, v            [B, H, L, d_head]       dt
+ *   k_ring, v_ring  [B, H, window, d_head]  dt (written)
+ */
+based_status_t based_window_ring_fill(const void* k, const void* v, int B, int H, int L,
+                                      int d_head, int window, void* k_ring, void* v_ring,
+                                      based_dtype_t dt, based_stream_t stream);
+
+/*
+ * One decode step for B sequences that all sit at position `pos` (0-based; the
+ * prefill length when decoding starts).  Either part may be skipped.
+ *
+ * Linear part (skipped when q == NULL and H == 0):
+ *   q, k  [B, H, d_feat] dt;  v [B, H, d_v] dt;  out [B, H, d_v] dt (written)
+ *   state_kv [B, H, 273, d_v] fp32, state_k [B, H, 273] fp32, updated in place:
+ *     S += phi(k) v^T ; z += phi(k) ; out = phi(q)^T S / (phi(q) . z + eps)
+ *   (the new token is folded in before the read-out: causality is inclusive).
+ * Window part (skipped when wq == NULL and H_w == 0):
+ *   wq, wk, wv [B, H_w, d_head] dt; wout [B, H_w, d_head] dt (written)
+ *   k_ring, v_ring [B, H_w, window, d_head] dt, updated in place: slot
+ *   pos mod window receives wk/wv, then softmax attention over the slots that
+ *   hold positions max(0, pos-window+1) .. pos.
+ */
+based_status_t based_decode_step(const void* q, const void* k, const void* v,
+                                 float* state_kv, float* state_k, void* out,
+                                 const void* wq, const void* wk, const void* wv,
+                                 void* k_ring, void* v_ring, void* wout,
+                                 long long pos, int B, int H, int d_feat, int d_v,
+                                 int H_w, int d_head, int window,
+                                 based_dtype_t dt, float eps, based_stream_t stream);
+
+/*
+ * Synchronise `stream`, then read and clear the library's device status word
+ * on the current device.  Returns BASED_OK, or the first error a kernel
+ * recorded since the last call (BASED_ERR_TIMEOUT), or BASED_ERR_CUDA if the
+ * synchronisation itself failed.
+ */
+based_status_t based_get_device_error(based_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BASED_H */

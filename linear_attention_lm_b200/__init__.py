@@ -1,0 +1,230 @@
+"""Python binding of the B200 Based attention library (``libbased.so``).
+
+The functions named ``based_*`` mirror the C ABI in ``include/based.h`` one to
+one: they only derive sizes from the tensors' shapes, check dtype, device and
+contiguity, pass raw device pointers and the current CUDA stream through ctypes,
+and turn a non-OK status into ``BasedError``.  Every step of the computation
+runs in the library's CUDA kernels; there is no CPU or PyTorch fallback -- if
+the library is missing or cannot be loaded, every call raises.
+
+The lower-case helpers (``linattn``, ``window_attn``, ``decode_step``, ...)
+allocate outputs with torch and call the ``based_*`` functions.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from .inputs import WORKLOADS, Workload  # noqa: F401  (re-exported for callers)
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbased.so")
+NUM_FEATURES = 273
+D_FEAT = 16
+
+BASED_F32, BASED_BF16 = 0, 1
+_STATUS = {0: "BASED_OK", 1: "BASED_ERR_INVALID_ARG", 2: "BASED_ERR_UNSUPPORTED",
+           3: "BASED_ERR_CUDA", 4: "BASED_ERR_TIMEOUT", 5: "BASED_ERR_WORKSPACE"}
+EXPORTED_SYMBOLS = ("based_abi_version", "based_status_string",
+                    "based_linattn_workspace_bytes", "based_linattn_fwd",
+                    "based_window_attn_fwd", "based_window_ring_fill", "based_decode_step",
+                    "based_get_device_error")
+
+
+class BasedError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {_STATUS.get(status, status)}")
+        self.status = status
+
+
+_lock = threading.Lock()
+_lib = None
+_vp, _fp = ctypes.c_void_p, ctypes.POINTER(ctypes.c_float)
+_i, _f, _ll, _sz = ctypes.c_int, ctypes.c_float, ctypes.c_longlong, ctypes.c_size_t
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libbased.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"CUDA library {path} is missing; build it with "
+                "`python -m linear_attention_lm_b200.build` (nvcc, sm_100a)")
+        lib = ctypes.CDLL(path)
+        lib.based_abi_version.restype = _i
+        lib.based_status_string.argtypes = [_i]
+        lib.based_status_string.restype = ctypes.c_char_p
+        lib.based_linattn_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
+        lib.based_linattn_workspace_bytes.restype = _sz
+        lib.based_linattn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f,
+                                          _vp, _vp, _vp, _sz, _vp]
+        lib.based_window_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
+        lib.based_window_ring_fill.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _i, _vp]
+        lib.based_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                          _vp, _vp, _ll, _i, _i, _i, _i, _i, _i, _i, _i, _f,
+                                          _vp]
+        lib.based_get_device_error.argtypes = [_vp]
+        for name in ("based_linattn_fwd", "based_window_attn_fwd", "based_window_ring_fill",
+                     "based_decode_step", "based_get_device_error"):
+            getattr(lib, name).restype = _i
+        _lib = lib
+        return lib
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return BASED_F32
+    if t.dtype == torch.bfloat16:
+        return BASED_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr() or None
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise BasedError(fn, status)
+
+
+def _same_dtype(*ts):
+    ts = [t for t in ts if t is not None]
+    for t in ts[1:]:
+        if t.dtype != ts[0].dtype:
+            raise TypeError("q/k/v/out must share one dtype")
+    return _dtype_code(ts[0])
+
+
+def _f32(t):
+    if t is not None and t.dtype != torch.float32:
+        raise TypeError("states must be float32")
+    return _ptr(t)
+
+
+# ---------------------------------------------------------------------------
+# one-to-one wrappers of the C entry points
+# ---------------------------------------------------------------------------
+
+def based_abi_version() -> int:
+    return load_library().based_abi_version()
+
+
+def based_status_string(status: int) -> str:
+    return load_library().based_status_string(int(status)).decode()
+
+
+def based_linattn_workspace_bytes(B, H, L, d_feat, d_v, dt) -> int:
+    n = load_library().based_linattn_workspace_bytes(B, H, L, d_feat, d_v, dt)
+    if n == ctypes.c_size_t(-1).value:
+        raise BasedError("based_linattn_workspace_bytes", 1)
+    return n
+
+
+def based_linattn_fwd(q, k, v, out, eps: float = 1e-6, state_kv=None, state_k=None,
+                      workspace=None, stream=None):
+    B, H, L, d = q.shape
+    d_v = v.shape[-1]
+    dt = _same_dtype(q, k, v, out)
+    if workspace is None:
+        nbytes = based_linattn_workspace_bytes(B, H, L, d, d_v, dt)
+        if nbytes:
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(q.device):
+        st = load_library().based_linattn_fwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, L, d, d_v, dt, float(eps),
+            _f32(state_kv), _f32(state_k), _ptr(workspace), ws_bytes, _stream(stream))
+    _check("based_linattn_fwd", st)
+    return out
+
+
+def based_window_attn_fwd(q, k, v, out, window: int = 64, stream=None):
+    B, H, L, dh = q.shape
+    dt = _same_dtype(q, k, v, out)
+    with torch.cuda.device(q.device):
+        st = load_library().based_window_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, L,
+                                                  dh, int(window), dt, _stream(stream))
+    _check("based_window_attn_fwd", st)
+    return out
+
+
+def based_window_ring_fill(k, v, k_ring, v_ring, window: int = 64, stream=None):
+    B, H, L, dh = k.shape
+    dt = _same_dtype(k, v, k_ring, v_ring)
+    with torch.cuda.device(k.device):
+        st = load_library().based_window_ring_fill(_ptr(k), _ptr(v), B, H, L, dh, int(window),
+                                                   _ptr(k_ring), _ptr(v_ring), dt,
+                                                   _stream(stream))
+    _check("based_window_ring_fill", st)
+
+
+def based_decode_step(q, k, v, state_kv, state_k, out, wq=None, wk=None, wv=None, k_ring=None,
+                      v_ring=None, wout=None, pos: int = 0, window: int = 64,
+                      eps: float = 1e-6, stream=None):
+    ref = q if q is not None else wq
+    B = ref.shape[0]
+    H, d_feat, d_v = (q.shape[1], q.shape[2], v.shape[2]) if q is not None else (0, D_FEAT, 64)
+    H_w, d_head = (wq.shape[1], wq.shape[2]) if wq is not None else (0, 64)
+    dt = _same_dtype(q, k, v, out, wq, wk, wv, k_ring, v_ring, wout)
+    with torch.cuda.device(ref.device):
+        st = load_library().based_decode_step(
+            _ptr(q), _ptr(k), _ptr(v), _f32(state_kv), _f32(state_k), _ptr(out), _ptr(wq),
+            _ptr(wk), _ptr(wv), _ptr(k_ring), _ptr(v_ring), _ptr(wout), int(pos), B, H,
+            d_feat, d_v, H_w, d_head, int(window), dt, float(eps), _stream(stream))
+    _check("based_decode_step", st)
+
+
+def based_get_device_error(stream=None) -> int:
+    return load_library().based_get_device_error(_stream(stream))
+
+
+# ---------------------------------------------------------------------------
+# allocating helpers
+# ---------------------------------------------------------------------------
+
+def linattn(q, k, v, eps: float = 1e-6, return_state: bool = False, stream=None):
+    """y [B,H,L,d_v] (and the final fp32 states S [B,H,273,d_v], z [B,H,273])."""
+    B, H, L, _ = q.shape
+    out = torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    S = z = None
+    if return_state:
+        S = torch.empty((B, H, NUM_FEATURES, v.shape[-1]), dtype=torch.float32, device=v.device)
+        z = torch.empty((B, H, NUM_FEATURES), dtype=torch.float32, device=v.device)
+    based_linattn_fwd(q, k, v, out, eps, S, z, stream=stream)
+    return (out, S, z) if return_state else out
+
+
+def window_attn(q, k, v, window: int = 64, stream=None):
+    out = torch.empty_like(q)
+    return based_window_attn_fwd(q, k, v, out, window, stream=stream)
+
+
+def window_ring_fill(k, v, window: int = 64, stream=None):
+    B, H, _, dh = k.shape
+    k_ring = torch.zeros((B, H, window, dh), dtype=k.dtype, device=k.device)
+    v_ring = torch.zeros_like(k_ring)
+    based_window_ring_fill(k, v, k_ring, v_ring, window, stream=stream)
+    return k_ring, v_ring

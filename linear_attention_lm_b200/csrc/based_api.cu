@@ -1,0 +1,274 @@
+// based_api.cu -- the extern "C" entry points declared in include/based.h.
+//
+// Host code only validates arguments, picks the kernel for the dtype/shape and
+// launches it on the caller's stream; every step of the computation runs in the
+// kernels included below.  The whole library is one translation unit so that
+// the device status word is a single object.
+#include <math.h>
+#include <stdint.h>
+
+#include "based.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "linattn_simt.cuh"
+#include "window_simt.cuh"
+
+namespace based {
+
+template <typename T>
+__global__ void __launch_bounds__(256) ring_fill_kernel(const T* __restrict__ k,
+                                                        const T* __restrict__ v,
+                                                        T* __restrict__ k_ring,
+                                                        T* __restrict__ v_ring, int L, int dh,
+                                                        int W) {
+  const size_t bh = blockIdx.x;
+  const int n = min(L, W);
+  const int p0 = L - n;
+  for (int i = threadIdx.x; i < n * dh; i += blockDim.x) {
+    const int r = i / dh, c = i - r * dh;
+    const int p = p0 + r, slot = p % W;
+    k_ring[(bh * W + slot) * dh + c] = k[(bh * L + p) * dh + c];
+    v_ring[(bh * W + slot) * dh + c] = v[(bh * L + p) * dh + c];
+  }
+}
+
+}  // namespace based
+
+namespace {
+
+using namespace based;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline based_status_t launch_status() {
+  return cudaGetLastError() == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
+}
+
+template <typename K>
+inline bool set_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)bytes) == cudaSuccess;
+}
+
+// Shared argument checks of the prefill entry points.  Null tensor pointers
+// are accepted only when the tensors are empty.
+inline based_status_t check_tensor(const void* p, bool empty) {
+  if (p == nullptr) return empty ? BASED_OK : BASED_ERR_INVALID_ARG;
+  return aligned16(p) ? BASED_OK : BASED_ERR_INVALID_ARG;
+}
+
+based_status_t check_linattn(const void* q, const void* k, const void* v, const void* out,
+                             int B, int H, int L, int d_feat, int d_v, based_dtype_t dt,
+                             float eps, const float* state_kv, const float* state_k) {
+  if (B < 0 || H < 0 || L < 0) return BASED_ERR_INVALID_ARG;
+  if (dt != BASED_F32 && dt != BASED_BF16) return BASED_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || !isfinite(eps)) return BASED_ERR_INVALID_ARG;
+  if (d_feat != kD) return BASED_ERR_UNSUPPORTED;
+  if (d_v != 64 && d_v != 128) return BASED_ERR_UNSUPPORTED;
+  if ((long long)B * H > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
+  const bool empty = (long long)B * H * L == 0;
+  based_status_t s;
+  if ((s = check_tensor(q, empty)) != BASED_OK) return s;
+  if ((s = check_tensor(k, empty)) != BASED_OK) return s;
+  if ((s = check_tensor(v, empty)) != BASED_OK) return s;
+  if ((s = check_tensor(out, empty)) != BASED_OK) return s;
+  if (state_kv && !aligned16(state_kv)) return BASED_ERR_INVALID_ARG;
+  if (state_k && !aligned16(state_k)) return BASED_ERR_INVALID_ARG;
+  return BASED_OK;
+}
+
+template <typename T>
+based_status_t launch_linattn_simt(const void* q, const void* k, const void* v, void* out,
+                                   int BH, int L, int d_v, float eps, float* state_kv,
+                                   float* state_k, cudaStream_t st) {
+  auto kern = linattn_simt_kernel<T>;
+  const size_t smem = linattn_simt_smem_bytes();
+  if (!set_smem(kern, smem)) return BASED_ERR_CUDA;
+  dim3 grid((unsigned)BH, (unsigned)(d_v / kSimtCols));
+  kern<<<grid, kSimtThreads, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
+                                         static_cast<const T*>(v), static_cast<T*>(out),
+                                         state_kv, state_k, L, d_v, eps);
+  return launch_status();
+}
+
+template <typename T>
+based_status_t launch_window_simt(const void* q, const void* k, const void* v, void* out,
+                                  int BH, int L, int dh, int W, cudaStream_t st) {
+  auto kern = window_simt_kernel<T>;
+  const size_t smem = window_simt_smem_bytes(dh);
+  if (!set_smem(kern, smem)) return BASED_ERR_CUDA;
+  const long long nblk = (L + kWinQ - 1) / kWinQ;
+  if (nblk > 0x7fffffffLL || BH > 65535) return BASED_ERR_UNSUPPORTED;
+  dim3 grid((unsigned)nblk, (unsigned)BH);
+  kern<<<grid, kWinQ, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
+                                  static_cast<const T*>(v), static_cast<T*>(out), L, dh, W);
+  return launch_status();
+}
+
+template <typename T, int DV>
+based_status_t launch_decode(const DecodeParams& p, cudaStream_t st) {
+  auto kern = decode_step_kernel<T, DV>;
+  size_t smem = sizeof(float) * (size_t)DecodeLinearLayout<DV>::kSmemFloats;
+  if (p.n_win > 0) {
+    const size_t w = sizeof(float) * (size_t)decode_window_smem_floats(p.dh, p.W);
+    if (w > smem) smem = w;
+  }
+  if (!set_smem(kern, smem)) return BASED_ERR_CUDA;
+  const long long nblk = (long long)p.n_lin + p.n_win;
+  kern<<<(unsigned)nblk, 4 * DV, smem, st>>>(p);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int based_abi_version(void) { return 1; }
+
+const char* based_status_string(based_status_t status) {
+  switch (status) {
+    case BASED_OK: return "BASED_OK";
+    case BASED_ERR_INVALID_ARG: return "BASED_ERR_INVALID_ARG";
+    case BASED_ERR_UNSUPPORTED: return "BASED_ERR_UNSUPPORTED";
+    case BASED_ERR_CUDA: return "BASED_ERR_CUDA";
+    case BASED_ERR_TIMEOUT: return "BASED_ERR_TIMEOUT";
+    case BASED_ERR_WORKSPACE: return "BASED_ERR_WORKSPACE";
+  }
+  return "BASED_ERR_UNKNOWN";
+}
+
+size_t based_linattn_workspace_bytes(int B, int H, int L, int d_feat, int d_v,
+                                     based_dtype_t dt) {
+  if (B < 0 || H < 0 || L < 0 || (dt != BASED_F32 && dt != BASED_BF16) || d_feat != kD ||
+      (d_v != 64 && d_v != 128))
+    return (size_t)-1;
+  return 0;
+}
+
+based_status_t based_linattn_fwd(const void* q, const void* k, const void* v, void* out,
+                                 int B, int H, int L, int d_feat, int d_v, based_dtype_t dt,
+                                 float eps, float* state_kv, float* state_k, void* workspace,
+                                 size_t workspace_bytes, based_stream_t stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  based_status_t s =
+      check_linattn(q, k, v, out, B, H, L, d_feat, d_v, dt, eps, state_kv, state_k);
+  if (s != BASED_OK) return s;
+  const int BH = B * H;
+  if (BH == 0) return BASED_OK;
+  if (L == 0 && !state_kv && !state_k) return BASED_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dt == BASED_F32)
+    return launch_linattn_simt<float>(q, k, v, out, BH, L, d_v, eps, state_kv, state_k, st);
+  return launch_linattn_simt<__nv_bfloat16>(q, k, v, out, BH, L, d_v, eps, state_kv, state_k,
+                                            st);
+}
+
+based_status_t based_window_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                                     int B, int H, int L, int d_head, int window,
+                                     based_dtype_t dt, based_stream_t stream) {
+  if (B < 0 || H < 0 || L < 0) return BASED_ERR_INVALID_ARG;
+  if (dt != BASED_F32 && dt != BASED_BF16) return BASED_ERR_INVALID_ARG;
+  if (window < 1) return BASED_ERR_INVALID_ARG;
+  if (window > kWinQ) return BASED_ERR_UNSUPPORTED;
+  if (d_head != 64 && d_head != 128) return BASED_ERR_UNSUPPORTED;
+  const bool empty = (long long)B * H * L == 0;
+  based_status_t s;
+  if ((s = check_tensor(q, empty)) != BASED_OK) return s;
+  if ((s = check_tensor(k, empty)) != BASED_OK) return s;
+  if ((s = check_tensor(v, empty)) != BASED_OK) return s;
+  if ((s = check_tensor(out, empty)) != BASED_OK) return s;
+  if (empty) return BASED_OK;
+  if ((long long)B * H > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dt == BASED_F32) return launch_window_simt<float>(q, k, v, out, B * H, L, d_head, window, st);
+  return launch_window_simt<__nv_bfloat16>(q, k, v, out, B * H, L, d_head, window, st);
+}
+
+based_status_t based_window_ring_fill(const void* k, const void* v, int B, int H, int L,
+                                      int d_head, int window, void* k_ring, void* v_ring,
+                                      based_dtype_t dt, based_stream_t stream) {
+  if (B < 0 || H < 0 || L < 0 || window < 1) return BASED_ERR_INVALID_ARG;
+  if (dt != BASED_F32 && dt != BASED_BF16) return BASED_ERR_INVALID_ARG;
+  if (window > kWinQ) return BASED_ERR_UNSUPPORTED;
+  if (d_head != 64 && d_head != 128) return BASED_ERR_UNSUPPORTED;
+  const long long BH = (long long)B * H;
+  if (BH > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
+  based_status_t s;
+  if ((s = check_tensor(k, BH * L == 0)) != BASED_OK) return s;
+  if ((s = check_tensor(v, BH * L == 0)) != BASED_OK) return s;
+  if ((s = check_tensor(k_ring, BH == 0)) != BASED_OK) return s;
+  if ((s = check_tensor(v_ring, BH == 0)) != BASED_OK) return s;
+  if (BH == 0 || L == 0) return BASED_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dt == BASED_F32)
+    ring_fill_kernel<float><<<(unsigned)BH, 256, 0, st>>>(
+        static_cast<const float*>(k), static_cast<const float*>(v), static_cast<float*>(k_ring),
+        static_cast<float*>(v_ring), L, d_head, window);
+  else
+    ring_fill_kernel<__nv_bfloat16><<<(unsigned)BH, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+        static_cast<__nv_bfloat16*>(k_ring), static_cast<__nv_bfloat16*>(v_ring), L, d_head,
+        window);
+  return launch_status();
+}
+
+based_status_t based_decode_step(const void* q, const void* k, const void* v, float* state_kv,
+                                 float* state_k, void* out, const void* wq, const void* wk,
+                                 const void* wv, void* k_ring, void* v_ring, void* wout,
+                                 long long pos, int B, int H, int d_feat, int d_v, int H_w,
+                                 int d_head, int window, based_dtype_t dt, float eps,
+                                 based_stream_t stream) {
+  if (B < 0 || H < 0 || H_w < 0 || pos < 0) return BASED_ERR_INVALID_ARG;
+  if (dt != BASED_F32 && dt != BASED_BF16) return BASED_ERR_INVALID_ARG;
+  const bool lin = q != nullptr || H > 0;
+  const bool win = wq != nullptr || H_w > 0;
+  if (!lin && !win) return BASED_ERR_INVALID_ARG;
+  if (lin) {
+    if (H < 1 || !q || !k || !v || !state_kv || !state_k || !out) return BASED_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state_kv) ||
+        !aligned16(state_k) || !aligned16(out))
+      return BASED_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f) || !isfinite(eps)) return BASED_ERR_INVALID_ARG;
+    if (d_feat != kD) return BASED_ERR_UNSUPPORTED;
+    if (d_v != 64 && d_v != 128) return BASED_ERR_UNSUPPORTED;
+  }
+  if (win) {
+    if (H_w < 1 || !wq || !wk || !wv || !k_ring || !v_ring || !wout) return BASED_ERR_INVALID_ARG;
+    if (!aligned16(wq) || !aligned16(wk) || !aligned16(wv) || !aligned16(k_ring) ||
+        !aligned16(v_ring) || !aligned16(wout))
+      return BASED_ERR_INVALID_ARG;
+    if (window < 1) return BASED_ERR_INVALID_ARG;
+    if (window > kWinQ) return BASED_ERR_UNSUPPORTED;
+    if (d_head != 64 && d_head != 128) return BASED_ERR_UNSUPPORTED;
+  }
+  const long long n_lin = lin ? (long long)B * H : 0, n_win = win ? (long long)B * H_w : 0;
+  if (n_lin + n_win > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
+  if (n_lin + n_win == 0) return BASED_OK;
+  DecodeParams p;
+  p.q = q; p.k = k; p.v = v; p.S = state_kv; p.z = state_k; p.out = out;
+  p.wq = wq; p.wk = wk; p.wv = wv; p.k_ring = k_ring; p.v_ring = v_ring; p.wout = wout;
+  p.pos = pos; p.n_lin = (int)n_lin; p.n_win = (int)n_win;
+  p.dh = d_head; p.W = window; p.eps = eps;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool wide = lin && d_v == 128;
+  if (dt == BASED_F32)
+    return wide ? launch_decode<float, 128>(p, st) : launch_decode<float, 64>(p, st);
+  return wide ? launch_decode<__nv_bfloat16, 128>(p, st) : launch_decode<__nv_bfloat16, 64>(p, st);
+}
+
+based_status_t based_get_device_error(based_stream_t stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return BASED_ERR_CUDA;
+  int v = BASED_OK;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess)
+    return BASED_ERR_CUDA;
+  if (v != BASED_OK) {
+    const int ok = BASED_OK;
+    if (cudaMemcpyToSymbol(g_device_status, &ok, sizeof(int)) != cudaSuccess)
+      return BASED_ERR_CUDA;
+  }
+  return static_cast<based_status_t>(v);
+}
+
+}  // extern "C"

@@ -1,0 +1,141 @@
+// linattn_simt.cuh -- causal Taylor linear attention on CUDA cores in fp32.
+//
+// The chunked ("fla_parallel") view of the based/train README, computed in fp32
+// for fp32 inputs: per chunk of 32 tokens
+//   A      = (phi(Q_c) phi(K_c)^T) masked to s <= t            (intra-chunk)
+//   num_t  = phi(q_t)^T S + sum_s A_ts v_s,  den_t = phi(q_t).z + sum_s A_ts
+//   y_t    = num_t / (den_t + eps)
+//   S     += phi(K_c)^T V_c,  z += sum_s phi(k_s)                (state update)
+// with S (273 x 64 fp32) and z resident in shared memory for the whole
+// sequence.  One CTA per (b, h, 64-column slice of d_v).  The feature rows use
+// a pitch of 273 floats (odd), so a warp reading one feature of 32 different
+// tokens touches 32 distinct banks.
+#pragma once
+
+#include "common.cuh"
+
+namespace based {
+
+constexpr int kSimtChunk = 32;
+constexpr int kSimtCols = 64;
+constexpr int kSimtThreads = 256;
+
+__host__ __device__ constexpr size_t linattn_simt_smem_bytes() {
+  return sizeof(float) * (size_t)(kF * kSimtCols + 276 + 2 * kSimtChunk * kF +
+                                  kSimtChunk * kSimtCols + kSimtChunk * 33 + kSimtChunk +
+                                  2 * kSimtChunk * kD);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
+    const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+    T* __restrict__ out, float* __restrict__ state_kv, float* __restrict__ state_k, int L,
+    int DV, float eps) {
+  constexpr int C = kSimtChunk, NC = kSimtCols, NT = kSimtThreads;
+  extern __shared__ __align__(16) float smem[];
+  float* S = smem;                 // [273][64]
+  float* z = S + kF * NC;          // [273] (+pad)
+  float* fq = z + 276;             // [32][273]
+  float* fk = fq + C * kF;         // [32][273]
+  float* vs = fk + C * kF;         // [32][64]
+  float* A = vs + C * NC;          // [32][33]
+  float* den = A + C * 33;         // [32]
+  float* xq = den + C;             // [32][16]
+  float* xk = xq + C * kD;         // [32][16]
+
+  const int tid = threadIdx.x;
+  const int bh = blockIdx.x, col0 = blockIdx.y * NC;
+  q += (size_t)bh * L * kD;
+  k += (size_t)bh * L * kD;
+  v += (size_t)bh * L * DV + col0;
+  out += (size_t)bh * L * DV + col0;
+
+  for (int i = tid; i < kF * NC; i += NT) S[i] = 0.0f;
+  for (int i = tid; i < 276; i += NT) z[i] = 0.0f;
+
+  const int j = tid % NC, grp = tid / NC;  // output column, row group (0..3)
+  for (int t0 = 0; t0 < L; t0 += C) {
+    const int n = min(C, L - t0);
+    __syncthreads();  // previous chunk's state update is complete
+    for (int i = tid; i < C * kD; i += NT) {
+      const int r = i / kD;
+      xq[i] = r < n ? to_f32(q[(size_t)t0 * kD + i]) : 0.0f;
+      xk[i] = r < n ? to_f32(k[(size_t)t0 * kD + i]) : 0.0f;
+    }
+    for (int i = tid; i < C * NC; i += NT) {
+      const int r = i / NC, c = i - r * NC;
+      vs[i] = r < n ? to_f32(v[(size_t)(t0 + r) * DV + c]) : 0.0f;
+    }
+    __syncthreads();
+    for (int i = tid; i < C * kF; i += NT) {
+      const int r = i / kF, f = i - r * kF;
+      fq[i] = phi_feature(xq + r * kD, f);
+      fk[i] = phi_feature(xk + r * kD, f);
+    }
+    __syncthreads();
+    // intra-chunk scores, causal mask s <= t
+    for (int i = tid; i < C * C; i += NT) {
+      const int t = i / C, s = i - t * C;
+      float a = 0.0f;
+      if (s <= t) {
+        const float* a_row = fq + t * kF;
+        const float* b_row = fk + s * kF;
+        for (int f = 0; f < kF; ++f) a = fmaf(a_row[f], b_row[f], a);
+      }
+      A[t * 33 + s] = a;
+    }
+    __syncthreads();
+    // denominators: inter (phi(q).z) + intra (row sum of A)
+    if (tid < C) {
+      float d = 0.0f;
+      const float* a_row = fq + tid * kF;
+      for (int f = 0; f < kF; ++f) d = fmaf(a_row[f], z[f], d);
+      for (int s = 0; s < C; ++s) d += A[tid * 33 + s];
+      den[tid] = d;
+    }
+    // numerators for rows grp, grp+4, ..., column j
+    float acc[C / 4];
+#pragma unroll
+    for (int i = 0; i < C / 4; ++i) acc[i] = 0.0f;
+    for (int f = 0; f < kF; ++f) {
+      const float sf = S[f * NC + j];
+#pragma unroll
+      for (int i = 0; i < C / 4; ++i) acc[i] = fmaf(fq[(grp + 4 * i) * kF + f], sf, acc[i]);
+    }
+    for (int s = 0; s < C; ++s) {
+      const float vj = vs[s * NC + j];
+#pragma unroll
+      for (int i = 0; i < C / 4; ++i) acc[i] = fmaf(A[(grp + 4 * i) * 33 + s], vj, acc[i]);
+    }
+    __syncthreads();  // den ready; all reads of S and z for this chunk done
+#pragma unroll
+    for (int i = 0; i < C / 4; ++i) {
+      const int t = grp + 4 * i;
+      if (t < n) out[(size_t)(t0 + t) * DV + j] = from_f32<T>(acc[i] / (den[t] + eps));
+    }
+    // state update
+    for (int f = grp; f < kF; f += 4) {
+      float s_acc = S[f * NC + j];
+      for (int s = 0; s < n; ++s) s_acc = fmaf(fk[s * kF + f], vs[s * NC + j], s_acc);
+      S[f * NC + j] = s_acc;
+    }
+    for (int f = tid; f < kF; f += NT) {
+      float z_acc = z[f];
+      for (int s = 0; s < n; ++s) z_acc += fk[s * kF + f];
+      z[f] = z_acc;
+    }
+  }
+  __syncthreads();
+  if (state_kv) {
+    float* dst = state_kv + (size_t)bh * kF * DV + col0;
+    for (int i = tid; i < kF * NC; i += NT) {
+      const int f = i / NC, c = i - f * NC;
+      dst[(size_t)f * DV + c] = S[i];
+    }
+  }
+  if (state_k && blockIdx.y == 0) {
+    for (int f = tid; f < kF; f += NT) state_k[(size_t)bh * kF + f] = z[f];
+  }
+}
+
+}  // namespace based

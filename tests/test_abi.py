@@ -1,0 +1,126 @@
+"""Host-only checks of the C ABI: the library builds, loads, exports every
+symbol include/based.h declares, and rejects bad arguments on the host before
+touching the GPU.  No kernel is launched here."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import linear_attention_lm_b200 as lab
+from linear_attention_lm_b200 import build as lab_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "based.h")
+
+INVALID, UNSUPPORTED = 1, 2
+
+
+@pytest.fixture(scope="module")
+def lib():
+    lab_build.build()
+    return lab.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(based_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_binding_symbols():
+    assert declared_functions() == sorted(lab.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert lib.based_abi_version() == 1
+
+
+def test_built_for_sm100a():
+    out = open(lab_build.LIB_PATH, "rb").read()
+    assert b"sm_100a" in out or b"sm_100" in out
+
+
+def test_status_strings(lib):
+    for code, name in [(0, "BASED_OK"), (1, "BASED_ERR_INVALID_ARG"), (2, "BASED_ERR_UNSUPPORTED"),
+                       (3, "BASED_ERR_CUDA"), (4, "BASED_ERR_TIMEOUT"), (5, "BASED_ERR_WORKSPACE")]:
+        assert lab.based_status_string(code) == name
+    assert lab.based_status_string(99) == "BASED_ERR_UNKNOWN"
+
+
+def test_workspace_query_rejects_bad_args(lib):
+    bad = ctypes.c_size_t(-1).value
+    f = lib.based_linattn_workspace_bytes
+    assert f(1, 1, 16, 8, 64, 1) == bad       # d_feat != 16
+    assert f(1, 1, 16, 16, 96, 1) == bad      # d_v not 64/128
+    assert f(-1, 1, 16, 16, 64, 1) == bad
+    assert f(1, 1, 16, 16, 64, 7) == bad      # dtype
+    assert f(1, 1, 16, 16, 64, 1) != bad
+
+
+FAKE = 1 << 20  # a 16-byte-aligned non-null address; never dereferenced here
+
+
+def lin_call(lib, q=FAKE, k=FAKE, v=FAKE, out=FAKE, B=1, H=1, L=8, d=16, dv=64, dt=1,
+             eps=1e-6, skv=None, sk=None):
+    return lib.based_linattn_fwd(q, k, v, out, B, H, L, d, dv, dt, eps, skv, sk, None, 0, None)
+
+
+def test_linattn_host_validation(lib):
+    assert lin_call(lib, d=8) == UNSUPPORTED
+    assert lin_call(lib, dv=32) == UNSUPPORTED
+    assert lin_call(lib, B=-1) == INVALID
+    assert lin_call(lib, q=None) == INVALID
+    assert lin_call(lib, k=FAKE + 4) == INVALID          # misaligned
+    assert lin_call(lib, eps=-1.0) == INVALID
+    assert lin_call(lib, eps=float("nan")) == INVALID
+    assert lin_call(lib, dt=5) == INVALID
+    assert lin_call(lib, skv=FAKE + 8) == INVALID
+    # empty problems are valid no-ops (no launch, no pointer needed)
+    assert lin_call(lib, q=None, k=None, v=None, out=None, B=0) == 0
+    assert lin_call(lib, q=None, k=None, v=None, out=None, L=0) == 0
+
+
+def test_window_host_validation(lib):
+    f = lib.based_window_attn_fwd
+    assert f(FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 64, 0, 1, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 64, 65, 1, None) == UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 96, 64, 1, None) == UNSUPPORTED
+    assert f(None, FAKE, FAKE, FAKE, 1, 1, 8, 64, 64, 1, None) == INVALID
+    assert f(None, None, None, None, 1, 1, 0, 64, 64, 1, None) == 0
+
+
+def test_decode_host_validation(lib):
+    f = lib.based_decode_step
+    N = None
+    # nothing to do
+    assert f(N, N, N, N, N, N, N, N, N, N, N, N, 0, 1, 0, 16, 64, 0, 64, 64, 1, 1e-6, N) == INVALID
+    # linear part missing its state
+    assert f(FAKE, FAKE, FAKE, N, FAKE, FAKE, N, N, N, N, N, N, 0, 1, 1, 16, 64, 0, 64, 64, 1,
+             1e-6, N) == INVALID
+    # negative position
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, N, N, N, N, N, N, -1, 1, 1, 16, 64, 0, 64, 64, 1,
+             1e-6, N) == INVALID
+    # window part with an unsupported head dim
+    assert f(N, N, N, N, N, N, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 3, 1, 0, 16, 64, 1, 32, 64, 1,
+             1e-6, N) == UNSUPPORTED
+
+
+def test_binding_refuses_cpu_tensors():
+    q = torch.zeros(1, 1, 8, 16, dtype=torch.bfloat16)
+    v = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        lab.based_linattn_fwd(q, q, v, v.clone())
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    saved = lab._lib
+    try:
+        lab._lib = None
+        with pytest.raises(RuntimeError):
+            lab.load_library(str(tmp_path / "nope.so"))
+    finally:
+        lab._lib = saved
