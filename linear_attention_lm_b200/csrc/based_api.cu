@@ -4,6 +4,7 @@
 // launches it on the caller's stream; every step of the computation runs in the
 // kernels included below.  The whole library is one translation unit so that
 // the device status word is a single object.
+#include <cudaTypedefs.h>
 #include <math.h>
 #include <stdint.h>
 
@@ -11,6 +12,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "linattn_simt.cuh"
+#include "linattn_tc.cuh"
 #include "window_simt.cuh"
 
 namespace based {
@@ -91,6 +93,49 @@ based_status_t launch_linattn_simt(const void* q, const void* k, const void* v, 
   return launch_status();
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) !=
+            cudaSuccess ||
+        qr != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// 3-D map over a [BH, L, cols] bf16 tensor with a (64 cols x rows x 1) box and
+// 128-byte swizzle; rows past L read as zero.
+bool make_rows_map(CUtensorMap* m, const void* base, int cols, int L, int BH, int box_rows) {
+  auto enc = encode_tiled();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)(L > 0 ? L : 1), (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)cols * 2 * (cuuint64_t)(L > 0 ? L : 1)};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int DV>
+based_status_t launch_linattn_tc(const void* q, const void* k, const void* v, void* out, int BH,
+                                 int L, float eps, float* state_kv, float* state_k,
+                                 cudaStream_t st) {
+  CUtensorMap vmap;
+  if (!make_rows_map(&vmap, v, DV, L, BH, kTcChunk)) return BASED_ERR_CUDA;
+  auto kern = linattn_tc_kernel<DV>;
+  const size_t smem = TcLayout<DV>::kSmem;
+  if (!set_smem(kern, smem)) return BASED_ERR_CUDA;
+  kern<<<(unsigned)BH, kTcThreads, smem, st>>>(
+      vmap, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+      static_cast<__nv_bfloat16*>(out), state_kv, state_k, L, eps);
+  return launch_status();
+}
+
 template <typename T>
 based_status_t launch_window_simt(const void* q, const void* k, const void* v, void* out,
                                   int BH, int L, int dh, int W, cudaStream_t st) {
@@ -160,8 +205,8 @@ based_status_t based_linattn_fwd(const void* q, const void* k, const void* v, vo
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dt == BASED_F32)
     return launch_linattn_simt<float>(q, k, v, out, BH, L, d_v, eps, state_kv, state_k, st);
-  return launch_linattn_simt<__nv_bfloat16>(q, k, v, out, BH, L, d_v, eps, state_kv, state_k,
-                                            st);
+  return d_v == 64 ? launch_linattn_tc<64>(q, k, v, out, BH, L, eps, state_kv, state_k, st)
+                   : launch_linattn_tc<128>(q, k, v, out, BH, L, eps, state_kv, state_k, st);
 }
 
 based_status_t based_window_attn_fwd(const void* q, const void* k, const void* v, void* out,
