@@ -14,6 +14,7 @@
 #include "linattn_simt.cuh"
 #include "linattn_tc.cuh"
 #include "window_simt.cuh"
+#include "window_tc.cuh"
 
 namespace based {
 
@@ -136,6 +137,24 @@ based_status_t launch_linattn_tc(const void* q, const void* k, const void* v, vo
   return launch_status();
 }
 
+template <int DH>
+based_status_t launch_window_tc(const void* q, const void* k, const void* v, void* out, int BH,
+                                int L, int W, cudaStream_t st) {
+  CUtensorMap qm, km, vm;
+  if (!make_rows_map(&qm, q, DH, L, BH, kWtQ) || !make_rows_map(&km, k, DH, L, BH, kWtKeys) ||
+      !make_rows_map(&vm, v, DH, L, BH, kWtKeys))
+    return BASED_ERR_CUDA;
+  auto kern = window_tc_kernel<DH>;
+  const size_t smem = WtLayout<DH>::kSmem;
+  if (!set_smem(kern, smem)) return BASED_ERR_CUDA;
+  const int n_tiles = (L + kWtQ - 1) / kWtQ;
+  const long long nblk = (long long)n_tiles * BH;
+  if (nblk > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
+  kern<<<(unsigned)nblk, kWtThreads, smem, st>>>(qm, km, vm, static_cast<__nv_bfloat16*>(out), L,
+                                                  W, n_tiles);
+  return launch_status();
+}
+
 template <typename T>
 based_status_t launch_window_simt(const void* q, const void* k, const void* v, void* out,
                                   int BH, int L, int dh, int W, cudaStream_t st) {
@@ -227,7 +246,8 @@ based_status_t based_window_attn_fwd(const void* q, const void* k, const void* v
   if ((long long)B * H > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dt == BASED_F32) return launch_window_simt<float>(q, k, v, out, B * H, L, d_head, window, st);
-  return launch_window_simt<__nv_bfloat16>(q, k, v, out, B * H, L, d_head, window, st);
+  return d_head == 64 ? launch_window_tc<64>(q, k, v, out, B * H, L, window, st)
+                      : launch_window_tc<128>(q, k, v, out, B * H, L, window, st);
 }
 
 based_status_t based_window_ring_fill(const void* k, const void* v, int B, int H, int L,

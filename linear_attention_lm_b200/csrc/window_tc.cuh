@@ -1,0 +1,217 @@
+// window_tc.cuh -- sliding-window causal softmax attention on the sm_100a tensor cores.
+//
+// Based README, introduction, item 1: exact softmax attention over a short
+// sliding window (size 64) models the fine-grained local interactions.  For
+// query t the keys are s in [max(0, t-W+1), t] (W <= 64), scores q_t.k_s/sqrt(dh).
+//
+// One CTA per tile of 128 queries [t0, t0+128) of one (b, h).  The keys any of
+// its queries can see lie in [t0-63, t0+127]; the CTA loads the 192 rows
+// [t0-64, t0+128) of K and V by TMA (rows before 0 or past L read as zero) and
+//   S = Q K^T        tcgen05, M=128, N=192, K=dh            -> TMEM (fp32)
+//   P = exp(S - m)   CUDA cores: thread r owns query row r; it reads the 96
+//                    TMEM columns covering its 64-key band, masks, takes the exact
+//                    row max, exponentiates, keeps the row sum l in a register
+//                    and writes P (bf16, zero outside the band) to shared memory
+//   O = P V          tcgen05, M=128, N=dh, K=192             -> TMEM (fp32)
+//   y = O / l        CUDA cores, straight from TMEM to global memory.
+// P reuses the shared memory of Q and K, which are dead once S is computed.
+#pragma once
+
+#include "common.cuh"
+#include "umma.cuh"
+
+namespace based {
+
+constexpr int kWtQ = 128;      // queries per CTA
+constexpr int kWtKeys = 192;   // staged key rows per CTA
+constexpr int kWtThreads = 128;
+
+template <int DH>
+struct WtLayout {
+  static constexpr int kQ = 0;                              // Q [128 x DH] K-major SW128
+  static constexpr int kK = kQ + kWtQ * DH * 2;             // K [192 x DH] K-major SW128
+  static constexpr int kP = 0;                              // P [128 x 192] bf16 K-major (aliases Q,K)
+  static constexpr int kPBytes = kWtQ * kWtKeys * 2;
+  static constexpr int kQKEnd = kK + kWtKeys * DH * 2;
+  static constexpr int kV = (kQKEnd > kPBytes ? kQKEnd : kPBytes);  // V [192 x DH] MN-major SW128
+  static constexpr int kBar = kV + kWtKeys * DH * 2;
+  static constexpr int kBytes = kBar + 64;
+  static constexpr size_t kSmem = kBytes + 1024;
+  static constexpr int kTmS = 0;
+  static constexpr int kTmO = kWtKeys;
+  static constexpr int kTmemCols = (kTmO + DH <= 256) ? 256 : 512;
+};
+
+template <int DH>
+__global__ void __launch_bounds__(kWtThreads)
+    window_tc_kernel(const __grid_constant__ CUtensorMap qmap,
+                     const __grid_constant__ CUtensorMap kmap,
+                     const __grid_constant__ CUtensorMap vmap, __nv_bfloat16* __restrict__ out,
+                     int L, int W, int n_tiles) {
+  using Lay = WtLayout<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + Lay::kBar);
+  uint64_t* bar_s = bar_tma + 1;
+  uint64_t* bar_o = bar_tma + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_tma + 3);
+  int* abort_flag = reinterpret_cast<int*>(bar_tma + 4);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tile = blockIdx.x % n_tiles;
+  const int bh = blockIdx.x / n_tiles;
+  const int t0 = tile * kWtQ;
+
+  if (tid == 0) {
+    umma::mbar_init(bar_tma, 1);
+    umma::mbar_init(bar_s, 1);
+    umma::mbar_init(bar_o, 1);
+    *abort_flag = 0;
+    umma::fence_mbar_init();
+    constexpr uint32_t bytes = (kWtQ + 2 * kWtKeys) * DH * 2;
+    umma::mbar_arrive_expect_tx(bar_tma, bytes);
+#pragma unroll
+    for (int b = 0; b < DH / 64; ++b) {
+      umma::tma_load_3d(sm + Lay::kQ + b * kWtQ * 128, &qmap, bar_tma, b * 64, t0, bh);
+      umma::tma_load_3d(sm + Lay::kK + b * kWtKeys * 128, &kmap, bar_tma, b * 64, t0 - 64, bh);
+      umma::tma_load_3d(sm + Lay::kV + b * kWtKeys * 128, &vmap, bar_tma, b * 64, t0 - 64, bh);
+    }
+  }
+  if (warp == 0) {
+    umma::tmem_alloc(tmem_slot, Lay::kTmemCols);
+    umma::tmem_relinquish();
+  }
+  umma::tc_fence_before();
+  __syncthreads();
+  umma::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tm_lane = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t sQ = umma::smem_u32(sm + Lay::kQ), sK = umma::smem_u32(sm + Lay::kK),
+                 sV = umma::smem_u32(sm + Lay::kV), sP = umma::smem_u32(sm + Lay::kP);
+
+  // ---- S = Q K^T ----------------------------------------------------------------
+  if (tid == 0) {
+    if (!umma::mbar_wait(bar_tma, 0)) {
+      record_device_error(BASED_ERR_TIMEOUT);
+      *abort_flag = 1;
+    } else {
+      umma::tc_fence_after();
+      const uint32_t id = umma::idesc_bf16(kWtQ, kWtKeys, false, false);
+#pragma unroll
+      for (int k0 = 0; k0 < DH; k0 += 16)
+        umma::mma_bf16(tmem + Lay::kTmS, umma::desc_kmajor_sw128(sQ, k0, kWtQ),
+                       umma::desc_kmajor_sw128(sK, k0, kWtKeys), id, k0 > 0);
+      umma::mma_commit(bar_s);
+    }
+  }
+  __syncthreads();
+  if (*abort_flag) goto done;
+  if (!umma::mbar_wait(bar_s, 0)) {
+    record_device_error(BASED_ERR_TIMEOUT);
+    *abort_flag = 1;
+  }
+  umma::tc_fence_after();
+
+  // ---- P = exp(S - m) over each row's band ---------------------------------------------
+  float l_row;
+  {
+    const int r = tid, t = t0 + r;
+    const int cb = warp * 32;  // first staged key column this warp reads
+    float sv[96];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) umma::tmem_ld32(tmem + Lay::kTmS + tm_lane + cb + 32 * j, sv + 32 * j);
+    // valid staged columns c (key s = t0 - 64 + c): s in [max(0, t-W+1), t]
+    const int c_hi = r + 64;
+    const int c_lo = max(max(r + 1, 64 - t0), t - W + 1 - (t0 - 64));
+    const float scale = rsqrtf((float)DH) * 1.4426950408889634f;  // 1/sqrt(dh) * log2(e)
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 96; ++i) {
+      const int c = cb + i;
+      if (c >= c_lo && c <= c_hi) m = fmaxf(m, sv[i]);
+    }
+    const bool live = t < L;
+    float l = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 96; ++i) {
+      const int c = cb + i;
+      const float p = (live && c >= c_lo && c <= c_hi) ? exp2f((sv[i] - m) * scale) : 0.0f;
+      sv[i] = p;
+      l += p;
+    }
+    l_row = live ? l : 1.0f;
+    // P row r: 24 chunks of 8 keys; chunks 4w .. 4w+11 carry the band, the rest are zero
+    __syncwarp();
+#pragma unroll
+    for (int kc = 0; kc < kWtKeys / 8; ++kc) {
+      const int rel = kc - warp * 4;
+      uint4 val = make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int j = 0; j < 12; ++j) {
+        if (rel == j) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 b = __floats2bfloat162_rn(sv[8 * j + 2 * e], sv[8 * j + 2 * e + 1]);
+            pk[e] = *reinterpret_cast<const uint32_t*>(&b);
+          }
+          val = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+      *reinterpret_cast<uint4*>(sm + Lay::kP + ((r >> 3) * (kWtKeys / 8) + kc) * 128 + (r & 7) * 16) = val;
+    }
+  }
+  umma::fence_async_smem();
+  umma::tc_fence_before();
+  __syncthreads();
+  umma::tc_fence_after();
+  if (*abort_flag) goto done;
+
+  // ---- O = P V --------------------------------------------------------------------------
+  if (tid == 0) {
+    const uint32_t id = umma::idesc_bf16(kWtQ, DH, false, true);
+#pragma unroll
+    for (int k0 = 0; k0 < kWtKeys; k0 += 16)
+      umma::mma_bf16(tmem + Lay::kTmO, umma::desc_kmajor_none(sP, k0, kWtKeys),
+                     umma::desc_mnmajor_sw128(sV, k0, kWtKeys), id, k0 > 0);
+    umma::mma_commit(bar_o);
+  }
+  __syncwarp();
+  if (!umma::mbar_wait(bar_o, 0)) {
+    record_device_error(BASED_ERR_TIMEOUT);
+    *abort_flag = 1;
+  }
+  umma::tc_fence_after();
+  {
+    const int r = tid, t = t0 + r;
+    const float inv = 1.0f / l_row;
+#pragma unroll
+    for (int c32 = 0; c32 < DH / 32; ++c32) {
+      float o[32];
+      umma::tmem_ld32(tmem + Lay::kTmO + tm_lane + c32 * 32, o);
+      if (t < L && !*abort_flag) {
+        uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)bh * L + t) * DH + c32 * 32);
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 b =
+                __floats2bfloat162_rn(o[ch * 8 + 2 * e] * inv, o[ch * 8 + 2 * e + 1] * inv);
+            pk[e] = *reinterpret_cast<const uint32_t*>(&b);
+          }
+          dst[ch] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+    }
+  }
+done:
+  // an aborted tile may still have its loads in flight: wait for them (bounded)
+  if (tid == 0 && *abort_flag) umma::mbar_wait(bar_tma, 0);
+  umma::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) umma::tmem_dealloc(tmem, Lay::kTmemCols);
+}
+
+}  // namespace based
