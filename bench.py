@@ -75,7 +75,7 @@ def decode_bytes(w):
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    QUERY = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -87,7 +87,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
@@ -104,23 +104,39 @@ class ClockSampler:
                 out, _ = self.proc.communicate()
             self.lines = [l for l in out.splitlines() if l.strip()]
 
+    def mark(self, which):
+        setattr(self, which, time.time())
+
     def summary(self):
-        sm, mx, reasons = [], None, set()
+        """Median SM clock and active throttle reasons over the samples taken
+        inside [t_start, t_stop]; if the window was shorter than the sampling
+        period, the samples nearest to it."""
+        import datetime
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        rows = []
         for line in getattr(self, "lines", []):
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(f[1]), float(f[2]), f[5:9]))
             except ValueError:
                 continue
-            for n, val in zip(names, f[5:9]):
+        t0, t1 = getattr(self, "t_start", None), getattr(self, "t_stop", None)
+        inside = [r for r in rows if t0 is not None and t0 <= r[0] <= t1]
+        sel = inside
+        if not sel and rows and t0 is not None:
+            mid = 0.5 * (t0 + t1)
+            sel = sorted(rows, key=lambda r: abs(r[0] - mid))[:2]
+        reasons = set()
+        for r in sel:
+            for n, val in zip(names, r[3]):
                 if val.lower().startswith("active"):
                     reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median([r[1] for r in sel]) if sel else None,
+                "sm_max_mhz": sel[0][2] if sel else None, "reasons": sorted(reasons),
+                "samples_in_window": len(inside)}
 
 
 # ---------------------------------------------------------------------------
@@ -170,14 +186,17 @@ def run_ours(args, rank, world, dev):
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index) as clk:
+        time.sleep(0.3)  # let the sampler start
         if world > 1:
             torch.distributed.barrier()
         torch.cuda.synchronize()
+        clk.mark("t_start")
         start.record()
         for i in range(args.steps):
             step(i, evs[i])
         stop.record()
         torch.cuda.synchronize()
+        clk.mark("t_stop")
         if world > 1:
             torch.distributed.barrier()
     elapsed_ms = start.elapsed_time(stop)
@@ -223,7 +242,7 @@ def run_ours(args, rank, world, dev):
         "e2e": e2e,
         "decode": decode,
         "gpu_launches": 2 * args.steps,
-        "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+        "clocks": clocks,
     }
     if rank == 0 and world == 1:
         line["cpu_baseline"] = cpu_baseline(w)
@@ -392,7 +411,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     args = ap.parse_args()

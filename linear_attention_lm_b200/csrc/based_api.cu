@@ -122,18 +122,75 @@ bool make_rows_map(CUtensorMap* m, const void* base, int cols, int L, int BH, in
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+// Segments per sequence for the tensor-core prefill: enough CTAs to cover the
+// SMs when B*H is small, at least two chunks per segment.
+struct TcPlan {
+  int n_seg = 1;
+  int seg_chunks = 1;
+  size_t workspace = 0;
+};
+TcPlan plan_linattn_tc(long long BH, int L, int d_v) {
+  TcPlan pl;
+  const int n_chunks = (L + kTcChunk - 1) / kTcChunk;
+  pl.seg_chunks = n_chunks > 0 ? n_chunks : 1;
+  if (BH <= 0 || n_chunks < 4) return pl;
+  const long long sms = device_sm_count();
+  long long want = sms / BH;
+  if (want < 2) return pl;
+  if (want > n_chunks / 2) want = n_chunks / 2;
+  const int seg_chunks = (int)((n_chunks + want - 1) / want);
+  const int n_seg = (n_chunks + seg_chunks - 1) / seg_chunks;
+  if (n_seg < 2) return pl;
+  pl.n_seg = n_seg;
+  pl.seg_chunks = seg_chunks;
+  pl.workspace = (size_t)BH * (size_t)(n_seg - 1) * kSymFP * (size_t)(d_v + 16) * sizeof(float);
+  return pl;
+}
+
 template <int DV>
 based_status_t launch_linattn_tc(const void* q, const void* k, const void* v, void* out, int BH,
                                  int L, float eps, float* state_kv, float* state_k,
-                                 cudaStream_t st) {
+                                 void* workspace, size_t workspace_bytes, cudaStream_t st) {
+  const TcPlan pl = plan_linattn_tc(BH, L, DV);
+  if (pl.workspace > 0 && (workspace == nullptr || workspace_bytes < pl.workspace))
+    return BASED_ERR_WORKSPACE;
+  if (pl.workspace > 0 && (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0)
+    return BASED_ERR_INVALID_ARG;
   CUtensorMap vmap;
   if (!make_rows_map(&vmap, v, DV, L, BH, kTcChunk)) return BASED_ERR_CUDA;
-  auto kern = linattn_tc_kernel<DV>;
+  TcParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.state_kv = state_kv;
+  p.state_k = state_k;
+  p.partial = static_cast<float*>(workspace);
+  p.L = L;
+  p.seg_chunks = pl.seg_chunks;
+  p.n_seg = pl.n_seg;
+  p.eps = eps;
   const size_t smem = TcLayout<DV>::kSmem;
+  if (pl.n_seg > 1) {
+    auto kst = linattn_tc_kernel<DV, true>;
+    if (!set_smem(kst, smem)) return BASED_ERR_CUDA;
+    const long long nblk = (long long)BH * (pl.n_seg - 1);
+    if (nblk > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
+    kst<<<(unsigned)nblk, kTcThreads, smem, st>>>(vmap, p);
+    if (cudaGetLastError() != cudaSuccess) return BASED_ERR_CUDA;
+  }
+  auto kern = linattn_tc_kernel<DV, false>;
   if (!set_smem(kern, smem)) return BASED_ERR_CUDA;
-  kern<<<(unsigned)BH, kTcThreads, smem, st>>>(
-      vmap, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-      static_cast<__nv_bfloat16*>(out), state_kv, state_k, L, eps);
+  const long long nblk = (long long)BH * pl.n_seg;
+  if (nblk > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
+  kern<<<(unsigned)nblk, kTcThreads, smem, st>>>(vmap, p);
   return launch_status();
 }
 
@@ -206,15 +263,14 @@ size_t based_linattn_workspace_bytes(int B, int H, int L, int d_feat, int d_v,
   if (B < 0 || H < 0 || L < 0 || (dt != BASED_F32 && dt != BASED_BF16) || d_feat != kD ||
       (d_v != 64 && d_v != 128))
     return (size_t)-1;
-  return 0;
+  if (dt == BASED_F32) return 0;
+  return plan_linattn_tc((long long)B * H, L, d_v).workspace;
 }
 
 based_status_t based_linattn_fwd(const void* q, const void* k, const void* v, void* out,
                                  int B, int H, int L, int d_feat, int d_v, based_dtype_t dt,
                                  float eps, float* state_kv, float* state_k, void* workspace,
                                  size_t workspace_bytes, based_stream_t stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   based_status_t s =
       check_linattn(q, k, v, out, B, H, L, d_feat, d_v, dt, eps, state_kv, state_k);
   if (s != BASED_OK) return s;
@@ -224,8 +280,10 @@ based_status_t based_linattn_fwd(const void* q, const void* k, const void* v, vo
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dt == BASED_F32)
     return launch_linattn_simt<float>(q, k, v, out, BH, L, d_v, eps, state_kv, state_k, st);
-  return d_v == 64 ? launch_linattn_tc<64>(q, k, v, out, BH, L, eps, state_kv, state_k, st)
-                   : launch_linattn_tc<128>(q, k, v, out, BH, L, eps, state_kv, state_k, st);
+  return d_v == 64 ? launch_linattn_tc<64>(q, k, v, out, BH, L, eps, state_kv, state_k,
+                                            workspace, workspace_bytes, st)
+                   : launch_linattn_tc<128>(q, k, v, out, BH, L, eps, state_kv, state_k,
+                                            workspace, workspace_bytes, st);
 }
 
 based_status_t based_window_attn_fwd(const void* q, const void* k, const void* v, void* out,

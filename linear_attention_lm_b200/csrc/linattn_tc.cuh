@@ -3,7 +3,7 @@
 // Method ("Базированная модель, часть 2", section "Что за линейное внимание?";
 // based/train README, training views): y_t = phi(q_t)^T S_t / (phi(q_t).z_t + eps)
 // with S_t = sum_{s<=t} phi(k_s) v_s^T, z_t = sum_{s<=t} phi(k_s).  The kernel runs
-// the chunked ("fla_parallel") view, one CTA per sequence, chunks of C = 128 tokens:
+// the chunked ("fla_parallel") view, chunks of C = 128 tokens:
 //
 //   #1  U   = Q_c K_c^T                      (tcgen05, K = 16)           -> TMEM
 //       P   = mask_{s<=t}(1 + U/4 + U^2/32)  (CUDA cores, from TMEM)     -> smem
@@ -30,6 +30,12 @@
 // copy is scaled by a power of two so it stays in fp16 range for any L, and P is
 // scaled by the same power so the ratio is unchanged).  All accumulation is fp32
 // in TMEM; the master state never leaves TMEM until the export.
+//
+// Long sequences are split into n_seg segments of seg_chunks chunks so that
+// B*H*n_seg CTAs fill the GPU: a state-only pass (kStateOnly) runs #5 alone
+// over every segment but the last and writes each segment's partial [S|z]
+// (fp32, 160 x (dv+16)) to the caller's workspace; the main pass then seeds
+// segment g's TMEM state with the sum of the partials of segments 0..g-1.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -45,7 +51,7 @@ constexpr int kSymF = 153;             // distinct Taylor features
 constexpr int kSymFP = 160;            // padded to the MMA K granularity (16)
 constexpr int kTcTmemCols = 512;
 
-// Symmetric-feature index -> (i, j, weight) for the quadratic block.
+// Symmetric-feature index (>= 17) -> (i, j) of the quadratic block, i <= j.
 __host__ __device__ constexpr int sym_pair_i(int p) {
   int i = 0;
   while (p >= 16 - i) { p -= 16 - i; ++i; }
@@ -60,6 +66,7 @@ __host__ __device__ constexpr int sym_pair_j(int p) {
 template <int DV>
 struct TcLayout {
   static constexpr int NA = DV + 16;                       // [V | 1 | 0..] columns
+  static constexpr int kTileCols = (NA + 31) / 32 * 32;    // TMEM columns per state tile
   // shared memory (byte offsets from a 1024-aligned base)
   static constexpr int kQ = 0;                             // Q tile  [128 x 16] bf16, K-major
   static constexpr int kK = kQ + 4096;                     // K tile  [128 x 16] bf16, K-major
@@ -74,29 +81,40 @@ struct TcLayout {
   static constexpr size_t kSmem = kBytes + 1024;           // + alignment slack
   // TMEM columns: [S|z] tiles (two 128-feature tiles) then the U / O accumulator
   static constexpr int kTmS = 0;
-  static constexpr int kTmO = 2 * NA;
-  static_assert(kTmO + 128 <= kTcTmemCols, "TMEM budget");
+  static constexpr int kTmO = 2 * kTileCols;
+  static_assert(kTmO + 160 <= kTcTmemCols, "TMEM budget");
   // #5 reads 32 feature groups past phiK (the second tile's unused rows); keep
   // that window inside the allocation.
   static_assert(kPhiK + 65536 <= kBytes, "phiK over-read window");
 };
 
+struct TcParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  __nv_bfloat16* out;
+  float* state_kv;   // [BH, 273, DV] or null (main pass, last segment)
+  float* state_k;    // [BH, 273] or null
+  float* partial;    // [BH, n_seg-1, 160, DV+16] fp32 segment partials (n_seg > 1)
+  int L;
+  int seg_chunks;    // chunks per segment
+  int n_seg;         // segments per sequence (1 = no split)
+  float eps;
+};
+
 // Power-of-two scale applied to the fp16 state copy (and to P) for the chunk
-// starting at t0, keeping every state entry (|z_0| <= t) below 2^15.
+// ending at t_end, keeping every state entry (|z_0| <= t) below 2^15.
 __device__ __forceinline__ float tc_chunk_scale(long long t_end) {
   int e = 0;
   while (t_end > (32768ll << e)) ++e;
   return __int_as_float((127 - e) << 23);
 }
 
-template <int DV>
+template <int DV, bool kStateOnly>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    linattn_tc_kernel(const __grid_constant__ CUtensorMap vmap,
-                      const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                      __nv_bfloat16* __restrict__ out, float* __restrict__ state_kv,
-                      float* __restrict__ state_k, int L, float eps) {
+    linattn_tc_kernel(const __grid_constant__ CUtensorMap vmap, const TcParams p) {
   using Lay = TcLayout<DV>;
   constexpr int NA = Lay::NA;
+  constexpr int NG = (NA + 31) / 32;  // 32-column groups of a state tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
@@ -107,11 +125,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   int* abort_flag = reinterpret_cast<int*>(bar_tma + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.x;
+  const int L = p.L;
   const int n_chunks = (L + kTcChunk - 1) / kTcChunk;
-  q += (size_t)bh * L * kD;
-  k += (size_t)bh * L * kD;
-  out += (size_t)bh * L * DV;
+  const int segs_here = kStateOnly ? p.n_seg - 1 : p.n_seg;
+  const int bh = blockIdx.x / segs_here;
+  const int seg = blockIdx.x - bh * segs_here;
+  const int c_begin = seg * p.seg_chunks;
+  const int c_end = min(c_begin + p.seg_chunks, n_chunks);
+  const bool has_init = !kStateOnly && seg > 0;
+  const __nv_bfloat16* q = p.q + (size_t)bh * L * kD;
+  const __nv_bfloat16* k = p.k + (size_t)bh * L * kD;
+  __nv_bfloat16* out = kStateOnly ? nullptr : p.out + (size_t)bh * L * DV;
 
   if (tid == 0) {
     umma::mbar_init(bar_tma, 1);
@@ -128,7 +152,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // ones block of [V | 1]: column DV of the augmented V is 1 for every token
   {
     uint8_t* ones = sm + Lay::kV + (DV / 64) * 16384;
-    for (int i = tid; i < 16384 / 16; i += kTcThreads) reinterpret_cast<uint4*>(ones)[i] = make_uint4(0, 0, 0, 0);
+    for (int i = tid; i < 16384 / 16; i += kTcThreads)
+      reinterpret_cast<uint4*>(ones)[i] = make_uint4(0, 0, 0, 0);
     __syncthreads();
     *reinterpret_cast<__nv_bfloat16*>(ones + umma::off_mnmajor_sw128(0, tid, kTcChunk)) =
         __float2bfloat16(1.0f);
@@ -144,6 +169,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                  sP = umma::smem_u32(sm + Lay::kP), sPhiQ = umma::smem_u32(sm + Lay::kPhiQ),
                  sS = umma::smem_u32(sm + Lay::kS);
   constexpr uint32_t kVBytes = DV * kTcChunk * 2;
+  // state tiles: tile 0 lanes 0..127 = features 0..127 (all warps); tile 1
+  // lanes 0..31 = features 128..159 (warp 0 only)
+  const int n_tiles_here = warp == 0 ? 2 : 1;
 
   auto issue_v = [&](int c) {
     umma::mbar_arrive_expect_tx(bar_tma, kVBytes);
@@ -151,43 +179,102 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int b = 0; b < DV / 64; ++b)
       umma::tma_load_3d(sm + Lay::kV + b * 16384, &vmap, bar_tma, b * 64, c * kTcChunk, bh);
   };
-  if (tid == 0 && n_chunks > 0) issue_v(0);
+  if (tid == 0 && c_begin < c_end) issue_v(c_begin);
+
+  // fp16 copy of the TMEM state, scaled by sn, as the B operand of #2
+  auto copy_state = [&](float sn) {
+    for (int mt = 0; mt < n_tiles_here; ++mt) {
+      const int f = mt * 128 + warp * 32 + lane;
+#pragma unroll
+      for (int g = 0; g < NG; ++g) {
+        float sv[32];
+        umma::tmem_ld32(tmem + Lay::kTmS + mt * Lay::kTileCols + tm_lane + g * 32, sv);
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const int j0 = g * 32 + h * 8;
+          if (j0 < NA) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __half2 hv = __floats2half2_rn(sv[h * 8 + 2 * e] * sn, sv[h * 8 + 2 * e + 1] * sn);
+              pk[e] = *reinterpret_cast<const uint32_t*>(&hv);
+            }
+            *reinterpret_cast<uint4*>(sm + Lay::kS + ((j0 >> 3) * 20 + (f >> 3)) * 128 + (f & 7) * 16) =
+                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+      }
+    }
+  };
+
+  // seed the TMEM state of a later segment with the sum of the earlier partials
+  if (has_init) {
+    const float* part = p.partial + (size_t)bh * (p.n_seg - 1) * kSymFP * NA;
+    for (int mt = 0; mt < n_tiles_here; ++mt) {
+      const int f = mt * 128 + warp * 32 + lane;
+#pragma unroll
+      for (int g = 0; g < NG; ++g) {
+        float acc[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
+        for (int sp = 0; sp < seg; ++sp) {
+          const float* row = part + ((size_t)sp * kSymFP + f) * NA + g * 32;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (g * 32 + i < NA) acc[i] += row[i];
+        }
+        umma::tmem_st32(tmem + Lay::kTmS + mt * Lay::kTileCols + tm_lane + g * 32, acc);
+      }
+    }
+    umma::tc_fence_before();
+    __syncthreads();
+    umma::tc_fence_after();
+    copy_state(tc_chunk_scale((long long)c_begin * kTcChunk + kTcChunk));
+  }
 
   // q/k rows of this thread's token, prefetched one chunk ahead
   uint4 qr[2], kr[2];
   auto load_qk = [&](int c) {
     const long long t = (long long)c * kTcChunk + tid;
-    if (c < n_chunks && t < L) {
-      const uint4* qp = reinterpret_cast<const uint4*>(q + t * kD);
+    if (c < c_end && t < L) {
       const uint4* kp = reinterpret_cast<const uint4*>(k + t * kD);
-      qr[0] = qp[0]; qr[1] = qp[1];
       kr[0] = kp[0]; kr[1] = kp[1];
+      if (!kStateOnly) {
+        const uint4* qp = reinterpret_cast<const uint4*>(q + t * kD);
+        qr[0] = qp[0]; qr[1] = qp[1];
+      } else {
+        qr[0] = qr[1] = make_uint4(0, 0, 0, 0);
+      }
     } else {
       qr[0] = qr[1] = kr[0] = kr[1] = make_uint4(0, 0, 0, 0);
     }
   };
-  load_qk(0);
+  load_qk(c_begin);
 
   uint32_t ph_tma = 0, ph_u = 0, ph_o = 0;
-  bool tma_pending = n_chunks > 0;
+  bool tma_pending = c_begin < c_end;
   const uint32_t id_u = umma::idesc_bf16(128, 128, false, false);
   const uint32_t id_o2 = umma::idesc_f16(128, NA, false, true);
   const uint32_t id_o4 = umma::idesc_bf16(128, NA, false, true);
   const uint32_t id_s5 = umma::idesc_bf16(128, NA, true, true);
 
-  for (int c = 0; c < n_chunks; ++c) {
+  __syncthreads();
+  for (int c = c_begin; c < c_end; ++c) {
     const int t0 = c * kTcChunk;
     const int n = min(kTcChunk, L - t0);
+    const bool has_state = has_init || c > c_begin;
     const float sc = tc_chunk_scale((long long)t0 + kTcChunk);
     // ---- (a) Q/K tiles and the feature maps of this thread's token -------------
     {
       const int t = tid;
-      uint8_t* qrow = sm + Lay::kQ + ((t >> 3) * 2) * 128 + (t & 7) * 16;
-      uint8_t* krow = sm + Lay::kK + ((t >> 3) * 2) * 128 + (t & 7) * 16;
-      *reinterpret_cast<uint4*>(qrow) = qr[0];
-      *reinterpret_cast<uint4*>(qrow + 128) = qr[1];
-      *reinterpret_cast<uint4*>(krow) = kr[0];
-      *reinterpret_cast<uint4*>(krow + 128) = kr[1];
+      if (!kStateOnly) {
+        uint8_t* qrow = sm + Lay::kQ + ((t >> 3) * 2) * 128 + (t & 7) * 16;
+        uint8_t* krow = sm + Lay::kK + ((t >> 3) * 2) * 128 + (t & 7) * 16;
+        *reinterpret_cast<uint4*>(qrow) = qr[0];
+        *reinterpret_cast<uint4*>(qrow + 128) = qr[1];
+        *reinterpret_cast<uint4*>(krow) = kr[0];
+        *reinterpret_cast<uint4*>(krow + 128) = kr[1];
+      }
       float xq[16], xk[16];
       const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(qr);
       const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(kr);
@@ -213,8 +300,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           hq[e] = *reinterpret_cast<const uint32_t*>(&h);
           bk[e] = *reinterpret_cast<const uint32_t*>(&b);
         }
-        *reinterpret_cast<uint4*>(sm + Lay::kPhiQ + ((t >> 3) * 20 + ch) * 128 + (t & 7) * 16) =
-            make_uint4(hq[0], hq[1], hq[2], hq[3]);
+        if (!kStateOnly)
+          *reinterpret_cast<uint4*>(sm + Lay::kPhiQ + ((t >> 3) * 20 + ch) * 128 + (t & 7) * 16) =
+              make_uint4(hq[0], hq[1], hq[2], hq[3]);
         *reinterpret_cast<uint4*>(sm + Lay::kPhiK + (ch * 16 + (t >> 3)) * 128 + (t & 7) * 16) =
             make_uint4(bk[0], bk[1], bk[2], bk[3]);
         ++ch;
@@ -244,49 +332,51 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     umma::tc_fence_before();
     __syncthreads();
     umma::tc_fence_after();
-    // ---- (b) #1: U = Q K^T ---------------------------------------------------------
-    if (tid == 0) {
-      umma::mma_bf16(tmem + Lay::kTmO, umma::desc_kmajor_none(sQ, 0, 16),
-                     umma::desc_kmajor_none(sK, 0, 16), id_u, 0);
-      umma::mma_commit(bar_u);
-    }
-    __syncwarp();
-    if (!umma::mbar_wait(bar_u, ph_u)) { record_device_error(BASED_ERR_TIMEOUT); *abort_flag = 1; }
-    ph_u ^= 1;
-    umma::tc_fence_after();
-    // ---- (c) scores: P = mask(1 + u/4 + u^2/32) * sc -> smem -------------------------
-    {
-      const int t = tid;
+    if (!kStateOnly) {
+      // ---- (b) #1: U = Q K^T -------------------------------------------------------
+      if (tid == 0) {
+        umma::mma_bf16(tmem + Lay::kTmO, umma::desc_kmajor_none(sQ, 0, 16),
+                       umma::desc_kmajor_none(sK, 0, 16), id_u, 0);
+        umma::mma_commit(bar_u);
+      }
+      __syncwarp();
+      if (!umma::mbar_wait(bar_u, ph_u)) { record_device_error(BASED_ERR_TIMEOUT); *abort_flag = 1; }
+      ph_u ^= 1;
+      umma::tc_fence_after();
+      // ---- (c) scores: P = mask(1 + u/4 + u^2/32) * sc -> smem -----------------------
+      {
+        const int t = tid;
 #pragma unroll
-      for (int c32 = 0; c32 < 4; ++c32) {
-        float u[32];
-        umma::tmem_ld32(tmem + Lay::kTmO + tm_lane + c32 * 32, u);
+        for (int c32 = 0; c32 < 4; ++c32) {
+          float u[32];
+          umma::tmem_ld32(tmem + Lay::kTmO + tm_lane + c32 * 32, u);
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          uint32_t pk[4];
+          for (int g = 0; g < 4; ++g) {
+            uint32_t pk[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int s0 = c32 * 32 + g * 8 + 2 * e;
-            const float u0 = u[g * 8 + 2 * e], u1 = u[g * 8 + 2 * e + 1];
-            const float w0 = s0 <= t ? fmaf(u0, fmaf(u0, 0.03125f, 0.25f), 1.0f) * sc : 0.0f;
-            const float w1 = s0 + 1 <= t ? fmaf(u1, fmaf(u1, 0.03125f, 0.25f), 1.0f) * sc : 0.0f;
-            const __nv_bfloat162 b = __floats2bfloat162_rn(w0, w1);
-            pk[e] = *reinterpret_cast<const uint32_t*>(&b);
+            for (int e = 0; e < 4; ++e) {
+              const int s0 = c32 * 32 + g * 8 + 2 * e;
+              const float u0 = u[g * 8 + 2 * e], u1 = u[g * 8 + 2 * e + 1];
+              const float w0 = s0 <= t ? fmaf(u0, fmaf(u0, 0.03125f, 0.25f), 1.0f) * sc : 0.0f;
+              const float w1 = s0 + 1 <= t ? fmaf(u1, fmaf(u1, 0.03125f, 0.25f), 1.0f) * sc : 0.0f;
+              const __nv_bfloat162 b = __floats2bfloat162_rn(w0, w1);
+              pk[e] = *reinterpret_cast<const uint32_t*>(&b);
+            }
+            const int ch = c32 * 4 + g;
+            *reinterpret_cast<uint4*>(sm + Lay::kP + ((t >> 3) * 16 + ch) * 128 + (t & 7) * 16) =
+                make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
-          const int ch = c32 * 4 + g;
-          *reinterpret_cast<uint4*>(sm + Lay::kP + ((t >> 3) * 16 + ch) * 128 + (t & 7) * 16) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
       }
+      umma::fence_async_smem();
+      umma::tc_fence_before();
+      __syncthreads();
+      umma::tc_fence_after();
+      if (*abort_flag) break;
     }
-    umma::fence_async_smem();
-    umma::tc_fence_before();
-    __syncthreads();
-    umma::tc_fence_after();
-    if (*abort_flag) break;
     // ---- (d) #2, #4, #5 ----------------------------------------------------------------
     if (tid == 0) {
-      bool ok = umma::mbar_wait(bar_tma, ph_tma);
+      const bool ok = umma::mbar_wait(bar_tma, ph_tma);
       ph_tma ^= 1;
       tma_pending = false;
       if (!ok) {
@@ -294,23 +384,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         *abort_flag = 1;
       } else {
         umma::tc_fence_after();
-        if (c > 0) {
+        if (!kStateOnly) {
+          if (has_state) {
 #pragma unroll
-          for (int k0 = 0; k0 < kSymFP; k0 += 16)
-            umma::mma_f16(tmem + Lay::kTmO, umma::desc_kmajor_none(sPhiQ, k0, kSymFP),
-                          umma::desc_mnmajor_none(sS, k0, kSymFP), id_o2, k0 > 0);
+            for (int k0 = 0; k0 < kSymFP; k0 += 16)
+              umma::mma_f16(tmem + Lay::kTmO, umma::desc_kmajor_none(sPhiQ, k0, kSymFP),
+                            umma::desc_mnmajor_none(sS, k0, kSymFP), id_o2, k0 > 0);
+          }
+#pragma unroll
+          for (int k0 = 0; k0 < kTcChunk; k0 += 16)
+            umma::mma_bf16(tmem + Lay::kTmO, umma::desc_kmajor_none(sP, k0, kTcChunk),
+                           umma::desc_mnmajor_sw128(sV, k0, kTcChunk), id_o4,
+                           has_state || (k0 > 0));
         }
-#pragma unroll
-        for (int k0 = 0; k0 < kTcChunk; k0 += 16)
-          umma::mma_bf16(tmem + Lay::kTmO, umma::desc_kmajor_none(sP, k0, kTcChunk),
-                         umma::desc_mnmajor_sw128(sV, k0, kTcChunk), id_o4, (c > 0) || (k0 > 0));
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
           for (int k0 = 0; k0 < kTcChunk; k0 += 16)
-            umma::mma_bf16(tmem + Lay::kTmS + mt * NA,
+            umma::mma_bf16(tmem + Lay::kTmS + mt * Lay::kTileCols,
                            umma::desc_mnmajor_none(sPhiK + mt * 16 * 2048, k0, kTcChunk),
-                           umma::desc_mnmajor_sw128(sV, k0, kTcChunk), id_s5, (c > 0) || (k0 > 0));
+                           umma::desc_mnmajor_sw128(sV, k0, kTcChunk), id_s5,
+                           has_state || (k0 > 0));
         umma::mma_commit(bar_o);
       }
     }
@@ -320,24 +414,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (!umma::mbar_wait(bar_o, ph_o)) { record_device_error(BASED_ERR_TIMEOUT); *abort_flag = 1; }
     ph_o ^= 1;
     umma::tc_fence_after();
-    if (tid == 0 && c + 1 < n_chunks && !*abort_flag) {
+    if (tid == 0 && c + 1 < c_end && !*abort_flag) {
       issue_v(c + 1);
       tma_pending = true;
     }
     // ---- (e) outputs and the fp16 state copy for the next chunk --------------------
-    {
+    if (!kStateOnly) {
       const int t = tid;
-      float o[NA];
+      float o[NG * 32];
 #pragma unroll
-      for (int c32 = 0; c32 < NA / 32 + (NA % 32 ? 1 : 0); ++c32) {
-        float tmp[32];
-        umma::tmem_ld32(tmem + Lay::kTmO + tm_lane + c32 * 32, tmp);
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (c32 * 32 + i < NA) o[c32 * 32 + i] = tmp[i];
-      }
+      for (int g = 0; g < NG; ++g) umma::tmem_ld32(tmem + Lay::kTmO + tm_lane + g * 32, o + g * 32);
       if (t < n) {
-        const float inv = 1.0f / (o[DV] + eps * sc);
+        const float inv = 1.0f / (o[DV] + p.eps * sc);
         uint4* dst = reinterpret_cast<uint4*>(out + (size_t)(t0 + t) * DV);
 #pragma unroll
         for (int ch = 0; ch < DV / 8; ++ch) {
@@ -351,33 +439,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           dst[ch] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
       }
-      if (c + 1 < n_chunks) {
-        const float sn = tc_chunk_scale((long long)t0 + 2 * kTcChunk);
-        // tile 0 holds features 0..127 (lane = feature); tile 1 lanes 0..31 hold 128..159
-        const int ntile = warp == 0 ? 2 : 1;
-        for (int mt = 0; mt < ntile; ++mt) {
-          const int f = mt * 128 + warp * 32 + lane;
-#pragma unroll
-          for (int c32 = 0; c32 < NA / 32 + (NA % 32 ? 1 : 0); ++c32) {
-            float sv[32];
-            umma::tmem_ld32(tmem + Lay::kTmS + mt * NA + tm_lane + c32 * 32, sv);
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              const int j0 = c32 * 32 + g * 8;
-              if (j0 < NA) {
-                uint32_t pk[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const __half2 h = __floats2half2_rn(sv[g * 8 + 2 * e] * sn, sv[g * 8 + 2 * e + 1] * sn);
-                  pk[e] = *reinterpret_cast<const uint32_t*>(&h);
-                }
-                *reinterpret_cast<uint4*>(sm + Lay::kS + ((j0 >> 3) * 20 + (f >> 3)) * 128 + (f & 7) * 16) =
-                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              }
-            }
-          }
-        }
-      }
+      if (c + 1 < c_end) copy_state(tc_chunk_scale((long long)t0 + 2 * kTcChunk));
     }
     umma::fence_async_smem();
     umma::tc_fence_before();
@@ -386,48 +448,59 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (*abort_flag) break;
   }
 
-  // ---- final state export: 153 symmetric rows -> 273-row layout ----------------------
-  if (!*abort_flag && (state_kv || state_k)) {
-    float* skv = state_kv ? state_kv + (size_t)bh * kF * DV : nullptr;
-    float* sk = state_k ? state_k + (size_t)bh * kF : nullptr;
-    const int ntile = warp == 0 ? 2 : 1;
-    for (int mt = 0; mt < ntile; ++mt) {
-      const int f = mt * 128 + warp * 32 + lane;
-      float s[NA];
-      if (n_chunks > 0) {
+  if (!*abort_flag) {
+    if (kStateOnly) {
+      // this segment's partial state, 160 symmetric rows x NA columns, fp32
+      float* part = p.partial + ((size_t)bh * (p.n_seg - 1) + seg) * kSymFP * NA;
+      for (int mt = 0; mt < n_tiles_here; ++mt) {
+        const int f = mt * 128 + warp * 32 + lane;
 #pragma unroll
-        for (int c32 = 0; c32 < NA / 32 + (NA % 32 ? 1 : 0); ++c32) {
-          float tmp[32];
-          umma::tmem_ld32(tmem + Lay::kTmS + mt * NA + tm_lane + c32 * 32, tmp);
+        for (int g = 0; g < NG; ++g) {
+          float s[32];
+          umma::tmem_ld32(tmem + Lay::kTmS + mt * Lay::kTileCols + tm_lane + g * 32, s);
+          float* row = part + (size_t)f * NA + g * 32;
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (c32 * 32 + i < NA) s[c32 * 32 + i] = tmp[i];
+            if (g * 32 + i < NA) row[i] = c_begin < c_end ? s[i] : 0.0f;
         }
-      } else {
-#pragma unroll
-        for (int i = 0; i < NA; ++i) s[i] = 0.0f;
       }
-      if (f >= kSymF) continue;
-      int r0, r1 = -1;
-      float scale = 1.0f;
-      if (f <= 16) {
-        r0 = f;
-      } else {
-        const int i = sym_pair_i(f - 17), j = sym_pair_j(f - 17);
-        r0 = 17 + 16 * i + j;
-        if (i != j) { r1 = 17 + 16 * j + i; scale = 0.70710678118654752f; }
-      }
-      for (int r = 0; r < 2; ++r) {
-        const int row = r == 0 ? r0 : r1;
-        if (row < 0) continue;
-        if (skv) {
-          float4* dst = reinterpret_cast<float4*>(skv + (size_t)row * DV);
+    } else if (seg == p.n_seg - 1 && (p.state_kv || p.state_k)) {
+      // final state export: 153 symmetric rows -> 273-row layout
+      float* skv = p.state_kv ? p.state_kv + (size_t)bh * kF * DV : nullptr;
+      float* sk = p.state_k ? p.state_k + (size_t)bh * kF : nullptr;
+      const bool any = has_init || c_begin < c_end;
+      for (int mt = 0; mt < n_tiles_here; ++mt) {
+        const int f = mt * 128 + warp * 32 + lane;
+        float s[NG * 32];
 #pragma unroll
-          for (int j = 0; j < DV / 4; ++j)
-            dst[j] = make_float4(s[4 * j] * scale, s[4 * j + 1] * scale, s[4 * j + 2] * scale,
-                                 s[4 * j + 3] * scale);
+        for (int g = 0; g < NG; ++g)
+          umma::tmem_ld32(tmem + Lay::kTmS + mt * Lay::kTileCols + tm_lane + g * 32, s + g * 32);
+        if (!any) {
+#pragma unroll
+          for (int i = 0; i < NG * 32; ++i) s[i] = 0.0f;
         }
-        if (sk) sk[row] = s[DV] * scale;
+        if (f >= kSymF) continue;
+        int r0, r1 = -1;
+        float scale = 1.0f;
+        if (f <= 16) {
+          r0 = f;
+        } else {
+          const int i = sym_pair_i(f - 17), j = sym_pair_j(f - 17);
+          r0 = 17 + 16 * i + j;
+          if (i != j) { r1 = 17 + 16 * j + i; scale = 0.70710678118654752f; }
+        }
+        for (int r = 0; r < 2; ++r) {
+          const int row = r == 0 ? r0 : r1;
+          if (row < 0) continue;
+          if (skv) {
+            float4* dst = reinterpret_cast<float4*>(skv + (size_t)row * DV);
+#pragma unroll
+            for (int j = 0; j < DV / 4; ++j)
+              dst[j] = make_float4(s[4 * j] * scale, s[4 * j + 1] * scale, s[4 * j + 2] * scale,
+                                   s[4 * j + 3] * scale);
+          }
+          if (sk) sk[row] = s[DV] * scale;
+        }
       }
     }
   }

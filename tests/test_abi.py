@@ -84,6 +84,18 @@ def test_linattn_host_validation(lib):
     assert lin_call(lib, q=None, k=None, v=None, out=None, L=0) == 0
 
 
+def test_linattn_workspace_required(lib):
+    """A long single sequence is split across CTAs and needs workspace; a
+    missing or short workspace is refused on the host."""
+    need = lib.based_linattn_workspace_bytes(1, 1, 4096, 16, 64, 1)
+    assert 0 < need < (1 << 26)
+    assert lib.based_linattn_workspace_bytes(1, 1, 4096, 16, 64, 0) == 0  # fp32 path
+    f = lib.based_linattn_fwd
+    assert f(FAKE, FAKE, FAKE, FAKE, 1, 1, 4096, 16, 64, 1, 1e-6, None, None, None, 0, None) == 5
+    assert f(FAKE, FAKE, FAKE, FAKE, 1, 1, 4096, 16, 64, 1, 1e-6, None, None, FAKE, need - 16,
+             None) == 5
+
+
 def test_window_host_validation(lib):
     f = lib.based_window_attn_fwd
     assert f(FAKE, FAKE, FAKE, FAKE, 1, 1, 8, 64, 0, 1, None) == INVALID

@@ -99,6 +99,15 @@ def test_linattn_head_dims(dv, dtype):
     run_linattn(w)
 
 
+@pytest.mark.parametrize("L", [3000, 1025])
+def test_linattn_split_segments(L):
+    """Few sequences, long L: the prefill splits each sequence into segments
+    (state-only pass + seeded main pass); ragged last chunk, state export."""
+    w = WORKLOADS["long_16k"].with_(B=1, H=2, L=L, name=f"split{L}")
+    assert lab.based_linattn_workspace_bytes(1, 2, L, 16, 64, lab.BASED_BF16) > 0
+    run_linattn(w)
+
+
 def test_linattn_empty_and_state_only():
     dev = torch.device("cuda:0")
     q = torch.empty((2, 2, 0, 16), dtype=torch.bfloat16, device=dev)
