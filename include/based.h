@@ -24,7 +24,8 @@
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers, owned by the caller, C-contiguous
  *     in the layouts given below, 16-byte aligned.  The library never keeps a
- *     pointer after the call returns and never allocates device memory.
+ *     pointer after the call returns and never allocates device memory
+ *     (based_linattn_fwd_noalloc uses a fixed array inside the library).
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
  *     asynchronous on it; the caller synchronises before reading results.
  *   - Argument errors are detected on the host, before any launch, and return
@@ -100,6 +101,33 @@ based_status_t based_linattn_fwd(const void* q, const void* k, const void* v, vo
                                  float* state_kv, float* state_k,
                                  void* workspace, size_t workspace_bytes,
                                  based_stream_t stream);
+
+/*
+ * Same computation and arguments as based_linattn_fwd, for callers that must
+ * not allocate device memory: a plugin or server whose host framework owns
+ * every device allocation, or a latency-critical loop where cudaMalloc's
+ * implicit device synchronisation is not acceptable.  Such callers cannot
+ * provide the workspace based_linattn_fwd may ask for.  (The paper has no
+ * counterpart to this entry point; it is a deployment convenience.)
+ *
+ * Scratch comes from a fixed array compiled into the library, 16 MiB on every
+ * GPU that loads the library, held until the process exits.  Nothing is
+ * allocated, here or later.  A problem whose scratch need
+ * (based_linattn_workspace_bytes) exceeds 16 MiB is refused with
+ * BASED_ERR_WORKSPACE before any launch.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls on one device share the array and it
+ * keeps the last call's contents (every call writes the parts it reads), so
+ * calls whose kernels overlap on the GPU -- concurrent streams, several host
+ * threads -- race on it: serialise them.
+ */
+based_status_t based_linattn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
+                                         int B, int H, int L, int d_feat, int d_v,
+                                         based_dtype_t dt, float eps,
+                                         float* state_kv, float* state_k,
+                                         based_stream_t stream);
 
 /*
  * Sliding-window causal softmax attention:

@@ -30,6 +30,7 @@ _STATUS = {0: "BASED_OK", 1: "BASED_ERR_INVALID_ARG", 2: "BASED_ERR_UNSUPPORTED"
            3: "BASED_ERR_CUDA", 4: "BASED_ERR_TIMEOUT", 5: "BASED_ERR_WORKSPACE"}
 EXPORTED_SYMBOLS = ("based_abi_version", "based_status_string",
                     "based_linattn_workspace_bytes", "based_linattn_fwd",
+                    "based_linattn_fwd_noalloc",
                     "based_window_attn_fwd", "based_window_ring_fill", "based_decode_step",
                     "based_get_device_error")
 
@@ -64,14 +65,16 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.based_linattn_workspace_bytes.restype = _sz
         lib.based_linattn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f,
                                           _vp, _vp, _vp, _sz, _vp]
+        lib.based_linattn_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                                  _f, _vp, _vp, _vp]
         lib.based_window_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
         lib.based_window_ring_fill.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _i, _vp]
         lib.based_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                           _vp, _vp, _ll, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                                           _vp]
         lib.based_get_device_error.argtypes = [_vp]
-        for name in ("based_linattn_fwd", "based_window_attn_fwd", "based_window_ring_fill",
-                     "based_decode_step", "based_get_device_error"):
+        for name in ("based_linattn_fwd", "based_linattn_fwd_noalloc", "based_window_attn_fwd",
+                     "based_window_ring_fill", "based_decode_step", "based_get_device_error"):
             getattr(lib, name).restype = _i
         _lib = lib
         return lib
@@ -158,6 +161,22 @@ def based_linattn_fwd(q, k, v, out, eps: float = 1e-6, state_kv=None, state_k=No
             _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, L, d, d_v, dt, float(eps),
             _f32(state_kv), _f32(state_k), _ptr(workspace), ws_bytes, _stream(stream))
     _check("based_linattn_fwd", st)
+    return out
+
+
+def based_linattn_fwd_noalloc(q, k, v, out, eps: float = 1e-6, state_kv=None, state_k=None,
+                              stream=None):
+    """based_linattn_fwd without a workspace: for callers that must not
+    allocate device memory (the library's fixed 16 MiB scratch array is used
+    instead; calls on one device must not overlap on the GPU)."""
+    B, H, L, d = q.shape
+    d_v = v.shape[-1]
+    dt = _same_dtype(q, k, v, out)
+    with torch.cuda.device(q.device):
+        st = load_library().based_linattn_fwd_noalloc(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, L, d, d_v, dt, float(eps),
+            _f32(state_kv), _f32(state_k), _stream(stream))
+    _check("based_linattn_fwd_noalloc", st)
     return out
 
 

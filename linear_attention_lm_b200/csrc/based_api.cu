@@ -8,6 +8,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "based.h"
 #include "common.cuh"
 #include "decode.cuh"
@@ -240,6 +242,39 @@ based_status_t launch_decode(const DecodeParams& p, cudaStream_t st) {
   return launch_status();
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free prefill (based_linattn_fwd_noalloc): the segment partials
+// live in this fixed array instead of a caller workspace.  Host code may not
+// pass the array's name to a kernel (on the host it is only a stand-in); the
+// device address is looked up once per device with cudaGetSymbolAddress.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+float* g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+}  // namespace
+
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+namespace {
+
+// Device address of g_noalloc_scratch on the current device (looked up on the
+// first call for that device).
+based_status_t noalloc_scratch(float** addr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BASED_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return BASED_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return BASED_ERR_CUDA;
+    g_noalloc_addr[dev] = static_cast<float*>(p);
+  }
+  *addr = g_noalloc_addr[dev];
+  return BASED_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -284,6 +319,29 @@ based_status_t based_linattn_fwd(const void* q, const void* k, const void* v, vo
                                             workspace, workspace_bytes, st)
                    : launch_linattn_tc<128>(q, k, v, out, BH, L, eps, state_kv, state_k,
                                             workspace, workspace_bytes, st);
+}
+
+based_status_t based_linattn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
+                                         int B, int H, int L, int d_feat, int d_v,
+                                         based_dtype_t dt, float eps, float* state_kv,
+                                         float* state_k, based_stream_t stream) {
+  based_status_t s =
+      check_linattn(q, k, v, out, B, H, L, d_feat, d_v, dt, eps, state_kv, state_k);
+  if (s != BASED_OK) return s;
+  const int BH = B * H;
+  if (BH == 0) return BASED_OK;
+  if (L == 0 && !state_kv && !state_k) return BASED_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dt == BASED_F32)  // the fp32 path needs no scratch
+    return launch_linattn_simt<float>(q, k, v, out, BH, L, d_v, eps, state_kv, state_k, st);
+  const size_t need = plan_linattn_tc(BH, L, d_v).workspace;
+  if (need > kNoAllocScratchBytes) return BASED_ERR_WORKSPACE;
+  float* scratch = nullptr;
+  if (need > 0 && (s = noalloc_scratch(&scratch)) != BASED_OK) return s;
+  return d_v == 64 ? launch_linattn_tc<64>(q, k, v, out, BH, L, eps, state_kv, state_k, scratch,
+                                           kNoAllocScratchBytes, st)
+                   : launch_linattn_tc<128>(q, k, v, out, BH, L, eps, state_kv, state_k, scratch,
+                                            kNoAllocScratchBytes, st);
 }
 
 based_status_t based_window_attn_fwd(const void* q, const void* k, const void* v, void* out,
