@@ -166,8 +166,9 @@ based_status_t launch_linattn_tc(const void* q, const void* k, const void* v, vo
     return BASED_ERR_WORKSPACE;
   if (pl.workspace > 0 && (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0)
     return BASED_ERR_INVALID_ARG;
-  CUtensorMap vmap;
+  CUtensorMap vmap, ymap;
   if (!make_rows_map(&vmap, v, DV, L, BH, kTcChunk)) return BASED_ERR_CUDA;
+  if (!make_rows_map(&ymap, out, DV, L, BH, kTcChunk)) return BASED_ERR_CUDA;
   TcParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k = static_cast<const __nv_bfloat16*>(k);
@@ -185,14 +186,14 @@ based_status_t launch_linattn_tc(const void* q, const void* k, const void* v, vo
     if (!set_smem(kst, smem)) return BASED_ERR_CUDA;
     const long long nblk = (long long)BH * (pl.n_seg - 1);
     if (nblk > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
-    kst<<<(unsigned)nblk, kTcThreads, smem, st>>>(vmap, p);
+    kst<<<(unsigned)nblk, kTcThreads, smem, st>>>(vmap, ymap, p);
     if (cudaGetLastError() != cudaSuccess) return BASED_ERR_CUDA;
   }
   auto kern = linattn_tc_kernel<DV, false>;
   if (!set_smem(kern, smem)) return BASED_ERR_CUDA;
   const long long nblk = (long long)BH * pl.n_seg;
   if (nblk > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
-  kern<<<(unsigned)nblk, kTcThreads, smem, st>>>(vmap, p);
+  kern<<<(unsigned)nblk, kTcThreads, smem, st>>>(vmap, ymap, p);
   return launch_status();
 }
 

@@ -16,20 +16,38 @@
 //  * the intra-chunk scores phi(q).phi(k) are evaluated in closed form,
 //    1 + u + u^2/2 with u = q.k / 4 (the expansion the blog post prints), so
 //    #1 contracts over the 16 input dims instead of the 273 features;
-//  * phi(q).phi(k) only needs the 153 distinct features [1, x_i/2,
-//    x_i x_j c_ij (i <= j)] with c_ii = 1/(4 sqrt 2), c_ij = 1/4 (i < j): the
-//    full map lists every off-diagonal product twice with weight 1/(4 sqrt 2).
-//    The state is kept over these 153 features and expanded to the 273-row
-//    layout (off-diagonal rows = value / sqrt 2, duplicated) only on export.
+//  * phi(q).phi(k) only needs the 153 distinct products: 1, x_i/2, and for each
+//    unordered pair {i, j} one feature (x_i/2)(x_j/2) c with c = 1/sqrt 2 on the
+//    diagonal and 1 off it (the full map lists every off-diagonal product twice
+//    with weight 1/(4 sqrt 2)).  The state is kept over these 153 features and
+//    expanded to the 273-row layout (off-diagonal rows = value / sqrt 2,
+//    duplicated) only on export.
 // The ones column appended to V makes the normaliser z and both parts of the
 // denominator come out of the same MMAs, with the same rounded operands as the
 // numerator.
+//
+// Feature order inside the kernel (160 = 20 chunks of 8): chunk 0 = [1, 0 x 7],
+// chunks 1-2 = x_i/2, chunks 3-4 = (x_i/2)^2/sqrt 2, then for d = 1..7 two chunks
+// of (x_i/2)(x_{i+d mod 16}/2), i = 0..15, and chunk 19 = (x_i/2)(x_{i+8}/2),
+// i = 0..7.  With x held as eight packed pairs X[m] = (x_2m, x_2m+1)/2 and the
+// shifted pairs Y[m] = (x_2m+1, x_2m+2)/2, every pair of features is a single
+// bf16x2 / f16x2 multiply X[m] * X[m + d/2] (d even) or X[m] * Y[m + (d-1)/2].
 //
 // Operand precision: Q, K, V, P and phiK are bf16; phiQ and the per-chunk copy
 // of the state used by #2 are fp16 (bf16 inputs are exact in fp16; the state
 // copy is scaled by a power of two so it stays in fp16 range for any L, and P is
 // scaled by the same power so the ratio is unchanged).  All accumulation is fp32
 // in TMEM; the master state never leaves TMEM until the export.
+//
+// Schedule (warp-specialised, chunks pipelined):
+//   group A (warps 0-3): feature maps and Q/K tiles of chunk c, then P of chunk c;
+//   group E (warps 4-7): epilogue of chunk c -- y from O, and the fp16 copy of the
+//            state for chunk c+1 -- while group A already builds chunk c+1;
+//   issue warp (warp 8, one thread): V tiles by TMA (double-buffered when shared
+//            memory allows) and the MMAs in the order #1, #5, #2, (P), #4.
+// The second state tile (features 128..191, of which 128..159 are used) is an
+// M=64 MMA.  Hand-offs are mbarriers (128 arrivals from a warp group, or a
+// tcgen05.commit); every wait is bounded.
 //
 // Long sequences are split into n_seg segments of seg_chunks chunks so that
 // B*H*n_seg CTAs fill the GPU: a state-only pass (kStateOnly) runs #5 alone
@@ -46,46 +64,51 @@
 namespace based {
 
 constexpr int kTcChunk = 128;          // tokens per chunk (MMA M)
-constexpr int kTcThreads = 128;        // 4 warps, one TMEM lane quadrant each
-constexpr int kSymF = 153;             // distinct Taylor features
-constexpr int kSymFP = 160;            // padded to the MMA K granularity (16)
+constexpr int kTcGroup = 128;          // threads of one CUDA-core warp group (4 warps)
+constexpr int kTcThreads = 2 * kTcGroup + 32;  // feature/score group, epilogue group, issue warp
+constexpr int kSymFP = 160;            // 153 distinct features + 7 zero pads
 constexpr int kTcTmemCols = 512;
-
-// Symmetric-feature index (>= 17) -> (i, j) of the quadratic block, i <= j.
-__host__ __device__ constexpr int sym_pair_i(int p) {
-  int i = 0;
-  while (p >= 16 - i) { p -= 16 - i; ++i; }
-  return i;
-}
-__host__ __device__ constexpr int sym_pair_j(int p) {
-  int i = 0;
-  while (p >= 16 - i) { p -= 16 - i; ++i; }
-  return i + p;
-}
 
 template <int DV>
 struct TcLayout {
   static constexpr int NA = DV + 16;                       // [V | 1 | 0..] columns
-  static constexpr int kTileCols = (NA + 31) / 32 * 32;    // TMEM columns per state tile
+  static constexpr int NG = (NA + 31) / 32;                // 32-column groups of a state tile
+  static constexpr int kTileCols = NG * 32;                // TMEM columns per state tile
+  // d_v = 64 fits phiQ and P in TMEM as A operands (and frees the shared memory
+  // for a second phiK buffer and a y staging tile stored by TMA); d_v = 128
+  // keeps them in shared memory
+  static constexpr bool kTm = DV == 64;
+  static constexpr int kVBuf = DV == 64 ? 2 : 1;           // V stages
+  static constexpr int kPhiKBuf = kTm ? 2 : 1;             // phiK buffers
+  static constexpr int kVStage = (DV / 64 + 1) * 16384;    // V blocks + ones block
   // shared memory (byte offsets from a 1024-aligned base)
   static constexpr int kQ = 0;                             // Q tile  [128 x 16] bf16, K-major
   static constexpr int kK = kQ + 4096;                     // K tile  [128 x 16] bf16, K-major
-  static constexpr int kV = kK + 4096;                     // [V | ones] MN-major SW128 blocks
-  static constexpr int kVBlocks = DV / 64 + 1;
-  static constexpr int kPhiK = kV + kVBlocks * 16384;      // phiK [160 x 128] bf16, MN-major
-  static constexpr int kP = kPhiK + 40960;                 // P [128 x 128] bf16, K-major
-  static constexpr int kPhiQ = kP + 32768;                 // phiQ [128 x 160] fp16, K-major
-  static constexpr int kS = kPhiQ + 40960;                 // [S|z] copy [160 x NA] fp16, MN-major
-  static constexpr int kBar = kS + NA * kSymFP * 2;        // mbarriers + TMEM address
-  static constexpr int kBytes = kBar + 64;
+  static constexpr int kV = kK + 4096;                     // [V | ones] MN-major SW128 stages
+  static constexpr int kPhiK = kV + kVBuf * kVStage;       // phiK [160 x 128] bf16, MN-major
+  static constexpr int kP = kPhiK + kPhiKBuf * 40960;      // P [128 x 128] bf16 (smem path)
+  static constexpr int kPhiQ = kP + (kTm ? 0 : 32768);     // phiQ [128 x 160] fp16 (smem path)
+  static constexpr int kS = kPhiQ + (kTm ? 0 : 40960);     // [S|z] copy [160 x NA] fp16, MN-major
+  static constexpr int kY = kS + NA * kSymFP * 2;          // y staging, 2 x [128 x 64] bf16 SW128
+  static constexpr int kBar = kY + (kTm ? 2 * 16384 : 0);  // mbarriers + TMEM address
+  static constexpr int kBytes = kBar + 128;
   static constexpr size_t kSmem = kBytes + 1024;           // + alignment slack
-  // TMEM columns: [S|z] tiles (two 128-feature tiles) then the U / O accumulator
-  static constexpr int kTmS = 0;
-  static constexpr int kTmO = 2 * kTileCols;
-  static_assert(kTmO + 160 <= kTcTmemCols, "TMEM budget");
-  // #5 reads 32 feature groups past phiK (the second tile's unused rows); keep
-  // that window inside the allocation.
-  static_assert(kPhiK + 65536 <= kBytes, "phiK over-read window");
+  // TMEM: state tile 0 (features 0..127, M=128), state tile 1 (features
+  // 128..191, M=64: row r in lane r%16 + 32*(r/16)), the score tile U (P is
+  // written over it), the output accumulator O -- separate from U when the
+  // columns allow it -- and phiQ (80 columns of fp16 pairs)
+  static constexpr bool kEarlyO = 3 * kTileCols + 128 <= kTcTmemCols;
+  static constexpr int kTmS0 = 0;
+  static constexpr int kTmS1 = kTileCols;
+  static constexpr int kTmU = 2 * kTileCols;
+  static constexpr int kTmO = kEarlyO ? kTmU + 128 : kTmU;
+  static constexpr int kTmQ = kTmO + kTileCols;
+  static_assert(kTmO + kTileCols + (kTm ? kSymFP / 2 : 0) <= kTcTmemCols, "TMEM budget");
+  static_assert(!kTm || kEarlyO, "TMEM operands need a separate O");
+  static_assert(kY % 1024 == 0, "TMA staging alignment");
+  // the M=64 state MMA reads feature groups 16..23 (8 past the 160 written)
+  static_assert(kPhiK + (kPhiKBuf - 1) * 40960 + 49152 <= kBytes, "phiK over-read window");
+  static_assert(kSmem <= 232448, "shared memory budget");
 };
 
 struct TcParams {
@@ -109,22 +132,117 @@ __device__ __forceinline__ float tc_chunk_scale(long long t_end) {
   return __int_as_float((127 - e) << 23);
 }
 
+// Row(s) of the 273-row layout a kernel feature f maps to, and the factor.
+// Returns the number of rows (0 for padding).
+__device__ __forceinline__ int tc_feature_rows(int f, int* r0, int* r1, float* scale) {
+  *scale = 1.0f;
+  if (f == 0) { *r0 = 0; return 1; }
+  if (f < 8) return 0;
+  if (f < 24) { *r0 = 1 + (f - 8); return 1; }
+  if (f < 40) { const int i = f - 24; *r0 = 17 + 17 * i; return 1; }
+  int i, j;
+  if (f < 152) {
+    const int d = 1 + (f - 40) / 16;
+    i = (f - 40) % 16;
+    j = (i + d) & 15;
+  } else {
+    i = f - 152;
+    j = i + 8;
+  }
+  *r0 = 17 + 16 * i + j;
+  *r1 = 17 + 16 * j + i;
+  *scale = 0.70710678118654752f;
+  return 2;
+}
+
+// Packed 2-wide arithmetic for the feature build (fp16 for phiQ, bf16 for phiK).
+struct H2Ops {
+  static __device__ __forceinline__ __half2 mul(__half2 a, __half2 b) { return __hmul2(a, b); }
+  static __device__ __forceinline__ __nv_bfloat162 mul(__nv_bfloat162 a, __nv_bfloat162 b) {
+    return __hmul2(a, b);
+  }
+  static __device__ __forceinline__ __half2 shift(__half2 a, __half2 b) {
+    return __halves2half2(__high2half(a), __low2half(b));
+  }
+  static __device__ __forceinline__ __nv_bfloat162 shift(__nv_bfloat162 a, __nv_bfloat162 b) {
+    return __halves2bfloat162(__high2bfloat16(a), __low2bfloat16(b));
+  }
+};
+
+template <typename T2>
+__device__ __forceinline__ uint32_t as_u32(T2 v) {
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+template <typename T2> __device__ __forceinline__ T2 pack2(float a, float b);
+template <> __device__ __forceinline__ __half2 pack2<__half2>(float a, float b) {
+  return __floats2half2_rn(a, b);
+}
+template <> __device__ __forceinline__ __nv_bfloat162 pack2<__nv_bfloat162>(float a, float b) {
+  return __floats2bfloat162_rn(a, b);
+}
+
+// Feature chunk ch (8 features) of one token from its packed pairs X[8] (x/2),
+// the shifted pairs Y[8], and its raw bf16 input pairs (the diagonal features are
+// formed in fp32 and rounded once).  ch must be a compile-time constant.
+template <typename T2>
+__device__ __forceinline__ uint4 tc_feature_chunk(const T2* X, const T2* Y,
+                                                  const __nv_bfloat162* raw, int ch) {
+  T2 v[4];
+  if (ch == 0) {
+    v[0] = pack2<T2>(1.0f, 0.0f);
+    v[1] = v[2] = v[3] = pack2<T2>(0.0f, 0.0f);
+  } else if (ch <= 2) {
+    const int m0 = (ch - 1) * 4;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[e] = X[m0 + e];
+  } else if (ch <= 4) {
+    const int m0 = (ch - 3) * 4;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 x = __bfloat1622float2(raw[m0 + e]);  // x_i^2 / (4 sqrt 2)
+      v[e] = pack2<T2>(x.x * x.x * 0.17677669529663687f, x.y * x.y * 0.17677669529663687f);
+    }
+  } else if (ch <= 18) {
+    const int d = 1 + (ch - 5) / 2, m0 = ((ch - 5) & 1) * 4;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int m = m0 + e;
+      v[e] = (d & 1) ? H2Ops::mul(X[m], Y[(m + (d - 1) / 2) & 7])
+                     : H2Ops::mul(X[m], X[(m + d / 2) & 7]);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[e] = H2Ops::mul(X[e], X[e + 4]);
+  }
+  return make_uint4(as_u32(v[0]), as_u32(v[1]), as_u32(v[2]), as_u32(v[3]));
+}
+
 template <int DV, bool kStateOnly>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    linattn_tc_kernel(const __grid_constant__ CUtensorMap vmap, const TcParams p) {
+    linattn_tc_kernel(const __grid_constant__ CUtensorMap vmap,
+                      const __grid_constant__ CUtensorMap ymap, const TcParams p) {
   using Lay = TcLayout<DV>;
   constexpr int NA = Lay::NA;
-  constexpr int NG = (NA + 31) / 32;  // 32-column groups of a state tile
+  constexpr int NG = Lay::NG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
-  uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + Lay::kBar);
-  uint64_t* bar_u = bar_tma + 1;
-  uint64_t* bar_o = bar_tma + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_tma + 3);
-  int* abort_flag = reinterpret_cast<int*>(bar_tma + 4);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::kBar);
+  uint64_t* bar_tma = bars;          // [2] V stage landed
+  uint64_t* bar_phi = bars + 2;      // feature maps + Q/K tiles written (group A)
+  uint64_t* bar_u = bars + 3;        // #1 done (commit)
+  uint64_t* bar_p = bars + 4;        // P written (group A)
+  uint64_t* bar_m25 = bars + 5;      // #5 and #2 done (commit): feature buffers free
+  uint64_t* bar_o = bars + 6;        // every MMA of the chunk done (commit)
+  uint64_t* bar_ss = bars + 7;       // state read + fp16 copy written, O read (group E)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 9);
+  uint64_t* bar_yfree = bars + 10;   // y staging tile free again (TMA store read it)
+  uint64_t* bar_yfull = bars + 11;   // y staging tile written (group E)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quad = warp & 3;
   const int L = p.L;
   const int n_chunks = (L + kTcChunk - 1) / kTcChunk;
   const int segs_here = kStateOnly ? p.n_seg - 1 : p.n_seg;
@@ -133,14 +251,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int c_begin = seg * p.seg_chunks;
   const int c_end = min(c_begin + p.seg_chunks, n_chunks);
   const bool has_init = !kStateOnly && seg > 0;
-  const __nv_bfloat16* q = p.q + (size_t)bh * L * kD;
-  const __nv_bfloat16* k = p.k + (size_t)bh * L * kD;
-  __nv_bfloat16* out = kStateOnly ? nullptr : p.out + (size_t)bh * L * DV;
 
   if (tid == 0) {
     umma::mbar_init(bar_tma, 1);
+    umma::mbar_init(bar_tma + 1, 1);
+    umma::mbar_init(bar_phi, kTcGroup);
     umma::mbar_init(bar_u, 1);
+    umma::mbar_init(bar_p, kTcGroup);
+    umma::mbar_init(bar_m25, 1);
     umma::mbar_init(bar_o, 1);
+    umma::mbar_init(bar_ss, kTcGroup);
+    umma::mbar_init(bar_yfree, 1);
+    umma::mbar_init(bar_yfull, kTcGroup);
     *abort_flag = 0;
     umma::fence_mbar_init();
     umma::tma_prefetch_desc(&vmap);
@@ -149,363 +271,474 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     umma::tmem_alloc(tmem_slot, kTcTmemCols);
     umma::tmem_relinquish();
   }
-  // ones block of [V | 1]: column DV of the augmented V is 1 for every token
-  {
-    uint8_t* ones = sm + Lay::kV + (DV / 64) * 16384;
+  // ones block of every V stage: column DV of the augmented V is 1 for every token
+  for (int b = 0; b < Lay::kVBuf; ++b) {
+    uint8_t* ones = sm + Lay::kV + b * Lay::kVStage + (DV / 64) * 16384;
     for (int i = tid; i < 16384 / 16; i += kTcThreads)
       reinterpret_cast<uint4*>(ones)[i] = make_uint4(0, 0, 0, 0);
-    __syncthreads();
-    *reinterpret_cast<__nv_bfloat16*>(ones + umma::off_mnmajor_sw128(0, tid, kTcChunk)) =
-        __float2bfloat16(1.0f);
   }
+  __syncthreads();
+  for (int b = 0; b < Lay::kVBuf; ++b)
+    if (tid < kTcChunk)
+      *reinterpret_cast<__nv_bfloat16*>(sm + Lay::kV + b * Lay::kVStage + (DV / 64) * 16384 +
+                                        umma::off_mnmajor_sw128(0, tid, kTcChunk)) =
+          __float2bfloat16(1.0f);
   umma::fence_async_smem();
   umma::tc_fence_before();
   __syncthreads();
   umma::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tm_lane = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t sQ = umma::smem_u32(sm + Lay::kQ), sK = umma::smem_u32(sm + Lay::kK),
-                 sV = umma::smem_u32(sm + Lay::kV), sPhiK = umma::smem_u32(sm + Lay::kPhiK),
-                 sP = umma::smem_u32(sm + Lay::kP), sPhiQ = umma::smem_u32(sm + Lay::kPhiQ),
-                 sS = umma::smem_u32(sm + Lay::kS);
-  constexpr uint32_t kVBytes = DV * kTcChunk * 2;
-  // state tiles: tile 0 lanes 0..127 = features 0..127 (all warps); tile 1
-  // lanes 0..31 = features 128..159 (warp 0 only)
-  const int n_tiles_here = warp == 0 ? 2 : 1;
-
-  auto issue_v = [&](int c) {
-    umma::mbar_arrive_expect_tx(bar_tma, kVBytes);
-#pragma unroll
-    for (int b = 0; b < DV / 64; ++b)
-      umma::tma_load_3d(sm + Lay::kV + b * 16384, &vmap, bar_tma, b * 64, c * kTcChunk, bh);
-  };
-  if (tid == 0 && c_begin < c_end) issue_v(c_begin);
-
-  // fp16 copy of the TMEM state, scaled by sn, as the B operand of #2
-  auto copy_state = [&](float sn) {
-    for (int mt = 0; mt < n_tiles_here; ++mt) {
-      const int f = mt * 128 + warp * 32 + lane;
-#pragma unroll
-      for (int g = 0; g < NG; ++g) {
-        float sv[32];
-        umma::tmem_ld32(tmem + Lay::kTmS + mt * Lay::kTileCols + tm_lane + g * 32, sv);
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const int j0 = g * 32 + h * 8;
-          if (j0 < NA) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const __half2 hv = __floats2half2_rn(sv[h * 8 + 2 * e] * sn, sv[h * 8 + 2 * e + 1] * sn);
-              pk[e] = *reinterpret_cast<const uint32_t*>(&hv);
-            }
-            *reinterpret_cast<uint4*>(sm + Lay::kS + ((j0 >> 3) * 20 + (f >> 3)) * 128 + (f & 7) * 16) =
-                make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          }
-        }
-      }
-    }
+  const uint32_t tm_lane = static_cast<uint32_t>(quad * 32) << 16;
+  auto fail = [&]() {
+    record_device_error(BASED_ERR_TIMEOUT);
+    *abort_flag = 1;
   };
 
-  // seed the TMEM state of a later segment with the sum of the earlier partials
-  if (has_init) {
-    const float* part = p.partial + (size_t)bh * (p.n_seg - 1) * kSymFP * NA;
-    for (int mt = 0; mt < n_tiles_here; ++mt) {
-      const int f = mt * 128 + warp * 32 + lane;
+  if (warp == 8) {
+    // ================= issue warp: lane 0 drives TMA and the tensor cores =================
+    if (lane == 0) {
+      const uint32_t sQ = umma::smem_u32(sm + Lay::kQ), sK = umma::smem_u32(sm + Lay::kK),
+                     sP = umma::smem_u32(sm + Lay::kP), sPhiQ = umma::smem_u32(sm + Lay::kPhiQ),
+                     sS = umma::smem_u32(sm + Lay::kS);
+      constexpr uint32_t kVBytes = DV * kTcChunk * 2;
+      auto issue_v = [&](int c, int stage) {
+        umma::mbar_arrive_expect_tx(bar_tma + stage, kVBytes);
 #pragma unroll
-      for (int g = 0; g < NG; ++g) {
-        float acc[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
-        for (int sp = 0; sp < seg; ++sp) {
-          const float* row = part + ((size_t)sp * kSymFP + f) * NA + g * 32;
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (g * 32 + i < NA) acc[i] += row[i];
-        }
-        umma::tmem_st32(tmem + Lay::kTmS + mt * Lay::kTileCols + tm_lane + g * 32, acc);
-      }
-    }
-    umma::tc_fence_before();
-    __syncthreads();
-    umma::tc_fence_after();
-    copy_state(tc_chunk_scale((long long)c_begin * kTcChunk + kTcChunk));
-  }
-
-  // q/k rows of this thread's token, prefetched one chunk ahead
-  uint4 qr[2], kr[2];
-  auto load_qk = [&](int c) {
-    const long long t = (long long)c * kTcChunk + tid;
-    if (c < c_end && t < L) {
-      const uint4* kp = reinterpret_cast<const uint4*>(k + t * kD);
-      kr[0] = kp[0]; kr[1] = kp[1];
-      if (!kStateOnly) {
-        const uint4* qp = reinterpret_cast<const uint4*>(q + t * kD);
-        qr[0] = qp[0]; qr[1] = qp[1];
-      } else {
-        qr[0] = qr[1] = make_uint4(0, 0, 0, 0);
-      }
-    } else {
-      qr[0] = qr[1] = kr[0] = kr[1] = make_uint4(0, 0, 0, 0);
-    }
-  };
-  load_qk(c_begin);
-
-  uint32_t ph_tma = 0, ph_u = 0, ph_o = 0;
-  bool tma_pending = c_begin < c_end;
-  const uint32_t id_u = umma::idesc_bf16(128, 128, false, false);
-  const uint32_t id_o2 = umma::idesc_f16(128, NA, false, true);
-  const uint32_t id_o4 = umma::idesc_bf16(128, NA, false, true);
-  const uint32_t id_s5 = umma::idesc_bf16(128, NA, true, true);
-
-  __syncthreads();
-  for (int c = c_begin; c < c_end; ++c) {
-    const int t0 = c * kTcChunk;
-    const int n = min(kTcChunk, L - t0);
-    const bool has_state = has_init || c > c_begin;
-    const float sc = tc_chunk_scale((long long)t0 + kTcChunk);
-    // ---- (a) Q/K tiles and the feature maps of this thread's token -------------
-    {
-      const int t = tid;
-      if (!kStateOnly) {
-        uint8_t* qrow = sm + Lay::kQ + ((t >> 3) * 2) * 128 + (t & 7) * 16;
-        uint8_t* krow = sm + Lay::kK + ((t >> 3) * 2) * 128 + (t & 7) * 16;
-        *reinterpret_cast<uint4*>(qrow) = qr[0];
-        *reinterpret_cast<uint4*>(qrow + 128) = qr[1];
-        *reinterpret_cast<uint4*>(krow) = kr[0];
-        *reinterpret_cast<uint4*>(krow + 128) = kr[1];
-      }
-      float xq[16], xk[16];
-      const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(qr);
-      const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(kr);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float2 a = __bfloat1622float2(q2[i]);
-        const float2 b = __bfloat1622float2(k2[i]);
-        xq[2 * i] = a.x; xq[2 * i + 1] = a.y;
-        xk[2 * i] = b.x; xk[2 * i + 1] = b.y;
-      }
-      const bool live = t < n;
-      // features in order: 1, x_i/2 (16), x_i x_j c_ij for i <= j (136), zero pad (7);
-      // every index below is a compile-time constant after unrolling
-      float fq8[8], fk8[8];
-      int slot = 0, ch = 0;
-      auto flush = [&]() {
-        uint32_t hq[4], bk[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const __half2 h = __floats2half2_rn(fq8[2 * e], fq8[2 * e + 1]);
-          const __nv_bfloat162 b = __floats2bfloat162_rn(live ? fk8[2 * e] : 0.0f,
-                                                          live ? fk8[2 * e + 1] : 0.0f);
-          hq[e] = *reinterpret_cast<const uint32_t*>(&h);
-          bk[e] = *reinterpret_cast<const uint32_t*>(&b);
-        }
-        if (!kStateOnly)
-          *reinterpret_cast<uint4*>(sm + Lay::kPhiQ + ((t >> 3) * 20 + ch) * 128 + (t & 7) * 16) =
-              make_uint4(hq[0], hq[1], hq[2], hq[3]);
-        *reinterpret_cast<uint4*>(sm + Lay::kPhiK + (ch * 16 + (t >> 3)) * 128 + (t & 7) * 16) =
-            make_uint4(bk[0], bk[1], bk[2], bk[3]);
-        ++ch;
-        slot = 0;
+        for (int blk = 0; blk < DV / 64; ++blk)
+          umma::tma_load_3d(sm + Lay::kV + stage * Lay::kVStage + blk * 16384, &vmap,
+                            bar_tma + stage, blk * 64, c * kTcChunk, bh);
       };
-      auto emit = [&](float a, float b) {
-        fq8[slot] = a;
-        fk8[slot] = b;
-        if (++slot == 8) flush();
-      };
-      emit(1.0f, 1.0f);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) emit(0.5f * xq[i], 0.5f * xk[i]);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-#pragma unroll
-        for (int j = i; j < 16; ++j) {
-          const float cw = i == j ? 0.17677669529663687f : 0.25f;
-          emit(xq[i] * xq[j] * cw, xk[i] * xk[j] * cw);
+      const uint32_t id_u = umma::idesc_bf16(128, 128, false, false);
+      const uint32_t id_o2 = umma::idesc_f16(128, NA, false, true);
+      const uint32_t id_o4 = umma::idesc_bf16(128, NA, false, true);
+      const uint32_t id_s0 = umma::idesc_bf16(128, NA, true, true);
+      const uint32_t id_s1 = umma::idesc_bf16(64, NA, true, true);
+      // per stage: a load in flight, and the parity of the phase it completes
+      bool inflight[2] = {false, false};
+      uint32_t vphase[2] = {0, 0};
+      if (c_begin < c_end) { issue_v(c_begin, 0); inflight[0] = true; }
+      if (Lay::kVBuf == 2 && c_begin + 1 < c_end) { issue_v(c_begin + 1, 1); inflight[1] = true; }
+      int n_done = 0;  // chunks whose MMAs were all issued and committed
+      for (int c = c_begin; c < c_end && !*abort_flag; ++c) {
+        const int it = c - c_begin;
+        const uint32_t ph = it & 1;
+        const int stage = Lay::kVBuf == 2 ? (it & 1) : 0;
+        const uint32_t sV = umma::smem_u32(sm + Lay::kV + stage * Lay::kVStage);
+        const uint32_t sPhiK = umma::smem_u32(sm + Lay::kPhiK + (it % Lay::kPhiKBuf) * 40960);
+        const bool has_state = has_init || it > 0;
+        const uint32_t ph_ss = (it + (has_init ? 0 : 1)) & 1;  // epilogue hand-off of chunk c-1
+        if (!umma::mbar_wait(bar_phi, ph)) { fail(); break; }
+        // when O shares TMEM with U, #1 may only overwrite it once the epilogue
+        // group has read the previous chunk's O
+        if (!kStateOnly && !Lay::kEarlyO && has_state) {
+          if (!umma::mbar_wait(bar_ss, ph_ss)) { fail(); break; }
         }
-      }
-#pragma unroll
-      for (int f = kSymF; f < kSymFP; ++f) emit(0.0f, 0.0f);
-    }
-    load_qk(c + 1);
-    umma::fence_async_smem();
-    umma::tc_fence_before();
-    __syncthreads();
-    umma::tc_fence_after();
-    if (!kStateOnly) {
-      // ---- (b) #1: U = Q K^T -------------------------------------------------------
-      if (tid == 0) {
-        umma::mma_bf16(tmem + Lay::kTmO, umma::desc_kmajor_none(sQ, 0, 16),
-                       umma::desc_kmajor_none(sK, 0, 16), id_u, 0);
-        umma::mma_commit(bar_u);
-      }
-      __syncwarp();
-      if (!umma::mbar_wait(bar_u, ph_u)) { record_device_error(BASED_ERR_TIMEOUT); *abort_flag = 1; }
-      ph_u ^= 1;
-      umma::tc_fence_after();
-      // ---- (c) scores: P = mask(1 + u/4 + u^2/32) * sc -> smem -----------------------
-      {
-        const int t = tid;
-#pragma unroll
-        for (int c32 = 0; c32 < 4; ++c32) {
-          float u[32];
-          umma::tmem_ld32(tmem + Lay::kTmO + tm_lane + c32 * 32, u);
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int s0 = c32 * 32 + g * 8 + 2 * e;
-              const float u0 = u[g * 8 + 2 * e], u1 = u[g * 8 + 2 * e + 1];
-              const float w0 = s0 <= t ? fmaf(u0, fmaf(u0, 0.03125f, 0.25f), 1.0f) * sc : 0.0f;
-              const float w1 = s0 + 1 <= t ? fmaf(u1, fmaf(u1, 0.03125f, 0.25f), 1.0f) * sc : 0.0f;
-              const __nv_bfloat162 b = __floats2bfloat162_rn(w0, w1);
-              pk[e] = *reinterpret_cast<const uint32_t*>(&b);
-            }
-            const int ch = c32 * 4 + g;
-            *reinterpret_cast<uint4*>(sm + Lay::kP + ((t >> 3) * 16 + ch) * 128 + (t & 7) * 16) =
-                make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          }
-        }
-      }
-      umma::fence_async_smem();
-      umma::tc_fence_before();
-      __syncthreads();
-      umma::tc_fence_after();
-      if (*abort_flag) break;
-    }
-    // ---- (d) #2, #4, #5 ----------------------------------------------------------------
-    if (tid == 0) {
-      const bool ok = umma::mbar_wait(bar_tma, ph_tma);
-      ph_tma ^= 1;
-      tma_pending = false;
-      if (!ok) {
-        record_device_error(BASED_ERR_TIMEOUT);
-        *abort_flag = 1;
-      } else {
         umma::tc_fence_after();
         if (!kStateOnly) {
+          umma::mma_bf16(tmem + Lay::kTmU, umma::desc_kmajor_none(sQ, 0, 16),
+                         umma::desc_kmajor_none(sK, 0, 16), id_u, 0);
+          umma::mma_commit(bar_u);
+        }
+        if (!umma::mbar_wait(bar_tma + stage, vphase[stage])) { fail(); break; }
+        inflight[stage] = false;
+        vphase[stage] ^= 1;
+        // the state copy of the previous chunk must have been read out of TMEM
+        // (and, for #2, written to shared memory) by the epilogue group
+        if (!kStateOnly && Lay::kEarlyO && has_state) {
+          if (!umma::mbar_wait(bar_ss, ph_ss)) { fail(); break; }
+        }
+        umma::tc_fence_after();
+#pragma unroll
+        for (int k0 = 0; k0 < kTcChunk; k0 += 16) {
+          const uint64_t bdesc = umma::desc_mnmajor_sw128(sV, k0, kTcChunk);
+          umma::mma_bf16(tmem + Lay::kTmS0, umma::desc_mnmajor_none(sPhiK, k0, kTcChunk), bdesc,
+                         id_s0, has_state || (k0 > 0));
+          umma::mma_bf16(tmem + Lay::kTmS1,
+                         umma::desc_mnmajor_none(sPhiK + 16 * 2048, k0, kTcChunk), bdesc, id_s1,
+                         has_state || (k0 > 0));
+        }
+        if (!kStateOnly) {
+          if (!Lay::kEarlyO) {  // O shares TMEM with U: wait until P has been read out
+            if (!umma::mbar_wait(bar_p, ph)) { fail(); break; }
+            umma::tc_fence_after();
+          }
           if (has_state) {
 #pragma unroll
-            for (int k0 = 0; k0 < kSymFP; k0 += 16)
-              umma::mma_f16(tmem + Lay::kTmO, umma::desc_kmajor_none(sPhiQ, k0, kSymFP),
-                            umma::desc_mnmajor_none(sS, k0, kSymFP), id_o2, k0 > 0);
+            for (int k0 = 0; k0 < kSymFP; k0 += 16) {
+              if constexpr (Lay::kTm)
+                umma::mma_ts(tmem + Lay::kTmO, tmem + Lay::kTmQ + k0 / 2,
+                             umma::desc_mnmajor_none(sS, k0, kSymFP), id_o2, k0 > 0);
+              else
+                umma::mma_f16(tmem + Lay::kTmO, umma::desc_kmajor_none(sPhiQ, k0, kSymFP),
+                              umma::desc_mnmajor_none(sS, k0, kSymFP), id_o2, k0 > 0);
+            }
+          }
+        }
+        umma::mma_commit(bar_m25);
+        if (!kStateOnly) {
+          if (Lay::kEarlyO) {
+            if (!umma::mbar_wait(bar_p, ph)) { fail(); break; }
+            umma::tc_fence_after();
           }
 #pragma unroll
-          for (int k0 = 0; k0 < kTcChunk; k0 += 16)
-            umma::mma_bf16(tmem + Lay::kTmO, umma::desc_kmajor_none(sP, k0, kTcChunk),
+          for (int k0 = 0; k0 < kTcChunk; k0 += 16) {
+            if constexpr (Lay::kTm)
+              umma::mma_ts(tmem + Lay::kTmO, tmem + Lay::kTmU + k0 / 2,
                            umma::desc_mnmajor_sw128(sV, k0, kTcChunk), id_o4,
                            has_state || (k0 > 0));
+            else
+              umma::mma_bf16(tmem + Lay::kTmO, umma::desc_kmajor_none(sP, k0, kTcChunk),
+                             umma::desc_mnmajor_sw128(sV, k0, kTcChunk), id_o4,
+                             has_state || (k0 > 0));
+          }
+        }
+        umma::mma_commit(bar_o);
+        ++n_done;
+        // refill the stage this chunk used once its MMAs are done
+        const int c_next = c + Lay::kVBuf;
+        if (c_next < c_end) {
+          if (!umma::mbar_wait(bar_o, ph)) { fail(); break; }
+          issue_v(c_next, stage);
+          inflight[stage] = true;
+        }
+      }
+      // the last chunk's MMAs must be complete before the state is read out
+      if (n_done > 0 && !umma::mbar_wait(bar_o, (n_done - 1) & 1)) fail();
+      // an aborted run may still have V loads in flight: wait for them (bounded)
+      for (int sidx = 0; sidx < 2; ++sidx)
+        if (inflight[sidx]) umma::mbar_wait(bar_tma + sidx, vphase[sidx]);
+    }
+  } else if (warp < 4) {
+    // ================= group A: feature maps (chunk c), scores (chunk c) =================
+    const int t = tid;  // token row of the chunk; also the TMEM lane (quadrant = warp)
+    const __nv_bfloat16* q = p.q + (size_t)bh * L * kD;
+    const __nv_bfloat16* k = p.k + (size_t)bh * L * kD;
+    uint4 qr[2], kr[2];
+    auto load_qk = [&](int c) {
+      const long long tt = (long long)c * kTcChunk + t;
+      if (c < c_end && tt < L) {
+        const uint4* kp = reinterpret_cast<const uint4*>(k + tt * kD);
+        kr[0] = kp[0]; kr[1] = kp[1];
+        if (!kStateOnly) {
+          const uint4* qp = reinterpret_cast<const uint4*>(q + tt * kD);
+          qr[0] = qp[0]; qr[1] = qp[1];
+        } else {
+          qr[0] = qr[1] = make_uint4(0, 0, 0, 0);
+        }
+      } else {
+        qr[0] = qr[1] = kr[0] = kr[1] = make_uint4(0, 0, 0, 0);
+      }
+    };
+    load_qk(c_begin);
+    for (int c = c_begin; c < c_end && !*abort_flag; ++c) {
+      const int it = c - c_begin;
+      const int t0 = c * kTcChunk;
+      const int n = min(kTcChunk, L - t0);
+      const bool live = t < n;
+      const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(qr);
+      const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(kr);
+      uint8_t* phik = sm + Lay::kPhiK + (it % Lay::kPhiKBuf) * 40960;
+      // With a single phiK buffer (and for the smem phiQ / Q / K tiles) wait
+      // until the previous chunk's #5 and #2 are done.  With two phiK buffers,
+      // this chunk's buffer was released by the wait of the previous iteration.
+      if (!Lay::kTm && it > 0 && !umma::mbar_wait(bar_m25, (it - 1) & 1)) { fail(); break; }
+      // ---- phiK and Q/K tiles -------------------------------------------------------
+      {
+        __nv_bfloat162 XK[8], YK[8];
+        const __nv_bfloat162 halfk = __floats2bfloat162_rn(0.5f, 0.5f);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) XK[m] = __hmul2(k2[m], halfk);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) YK[m] = H2Ops::shift(XK[m], XK[(m + 1) & 7]);
+#pragma unroll
+        for (int ch = 0; ch < 20; ++ch)
+          *reinterpret_cast<uint4*>(phik + (ch * 16 + (t >> 3)) * 128 + (t & 7) * 16) =
+              live ? tc_feature_chunk(XK, YK, k2, ch) : make_uint4(0, 0, 0, 0);
+        if (!kStateOnly) {
+          uint8_t* qrow = sm + Lay::kQ + ((t >> 3) * 2) * 128 + (t & 7) * 16;
+          uint8_t* krow = sm + Lay::kK + ((t >> 3) * 2) * 128 + (t & 7) * 16;
+          *reinterpret_cast<uint4*>(qrow) = qr[0];
+          *reinterpret_cast<uint4*>(qrow + 128) = qr[1];
+          *reinterpret_cast<uint4*>(krow) = kr[0];
+          *reinterpret_cast<uint4*>(krow + 128) = kr[1];
+        }
+      }
+      if (Lay::kTm && it > 0 && !umma::mbar_wait(bar_m25, (it - 1) & 1)) { fail(); break; }
+      // ---- phiQ (TMEM operand, or smem) ------------------------------------------------
+      if (!kStateOnly) {
+        __half2 XQ[8], YQ[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const float2 a = __bfloat1622float2(q2[m]);
+          XQ[m] = __floats2half2_rn(0.5f * a.x, 0.5f * a.y);
         }
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
+        for (int m = 0; m < 8; ++m) YQ[m] = H2Ops::shift(XQ[m], XQ[(m + 1) & 7]);
+        if constexpr (Lay::kTm) {
+          umma::tc_fence_after();
+          uint32_t buf[32];
 #pragma unroll
-          for (int k0 = 0; k0 < kTcChunk; k0 += 16)
-            umma::mma_bf16(tmem + Lay::kTmS + mt * Lay::kTileCols,
-                           umma::desc_mnmajor_none(sPhiK + mt * 16 * 2048, k0, kTcChunk),
-                           umma::desc_mnmajor_sw128(sV, k0, kTcChunk), id_s5,
-                           has_state || (k0 > 0));
-        umma::mma_commit(bar_o);
+          for (int ch = 0; ch < 20; ++ch) {
+            const uint4 v = tc_feature_chunk(XQ, YQ, q2, ch);
+            const int s4 = (ch * 4) & 31;
+            buf[s4] = v.x; buf[s4 + 1] = v.y; buf[s4 + 2] = v.z; buf[s4 + 3] = v.w;
+            if (ch == 7 || ch == 15)
+              umma::tmem_st32(tmem + Lay::kTmQ + tm_lane + (ch - 7) * 4,
+                              reinterpret_cast<const float*>(buf));
+            if (ch == 19) umma::tmem_st16(tmem + Lay::kTmQ + tm_lane + 64, buf);
+          }
+        } else {
+#pragma unroll
+          for (int ch = 0; ch < 20; ++ch)
+            *reinterpret_cast<uint4*>(sm + Lay::kPhiQ + ((t >> 3) * 20 + ch) * 128 + (t & 7) * 16) =
+                tc_feature_chunk(XQ, YQ, q2, ch);
+        }
       }
-    }
-    __syncwarp();
-    __syncthreads();
-    if (*abort_flag) break;
-    if (!umma::mbar_wait(bar_o, ph_o)) { record_device_error(BASED_ERR_TIMEOUT); *abort_flag = 1; }
-    ph_o ^= 1;
-    umma::tc_fence_after();
-    if (tid == 0 && c + 1 < c_end && !*abort_flag) {
-      issue_v(c + 1);
-      tma_pending = true;
-    }
-    // ---- (e) outputs and the fp16 state copy for the next chunk --------------------
-    if (!kStateOnly) {
-      const int t = tid;
-      float o[NG * 32];
+      load_qk(c + 1);
+      umma::fence_async_smem();
+      umma::tc_fence_before();
+      umma::mbar_arrive(bar_phi);
+      if (kStateOnly) continue;
+      // ---- scores: P = mask(1 + u/4 + u^2/32) * sc ------------------------------------
+      if (!umma::mbar_wait(bar_u, it & 1)) { fail(); break; }
+      if (!Lay::kTm && it > 0 && !umma::mbar_wait(bar_o, (it - 1) & 1)) { fail(); break; }
+      umma::tc_fence_after();
+      const float sc = tc_chunk_scale((long long)t0 + kTcChunk);
+      const float c0 = sc, c1 = 0.25f * sc, c2 = 0.03125f * sc;
+      auto poly_pack = [&](const float* u, int c32, uint32_t* pk) {
+        const bool diag = c32 == quad;
 #pragma unroll
-      for (int g = 0; g < NG; ++g) umma::tmem_ld32(tmem + Lay::kTmO + tm_lane + g * 32, o + g * 32);
-      if (t < n) {
-        const float inv = 1.0f / (o[DV] + p.eps * sc);
-        uint4* dst = reinterpret_cast<uint4*>(out + (size_t)(t0 + t) * DV);
+        for (int e = 0; e < 16; ++e) {
+          float w0 = fmaf(u[2 * e], fmaf(u[2 * e], c2, c1), c0);
+          float w1 = fmaf(u[2 * e + 1], fmaf(u[2 * e + 1], c2, c1), c0);
+          if (diag) {
+            if (2 * e > lane) w0 = 0.0f;
+            if (2 * e + 1 > lane) w1 = 0.0f;
+          }
+          pk[e] = as_u32(__floats2bfloat162_rn(w0, w1));
+        }
+      };
+      if constexpr (Lay::kTm) {
+        // P (bf16 pairs) over the first 64 columns of U; this thread reads its
+        // whole U row before writing any of it
+        uint32_t pk[64];
+        float u[64];
+        umma::tmem_ld64(tmem + Lay::kTmU + tm_lane, u);
+        poly_pack(u, 0, pk);
+        if (quad >= 1) poly_pack(u + 32, 1, pk + 16);
+        else
 #pragma unroll
-        for (int ch = 0; ch < DV / 8; ++ch) {
+          for (int e = 0; e < 16; ++e) pk[16 + e] = 0u;
+        if (quad >= 2) {
+          umma::tmem_ld64(tmem + Lay::kTmU + tm_lane + 64, u);
+          poly_pack(u, 2, pk + 32);
+          if (quad >= 3) poly_pack(u + 32, 3, pk + 48);
+          else
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[48 + e] = 0u;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) pk[32 + e] = 0u;
+        }
+        umma::tmem_st32(tmem + Lay::kTmU + tm_lane, reinterpret_cast<const float*>(pk));
+        umma::tmem_st32(tmem + Lay::kTmU + tm_lane + 32, reinterpret_cast<const float*>(pk + 32));
+        umma::tc_fence_before();
+      } else {
+#pragma unroll
+        for (int c32 = 0; c32 < 4; ++c32) {
+          if (c32 > quad) {  // strictly above the diagonal: zeros (warp-uniform)
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+              *reinterpret_cast<uint4*>(sm + Lay::kP + ((t >> 3) * 16 + c32 * 4 + g) * 128 + (t & 7) * 16) =
+                  make_uint4(0, 0, 0, 0);
+            continue;
+          }
+          float u[32];
+          umma::tmem_ld32(tmem + Lay::kTmU + tm_lane + c32 * 32, u);
+          uint32_t pk[16];
+          poly_pack(u, c32, pk);
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            *reinterpret_cast<uint4*>(sm + Lay::kP + ((t >> 3) * 16 + c32 * 4 + g) * 128 + (t & 7) * 16) =
+                make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
+        }
+        umma::fence_async_smem();
+        umma::tc_fence_before();
+      }
+      umma::mbar_arrive(bar_p);
+    }
+  } else if (!kStateOnly) {
+    // ================= group E: epilogue of chunk c (output, fp16 state copy) =================
+    const int t = tid - kTcGroup;  // TMEM lane of this thread (quadrant = warp - 4)
+    __nv_bfloat16* out = p.out + (size_t)bh * L * DV;
+    // fp16 copy (scaled by sn) of the state rows this thread holds, as #2's B operand:
+    // tile 0 row t = feature t; tile 1 (M=64) lanes 0..15 of quadrants 0, 1 = features
+    // 128 + 16 * quad + lane
+    auto copy_state = [&](float sn) {
+      for (int tile = 0; tile < 2; ++tile) {
+        if (tile == 1 && (quad > 1)) break;
+        const int f = tile == 0 ? t : 128 + quad * 16 + lane;
+        const uint32_t base = tmem + (tile == 0 ? Lay::kTmS0 : Lay::kTmS1) + tm_lane;
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+          float sv[32];
+          umma::tmem_ld32(base + g * 32, sv);
+          if (tile == 1 && lane >= 16) continue;
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const int j0 = g * 32 + h * 8;
+            if (j0 < NA) {
+              uint32_t pk[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                pk[e] = as_u32(__floats2half2_rn(sv[h * 8 + 2 * e] * sn, sv[h * 8 + 2 * e + 1] * sn));
+              *reinterpret_cast<uint4*>(sm + Lay::kS + ((j0 >> 3) * 20 + (f >> 3)) * 128 + (f & 7) * 16) =
+                  make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+          }
+        }
+      }
+    };
+    if (has_init) {
+      // seed the TMEM state of a later segment with the sum of the earlier partials
+      const float* part = p.partial + (size_t)bh * (p.n_seg - 1) * kSymFP * NA;
+      for (int tile = 0; tile < 2; ++tile) {
+        if (tile == 1 && quad > 1) break;
+        const int f = tile == 0 ? t : 128 + quad * 16 + (lane & 15);
+        const uint32_t base = tmem + (tile == 0 ? Lay::kTmS0 : Lay::kTmS1) + tm_lane;
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+          float acc[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
+          if (tile == 0 || lane < 16) {
+            for (int sp = 0; sp < seg; ++sp) {
+              const float* row = part + ((size_t)sp * kSymFP + f) * NA + g * 32;
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (g * 32 + i < NA) acc[i] += row[i];
+            }
+          }
+          umma::tmem_st32(base + g * 32, acc);
+        }
+      }
+      copy_state(tc_chunk_scale((long long)c_begin * kTcChunk + kTcChunk));
+      umma::fence_async_smem();
+      umma::tc_fence_before();
+      umma::mbar_arrive(bar_ss);
+    }
+    for (int c = c_begin; c < c_end && !*abort_flag; ++c) {
+      const int it = c - c_begin;
+      const int t0 = c * kTcChunk;
+      const int n = min(kTcChunk, L - t0);
+      const float sc = tc_chunk_scale((long long)t0 + kTcChunk);
+      if (!umma::mbar_wait(bar_o, it & 1)) { fail(); break; }
+      umma::tc_fence_after();
+      const float den = umma::tmem_ld1(tmem + Lay::kTmO + tm_lane + DV);
+      const float inv = 1.0f / (den + p.eps * sc);
+      if constexpr (Lay::kTm) {
+        // y row t into the swizzled staging tile of this chunk; one TMA store per chunk
+        uint8_t* ybuf = sm + Lay::kY + (it & 1) * 16384;
+        if (t == 0) {  // the store of chunk c-2 has finished reading ybuf
+          umma::bulk_wait_read<1>();
+          umma::mbar_arrive(bar_yfree);
+        }
+        if (!umma::mbar_wait(bar_yfree, it & 1)) { fail(); break; }
+        float o[64];
+        umma::tmem_ld64(tmem + Lay::kTmO + tm_lane, o);
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
           uint32_t pk[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 b =
-                __floats2bfloat162_rn(o[ch * 8 + 2 * e] * inv, o[ch * 8 + 2 * e + 1] * inv);
-            pk[e] = *reinterpret_cast<const uint32_t*>(&b);
+          for (int e = 0; e < 4; ++e)
+            pk[e] = as_u32(__floats2bfloat162_rn(o[ch * 8 + 2 * e] * inv, o[ch * 8 + 2 * e + 1] * inv));
+          *reinterpret_cast<uint4*>(ybuf + t * 128 + ((ch ^ (t & 7)) << 4)) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+      } else {
+#pragma unroll
+        for (int g = 0; g < DV / 64; ++g) {
+          float o[64];
+          umma::tmem_ld64(tmem + Lay::kTmO + tm_lane + g * 64, o);
+          if (t < n) {
+            uint4* dst = reinterpret_cast<uint4*>(out + (size_t)(t0 + t) * DV + g * 64);
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+              uint32_t pk[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                pk[e] = as_u32(__floats2bfloat162_rn(o[ch * 8 + 2 * e] * inv, o[ch * 8 + 2 * e + 1] * inv));
+              dst[ch] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
           }
-          dst[ch] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
       }
       if (c + 1 < c_end) copy_state(tc_chunk_scale((long long)t0 + 2 * kTcChunk));
+      umma::fence_async_smem();
+      umma::tc_fence_before();
+      if (c + 1 < c_end) umma::mbar_arrive(bar_ss);
+      if constexpr (Lay::kTm) {
+        umma::mbar_arrive(bar_yfull);
+        if (t == 0) {
+          if (!umma::mbar_wait(bar_yfull, it & 1)) { fail(); break; }
+          umma::tma_store_3d(&ymap, sm + Lay::kY + (it & 1) * 16384, 0, t0, bh);
+          umma::bulk_commit();
+        }
+      }
     }
-    umma::fence_async_smem();
-    umma::tc_fence_before();
-    __syncthreads();
-    umma::tc_fence_after();
-    if (*abort_flag) break;
+    if (Lay::kTm && t == 0) umma::bulk_wait<0>();
   }
 
-  if (!*abort_flag) {
-    if (kStateOnly) {
-      // this segment's partial state, 160 symmetric rows x NA columns, fp32
-      float* part = p.partial + ((size_t)bh * (p.n_seg - 1) + seg) * kSymFP * NA;
-      for (int mt = 0; mt < n_tiles_here; ++mt) {
-        const int f = mt * 128 + warp * 32 + lane;
-#pragma unroll
-        for (int g = 0; g < NG; ++g) {
-          float s[32];
-          umma::tmem_ld32(tmem + Lay::kTmS + mt * Lay::kTileCols + tm_lane + g * 32, s);
-          float* row = part + (size_t)f * NA + g * 32;
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (g * 32 + i < NA) row[i] = c_begin < c_end ? s[i] : 0.0f;
-        }
-      }
-    } else if (seg == p.n_seg - 1 && (p.state_kv || p.state_k)) {
-      // final state export: 153 symmetric rows -> 273-row layout
-      float* skv = p.state_kv ? p.state_kv + (size_t)bh * kF * DV : nullptr;
-      float* sk = p.state_k ? p.state_k + (size_t)bh * kF : nullptr;
+  umma::tc_fence_before();
+  __syncthreads();
+  umma::tc_fence_after();
+  if (!*abort_flag && warp >= 4 && warp < 8) {
+    // ---- state out of TMEM (group E lanes): segment partials or the final export ----
+    const int t = tid - kTcGroup;
+    for (int tile = 0; tile < 2; ++tile) {
+      if (tile == 1 && quad > 1) break;
+      const int f = tile == 0 ? t : 128 + quad * 16 + (lane & 15);
+      const bool mine = tile == 0 || lane < 16;
+      const uint32_t base = tmem + (tile == 0 ? Lay::kTmS0 : Lay::kTmS1) + tm_lane;
       const bool any = has_init || c_begin < c_end;
-      for (int mt = 0; mt < n_tiles_here; ++mt) {
-        const int f = mt * 128 + warp * 32 + lane;
-        float s[NG * 32];
+      int r0 = -1, r1 = -1;
+      float scale = 1.0f;
+      const int nrows = (mine && f < kSymFP && !kStateOnly) ? tc_feature_rows(f, &r0, &r1, &scale) : 0;
 #pragma unroll
-        for (int g = 0; g < NG; ++g)
-          umma::tmem_ld32(tmem + Lay::kTmS + mt * Lay::kTileCols + tm_lane + g * 32, s + g * 32);
+      for (int g = 0; g < NG; ++g) {
+        float s[32];
+        umma::tmem_ld32(base + g * 32, s);
         if (!any) {
 #pragma unroll
-          for (int i = 0; i < NG * 32; ++i) s[i] = 0.0f;
+          for (int i = 0; i < 32; ++i) s[i] = 0.0f;
         }
-        if (f >= kSymF) continue;
-        int r0, r1 = -1;
-        float scale = 1.0f;
-        if (f <= 16) {
-          r0 = f;
-        } else {
-          const int i = sym_pair_i(f - 17), j = sym_pair_j(f - 17);
-          r0 = 17 + 16 * i + j;
-          if (i != j) { r1 = 17 + 16 * j + i; scale = 0.70710678118654752f; }
-        }
-        for (int r = 0; r < 2; ++r) {
-          const int row = r == 0 ? r0 : r1;
-          if (row < 0) continue;
-          if (skv) {
-            float4* dst = reinterpret_cast<float4*>(skv + (size_t)row * DV);
+        if (!mine) continue;
+        if (kStateOnly) {
+          float* row = p.partial + (((size_t)bh * (p.n_seg - 1) + seg) * kSymFP + f) * NA + g * 32;
 #pragma unroll
-            for (int j = 0; j < DV / 4; ++j)
-              dst[j] = make_float4(s[4 * j] * scale, s[4 * j + 1] * scale, s[4 * j + 2] * scale,
-                                   s[4 * j + 3] * scale);
+          for (int i = 0; i < 32; ++i)
+            if (g * 32 + i < NA) row[i] = s[i];
+        } else if (seg == p.n_seg - 1) {
+          float* skv = p.state_kv ? p.state_kv + (size_t)bh * kF * DV : nullptr;
+          float* sk = p.state_k ? p.state_k + (size_t)bh * kF : nullptr;
+          for (int r = 0; r < nrows; ++r) {
+            const int row = r == 0 ? r0 : r1;
+            if (skv) {
+#pragma unroll
+              for (int i4 = 0; i4 < 8; ++i4) {
+                const int j = g * 32 + 4 * i4;
+                if (j < DV)
+                  *reinterpret_cast<float4*>(skv + (size_t)row * DV + j) =
+                      make_float4(s[4 * i4] * scale, s[4 * i4 + 1] * scale,
+                                  s[4 * i4 + 2] * scale, s[4 * i4 + 3] * scale);
+              }
+            }
+            if (sk && DV / 32 == g) sk[row] = s[0] * scale;
           }
-          if (sk) sk[row] = s[DV] * scale;
         }
       }
     }
   }
-  // an aborted run may still have a V load in flight: wait for it (bounded)
-  if (tid == 0 && tma_pending && *abort_flag) umma::mbar_wait(bar_tma, ph_tma);
   umma::tc_fence_before();
   __syncthreads();
   if (warp == 0) umma::tmem_dealloc(tmem, kTcTmemCols);
