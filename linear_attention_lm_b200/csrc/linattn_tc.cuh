@@ -88,9 +88,11 @@ struct TcLayout {
   static constexpr int kPhiK = kV + kVBuf * kVStage;       // phiK [160 x 128] bf16, MN-major
   static constexpr int kP = kPhiK + kPhiKBuf * 40960;      // P [128 x 128] bf16 (smem path)
   static constexpr int kPhiQ = kP + (kTm ? 0 : 32768);     // phiQ [128 x 160] fp16 (smem path)
-  static constexpr int kS = kPhiQ + (kTm ? 0 : 40960);     // [S|z] copy [160 x NA] fp16, MN-major
-  static constexpr int kY = kS + NA * kSymFP * 2;          // y staging, 2 x [128 x 64] bf16 SW128
-  static constexpr int kBar = kY + (kTm ? 2 * 16384 : 0);  // mbarriers + TMEM address
+  static constexpr int kSBuf = kTm ? 2 : 1;                // fp16 state copies
+  static constexpr int kSBytes = NA * kSymFP * 2;
+  static constexpr int kS = kPhiQ + (kTm ? 0 : 40960);     // [S|z] copies [160 x NA] fp16, MN-major
+  static constexpr int kY = kS + kSBuf * kSBytes;          // y staging [128 x 64] bf16 SW128
+  static constexpr int kBar = kY + (kTm ? 16384 : 0);      // mbarriers + TMEM address
   static constexpr int kBytes = kBar + 128;
   static constexpr size_t kSmem = kBytes + 1024;           // + alignment slack
   // TMEM: state tile 0 (features 0..127, M=128), state tile 1 (features
@@ -240,6 +242,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 9);
   uint64_t* bar_yfree = bars + 10;   // y staging tile free again (TMA store read it)
   uint64_t* bar_yfull = bars + 11;   // y staging tile written (group E)
+  uint64_t* bar_m5 = bars + 12;      // #5 done (commit): the state can be read
+  uint64_t* bar_sread = bars + 13;   // state read and its fp16 copy written (group E)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quad = warp & 3;
@@ -263,6 +267,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     umma::mbar_init(bar_ss, kTcGroup);
     umma::mbar_init(bar_yfree, 1);
     umma::mbar_init(bar_yfull, kTcGroup);
+    umma::mbar_init(bar_m5, 1);
+    umma::mbar_init(bar_sread, kTcGroup);
     *abort_flag = 0;
     umma::fence_mbar_init();
     umma::tma_prefetch_desc(&vmap);
@@ -308,6 +314,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           umma::tma_load_3d(sm + Lay::kV + stage * Lay::kVStage + blk * 16384, &vmap,
                             bar_tma + stage, blk * 64, c * kTcChunk, bh);
       };
+      // descriptors are computed once per buffer and stepped along K by adding
+      // the start-address increment (16-byte units) to their low word
+      const uint64_t d_q = umma::desc_kmajor_none(sQ, 0, 16), d_k = umma::desc_kmajor_none(sK, 0, 16);
+      const uint64_t d_s0 = umma::desc_mnmajor_none(sS, 0, kSymFP);
+      const uint64_t d_s1 = umma::desc_mnmajor_none(sS + (Lay::kSBuf - 1) * Lay::kSBytes, 0, kSymFP);
+      const uint64_t d_p = umma::desc_kmajor_none(sP, 0, kTcChunk);
+      const uint64_t d_phiq = umma::desc_kmajor_none(sPhiQ, 0, kSymFP);
       const uint32_t id_u = umma::idesc_bf16(128, 128, false, false);
       const uint32_t id_o2 = umma::idesc_f16(128, NA, false, true);
       const uint32_t id_o4 = umma::idesc_bf16(128, NA, false, true);
@@ -323,10 +336,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int it = c - c_begin;
         const uint32_t ph = it & 1;
         const int stage = Lay::kVBuf == 2 ? (it & 1) : 0;
-        const uint32_t sV = umma::smem_u32(sm + Lay::kV + stage * Lay::kVStage);
+        const uint64_t d_v =
+            umma::desc_mnmajor_sw128(umma::smem_u32(sm + Lay::kV + stage * Lay::kVStage), 0, kTcChunk);
         const uint32_t sPhiK = umma::smem_u32(sm + Lay::kPhiK + (it % Lay::kPhiKBuf) * 40960);
+        const uint64_t d_k0 = umma::desc_mnmajor_none(sPhiK, 0, kTcChunk);
+        const uint64_t d_k1 = umma::desc_mnmajor_none(sPhiK + 16 * 2048, 0, kTcChunk);
         const bool has_state = has_init || it > 0;
-        const uint32_t ph_ss = (it + (has_init ? 0 : 1)) & 1;  // epilogue hand-off of chunk c-1
+        // index of the epilogue hand-off (state copy) of chunk c-1
+        const int kk = has_init ? it : it - 1;
+        const uint32_t ph_ss = kk & 1;
+        const uint64_t d_s = (kk & 1) ? d_s1 : d_s0;
         if (!umma::mbar_wait(bar_phi, ph)) { fail(); break; }
         // when O shares TMEM with U, #1 may only overwrite it once the epilogue
         // group has read the previous chunk's O
@@ -335,27 +354,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         umma::tc_fence_after();
         if (!kStateOnly) {
-          umma::mma_bf16(tmem + Lay::kTmU, umma::desc_kmajor_none(sQ, 0, 16),
-                         umma::desc_kmajor_none(sK, 0, 16), id_u, 0);
+          umma::mma_bf16(tmem + Lay::kTmU, d_q, d_k, id_u, 0);
           umma::mma_commit(bar_u);
         }
         if (!umma::mbar_wait(bar_tma + stage, vphase[stage])) { fail(); break; }
         inflight[stage] = false;
         vphase[stage] ^= 1;
-        // the state copy of the previous chunk must have been read out of TMEM
-        // (and, for #2, written to shared memory) by the epilogue group
+        // #5 overwrites the state: the epilogue group must have read (and copied)
+        // the previous chunk's state out of TMEM
         if (!kStateOnly && Lay::kEarlyO && has_state) {
-          if (!umma::mbar_wait(bar_ss, ph_ss)) { fail(); break; }
+          if (!umma::mbar_wait(Lay::kTm ? bar_sread : bar_ss, ph_ss)) { fail(); break; }
         }
         umma::tc_fence_after();
+        // K step of 16 tokens: +256 B in the no-swizzle phiK layout (2 core
+        // matrices), +2048 B (16 rows of 128 B) in the swizzled V tile
 #pragma unroll
-        for (int k0 = 0; k0 < kTcChunk; k0 += 16) {
-          const uint64_t bdesc = umma::desc_mnmajor_sw128(sV, k0, kTcChunk);
-          umma::mma_bf16(tmem + Lay::kTmS0, umma::desc_mnmajor_none(sPhiK, k0, kTcChunk), bdesc,
-                         id_s0, has_state || (k0 > 0));
-          umma::mma_bf16(tmem + Lay::kTmS1,
-                         umma::desc_mnmajor_none(sPhiK + 16 * 2048, k0, kTcChunk), bdesc, id_s1,
-                         has_state || (k0 > 0));
+        for (int ks = 0; ks < kTcChunk / 16; ++ks) {
+          const uint32_t acc = has_state || ks > 0;
+          umma::mma_bf16(tmem + Lay::kTmS0, d_k0 + ks * 16, d_v + ks * 128, id_s0, acc);
+          umma::mma_bf16(tmem + Lay::kTmS1, d_k1 + ks * 16, d_v + ks * 128, id_s1, acc);
+        }
+        if (Lay::kTm) {
+          umma::mma_commit(bar_m5);
+          // refill the stage of chunk c-1 (its MMAs are done by now) with chunk c+1
+          if (Lay::kVBuf == 2 && it > 0 && c + 1 < c_end) {
+            if (!umma::mbar_wait(bar_o, (it - 1) & 1)) { fail(); break; }
+            issue_v(c + 1, (it - 1) & 1);
+            inflight[(it - 1) & 1] = true;
+          }
         }
         if (!kStateOnly) {
           if (!Lay::kEarlyO) {  // O shares TMEM with U: wait until P has been read out
@@ -363,14 +389,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             umma::tc_fence_after();
           }
           if (has_state) {
+            // #2 overwrites O: the epilogue group must have read the previous O
+            if (Lay::kTm) {
+              if (!umma::mbar_wait(bar_ss, ph_ss)) { fail(); break; }
+              umma::tc_fence_after();
+            }
+            // K step of 16 features: +256 B in both no-swizzle layouts, 8 TMEM columns
 #pragma unroll
-            for (int k0 = 0; k0 < kSymFP; k0 += 16) {
+            for (int ks = 0; ks < kSymFP / 16; ++ks) {
               if constexpr (Lay::kTm)
-                umma::mma_ts(tmem + Lay::kTmO, tmem + Lay::kTmQ + k0 / 2,
-                             umma::desc_mnmajor_none(sS, k0, kSymFP), id_o2, k0 > 0);
+                umma::mma_ts(tmem + Lay::kTmO, tmem + Lay::kTmQ + ks * 8, d_s + ks * 16, id_o2,
+                             ks > 0);
               else
-                umma::mma_f16(tmem + Lay::kTmO, umma::desc_kmajor_none(sPhiQ, k0, kSymFP),
-                              umma::desc_mnmajor_none(sS, k0, kSymFP), id_o2, k0 > 0);
+                umma::mma_f16(tmem + Lay::kTmO, d_phiq + ks * 16, d_s + ks * 16, id_o2, ks > 0);
             }
           }
         }
@@ -381,22 +412,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             umma::tc_fence_after();
           }
 #pragma unroll
-          for (int k0 = 0; k0 < kTcChunk; k0 += 16) {
+          for (int ks = 0; ks < kTcChunk / 16; ++ks) {
+            const uint32_t acc = has_state || ks > 0;
             if constexpr (Lay::kTm)
-              umma::mma_ts(tmem + Lay::kTmO, tmem + Lay::kTmU + k0 / 2,
-                           umma::desc_mnmajor_sw128(sV, k0, kTcChunk), id_o4,
-                           has_state || (k0 > 0));
+              umma::mma_ts(tmem + Lay::kTmO, tmem + Lay::kTmU + ks * 8, d_v + ks * 128, id_o4, acc);
             else
-              umma::mma_bf16(tmem + Lay::kTmO, umma::desc_kmajor_none(sP, k0, kTcChunk),
-                             umma::desc_mnmajor_sw128(sV, k0, kTcChunk), id_o4,
-                             has_state || (k0 > 0));
+              umma::mma_bf16(tmem + Lay::kTmO, d_p + ks * 16, d_v + ks * 128, id_o4, acc);
           }
         }
         umma::mma_commit(bar_o);
         ++n_done;
         // refill the stage this chunk used once its MMAs are done
         const int c_next = c + Lay::kVBuf;
-        if (c_next < c_end) {
+        if (!Lay::kTm && c_next < c_end) {
           if (!umma::mbar_wait(bar_o, ph)) { fail(); break; }
           issue_v(c_next, stage);
           inflight[stage] = true;
@@ -482,11 +510,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const uint4 v = tc_feature_chunk(XQ, YQ, q2, ch);
             const int s4 = (ch * 4) & 31;
             buf[s4] = v.x; buf[s4 + 1] = v.y; buf[s4 + 2] = v.z; buf[s4 + 3] = v.w;
-            if (ch == 7 || ch == 15)
-              umma::tmem_st32(tmem + Lay::kTmQ + tm_lane + (ch - 7) * 4,
-                              reinterpret_cast<const float*>(buf));
-            if (ch == 19) umma::tmem_st16(tmem + Lay::kTmQ + tm_lane + 64, buf);
+            if (ch == 7 || ch == 15) umma::tmem_st32_nowait(tmem + Lay::kTmQ + tm_lane + (ch - 7) * 4, buf);
+            if (ch == 19) umma::tmem_st16_nowait(tmem + Lay::kTmQ + tm_lane + 64, buf);
           }
+          umma::tmem_wait_st();
         } else {
 #pragma unroll
           for (int ch = 0; ch < 20; ++ch)
@@ -540,8 +567,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) pk[32 + e] = 0u;
         }
-        umma::tmem_st32(tmem + Lay::kTmU + tm_lane, reinterpret_cast<const float*>(pk));
-        umma::tmem_st32(tmem + Lay::kTmU + tm_lane + 32, reinterpret_cast<const float*>(pk + 32));
+        umma::tmem_st32_nowait(tmem + Lay::kTmU + tm_lane, pk);
+        umma::tmem_st32_nowait(tmem + Lay::kTmU + tm_lane + 32, pk + 32);
+        umma::tmem_wait_st();
         umma::tc_fence_before();
       } else {
 #pragma unroll
@@ -574,27 +602,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // fp16 copy (scaled by sn) of the state rows this thread holds, as #2's B operand:
     // tile 0 row t = feature t; tile 1 (M=64) lanes 0..15 of quadrants 0, 1 = features
     // 128 + 16 * quad + lane
+    int kk = 0;  // number of state copies handed off so far (buffer kk % kSBuf)
     auto copy_state = [&](float sn) {
+      uint8_t* sbuf = sm + Lay::kS + (kk % Lay::kSBuf) * Lay::kSBytes;
       for (int tile = 0; tile < 2; ++tile) {
         if (tile == 1 && (quad > 1)) break;
         const int f = tile == 0 ? t : 128 + quad * 16 + lane;
         const uint32_t base = tmem + (tile == 0 ? Lay::kTmS0 : Lay::kTmS1) + tm_lane;
+        auto put = [&](const float* sv, int j0) {
+          uint32_t pk[4];
 #pragma unroll
-        for (int g = 0; g < NG; ++g) {
-          float sv[32];
-          umma::tmem_ld32(base + g * 32, sv);
+          for (int e = 0; e < 4; ++e)
+            pk[e] = as_u32(__floats2half2_rn(sv[2 * e] * sn, sv[2 * e + 1] * sn));
+          *reinterpret_cast<uint4*>(sbuf + ((j0 >> 3) * 20 + (f >> 3)) * 128 + (f & 7) * 16) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        };
+        if constexpr (NG == 3) {
+          float sv[96];  // the whole tile row in one TMEM round trip
+          umma::tmem_ld64_32(base, base + 64, sv);
           if (tile == 1 && lane >= 16) continue;
 #pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const int j0 = g * 32 + h * 8;
-            if (j0 < NA) {
-              uint32_t pk[4];
+          for (int j0 = 0; j0 < NA; j0 += 8) put(sv + j0, j0);
+        } else {
 #pragma unroll
-              for (int e = 0; e < 4; ++e)
-                pk[e] = as_u32(__floats2half2_rn(sv[h * 8 + 2 * e] * sn, sv[h * 8 + 2 * e + 1] * sn));
-              *reinterpret_cast<uint4*>(sm + Lay::kS + ((j0 >> 3) * 20 + (f >> 3)) * 128 + (f & 7) * 16) =
-                  make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            }
+          for (int g = 0; g < NG; ++g) {
+            float sv[32];
+            umma::tmem_ld32(base + g * 32, sv);
+            if (tile == 1 && lane >= 16) continue;
+#pragma unroll
+            for (int h = 0; h < 4; ++h)
+              if (g * 32 + h * 8 < NA) put(sv + h * 8, g * 32 + h * 8);
           }
         }
       }
@@ -625,27 +662,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       copy_state(tc_chunk_scale((long long)c_begin * kTcChunk + kTcChunk));
       umma::fence_async_smem();
       umma::tc_fence_before();
+      if (Lay::kTm) umma::mbar_arrive(bar_sread);
       umma::mbar_arrive(bar_ss);
+      ++kk;
     }
     for (int c = c_begin; c < c_end && !*abort_flag; ++c) {
       const int it = c - c_begin;
       const int t0 = c * kTcChunk;
       const int n = min(kTcChunk, L - t0);
       const float sc = tc_chunk_scale((long long)t0 + kTcChunk);
+      if (Lay::kTm && c + 1 < c_end) {
+        // the state after #5 of this chunk, copied while #2 and #4 still run
+        if (!umma::mbar_wait(bar_m5, it & 1)) { fail(); break; }
+        umma::tc_fence_after();
+        copy_state(tc_chunk_scale((long long)t0 + 2 * kTcChunk));
+        umma::fence_async_smem();
+        umma::tc_fence_before();
+        umma::mbar_arrive(bar_sread);
+      }
       if (!umma::mbar_wait(bar_o, it & 1)) { fail(); break; }
       umma::tc_fence_after();
-      const float den = umma::tmem_ld1(tmem + Lay::kTmO + tm_lane + DV);
-      const float inv = 1.0f / (den + p.eps * sc);
       if constexpr (Lay::kTm) {
-        // y row t into the swizzled staging tile of this chunk; one TMA store per chunk
-        uint8_t* ybuf = sm + Lay::kY + (it & 1) * 16384;
-        if (t == 0) {  // the store of chunk c-2 has finished reading ybuf
-          umma::bulk_wait_read<1>();
+        // y row t into the swizzled staging tile; one TMA store per chunk
+        uint8_t* ybuf = sm + Lay::kY;
+        if (t == 0) {  // the store of chunk c-1 has finished reading ybuf
+          umma::bulk_wait_read<0>();
           umma::mbar_arrive(bar_yfree);
         }
         if (!umma::mbar_wait(bar_yfree, it & 1)) { fail(); break; }
-        float o[64];
-        umma::tmem_ld64(tmem + Lay::kTmO + tm_lane, o);
+        float o[64], den;
+        umma::tmem_ld64_1(tmem + Lay::kTmO + tm_lane, tmem + Lay::kTmO + tm_lane + DV, o, &den);
+        const float inv = 1.0f / (den + p.eps * sc);
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
           uint32_t pk[4];
@@ -656,6 +703,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
       } else {
+        const float den = umma::tmem_ld1(tmem + Lay::kTmO + tm_lane + DV);
+        const float inv = 1.0f / (den + p.eps * sc);
 #pragma unroll
         for (int g = 0; g < DV / 64; ++g) {
           float o[64];
@@ -673,15 +722,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
       }
-      if (c + 1 < c_end) copy_state(tc_chunk_scale((long long)t0 + 2 * kTcChunk));
+      if (!Lay::kTm && c + 1 < c_end) copy_state(tc_chunk_scale((long long)t0 + 2 * kTcChunk));
       umma::fence_async_smem();
       umma::tc_fence_before();
-      if (c + 1 < c_end) umma::mbar_arrive(bar_ss);
+      if (c + 1 < c_end) {  // O (and, without a second copy buffer, the state) read
+        umma::mbar_arrive(bar_ss);
+        ++kk;
+      }
       if constexpr (Lay::kTm) {
         umma::mbar_arrive(bar_yfull);
         if (t == 0) {
           if (!umma::mbar_wait(bar_yfull, it & 1)) { fail(); break; }
-          umma::tma_store_3d(&ymap, sm + Lay::kY + (it & 1) * 16384, 0, t0, bh);
+          umma::tma_store_3d(&ymap, sm + Lay::kY, 0, t0, bh);
           umma::bulk_commit();
         }
       }
