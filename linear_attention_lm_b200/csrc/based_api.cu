@@ -230,16 +230,25 @@ based_status_t launch_window_simt(const void* q, const void* k, const void* v, v
 }
 
 template <typename T, int DV>
-based_status_t launch_decode(const DecodeParams& p, cudaStream_t st) {
+based_status_t launch_decode(DecodeParams p, cudaStream_t st) {
   auto kern = decode_step_kernel<T, DV>;
+  constexpr int kThreads = 4 * DV;
   size_t smem = sizeof(float) * (size_t)DecodeLinearLayout<DV>::kSmemFloats;
+  p.wg = 1;
+  p.n_wblk = 0;
   if (p.n_win > 0) {
-    const size_t w = sizeof(float) * (size_t)decode_window_smem_floats(p.dh, p.W);
+    // up to 4 heads per window CTA, within 64 KiB of ring buffers
+    const int ring_pair = 2 * p.W * p.dh * (int)sizeof(T);
+    p.wg = 65536 / ring_pair;
+    p.wg = p.wg < 1 ? 1 : (p.wg > 4 ? 4 : p.wg);
+    p.n_wblk = (p.n_win + p.wg - 1) / p.wg;
+    const size_t w = (size_t)DecodeWindowLayout(p.wg, p.dh, p.W, kThreads, sizeof(T)).bytes;
     if (w > smem) smem = w;
   }
   if (!set_smem(kern, smem)) return BASED_ERR_CUDA;
-  const long long nblk = (long long)p.n_lin + p.n_win;
-  kern<<<(unsigned)nblk, 4 * DV, smem, st>>>(p);
+  const long long nblk = (long long)p.n_lin + p.n_wblk;
+  p.wstride = p.n_wblk > 0 ? (int)(nblk / p.n_wblk) : 1;
+  kern<<<(unsigned)nblk, kThreads, smem, st>>>(p);
   return launch_status();
 }
 

@@ -12,10 +12,15 @@
 //
 // Window part (Based README, introduction, item 1: short sliding-window softmax
 // attention): the new k/v go to ring slot pos mod W, then softmax over the slots
-// holding positions max(0, pos-W+1)..pos.
+// holding positions max(0, pos-W+1)..pos.  A window CTA serves up to G heads:
+// it issues one bulk copy per ring (the valid rows of one (b, h) ring are
+// contiguous) for all its heads at once, so the ring reads overlap each other
+// and the linear CTAs' state streaming; window CTAs are spread evenly through
+// the grid among the linear ones.
 #pragma once
 
 #include "common.cuh"
+#include "umma.cuh"
 
 namespace based {
 
@@ -26,8 +31,11 @@ struct DecodeParams {
   const void *wq, *wk, *wv;
   void *k_ring, *v_ring, *wout;
   long long pos;
-  int n_lin;  // B * H   (CTAs of the linear part)
-  int n_win;  // B * H_w (CTAs of the window part)
+  int n_lin;   // B * H   (one CTA each)
+  int n_win;   // B * H_w window heads
+  int n_wblk;  // window CTAs, each serving up to wg heads
+  int wg;
+  int wstride;  // (n_lin + n_wblk) / n_wblk: spacing of the window CTAs
   int dh, W;
   float eps;
 };
@@ -132,75 +140,154 @@ __device__ __forceinline__ void decode_linear_block(const DecodeParams& p, int b
   }
 }
 
-__host__ __device__ constexpr int decode_window_smem_floats(int dh, int W) {
-  return 128 + 2 * W * dh + 64 + 32;
+// Shared-memory layout of a window CTA (bytes), for G heads of d_h = dh and
+// element size es: the K and V rings of each head (W rows), one mbarrier per
+// head, then q and the new k/v of each head, scores, partial outputs.
+struct DecodeWindowLayout {
+  int ring, bar, qs, kvn, pr, part, red, bytes;
+  __host__ __device__ DecodeWindowLayout(int G, int dh, int W, int NT, int es) {
+    ring = W * dh * es;  // one ring; multiple of 16 for dh in {64, 128}
+    bar = 2 * G * ring;
+    qs = bar + 8 * G + 16;
+    kvn = qs + 4 * G * dh;
+    pr = kvn + ((2 * G * dh * es + 15) & ~15);
+    part = pr + 4 * 64;
+    red = part + 4 * NT;
+    bytes = red + 16;
+  }
+};
+
+// 16 bytes of T at p (16-byte aligned) as floats
+template <typename T>
+__device__ __forceinline__ void load16_f32(const T* p, float* f);
+template <>
+__device__ __forceinline__ void load16_f32<float>(const float* p, float* f) {
+  const float4 v = *reinterpret_cast<const float4*>(p);
+  f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+}
+template <>
+__device__ __forceinline__ void load16_f32<__nv_bfloat16>(const __nv_bfloat16* p, float* f) {
+  const uint4 v = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
 }
 
 template <typename T>
-__device__ __forceinline__ void decode_window_block(const DecodeParams& p, int bhw, float* smem) {
-  const int dh = p.dh, W = p.W, NT = blockDim.x;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = NT >> 5;
-  float* qs = smem;              // [dh]
-  float* kr = qs + 128;          // [W][dh]
-  float* vr = kr + W * dh;       // [W][dh]
-  float* pr = vr + W * dh;       // [W] scores, then weights
-  float* red = pr + 64;          // [2] max, sum
-  T* kring = static_cast<T*>(p.k_ring) + (size_t)bhw * W * dh;
-  T* vring = static_cast<T*>(p.v_ring) + (size_t)bhw * W * dh;
-  const T* q = static_cast<const T*>(p.wq) + (size_t)bhw * dh;
-  const T* kn = static_cast<const T*>(p.wk) + (size_t)bhw * dh;
-  const T* vn = static_cast<const T*>(p.wv) + (size_t)bhw * dh;
+__device__ __forceinline__ void decode_window_block(const DecodeParams& p, int wblk, uint8_t* sm) {
+  constexpr int VEC = 16 / sizeof(T);
+  const int dh = p.dh, W = p.W, NT = blockDim.x, G = p.wg;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int w0 = wblk * G;
+  const int n_items = min(G, p.n_win - w0);
+  const DecodeWindowLayout lay(G, dh, W, NT, sizeof(T));
+  T* rings = reinterpret_cast<T*>(sm);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + lay.bar);
+  float* qs = reinterpret_cast<float*>(sm + lay.qs);
+  T* kvn = reinterpret_cast<T*>(sm + lay.kvn);
+  float* pr = reinterpret_cast<float*>(sm + lay.pr);
+  float* part = reinterpret_cast<float*>(sm + lay.part);
+  float* red = reinterpret_cast<float*>(sm + lay.red);
   const long long pos = p.pos;
   const int slot = (int)(pos % W);
   const int nvalid = pos + 1 < W ? (int)(pos + 1) : W;  // valid slots are 0..nvalid-1
+  const uint32_t load_bytes = (uint32_t)(nvalid * dh * sizeof(T));
+  T* kring = static_cast<T*>(p.k_ring);
+  T* vring = static_cast<T*>(p.v_ring);
 
-  for (int i = tid; i < nvalid * dh; i += NT) {
-    kr[i] = to_f32(kring[i]);
-    vr[i] = to_f32(vring[i]);
+  if (tid == 0) {
+    for (int g = 0; g < n_items; ++g) umma::mbar_init(bar + g, 1);
+    umma::fence_mbar_init();
+    for (int g = 0; g < n_items; ++g) {
+      const size_t ro = (size_t)(w0 + g) * W * dh;
+      T* dst = rings + (size_t)g * 2 * W * dh;
+      umma::mbar_arrive_expect_tx(bar + g, 2 * load_bytes);
+      umma::bulk_load(dst, kring + ro, load_bytes, bar + g);
+      umma::bulk_load(dst + W * dh, vring + ro, load_bytes, bar + g);
+    }
   }
-  if (tid < dh) qs[tid] = to_f32(q[tid]);
-  __syncthreads();
-  if (tid < dh) {
-    const T kt = kn[tid], vt = vn[tid];
-    kring[(size_t)slot * dh + tid] = kt;
-    vring[(size_t)slot * dh + tid] = vt;
-    kr[slot * dh + tid] = to_f32(kt);
-    vr[slot * dh + tid] = to_f32(vt);
+  for (int i = tid; i < n_items * dh; i += NT) {
+    const size_t gi = (size_t)w0 * dh + i;
+    qs[i] = to_f32(static_cast<const T*>(p.wq)[gi]);
+    kvn[2 * i] = static_cast<const T*>(p.wk)[gi];
+    kvn[2 * i + 1] = static_cast<const T*>(p.wv)[gi];
   }
   __syncthreads();
+
   const float scale = rsqrtf((float)dh);
-  for (int s = warp; s < nvalid; s += nwarps) {
+  const int tps = NT / 64, s_me = tid / tps, u = tid % tps, dpt = dh / tps;
+  const int ng = NT / dh, c_me = tid % dh, grp = tid / dh;
+  int g = 0;
+  for (; g < n_items; ++g) {
+    const bool ok = umma::mbar_wait(bar + g, 0);
+    if (!ok) record_device_error(BASED_ERR_TIMEOUT);
+    if (__syncthreads_or(!ok)) break;
+    T* K = rings + (size_t)g * 2 * W * dh;
+    T* V = K + W * dh;
+    if (tid < dh) {
+      const T kt = kvn[2 * (g * dh + tid)], vt = kvn[2 * (g * dh + tid) + 1];
+      const size_t ro = (size_t)(w0 + g) * W * dh + (size_t)slot * dh + tid;
+      K[slot * dh + tid] = kt;
+      V[slot * dh + tid] = vt;
+      kring[ro] = kt;
+      vring[ro] = vt;
+    }
+    __syncthreads();
+    // scores: tps consecutive threads share slot s_me, dpt dims each
     float a = 0.0f;
-    for (int j = lane; j < dh; j += 32) a = fmaf(qs[j], kr[s * dh + j], a);
-    a = warp_sum(a);
-    if (lane == 0) pr[s] = a * scale;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    const float a0 = lane < nvalid ? pr[lane] : -INFINITY;
-    const float a1 = lane + 32 < nvalid ? pr[lane + 32] : -INFINITY;
-    const float m = warp_max(fmaxf(a0, a1));
-    const float e0 = lane < nvalid ? expf(a0 - m) : 0.0f;
-    const float e1 = lane + 32 < nvalid ? expf(a1 - m) : 0.0f;
-    if (lane < nvalid) pr[lane] = e0;
-    if (lane + 32 < nvalid) pr[lane + 32] = e1;
-    const float sum = warp_sum(e0 + e1);
-    if (lane == 0) red[0] = sum;
-  }
-  __syncthreads();
-  if (tid < dh) {
+    if (s_me < nvalid) {
+      const T* kr = K + s_me * dh + u * dpt;
+      const float* qg = qs + g * dh + u * dpt;
+      for (int e = 0; e < dpt; e += VEC) {
+        float kf[VEC];
+        load16_f32<T>(kr + e, kf);
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) a = fmaf(qg[e + i], kf[i], a);
+      }
+    }
+    for (int o = tps >> 1; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    if (u == 0) pr[s_me] = a * scale;
+    __syncthreads();
+    if (warp == 0) {
+      const float a0 = lane < nvalid ? pr[lane] : -INFINITY;
+      const float a1 = lane + 32 < nvalid ? pr[lane + 32] : -INFINITY;
+      const float m = warp_max(fmaxf(a0, a1));
+      const float e0 = lane < nvalid ? expf(a0 - m) : 0.0f;
+      const float e1 = lane + 32 < nvalid ? expf(a1 - m) : 0.0f;
+      pr[lane] = e0;
+      pr[lane + 32] = e1;
+      const float sum = warp_sum(e0 + e1);
+      if (lane == 0) red[0] = sum;
+    }
+    __syncthreads();
+    // output column c_me over the slots of group grp
     float acc = 0.0f;
-    for (int s = 0; s < nvalid; ++s) acc = fmaf(pr[s], vr[s * dh + tid], acc);
-    static_cast<T*>(p.wout)[(size_t)bhw * dh + tid] = from_f32<T>(acc / red[0]);
+    for (int s = grp; s < nvalid; s += ng) acc = fmaf(pr[s], to_f32(V[s * dh + c_me]), acc);
+    part[tid] = acc;
+    __syncthreads();
+    if (tid < dh) {
+      float y = 0.0f;
+      for (int j = 0; j < ng; ++j) y += part[j * dh + tid];
+      static_cast<T*>(p.wout)[(size_t)(w0 + g) * dh + tid] = from_f32<T>(y / red[0]);
+    }
   }
+  // after an abort, loads of the heads not reached may still be in flight
+  if (tid == 0)
+    for (int i = g + 1; i < n_items; ++i) umma::mbar_wait(bar + i, 0);
 }
 
 template <typename T, int DV>
-__global__ void __launch_bounds__(4 * DV) decode_step_kernel(const DecodeParams p) {
-  extern __shared__ __align__(16) float smem[];
-  const int b = blockIdx.x;
-  if (b < p.n_lin) decode_linear_block<T, DV>(p, b, smem);
-  else decode_window_block<T>(p, b - p.n_lin, smem);
+__global__ void __launch_bounds__(4 * DV, 1) decode_step_kernel(const DecodeParams p) {
+  extern __shared__ __align__(16) uint8_t dec_smem[];
+  // window CTAs are interleaved evenly: with stride = n / n_wblk, CTA b is a
+  // window CTA iff b mod stride = stride - 1 and b / stride < n_wblk
+  const int b = blockIdx.x, q = b / p.wstride, r = b - q * p.wstride;
+  if (q < p.n_wblk && r == p.wstride - 1) decode_window_block<T>(p, q, dec_smem);
+  else decode_linear_block<T, DV>(p, b - min(q, p.n_wblk), reinterpret_cast<float*>(dec_smem));
 }
 
 }  // namespace based
