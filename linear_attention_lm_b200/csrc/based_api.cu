@@ -200,9 +200,9 @@ based_status_t launch_linattn_tc(const void* q, const void* k, const void* v, vo
 template <int DH>
 based_status_t launch_window_tc(const void* q, const void* k, const void* v, void* out, int BH,
                                 int L, int W, cudaStream_t st) {
-  CUtensorMap qm, km, vm;
+  CUtensorMap qm, km, vm, ym;
   if (!make_rows_map(&qm, q, DH, L, BH, kWtQ) || !make_rows_map(&km, k, DH, L, BH, kWtKeys) ||
-      !make_rows_map(&vm, v, DH, L, BH, kWtKeys))
+      !make_rows_map(&vm, v, DH, L, BH, kWtKeys) || !make_rows_map(&ym, out, DH, L, BH, kWtQ))
     return BASED_ERR_CUDA;
   auto kern = window_tc_kernel<DH>;
   const size_t smem = WtLayout<DH>::kSmem;
@@ -210,8 +210,7 @@ based_status_t launch_window_tc(const void* q, const void* k, const void* v, voi
   const int n_tiles = (L + kWtQ - 1) / kWtQ;
   const long long nblk = (long long)n_tiles * BH;
   if (nblk > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
-  kern<<<(unsigned)nblk, kWtThreads, smem, st>>>(qm, km, vm, static_cast<__nv_bfloat16*>(out), L,
-                                                  W, n_tiles);
+  kern<<<(unsigned)nblk, kWtThreads, smem, st>>>(qm, km, vm, ym, L, W, n_tiles);
   return launch_status();
 }
 

@@ -13,8 +13,9 @@
 //                    row max, exponentiates, keeps the row sum l in a register
 //                    and writes P (bf16, zero outside the band) to shared memory
 //   O = P V          tcgen05, M=128, N=dh, K=192             -> TMEM (fp32)
-//   y = O / l        CUDA cores, straight from TMEM to global memory.
-// P reuses the shared memory of Q and K, which are dead once S is computed.
+//   y = O / l        CUDA cores: TMEM -> 128B-swizzled staging tile -> TMA store.
+// P reuses the shared memory of Q and K, which are dead once S is computed, and
+// the y staging tile reuses that of P once O is complete.
 #pragma once
 
 #include "common.cuh"
@@ -31,6 +32,7 @@ struct WtLayout {
   static constexpr int kQ = 0;                              // Q [128 x DH] K-major SW128
   static constexpr int kK = kQ + kWtQ * DH * 2;             // K [192 x DH] K-major SW128
   static constexpr int kP = 0;                              // P [128 x 192] bf16 K-major (aliases Q,K)
+  static constexpr int kY = 0;                              // y [128 x DH] bf16 SW128 (aliases P)
   static constexpr int kPBytes = kWtQ * kWtKeys * 2;
   static constexpr int kQKEnd = kK + kWtKeys * DH * 2;
   static constexpr int kV = (kQKEnd > kPBytes ? kQKEnd : kPBytes);  // V [192 x DH] MN-major SW128
@@ -43,11 +45,11 @@ struct WtLayout {
 };
 
 template <int DH>
-__global__ void __launch_bounds__(kWtThreads)
+__global__ void __launch_bounds__(kWtThreads, 1)
     window_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                      const __grid_constant__ CUtensorMap kmap,
-                     const __grid_constant__ CUtensorMap vmap, __nv_bfloat16* __restrict__ out,
-                     int L, int W, int n_tiles) {
+                     const __grid_constant__ CUtensorMap vmap,
+                     const __grid_constant__ CUtensorMap ymap, int L, int W, int n_tiles) {
   using Lay = WtLayout<DH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -114,52 +116,50 @@ __global__ void __launch_bounds__(kWtThreads)
   umma::tc_fence_after();
 
   // ---- P = exp(S - m) over each row's band ---------------------------------------------
+  // Row r = 32 w + lane (w = warp) reads the 96 staged columns [32 w, 32 w + 96);
+  // relative to that base its band is [lo, lane + 64] (lo = lane + 1 away from
+  // the sequence start and for W = 64).  Rows past L see zero-filled Q, so their
+  // scores are finite and their output is simply not stored.
   float l_row;
   {
     const int r = tid, t = t0 + r;
-    const int cb = warp * 32;  // first staged key column this warp reads
+    const int cb = warp * 32;
     float sv[96];
-#pragma unroll
-    for (int j = 0; j < 3; ++j) umma::tmem_ld32(tmem + Lay::kTmS + tm_lane + cb + 32 * j, sv + 32 * j);
-    // valid staged columns c (key s = t0 - 64 + c): s in [max(0, t-W+1), t]
-    const int c_hi = r + 64;
-    const int c_lo = max(max(r + 1, 64 - t0), t - W + 1 - (t0 - 64));
+    umma::tmem_ld64_32(tmem + Lay::kTmS + tm_lane + cb, tmem + Lay::kTmS + tm_lane + cb + 64, sv);
+    // staged column c holds key s = t0 - 64 + c; row t sees s in [max(0, t-W+1), t]
+    const int lo = max(max(r + 1, 64 - t0), t - W + 1 - (t0 - 64)) - cb;
+    const int hi = lane + 64;
     const float scale = rsqrtf((float)DH) * 1.4426950408889634f;  // 1/sqrt(dh) * log2(e)
-    float m = -INFINITY;
+    // four interleaved partial maxima / sums keep the dependent chains short
+    float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int i = 0; i < 96; ++i)
+      if (i >= lo && (i < 64 || i <= hi)) mp[i & 3] = fmaxf(mp[i & 3], sv[i]);
+    const float ms = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])) * scale;
+    float lp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
     for (int i = 0; i < 96; ++i) {
-      const int c = cb + i;
-      if (c >= c_lo && c <= c_hi) m = fmaxf(m, sv[i]);
+      const float e = ex2_approx(fmaf(sv[i], scale, -ms));
+      sv[i] = (i >= lo && (i < 64 || i <= hi)) ? e : 0.0f;
+      lp[i & 3] += sv[i];
     }
-    const bool live = t < L;
-    float l = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 96; ++i) {
-      const int c = cb + i;
-      const float p = (live && c >= c_lo && c <= c_hi) ? exp2f((sv[i] - m) * scale) : 0.0f;
-      sv[i] = p;
-      l += p;
-    }
-    l_row = live ? l : 1.0f;
-    // P row r: 24 chunks of 8 keys; chunks 4w .. 4w+11 carry the band, the rest are zero
+    l_row = (lp[0] + lp[1]) + (lp[2] + lp[3]);  // >= 1: the row maximum contributes exp2(0)
+    // P row r (K-major, 24 chunks of 8 keys): chunks 4w .. 4w+11 carry the band
+    uint8_t* prow = sm + Lay::kP + (r >> 3) * (kWtKeys / 8) * 128 + (r & 7) * 16;
     __syncwarp();
+    for (int kc = 0; kc < 4 * warp; ++kc)
+      *reinterpret_cast<uint4*>(prow + kc * 128) = make_uint4(0, 0, 0, 0);
+    for (int kc = 4 * warp + 12; kc < kWtKeys / 8; ++kc)
+      *reinterpret_cast<uint4*>(prow + kc * 128) = make_uint4(0, 0, 0, 0);
 #pragma unroll
-    for (int kc = 0; kc < kWtKeys / 8; ++kc) {
-      const int rel = kc - warp * 4;
-      uint4 val = make_uint4(0, 0, 0, 0);
+    for (int j = 0; j < 12; ++j) {
+      uint32_t pk[4];
 #pragma unroll
-      for (int j = 0; j < 12; ++j) {
-        if (rel == j) {
-          uint32_t pk[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 b = __floats2bfloat162_rn(sv[8 * j + 2 * e], sv[8 * j + 2 * e + 1]);
-            pk[e] = *reinterpret_cast<const uint32_t*>(&b);
-          }
-          val = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        }
+      for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(sv[8 * j + 2 * e], sv[8 * j + 2 * e + 1]);
+        pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
       }
-      *reinterpret_cast<uint4*>(sm + Lay::kP + ((r >> 3) * (kWtKeys / 8) + kc) * 128 + (r & 7) * 16) = val;
+      *reinterpret_cast<uint4*>(prow + (4 * warp + j) * 128) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
   }
   umma::fence_async_smem();
@@ -178,33 +178,43 @@ __global__ void __launch_bounds__(kWtThreads)
     umma::mma_commit(bar_o);
   }
   __syncwarp();
-  if (!umma::mbar_wait(bar_o, 0)) {
-    record_device_error(BASED_ERR_TIMEOUT);
-    *abort_flag = 1;
-  }
-  umma::tc_fence_after();
   {
-    const int r = tid, t = t0 + r;
+    const bool ok = umma::mbar_wait(bar_o, 0);
+    if (!ok) record_device_error(BASED_ERR_TIMEOUT);
+    umma::tc_fence_after();
+    if (__syncthreads_or(!ok)) goto done;
+  }
+  // ---- y = O / l, staged over P (128B-swizzled rows) and stored by TMA ------------------
+  {
+    const int r = tid;
     const float inv = 1.0f / l_row;
 #pragma unroll
-    for (int c32 = 0; c32 < DH / 32; ++c32) {
-      float o[32];
-      umma::tmem_ld32(tmem + Lay::kTmO + tm_lane + c32 * 32, o);
-      if (t < L && !*abort_flag) {
-        uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)bh * L + t) * DH + c32 * 32);
+    for (int blk = 0; blk < DH / 64; ++blk) {
+      float o[64];
+      umma::tmem_ld64(tmem + Lay::kTmO + tm_lane + blk * 64, o);
+      uint8_t* yrow = sm + Lay::kY + blk * (kWtQ * 128) + r * 128;
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t pk[4];
+      for (int ch = 0; ch < 8; ++ch) {
+        uint32_t pk[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 b =
-                __floats2bfloat162_rn(o[ch * 8 + 2 * e] * inv, o[ch * 8 + 2 * e + 1] * inv);
-            pk[e] = *reinterpret_cast<const uint32_t*>(&b);
-          }
-          dst[ch] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        for (int e = 0; e < 4; ++e) {
+          const __nv_bfloat162 b2 =
+              __floats2bfloat162_rn(o[ch * 8 + 2 * e] * inv, o[ch * 8 + 2 * e + 1] * inv);
+          pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
         }
+        *reinterpret_cast<uint4*>(yrow + ((ch ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
     }
+    umma::fence_async_smem();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    // rows past L are clipped by the tensor map
+#pragma unroll
+    for (int b = 0; b < DH / 64; ++b)
+      umma::tma_store_3d(&ymap, sm + Lay::kY + b * kWtQ * 128, b * 64, t0, bh);
+    umma::bulk_commit();
+    umma::bulk_wait_read<0>();
   }
 done:
   // an aborted tile may still have its loads in flight: wait for them (bounded)
