@@ -441,23 +441,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int t = tid;  // token row of the chunk; also the TMEM lane (quadrant = warp)
     const __nv_bfloat16* q = p.q + (size_t)bh * L * kD;
     const __nv_bfloat16* k = p.k + (size_t)bh * L * kD;
-    uint4 qr[2], kr[2];
-    auto load_qk = [&](int c) {
+    // q/k rows of this thread's token, loaded two chunks ahead of their use
+    uint4 qr[2], kr[2], qn[2], kn[2];
+    auto load_qk = [&](int c, uint4* qd, uint4* kd) {
       const long long tt = (long long)c * kTcChunk + t;
       if (c < c_end && tt < L) {
         const uint4* kp = reinterpret_cast<const uint4*>(k + tt * kD);
-        kr[0] = kp[0]; kr[1] = kp[1];
+        kd[0] = kp[0]; kd[1] = kp[1];
         if (!kStateOnly) {
           const uint4* qp = reinterpret_cast<const uint4*>(q + tt * kD);
-          qr[0] = qp[0]; qr[1] = qp[1];
+          qd[0] = qp[0]; qd[1] = qp[1];
         } else {
-          qr[0] = qr[1] = make_uint4(0, 0, 0, 0);
+          qd[0] = qd[1] = make_uint4(0, 0, 0, 0);
         }
       } else {
-        qr[0] = qr[1] = kr[0] = kr[1] = make_uint4(0, 0, 0, 0);
+        qd[0] = qd[1] = kd[0] = kd[1] = make_uint4(0, 0, 0, 0);
       }
     };
-    load_qk(c_begin);
+    load_qk(c_begin, qr, kr);
+    load_qk(c_begin + 1, qn, kn);
     for (int c = c_begin; c < c_end && !*abort_flag; ++c) {
       const int it = c - c_begin;
       const int t0 = c * kTcChunk;
@@ -521,7 +523,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tc_feature_chunk(XQ, YQ, q2, ch);
         }
       }
-      load_qk(c + 1);
+      qr[0] = qn[0]; qr[1] = qn[1]; kr[0] = kn[0]; kr[1] = kn[1];
+      load_qk(c + 2, qn, kn);
       umma::fence_async_smem();
       umma::tc_fence_before();
       umma::mbar_arrive(bar_phi);
@@ -546,29 +549,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       };
       if constexpr (Lay::kTm) {
-        // P (bf16 pairs) over the first 64 columns of U; this thread reads its
-        // whole U row before writing any of it
-        uint32_t pk[64];
+        // P (bf16 pairs) over the first 64 columns of U, one 64-key half at a
+        // time: the pairs of half h land in U columns [32h, 32h + 32), which this
+        // thread has already read (they belong to half 0)
         float u[64];
-        umma::tmem_ld64(tmem + Lay::kTmU + tm_lane, u);
-        poly_pack(u, 0, pk);
-        if (quad >= 1) poly_pack(u + 32, 1, pk + 16);
-        else
+        uint32_t pk[32];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) pk[16 + e] = 0u;
-        if (quad >= 2) {
-          umma::tmem_ld64(tmem + Lay::kTmU + tm_lane + 64, u);
-          poly_pack(u, 2, pk + 32);
-          if (quad >= 3) poly_pack(u + 32, 3, pk + 48);
-          else
+        for (int h = 0; h < 2; ++h) {
+          if (quad >= 2 * h) {
+            umma::tmem_ld64(tmem + Lay::kTmU + tm_lane + 64 * h, u);
+            poly_pack(u, 2 * h, pk);
+            if (quad >= 2 * h + 1) poly_pack(u + 32, 2 * h + 1, pk + 16);
+            else
 #pragma unroll
-            for (int e = 0; e < 16; ++e) pk[48 + e] = 0u;
-        } else {
+              for (int e = 0; e < 16; ++e) pk[16 + e] = 0u;
+          } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) pk[32 + e] = 0u;
+            for (int e = 0; e < 32; ++e) pk[e] = 0u;
+          }
+          umma::tmem_st32_nowait(tmem + Lay::kTmU + tm_lane + 32 * h, pk);
         }
-        umma::tmem_st32_nowait(tmem + Lay::kTmU + tm_lane, pk);
-        umma::tmem_st32_nowait(tmem + Lay::kTmU + tm_lane + 32, pk + 32);
         umma::tmem_wait_st();
         umma::tc_fence_before();
       } else {
