@@ -40,11 +40,15 @@
 // in TMEM; the master state never leaves TMEM until the export.
 //
 // Schedule (warp-specialised, chunks pipelined):
-//   group A (warps 0-3): feature maps and Q/K tiles of chunk c, then P of chunk c;
-//   group E (warps 4-7): epilogue of chunk c -- y from O, and the fp16 copy of the
-//            state for chunk c+1 -- while group A already builds chunk c+1;
-//   issue warp (warp 8, one thread): V tiles by TMA (double-buffered when shared
+//   group P (warps 0-3):  P of chunk c from U;
+//   group F (warps 4-7):  feature maps and Q/K tiles of chunk c+1, while group P
+//            still works on chunk c;
+//   group E (warps 8-11): epilogue of chunk c -- y from O, and the fp16 copy of the
+//            state for chunk c+1;
+//   issue warp (warp 12, one thread): V tiles by TMA (double-buffered when shared
 //            memory allows) and the MMAs in the order #1, #5, #2, (P), #4.
+// Warps w, w+4 and w+8 share TMEM lane quadrant w, so each group reads and writes
+// the TMEM rows of its own 32 tokens.
 // The second state tile (features 128..191, of which 128..159 are used) is an
 // M=64 MMA.  Hand-offs are mbarriers (128 arrivals from a warp group, or a
 // tcgen05.commit); every wait is bounded.
@@ -65,7 +69,7 @@ namespace based {
 
 constexpr int kTcChunk = 128;          // tokens per chunk (MMA M)
 constexpr int kTcGroup = 128;          // threads of one CUDA-core warp group (4 warps)
-constexpr int kTcThreads = 2 * kTcGroup + 32;  // feature/score group, epilogue group, issue warp
+constexpr int kTcThreads = 3 * kTcGroup + 32;  // score, feature and epilogue groups, issue warp
 constexpr int kSymFP = 160;            // 153 distinct features + 7 zero pads
 constexpr int kTcTmemCols = 512;
 
@@ -300,7 +304,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     *abort_flag = 1;
   };
 
-  if (warp == 8) {
+  if (warp == 12) {
     // ================= issue warp: lane 0 drives TMA and the tensor cores =================
     if (lane == 0) {
       const uint32_t sQ = umma::smem_u32(sm + Lay::kQ), sK = umma::smem_u32(sm + Lay::kK),
@@ -326,11 +330,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint32_t id_o4 = umma::idesc_bf16(128, NA, false, true);
       const uint32_t id_s0 = umma::idesc_bf16(128, NA, true, true);
       const uint32_t id_s1 = umma::idesc_bf16(64, NA, true, true);
-      // per stage: a load in flight, and the parity of the phase it completes
-      bool inflight[2] = {false, false};
-      uint32_t vphase[2] = {0, 0};
-      if (c_begin < c_end) { issue_v(c_begin, 0); inflight[0] = true; }
-      if (Lay::kVBuf == 2 && c_begin + 1 < c_end) { issue_v(c_begin + 1, 1); inflight[1] = true; }
+      // per stage (bit s): a load in flight, and the parity of the phase it completes
+      // (bit masks rather than arrays, which would live in local memory)
+      uint32_t inflight = 0, vphase = 0;
+      if (c_begin < c_end) { issue_v(c_begin, 0); inflight |= 1u; }
+      if (Lay::kVBuf == 2 && c_begin + 1 < c_end) { issue_v(c_begin + 1, 1); inflight |= 2u; }
       int n_done = 0;  // chunks whose MMAs were all issued and committed
       for (int c = c_begin; c < c_end && !*abort_flag; ++c) {
         const int it = c - c_begin;
@@ -357,9 +361,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           umma::mma_bf16(tmem + Lay::kTmU, d_q, d_k, id_u, 0);
           umma::mma_commit(bar_u);
         }
-        if (!umma::mbar_wait(bar_tma + stage, vphase[stage])) { fail(); break; }
-        inflight[stage] = false;
-        vphase[stage] ^= 1;
+        if (!umma::mbar_wait(bar_tma + stage, (vphase >> stage) & 1u)) { fail(); break; }
+        inflight &= ~(1u << stage);
+        vphase ^= 1u << stage;
         // #5 overwrites the state: the epilogue group must have read (and copied)
         // the previous chunk's state out of TMEM
         if (!kStateOnly && Lay::kEarlyO && has_state) {
@@ -380,7 +384,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (Lay::kVBuf == 2 && it > 0 && c + 1 < c_end) {
             if (!umma::mbar_wait(bar_o, (it - 1) & 1)) { fail(); break; }
             issue_v(c + 1, (it - 1) & 1);
-            inflight[(it - 1) & 1] = true;
+            inflight |= 1u << ((it - 1) & 1);
           }
         }
         if (!kStateOnly) {
@@ -427,18 +431,95 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!Lay::kTm && c_next < c_end) {
           if (!umma::mbar_wait(bar_o, ph)) { fail(); break; }
           issue_v(c_next, stage);
-          inflight[stage] = true;
+          inflight |= 1u << stage;
         }
       }
       // the last chunk's MMAs must be complete before the state is read out
       if (n_done > 0 && !umma::mbar_wait(bar_o, (n_done - 1) & 1)) fail();
       // an aborted run may still have V loads in flight: wait for them (bounded)
       for (int sidx = 0; sidx < 2; ++sidx)
-        if (inflight[sidx]) umma::mbar_wait(bar_tma + sidx, vphase[sidx]);
+        if ((inflight >> sidx) & 1u) umma::mbar_wait(bar_tma + sidx, (vphase >> sidx) & 1u);
     }
   } else if (warp < 4) {
-    // ================= group A: feature maps (chunk c), scores (chunk c) =================
+    // ================= group P: scores of chunk c =================
     const int t = tid;  // token row of the chunk; also the TMEM lane (quadrant = warp)
+    for (int c = c_begin; c < c_end && !kStateOnly && !*abort_flag; ++c) {
+      const int it = c - c_begin;
+      const int t0 = c * kTcChunk;
+      // ---- scores: P = mask(1 + u/4 + u^2/32) * sc ------------------------------------
+      if (!umma::mbar_wait(bar_u, it & 1)) { fail(); break; }
+      if (!Lay::kTm && it > 0 && !umma::mbar_wait(bar_o, (it - 1) & 1)) { fail(); break; }
+      umma::tc_fence_after();
+      const float sc = tc_chunk_scale((long long)t0 + kTcChunk);
+      const float c0 = sc, c1 = 0.25f * sc, c2 = 0.03125f * sc;
+      auto poly_pack = [&](const float* u, int c32, uint32_t* pk) {
+        const bool diag = c32 == quad;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float w0 = fmaf(u[2 * e], fmaf(u[2 * e], c2, c1), c0);
+          float w1 = fmaf(u[2 * e + 1], fmaf(u[2 * e + 1], c2, c1), c0);
+          if (diag) {
+            if (2 * e > lane) w0 = 0.0f;
+            if (2 * e + 1 > lane) w1 = 0.0f;
+          }
+          pk[e] = as_u32(__floats2bfloat162_rn(w0, w1));
+        }
+      };
+      if constexpr (Lay::kTm) {
+        // P (bf16 pairs) of key block b (32 keys) goes to U columns [16b, 16b + 16),
+        // which this thread has read already (they belong to block b / 2 <= b);
+        // one loop body for every block keeps the code small
+        const int row = lane + 32 * quad;  // this thread's token within the chunk
+#pragma unroll 1
+        for (int b = 0; b <= quad; ++b) {
+          float u[32];
+          umma::tmem_ld32(tmem + Lay::kTmU + tm_lane + 32 * b, u);
+          const int lim = row - 32 * b;  // keys 32b + j with j > lim lie in the future
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float w0 = fmaf(u[2 * e], fmaf(u[2 * e], c2, c1), c0);
+            float w1 = fmaf(u[2 * e + 1], fmaf(u[2 * e + 1], c2, c1), c0);
+            if (2 * e > lim) w0 = 0.0f;
+            if (2 * e + 1 > lim) w1 = 0.0f;
+            pk[e] = as_u32(__floats2bfloat162_rn(w0, w1));
+          }
+          umma::tmem_st16_nowait(tmem + Lay::kTmU + tm_lane + 16 * b, pk);
+        }
+        uint32_t zero[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) zero[e] = 0u;
+#pragma unroll 1
+        for (int b = quad + 1; b < 4; ++b) umma::tmem_st16_nowait(tmem + Lay::kTmU + tm_lane + 16 * b, zero);
+        umma::tmem_wait_st();
+        umma::tc_fence_before();
+      } else {
+#pragma unroll
+        for (int c32 = 0; c32 < 4; ++c32) {
+          if (c32 > quad) {  // strictly above the diagonal: zeros (warp-uniform)
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+              *reinterpret_cast<uint4*>(sm + Lay::kP + ((t >> 3) * 16 + c32 * 4 + g) * 128 + (t & 7) * 16) =
+                  make_uint4(0, 0, 0, 0);
+            continue;
+          }
+          float u[32];
+          umma::tmem_ld32(tmem + Lay::kTmU + tm_lane + c32 * 32, u);
+          uint32_t pk[16];
+          poly_pack(u, c32, pk);
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            *reinterpret_cast<uint4*>(sm + Lay::kP + ((t >> 3) * 16 + c32 * 4 + g) * 128 + (t & 7) * 16) =
+                make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
+        }
+        umma::fence_async_smem();
+        umma::tc_fence_before();
+      }
+      umma::mbar_arrive(bar_p);
+    }
+  } else if (warp < 8) {
+    // ================= group F: feature maps and Q/K tiles of chunk c =================
+    const int t = tid - kTcGroup;  // token row of the chunk; also the TMEM lane (quadrant = warp & 3)
     const __nv_bfloat16* q = p.q + (size_t)bh * L * kD;
     const __nv_bfloat16* k = p.k + (size_t)bh * L * kD;
     // q/k rows of this thread's token, loaded two chunks ahead of their use
@@ -468,10 +549,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(qr);
       const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(kr);
       uint8_t* phik = sm + Lay::kPhiK + (it % Lay::kPhiKBuf) * 40960;
-      // With a single phiK buffer (and for the smem phiQ / Q / K tiles) wait
-      // until the previous chunk's #5 and #2 are done.  With two phiK buffers,
-      // this chunk's buffer was released by the wait of the previous iteration.
+      // With a single phiK buffer (and for the smem phiQ tile) wait until the
+      // previous chunk's #5 and #2 are done.  With two phiK buffers, this chunk's
+      // buffer was released by the wait of the previous iteration.
       if (!Lay::kTm && it > 0 && !umma::mbar_wait(bar_m25, (it - 1) & 1)) { fail(); break; }
+      // the Q/K tiles are rewritten once #1 of the previous chunk has read them
+      if (!kStateOnly && it > 0 && !umma::mbar_wait(bar_u, (it - 1) & 1)) { fail(); break; }
       // ---- phiK and Q/K tiles -------------------------------------------------------
       {
         __nv_bfloat162 XK[8], YK[8];
@@ -528,76 +611,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       umma::fence_async_smem();
       umma::tc_fence_before();
       umma::mbar_arrive(bar_phi);
-      if (kStateOnly) continue;
-      // ---- scores: P = mask(1 + u/4 + u^2/32) * sc ------------------------------------
-      if (!umma::mbar_wait(bar_u, it & 1)) { fail(); break; }
-      if (!Lay::kTm && it > 0 && !umma::mbar_wait(bar_o, (it - 1) & 1)) { fail(); break; }
-      umma::tc_fence_after();
-      const float sc = tc_chunk_scale((long long)t0 + kTcChunk);
-      const float c0 = sc, c1 = 0.25f * sc, c2 = 0.03125f * sc;
-      auto poly_pack = [&](const float* u, int c32, uint32_t* pk) {
-        const bool diag = c32 == quad;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float w0 = fmaf(u[2 * e], fmaf(u[2 * e], c2, c1), c0);
-          float w1 = fmaf(u[2 * e + 1], fmaf(u[2 * e + 1], c2, c1), c0);
-          if (diag) {
-            if (2 * e > lane) w0 = 0.0f;
-            if (2 * e + 1 > lane) w1 = 0.0f;
-          }
-          pk[e] = as_u32(__floats2bfloat162_rn(w0, w1));
-        }
-      };
-      if constexpr (Lay::kTm) {
-        // P (bf16 pairs) over the first 64 columns of U, one 64-key half at a
-        // time: the pairs of half h land in U columns [32h, 32h + 32), which this
-        // thread has already read (they belong to half 0)
-        float u[64];
-        uint32_t pk[32];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (quad >= 2 * h) {
-            umma::tmem_ld64(tmem + Lay::kTmU + tm_lane + 64 * h, u);
-            poly_pack(u, 2 * h, pk);
-            if (quad >= 2 * h + 1) poly_pack(u + 32, 2 * h + 1, pk + 16);
-            else
-#pragma unroll
-              for (int e = 0; e < 16; ++e) pk[16 + e] = 0u;
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) pk[e] = 0u;
-          }
-          umma::tmem_st32_nowait(tmem + Lay::kTmU + tm_lane + 32 * h, pk);
-        }
-        umma::tmem_wait_st();
-        umma::tc_fence_before();
-      } else {
-#pragma unroll
-        for (int c32 = 0; c32 < 4; ++c32) {
-          if (c32 > quad) {  // strictly above the diagonal: zeros (warp-uniform)
-#pragma unroll
-            for (int g = 0; g < 4; ++g)
-              *reinterpret_cast<uint4*>(sm + Lay::kP + ((t >> 3) * 16 + c32 * 4 + g) * 128 + (t & 7) * 16) =
-                  make_uint4(0, 0, 0, 0);
-            continue;
-          }
-          float u[32];
-          umma::tmem_ld32(tmem + Lay::kTmU + tm_lane + c32 * 32, u);
-          uint32_t pk[16];
-          poly_pack(u, c32, pk);
-#pragma unroll
-          for (int g = 0; g < 4; ++g)
-            *reinterpret_cast<uint4*>(sm + Lay::kP + ((t >> 3) * 16 + c32 * 4 + g) * 128 + (t & 7) * 16) =
-                make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
-        }
-        umma::fence_async_smem();
-        umma::tc_fence_before();
-      }
-      umma::mbar_arrive(bar_p);
     }
   } else if (!kStateOnly) {
     // ================= group E: epilogue of chunk c (output, fp16 state copy) =================
-    const int t = tid - kTcGroup;  // TMEM lane of this thread (quadrant = warp - 4)
+    const int t = tid - 2 * kTcGroup;  // TMEM lane of this thread (quadrant = warp - 8)
     __nv_bfloat16* out = p.out + (size_t)bh * L * DV;
     // fp16 copy (scaled by sn) of the state rows this thread holds, as #2's B operand:
     // tile 0 row t = feature t; tile 1 (M=64) lanes 0..15 of quadrants 0, 1 = features
@@ -618,11 +635,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               make_uint4(pk[0], pk[1], pk[2], pk[3]);
         };
         if constexpr (NG == 3) {
-          float sv[96];  // the whole tile row in one TMEM round trip
-          umma::tmem_ld64_32(base, base + 64, sv);
+          {
+            float sv[64];
+            umma::tmem_ld64(base, sv);
+            if (tile == 0 || lane < 16) {
+#pragma unroll
+              for (int j0 = 0; j0 < 64; j0 += 8) put(sv + j0, j0);
+            }
+          }
+          float sv[32];
+          umma::tmem_ld32(base + 64, sv);
           if (tile == 1 && lane >= 16) continue;
 #pragma unroll
-          for (int j0 = 0; j0 < NA; j0 += 8) put(sv + j0, j0);
+          for (int j0 = 64; j0 < NA; j0 += 8) put(sv + j0 - 64, j0);
         } else {
 #pragma unroll
           for (int g = 0; g < NG; ++g) {
@@ -744,9 +769,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   umma::tc_fence_before();
   __syncthreads();
   umma::tc_fence_after();
-  if (!*abort_flag && warp >= 4 && warp < 8) {
+  if (!*abort_flag && warp >= 8 && warp < 12) {
     // ---- state out of TMEM (group E lanes): segment partials or the final export ----
-    const int t = tid - kTcGroup;
+    const int t = tid - 2 * kTcGroup;
     for (int tile = 0; tile < 2; ++tile) {
       if (tile == 1 && quad > 1) break;
       const int f = tile == 0 ? t : 128 + quad * 16 + (lane & 15);

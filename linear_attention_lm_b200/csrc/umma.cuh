@@ -64,15 +64,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Wait for the phase with the given parity to complete; false after kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
+// The spin part of mbar_wait, kept out of line so that the many wait sites of a
+// warp-specialised kernel stay small in the instruction cache.
+__device__ __noinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = global_timer_ns();
   while (true) {
     for (int i = 0; i < 256; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (global_timer_ns() - t0 > kWaitLimitNs) return false;
   }
+}
+// Wait for the phase with the given parity to complete; false after kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_spin(bar, parity);
 }
 
 // ---------------------------------------------------------------- fences
