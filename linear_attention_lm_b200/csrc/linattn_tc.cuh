@@ -103,11 +103,17 @@ struct TcLayout {
   // 128..191, M=64: row r in lane r%16 + 32*(r/16)), the score tile U (P is
   // written over it), the output accumulator O -- separate from U when the
   // columns allow it -- and phiQ (80 columns of fp16 pairs)
-  static constexpr bool kEarlyO = 3 * kTileCols + 128 <= kTcTmemCols;
+  // d_v = 64 keeps the state transposed, [S|z]^T: TMEM lane = value column (64
+  // columns, then z in lane 64), TMEM column = feature; #5 is then one N=160 MMA
+  // per K step.  d_v = 128 keeps features on the lanes (tile 0: features
+  // 0..127, M=128; tile 1: features 128..191, M=64).
+  static constexpr bool kSt = DV == 64;
   static constexpr int kTmS0 = 0;
-  static constexpr int kTmS1 = kTileCols;
-  static constexpr int kTmU = 2 * kTileCols;
+  static constexpr int kTmS1 = kSt ? 0 : kTileCols;
+  static constexpr int kTmU = kSt ? kSymFP : 2 * kTileCols;
+  static constexpr bool kEarlyO = kTmU + 128 + kTileCols <= kTcTmemCols;
   static constexpr int kTmO = kEarlyO ? kTmU + 128 : kTmU;
+  static_assert(kTmU % 32 == 0, "TMEM region alignment");
   static constexpr int kTmQ = kTmO + kTileCols;
   static_assert(kTmO + kTileCols + (kTm ? kSymFP / 2 : 0) <= kTcTmemCols, "TMEM budget");
   static_assert(!kTm || kEarlyO, "TMEM operands need a separate O");
@@ -293,6 +299,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       *reinterpret_cast<__nv_bfloat16*>(sm + Lay::kV + b * Lay::kVStage + (DV / 64) * 16384 +
                                         umma::off_mnmajor_sw128(0, tid, kTcChunk)) =
           __float2bfloat16(1.0f);
+  if constexpr (Lay::kSt) {
+    // rows DV..NA-1 of the transposed fp16 state copies: row DV (z) is rewritten
+    // for every chunk, the rows after it stay zero
+    for (int b = 0; b < Lay::kSBuf; ++b)
+      for (int i = tid; i < (NA - DV) * kSymFP * 2 / 16; i += kTcThreads)
+        reinterpret_cast<uint4*>(sm + Lay::kS + b * Lay::kSBytes + DV * kSymFP * 2)[i] =
+            make_uint4(0, 0, 0, 0);
+  }
   umma::fence_async_smem();
   umma::tc_fence_before();
   __syncthreads();
@@ -321,15 +335,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // descriptors are computed once per buffer and stepped along K by adding
       // the start-address increment (16-byte units) to their low word
       const uint64_t d_q = umma::desc_kmajor_none(sQ, 0, 16), d_k = umma::desc_kmajor_none(sK, 0, 16);
-      const uint64_t d_s0 = umma::desc_mnmajor_none(sS, 0, kSymFP);
-      const uint64_t d_s1 = umma::desc_mnmajor_none(sS + (Lay::kSBuf - 1) * Lay::kSBytes, 0, kSymFP);
+      // fp16 state copy: [value column x feature] K-major (transposed state) or
+      // [feature x value column] MN-major
+      const uint32_t sS1 = sS + (Lay::kSBuf - 1) * Lay::kSBytes;
+      const uint64_t d_s0 = Lay::kSt ? umma::desc_kmajor_none(sS, 0, kSymFP)
+                                     : umma::desc_mnmajor_none(sS, 0, kSymFP);
+      const uint64_t d_s1 = Lay::kSt ? umma::desc_kmajor_none(sS1, 0, kSymFP)
+                                     : umma::desc_mnmajor_none(sS1, 0, kSymFP);
       const uint64_t d_p = umma::desc_kmajor_none(sP, 0, kTcChunk);
       const uint64_t d_phiq = umma::desc_kmajor_none(sPhiQ, 0, kSymFP);
       const uint32_t id_u = umma::idesc_bf16(128, 128, false, false);
-      const uint32_t id_o2 = umma::idesc_f16(128, NA, false, true);
+      const uint32_t id_o2 = umma::idesc_f16(128, NA, false, !Lay::kSt);
       const uint32_t id_o4 = umma::idesc_bf16(128, NA, false, true);
       const uint32_t id_s0 = umma::idesc_bf16(128, NA, true, true);
       const uint32_t id_s1 = umma::idesc_bf16(64, NA, true, true);
+      const uint32_t id_st = umma::idesc_bf16(128, kSymFP, true, true);
       // per stage (bit s): a load in flight, and the parity of the phase it completes
       // (bit masks rather than arrays, which would live in local memory)
       uint32_t inflight = 0, vphase = 0;
@@ -372,11 +392,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         umma::tc_fence_after();
         // K step of 16 tokens: +256 B in the no-swizzle phiK layout (2 core
         // matrices), +2048 B (16 rows of 128 B) in the swizzled V tile
+        if constexpr (Lay::kSt) {
+          // [S|z]^T += [V|1]^T phiK: A = the V stage (value columns x tokens,
+          // MN-major; the ones block supplies row DV), B = phiK (N = 160 features)
 #pragma unroll
-        for (int ks = 0; ks < kTcChunk / 16; ++ks) {
-          const uint32_t acc = has_state || ks > 0;
-          umma::mma_bf16(tmem + Lay::kTmS0, d_k0 + ks * 16, d_v + ks * 128, id_s0, acc);
-          umma::mma_bf16(tmem + Lay::kTmS1, d_k1 + ks * 16, d_v + ks * 128, id_s1, acc);
+          for (int ks = 0; ks < kTcChunk / 16; ++ks)
+            umma::mma_bf16(tmem + Lay::kTmS0, d_v + ks * 128, d_k0 + ks * 16, id_st,
+                           has_state || ks > 0);
+        } else {
+#pragma unroll
+          for (int ks = 0; ks < kTcChunk / 16; ++ks) {
+            const uint32_t acc = has_state || ks > 0;
+            umma::mma_bf16(tmem + Lay::kTmS0, d_k0 + ks * 16, d_v + ks * 128, id_s0, acc);
+            umma::mma_bf16(tmem + Lay::kTmS1, d_k1 + ks * 16, d_v + ks * 128, id_s1, acc);
+          }
         }
         if (Lay::kTm) {
           umma::mma_commit(bar_m5);
@@ -622,6 +651,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     int kk = 0;  // number of state copies handed off so far (buffer kk % kSBuf)
     auto copy_state = [&](float sn) {
       uint8_t* sbuf = sm + Lay::kS + (kk % Lay::kSBuf) * Lay::kSBytes;
+      if constexpr (Lay::kSt) {
+        // row t of [S|z]^T (value column t, or z for t = DV) -> row t of the
+        // K-major copy; lanes past DV hold nothing (quadrant 3 skips the loads)
+        if (quad == 3) return;
+        uint8_t* dst = sbuf + (t >> 3) * (kSymFP * 16) + (t & 7) * 16;
+        const uint32_t base = tmem + Lay::kTmS0 + tm_lane;
+        auto put8 = [&](const float* sv, int fg) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            pk[e] = as_u32(__floats2half2_rn(sv[2 * e] * sn, sv[2 * e + 1] * sn));
+          if (t <= DV) *reinterpret_cast<uint4*>(dst + fg * 128) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        };
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          float sv[64];
+          umma::tmem_ld64(base + 64 * h, sv);
+#pragma unroll
+          for (int g = 0; g < 8; ++g) put8(sv + 8 * g, 8 * h + g);
+        }
+        float sv[32];
+        umma::tmem_ld32(base + 128, sv);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) put8(sv + 8 * g, 16 + g);
+        return;
+      }
       for (int tile = 0; tile < 2; ++tile) {
         if (tile == 1 && (quad > 1)) break;
         const int f = tile == 0 ? t : 128 + quad * 16 + lane;
@@ -664,7 +719,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (has_init) {
       // seed the TMEM state of a later segment with the sum of the earlier partials
       const float* part = p.partial + (size_t)bh * (p.n_seg - 1) * kSymFP * NA;
-      for (int tile = 0; tile < 2; ++tile) {
+      if (Lay::kSt && quad < 3) {
+        // partials are [feature][value column]; this lane seeds row t of [S|z]^T
+        for (int g = 0; g < kSymFP / 32; ++g) {
+          float acc[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
+          if (t <= DV) {
+            for (int sp = 0; sp < seg; ++sp) {
+              const float* col = part + ((size_t)sp * kSymFP + g * 32) * NA + t;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) acc[i] += col[(size_t)i * NA];
+            }
+          }
+          umma::tmem_st32(tmem + Lay::kTmS0 + tm_lane + g * 32, acc);
+        }
+      }
+      for (int tile = 0; tile < 2 && !Lay::kSt; ++tile) {
         if (tile == 1 && quad > 1) break;
         const int f = tile == 0 ? t : 128 + quad * 16 + (lane & 15);
         const uint32_t base = tmem + (tile == 0 ? Lay::kTmS0 : Lay::kTmS1) + tm_lane;
@@ -772,7 +843,62 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (!*abort_flag && warp >= 8 && warp < 12) {
     // ---- state out of TMEM (group E lanes): segment partials or the final export ----
     const int t = tid - 2 * kTcGroup;
-    for (int tile = 0; tile < 2; ++tile) {
+    const bool any_st = has_init || c_begin < c_end;
+    if constexpr (Lay::kSt) {
+      // [S|z]^T -> shared memory as [feature][value column | z] (stride DV + 1),
+      // then coalesced rows of the 273-row layout (or of the segment partial).
+      // The feature-map buffers are free: every MMA has completed.
+      constexpr int kStr = DV + 1;
+      float* stage = reinterpret_cast<float*>(sm + Lay::kPhiK);
+      int* rowmap = reinterpret_cast<int*>(stage + kSymFP * kStr);  // [273]: 2 f + (1 if / sqrt 2)
+      static_assert(Lay::kPhiKBuf * 40960 >= (kSymFP * (DV + 1) + kF) * 4, "export staging");
+      if (quad < 3) {
+#pragma unroll 1
+        for (int g = 0; g < kSymFP / 32; ++g) {
+          float sv[32];
+          umma::tmem_ld32(tmem + Lay::kTmS0 + tm_lane + g * 32, sv);
+          if (t <= DV) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) stage[(g * 32 + i) * kStr + t] = any_st ? sv[i] : 0.0f;
+          }
+        }
+      }
+      for (int f = t; f < kSymFP; f += kTcGroup) {
+        int r0 = -1, r1 = -1;
+        float scale = 1.0f;
+        const int nrows = tc_feature_rows(f, &r0, &r1, &scale);
+        const int code = 2 * f + (nrows == 2 ? 1 : 0);
+        if (nrows >= 1) rowmap[r0] = code;
+        if (nrows == 2) rowmap[r1] = code;
+      }
+      umma::named_sync(1, kTcGroup);
+      if (kStateOnly) {
+        float* part = p.partial + ((size_t)bh * (p.n_seg - 1) + seg) * kSymFP * NA;
+        for (int i = t; i < kSymFP * NA; i += kTcGroup) {
+          const int f = i / NA, j = i - f * NA;
+          part[i] = j <= DV ? stage[f * kStr + j] : 0.0f;
+        }
+      } else if (seg == p.n_seg - 1) {
+        if (p.state_kv) {
+          float4* skv = reinterpret_cast<float4*>(p.state_kv + (size_t)bh * kF * DV);
+          for (int i = t; i < kF * (DV / 4); i += kTcGroup) {
+            const int r = i / (DV / 4), j = (i - r * (DV / 4)) * 4;
+            const int code = rowmap[r];
+            const float sc = (code & 1) ? 0.70710678118654752f : 1.0f;
+            const float* src = stage + (code >> 1) * kStr + j;
+            skv[i] = make_float4(src[0] * sc, src[1] * sc, src[2] * sc, src[3] * sc);
+          }
+        }
+        if (p.state_k) {
+          float* sk = p.state_k + (size_t)bh * kF;
+          for (int r = t; r < kF; r += kTcGroup) {
+            const int code = rowmap[r];
+            sk[r] = stage[(code >> 1) * kStr + DV] * ((code & 1) ? 0.70710678118654752f : 1.0f);
+          }
+        }
+      }
+    }
+    for (int tile = 0; tile < 2 && !Lay::kSt; ++tile) {
       if (tile == 1 && quad > 1) break;
       const int f = tile == 0 ? t : 128 + quad * 16 + (lane & 15);
       const bool mine = tile == 0 || lane < 16;
