@@ -82,14 +82,25 @@ struct TcLayout {
   // for a second phiK buffer and a y staging tile stored by TMA); d_v = 128
   // keeps them in shared memory
   static constexpr bool kTm = DV == 64;
-  static constexpr int kVBuf = DV == 64 ? 2 : 1;           // V stages
+  static constexpr int kVBuf = DV == 64 ? 3 : 1;           // V stages
   static constexpr int kPhiKBuf = kTm ? 2 : 1;             // phiK buffers
-  static constexpr int kVStage = (DV / 64 + 1) * 16384;    // V blocks + ones block
+  // d_v = 64: three V stages share one ones block placed after them (each stage's
+  // descriptor reaches it through its own block stride); d_v = 128: one stage
+  // holding its V blocks and its ones block
+  static constexpr int kVStage = DV == 64 ? 16384 : (DV / 64 + 1) * 16384;
+  static constexpr int kNOnes = DV == 64 ? 1 : kVBuf;
+  static constexpr int kVBytes = DV == 64 ? (kVBuf + 1) * 16384 : kVBuf * kVStage;
+  // ones block used by V stage s, and the stride from the stage's first V block
+  // to it (the descriptor's block stride), relative to kV
+  static __host__ __device__ constexpr int ones_off(int s) {
+    return DV == 64 ? kVBuf * 16384 : s * kVStage + (DV / 64) * 16384;
+  }
+  static __host__ __device__ constexpr int v_lbo(int s) { return DV == 64 ? (kVBuf - s) * 16384 : 16384; }
   // shared memory (byte offsets from a 1024-aligned base)
   static constexpr int kQ = 0;                             // Q tile  [128 x 16] bf16, K-major
   static constexpr int kK = kQ + 4096;                     // K tile  [128 x 16] bf16, K-major
   static constexpr int kV = kK + 4096;                     // [V | ones] MN-major SW128 stages
-  static constexpr int kPhiK = kV + kVBuf * kVStage;       // phiK [160 x 128] bf16, MN-major
+  static constexpr int kPhiK = kV + kVBytes;               // phiK [160 x 128] bf16, MN-major
   static constexpr int kP = kPhiK + kPhiKBuf * 40960;      // P [128 x 128] bf16 (smem path)
   static constexpr int kPhiQ = kP + (kTm ? 0 : 32768);     // phiQ [128 x 160] fp16 (smem path)
   static constexpr int kSBuf = kTm ? 2 : 1;                // fp16 state copies
@@ -97,7 +108,7 @@ struct TcLayout {
   static constexpr int kS = kPhiQ + (kTm ? 0 : 40960);     // [S|z] copies [160 x NA] fp16, MN-major
   static constexpr int kY = kS + kSBuf * kSBytes;          // y staging [128 x 64] bf16 SW128
   static constexpr int kBar = kY + (kTm ? 16384 : 0);      // mbarriers + TMEM address
-  static constexpr int kBytes = kBar + 128;
+  static constexpr int kBytes = kBar + 256;
   static constexpr size_t kSmem = kBytes + 1024;           // + alignment slack
   // TMEM: state tile 0 (features 0..127, M=128), state tile 1 (features
   // 128..191, M=64: row r in lane r%16 + 32*(r/16)), the score tile U (P is
@@ -241,7 +252,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::kBar);
-  uint64_t* bar_tma = bars;          // [2] V stage landed
+  uint64_t* bar_tma = bars + 16;     // [kVBuf] V stage landed
   uint64_t* bar_phi = bars + 2;      // feature maps + Q/K tiles written (group A)
   uint64_t* bar_u = bars + 3;        // #1 done (commit)
   uint64_t* bar_p = bars + 4;        // P written (group A)
@@ -267,8 +278,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const bool has_init = !kStateOnly && seg > 0;
 
   if (tid == 0) {
-    umma::mbar_init(bar_tma, 1);
-    umma::mbar_init(bar_tma + 1, 1);
+    for (int sidx = 0; sidx < Lay::kVBuf; ++sidx) umma::mbar_init(bar_tma + sidx, 1);
     umma::mbar_init(bar_phi, kTcGroup);
     umma::mbar_init(bar_u, 1);
     umma::mbar_init(bar_p, kTcGroup);
@@ -288,15 +298,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     umma::tmem_relinquish();
   }
   // ones block of every V stage: column DV of the augmented V is 1 for every token
-  for (int b = 0; b < Lay::kVBuf; ++b) {
-    uint8_t* ones = sm + Lay::kV + b * Lay::kVStage + (DV / 64) * 16384;
+  for (int b = 0; b < Lay::kNOnes; ++b) {
+    uint8_t* ones = sm + Lay::kV + Lay::ones_off(b);
     for (int i = tid; i < 16384 / 16; i += kTcThreads)
       reinterpret_cast<uint4*>(ones)[i] = make_uint4(0, 0, 0, 0);
   }
   __syncthreads();
-  for (int b = 0; b < Lay::kVBuf; ++b)
+  for (int b = 0; b < Lay::kNOnes; ++b)
     if (tid < kTcChunk)
-      *reinterpret_cast<__nv_bfloat16*>(sm + Lay::kV + b * Lay::kVStage + (DV / 64) * 16384 +
+      *reinterpret_cast<__nv_bfloat16*>(sm + Lay::kV + Lay::ones_off(b) +
                                         umma::off_mnmajor_sw128(0, tid, kTcChunk)) =
           __float2bfloat16(1.0f);
   if constexpr (Lay::kSt) {
@@ -353,15 +363,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // per stage (bit s): a load in flight, and the parity of the phase it completes
       // (bit masks rather than arrays, which would live in local memory)
       uint32_t inflight = 0, vphase = 0;
-      if (c_begin < c_end) { issue_v(c_begin, 0); inflight |= 1u; }
-      if (Lay::kVBuf == 2 && c_begin + 1 < c_end) { issue_v(c_begin + 1, 1); inflight |= 2u; }
+      for (int sidx = 0; sidx < Lay::kVBuf && c_begin + sidx < c_end; ++sidx) {
+        issue_v(c_begin + sidx, sidx);
+        inflight |= 1u << sidx;
+      }
       int n_done = 0;  // chunks whose MMAs were all issued and committed
       for (int c = c_begin; c < c_end && !*abort_flag; ++c) {
         const int it = c - c_begin;
         const uint32_t ph = it & 1;
-        const int stage = Lay::kVBuf == 2 ? (it & 1) : 0;
-        const uint64_t d_v =
-            umma::desc_mnmajor_sw128(umma::smem_u32(sm + Lay::kV + stage * Lay::kVStage), 0, kTcChunk);
+        const int stage = it % Lay::kVBuf;
+        const uint64_t d_v = umma::smem_desc(umma::smem_u32(sm + Lay::kV + stage * Lay::kVStage),
+                                             Lay::v_lbo(stage), 1024, umma::kLayoutSW128);
         const uint32_t sPhiK = umma::smem_u32(sm + Lay::kPhiK + (it % Lay::kPhiKBuf) * 40960);
         const uint64_t d_k0 = umma::desc_mnmajor_none(sPhiK, 0, kTcChunk);
         const uint64_t d_k1 = umma::desc_mnmajor_none(sPhiK + 16 * 2048, 0, kTcChunk);
@@ -409,11 +421,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         if (Lay::kTm) {
           umma::mma_commit(bar_m5);
-          // refill the stage of chunk c-1 (its MMAs are done by now) with chunk c+1
-          if (Lay::kVBuf == 2 && it > 0 && c + 1 < c_end) {
+          // refill the stage of chunk c-1 (its MMAs are done by now) with chunk
+          // c + kVBuf - 1
+          if (Lay::kVBuf > 1 && it > 0 && c + Lay::kVBuf - 1 < c_end) {
             if (!umma::mbar_wait(bar_o, (it - 1) & 1)) { fail(); break; }
-            issue_v(c + 1, (it - 1) & 1);
-            inflight |= 1u << ((it - 1) & 1);
+            issue_v(c + Lay::kVBuf - 1, (it - 1) % Lay::kVBuf);
+            inflight |= 1u << ((it - 1) % Lay::kVBuf);
           }
         }
         if (!kStateOnly) {
@@ -466,7 +479,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // the last chunk's MMAs must be complete before the state is read out
       if (n_done > 0 && !umma::mbar_wait(bar_o, (n_done - 1) & 1)) fail();
       // an aborted run may still have V loads in flight: wait for them (bounded)
-      for (int sidx = 0; sidx < 2; ++sidx)
+      for (int sidx = 0; sidx < Lay::kVBuf; ++sidx)
         if ((inflight >> sidx) & 1u) umma::mbar_wait(bar_tma + sidx, (vphase >> sidx) & 1u);
     }
   } else if (warp < 4) {
@@ -779,6 +792,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!umma::mbar_wait(bar_o, it & 1)) { fail(); break; }
       umma::tc_fence_after();
       if constexpr (Lay::kTm) {
+        float o[64], den;
+        umma::tmem_ld64_1(tmem + Lay::kTmO + tm_lane, tmem + Lay::kTmO + tm_lane + DV, o, &den);
+        // O is in registers: #2 of the next chunk may overwrite it
+        umma::tc_fence_before();
+        if (c + 1 < c_end) {
+          umma::mbar_arrive(bar_ss);
+          ++kk;
+        }
         // y row t into the swizzled staging tile; one TMA store per chunk
         uint8_t* ybuf = sm + Lay::kY;
         if (t == 0) {  // the store of chunk c-1 has finished reading ybuf
@@ -786,8 +807,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           umma::mbar_arrive(bar_yfree);
         }
         if (!umma::mbar_wait(bar_yfree, it & 1)) { fail(); break; }
-        float o[64], den;
-        umma::tmem_ld64_1(tmem + Lay::kTmO + tm_lane, tmem + Lay::kTmO + tm_lane + DV, o, &den);
         const float inv = 1.0f / (den + p.eps * sc);
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
@@ -821,7 +840,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!Lay::kTm && c + 1 < c_end) copy_state(tc_chunk_scale((long long)t0 + 2 * kTcChunk));
       umma::fence_async_smem();
       umma::tc_fence_before();
-      if (c + 1 < c_end) {  // O (and, without a second copy buffer, the state) read
+      if (!Lay::kTm && c + 1 < c_end) {  // O and the state read
         umma::mbar_arrive(bar_ss);
         ++kk;
       }
