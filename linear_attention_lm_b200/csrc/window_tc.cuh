@@ -11,11 +11,12 @@
 //   P = exp(S - m)   CUDA cores: thread r owns query row r; it reads the 96
 //                    TMEM columns covering its 64-key band, masks, takes the exact
 //                    row max, exponentiates, keeps the row sum l in a register
-//                    and writes P (bf16, zero outside the band) to shared memory
-//   O = P V          tcgen05, M=128, N=dh, K=192             -> TMEM (fp32)
+//                    and writes P (bf16 pairs, zero outside the band) back over
+//                    S in its own TMEM lane
+//   O = P V          tcgen05, A = P from TMEM, M=128, N=dh, K=192 -> TMEM (fp32)
 //   y = O / l        CUDA cores: TMEM -> 128B-swizzled staging tile -> TMA store.
-// P reuses the shared memory of Q and K, which are dead once S is computed, and
-// the y staging tile reuses that of P once O is complete.
+// Keeping P in TMEM leaves shared memory to the Q, K, V tiles (the y staging tile
+// reuses Q's once O is complete) and spares the tensor core the P reads.
 #pragma once
 
 #include "common.cuh"
@@ -31,11 +32,8 @@ template <int DH>
 struct WtLayout {
   static constexpr int kQ = 0;                              // Q [128 x DH] K-major SW128
   static constexpr int kK = kQ + kWtQ * DH * 2;             // K [192 x DH] K-major SW128
-  static constexpr int kP = 0;                              // P [128 x 192] bf16 K-major (aliases Q,K)
-  static constexpr int kY = 0;                              // y [128 x DH] bf16 SW128 (aliases P)
-  static constexpr int kPBytes = kWtQ * kWtKeys * 2;
-  static constexpr int kQKEnd = kK + kWtKeys * DH * 2;
-  static constexpr int kV = (kQKEnd > kPBytes ? kQKEnd : kPBytes);  // V [192 x DH] MN-major SW128
+  static constexpr int kY = 0;                              // y [128 x DH] bf16 SW128 (over Q)
+  static constexpr int kV = kK + kWtKeys * DH * 2;          // V [192 x DH] MN-major SW128
   static constexpr int kBar = kV + kWtKeys * DH * 2;
   static constexpr int kBytes = kBar + 64;
   static constexpr size_t kSmem = kBytes + 1024;
@@ -90,7 +88,7 @@ __global__ void __launch_bounds__(kWtThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tm_lane = static_cast<uint32_t>(warp * 32) << 16;
   const uint32_t sQ = umma::smem_u32(sm + Lay::kQ), sK = umma::smem_u32(sm + Lay::kK),
-                 sV = umma::smem_u32(sm + Lay::kV), sP = umma::smem_u32(sm + Lay::kP);
+                 sV = umma::smem_u32(sm + Lay::kV);
 
   // ---- S = Q K^T ----------------------------------------------------------------
   if (tid == 0) {
@@ -144,25 +142,40 @@ __global__ void __launch_bounds__(kWtThreads, 1)
       lp[i & 3] += sv[i];
     }
     l_row = (lp[0] + lp[1]) + (lp[2] + lp[3]);  // >= 1: the row maximum contributes exp2(0)
-    // P row r (K-major, 24 chunks of 8 keys): chunks 4w .. 4w+11 carry the band
-    uint8_t* prow = sm + Lay::kP + (r >> 3) * (kWtKeys / 8) * 128 + (r & 7) * 16;
-    __syncwarp();
-    for (int kc = 0; kc < 4 * warp; ++kc)
-      *reinterpret_cast<uint4*>(prow + kc * 128) = make_uint4(0, 0, 0, 0);
-    for (int kc = 4 * warp + 12; kc < kWtKeys / 8; ++kc)
-      *reinterpret_cast<uint4*>(prow + kc * 128) = make_uint4(0, 0, 0, 0);
+    // P (bf16 pairs, column j = keys 2j, 2j+1) replaces S in this lane: the band
+    // of quadrant w lands in columns [16w, 16w + 48), the rest of [0, 96) is zero
+    uint32_t pk[48], zero[32];
 #pragma unroll
-    for (int j = 0; j < 12; ++j) {
-      uint32_t pk[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const __nv_bfloat162 b2 = __floats2bfloat162_rn(sv[8 * j + 2 * e], sv[8 * j + 2 * e + 1]);
-        pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
-      }
-      *reinterpret_cast<uint4*>(prow + (4 * warp + j) * 128) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    for (int j = 0; j < 48; ++j) {
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(sv[2 * j], sv[2 * j + 1]);
+      pk[j] = *reinterpret_cast<const uint32_t*>(&b2);
     }
+#pragma unroll
+    for (int j = 0; j < 32; ++j) zero[j] = 0u;
+    const uint32_t prow = tmem + Lay::kTmS + tm_lane;
+    if (warp == 0) {
+      umma::tmem_st32_nowait(prow, pk);
+      umma::tmem_st16_nowait(prow + 32, pk + 32);
+      umma::tmem_st32_nowait(prow + 48, zero);
+      umma::tmem_st16_nowait(prow + 80, zero);
+    } else if (warp == 1) {
+      umma::tmem_st16_nowait(prow, zero);
+      umma::tmem_st32_nowait(prow + 16, pk);
+      umma::tmem_st16_nowait(prow + 48, pk + 32);
+      umma::tmem_st32_nowait(prow + 64, zero);
+    } else if (warp == 2) {
+      umma::tmem_st32_nowait(prow, zero);
+      umma::tmem_st32_nowait(prow + 32, pk);
+      umma::tmem_st16_nowait(prow + 64, pk + 32);
+      umma::tmem_st16_nowait(prow + 80, zero);
+    } else {
+      umma::tmem_st32_nowait(prow, zero);
+      umma::tmem_st16_nowait(prow + 32, zero);
+      umma::tmem_st32_nowait(prow + 48, pk);
+      umma::tmem_st16_nowait(prow + 80, pk + 32);
+    }
+    umma::tmem_wait_st();
   }
-  umma::fence_async_smem();
   umma::tc_fence_before();
   __syncthreads();
   umma::tc_fence_after();
@@ -173,8 +186,8 @@ __global__ void __launch_bounds__(kWtThreads, 1)
     const uint32_t id = umma::idesc_bf16(kWtQ, DH, false, true);
 #pragma unroll
     for (int k0 = 0; k0 < kWtKeys; k0 += 16)
-      umma::mma_bf16(tmem + Lay::kTmO, umma::desc_kmajor_none(sP, k0, kWtKeys),
-                     umma::desc_mnmajor_sw128(sV, k0, kWtKeys), id, k0 > 0);
+      umma::mma_ts(tmem + Lay::kTmO, tmem + Lay::kTmS + k0 / 2,
+                   umma::desc_mnmajor_sw128(sV, k0, kWtKeys), id, k0 > 0);
     umma::mma_commit(bar_o);
   }
   __syncwarp();
