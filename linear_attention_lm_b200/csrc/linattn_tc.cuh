@@ -864,21 +864,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int t = tid - 2 * kTcGroup;
     const bool any_st = has_init || c_begin < c_end;
     if constexpr (Lay::kSt) {
-      // [S|z]^T -> shared memory as [feature][value column | z] (stride DV + 1),
+      // [S|z]^T -> shared memory as [feature][value column | z] (stride DV + 4),
       // then coalesced rows of the 273-row layout (or of the segment partial).
       // The feature-map buffers are free: every MMA has completed.
-      constexpr int kStr = DV + 1;
+      constexpr int kStr = DV + 4;  // keeps each feature row 16-byte aligned
       float* stage = reinterpret_cast<float*>(sm + Lay::kPhiK);
       int* rowmap = reinterpret_cast<int*>(stage + kSymFP * kStr);  // [273]: 2 f + (1 if / sqrt 2)
-      static_assert(Lay::kPhiKBuf * 40960 >= (kSymFP * (DV + 1) + kF) * 4, "export staging");
+      static_assert(Lay::kPhiKBuf * 40960 >= (kSymFP * kStr + kF) * 4, "export staging");
       if (quad < 3) {
+        // two TMEM round trips of 80 features each
 #pragma unroll 1
-        for (int g = 0; g < kSymFP / 32; ++g) {
-          float sv[32];
-          umma::tmem_ld32(tmem + Lay::kTmS0 + tm_lane + g * 32, sv);
+        for (int g = 0; g < 2; ++g) {
+          float sv[80];
+          umma::tmem_ld80(tmem + Lay::kTmS0 + tm_lane + g * 80, sv);
           if (t <= DV) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) stage[(g * 32 + i) * kStr + t] = any_st ? sv[i] : 0.0f;
+            for (int i = 0; i < 80; ++i) stage[(g * 80 + i) * kStr + t] = any_st ? sv[i] : 0.0f;
           }
         }
       }
@@ -904,8 +905,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int r = i / (DV / 4), j = (i - r * (DV / 4)) * 4;
             const int code = rowmap[r];
             const float sc = (code & 1) ? 0.70710678118654752f : 1.0f;
-            const float* src = stage + (code >> 1) * kStr + j;
-            skv[i] = make_float4(src[0] * sc, src[1] * sc, src[2] * sc, src[3] * sc);
+            const float4 v4 = *reinterpret_cast<const float4*>(stage + (code >> 1) * kStr + j);
+            skv[i] = make_float4(v4.x * sc, v4.y * sc, v4.z * sc, v4.w * sc);
           }
         }
         if (p.state_k) {
