@@ -142,18 +142,18 @@ __device__ __forceinline__ void decode_linear_block(const DecodeParams& p, int b
 
 // Shared-memory layout of a window CTA (bytes), for G heads of d_h = dh and
 // element size es: the K and V rings of each head (W rows), one mbarrier per
-// head, then q and the new k/v of each head, scores, partial outputs.
+// head, then q and the new k/v of each head, the weights and the reductions.
 struct DecodeWindowLayout {
-  int ring, bar, qs, kvn, pr, part, red, bytes;
+  int ring, bar, qs, kvn, pr, red, bytes;
   __host__ __device__ DecodeWindowLayout(int G, int dh, int W, int NT, int es) {
+    (void)NT;
     ring = W * dh * es;  // one ring; multiple of 16 for dh in {64, 128}
     bar = 2 * G * ring;
     qs = bar + 8 * G + 16;
     kvn = qs + 4 * G * dh;
     pr = kvn + ((2 * G * dh * es + 15) & ~15);
-    part = pr + 4 * 64;
-    red = part + 4 * NT;
-    bytes = red + 16;
+    red = pr + 4 * 64 * G;
+    bytes = red + 4 * 4 * G;
   }
 };
 
@@ -177,11 +177,14 @@ __device__ __forceinline__ void load16_f32<__nv_bfloat16>(const __nv_bfloat16* p
   }
 }
 
+// The G heads of a window CTA run side by side, 64 threads each (thread s owns
+// ring slot s for the scores and value columns s, s+64, ... for the output), so
+// the CTA needs four block barriers in all, whatever G.
 template <typename T>
 __device__ __forceinline__ void decode_window_block(const DecodeParams& p, int wblk, uint8_t* sm) {
   constexpr int VEC = 16 / sizeof(T);
   const int dh = p.dh, W = p.W, NT = blockDim.x, G = p.wg;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, lane = tid & 31;
   const int w0 = wblk * G;
   const int n_items = min(G, p.n_win - w0);
   const DecodeWindowLayout lay(G, dh, W, NT, sizeof(T));
@@ -190,7 +193,6 @@ __device__ __forceinline__ void decode_window_block(const DecodeParams& p, int w
   float* qs = reinterpret_cast<float*>(sm + lay.qs);
   T* kvn = reinterpret_cast<T*>(sm + lay.kvn);
   float* pr = reinterpret_cast<float*>(sm + lay.pr);
-  float* part = reinterpret_cast<float*>(sm + lay.part);
   float* red = reinterpret_cast<float*>(sm + lay.red);
   const long long pos = p.pos;
   const int slot = (int)(pos % W);
@@ -218,66 +220,70 @@ __device__ __forceinline__ void decode_window_block(const DecodeParams& p, int w
   }
   __syncthreads();
 
-  const float scale = rsqrtf((float)dh);
-  const int tps = NT / 64, s_me = tid / tps, u = tid % tps, dpt = dh / tps;
-  const int ng = NT / dh, c_me = tid % dh, grp = tid / dh;
-  int g = 0;
-  for (; g < n_items; ++g) {
-    const bool ok = umma::mbar_wait(bar + g, 0);
+  const int g = tid >> 6, s = tid & 63;  // head and slot / column of this thread
+  const bool active = g < n_items;
+  T* K = rings + (size_t)g * 2 * W * dh;
+  T* V = K + W * dh;
+  bool ok = true;
+  if (active) {
+    ok = umma::mbar_wait(bar + g, 0);
     if (!ok) record_device_error(BASED_ERR_TIMEOUT);
-    if (__syncthreads_or(!ok)) break;
-    T* K = rings + (size_t)g * 2 * W * dh;
-    T* V = K + W * dh;
-    if (tid < dh) {
-      const T kt = kvn[2 * (g * dh + tid)], vt = kvn[2 * (g * dh + tid) + 1];
-      const size_t ro = (size_t)(w0 + g) * W * dh + (size_t)slot * dh + tid;
-      K[slot * dh + tid] = kt;
-      V[slot * dh + tid] = vt;
+  }
+  // every head's loads must be complete (or abandoned) before any thread leaves
+  if (__syncthreads_or(!ok)) {
+    if (tid == 0)
+      for (int i = 0; i < n_items; ++i) umma::mbar_wait(bar + i, 0);
+    return;
+  }
+  if (active) {
+    // the new k/v into slot pos mod W, in shared memory and in the ring
+    for (int c = s; c < dh; c += 64) {
+      const T kt = kvn[2 * (g * dh + c)], vt = kvn[2 * (g * dh + c) + 1];
+      const size_t ro = (size_t)(w0 + g) * W * dh + (size_t)slot * dh + c;
+      K[slot * dh + c] = kt;
+      V[slot * dh + c] = vt;
       kring[ro] = kt;
       vring[ro] = vt;
     }
-    __syncthreads();
-    // scores: tps consecutive threads share slot s_me, dpt dims each
-    float a = 0.0f;
-    if (s_me < nvalid) {
-      const T* kr = K + s_me * dh + u * dpt;
-      const float* qg = qs + g * dh + u * dpt;
-      for (int e = 0; e < dpt; e += VEC) {
-        float kf[VEC];
-        load16_f32<T>(kr + e, kf);
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) a = fmaf(qg[e + i], kf[i], a);
-      }
-    }
-    for (int o = tps >> 1; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-    if (u == 0) pr[s_me] = a * scale;
-    __syncthreads();
-    if (warp == 0) {
-      const float a0 = lane < nvalid ? pr[lane] : -INFINITY;
-      const float a1 = lane + 32 < nvalid ? pr[lane + 32] : -INFINITY;
-      const float m = warp_max(fmaxf(a0, a1));
-      const float e0 = lane < nvalid ? expf(a0 - m) : 0.0f;
-      const float e1 = lane + 32 < nvalid ? expf(a1 - m) : 0.0f;
-      pr[lane] = e0;
-      pr[lane + 32] = e1;
-      const float sum = warp_sum(e0 + e1);
-      if (lane == 0) red[0] = sum;
-    }
-    __syncthreads();
-    // output column c_me over the slots of group grp
+  }
+  __syncthreads();
+  // score of slot s: 16-byte chunks taken in an order rotated by s, so the eight
+  // lanes of a shared-memory phase touch eight different bank groups
+  float a = -INFINITY;
+  if (active && s < nvalid) {
+    const int nch = dh / VEC;
+    const T* kr = K + s * dh;
+    const float* qg = qs + g * dh;
     float acc = 0.0f;
-    for (int s = grp; s < nvalid; s += ng) acc = fmaf(pr[s], to_f32(V[s * dh + c_me]), acc);
-    part[tid] = acc;
-    __syncthreads();
-    if (tid < dh) {
-      float y = 0.0f;
-      for (int j = 0; j < ng; ++j) y += part[j * dh + tid];
-      static_cast<T*>(p.wout)[(size_t)(w0 + g) * dh + tid] = from_f32<T>(y / red[0]);
+    for (int c = 0; c < nch; ++c) {
+      const int ch = (c + s) & (nch - 1);
+      float kf[VEC];
+      load16_f32<T>(kr + ch * VEC, kf);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) acc = fmaf(qg[ch * VEC + i], kf[i], acc);
+    }
+    a = acc * rsqrtf((float)dh);
+  }
+  // softmax over the head's 64 slots (two warps)
+  const int hw = (tid >> 5) & 1;  // warp within the head
+  float m = warp_max(a);
+  if (active && lane == 0) red[g * 4 + hw] = m;
+  __syncthreads();
+  if (active) m = fmaxf(red[g * 4], red[g * 4 + 1]);
+  const float e = (active && s < nvalid) ? expf(a - m) : 0.0f;
+  if (active) pr[g * 64 + s] = e;
+  const float es = warp_sum(e);
+  if (active && lane == 0) red[g * 4 + 2 + hw] = es;
+  __syncthreads();
+  if (active) {
+    const float inv = 1.0f / (red[g * 4 + 2] + red[g * 4 + 3]);
+    const float* pw = pr + g * 64;
+    for (int c = s; c < dh; c += 64) {
+      float acc = 0.0f;
+      for (int j = 0; j < nvalid; ++j) acc = fmaf(pw[j], to_f32(V[j * dh + c]), acc);
+      static_cast<T*>(p.wout)[(size_t)(w0 + g) * dh + c] = from_f32<T>(acc * inv);
     }
   }
-  // after an abort, loads of the heads not reached may still be in flight
-  if (tid == 0)
-    for (int i = g + 1; i < n_items; ++i) umma::mbar_wait(bar + i, 0);
 }
 
 template <typename T, int DV>
