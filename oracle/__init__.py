@@ -20,6 +20,11 @@ wrapper names the passage the C routine follows:
 * ``decode_linear`` / ``decode_window`` -- one recurrent generation step
   over the KV / K states (blog post part 2, state-size paragraph) and over a
   ring cache of the last W window keys/values.
+* ``proj_heads`` -- x W^T split into heads (blog post part 2, state-size
+  paragraph: the states are made smaller by projections of the input).
+* ``baseconv`` -- y = linear(x) (.) conv(h, x) ("Базированная модель, часть 1",
+  section "Кто виноват?"), a dense map with bias gated by a causal per-channel
+  convolution.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (closed forms, brute force on tiny inputs, library softmax attention,
@@ -92,6 +97,11 @@ def _load():
                 _dp, _dp, _dp, _dp, _dp, ctypes.c_longlong, ctypes.c_int, ctypes.c_int,
                 ctypes.c_int, _dp]
             lib.oracle_decode_window.restype = None
+            _i = ctypes.c_int
+            lib.oracle_proj_heads.argtypes = [_dp, _dp, _dp, _i, _i, _i, _i, _i, _i]
+            lib.oracle_proj_heads.restype = None
+            lib.oracle_baseconv.argtypes = [_dp, _dp, _dp, _dp, _dp, _i, _i, _i, _i, _i]
+            lib.oracle_baseconv.restype = None
             _lib = lib
     return _lib
 
@@ -218,4 +228,31 @@ def decode_window(q, k, v, k_ring, v_ring, pos: int, window: int = 64):
     y = np.empty(q.shape, dtype=np.float64)
     _load().oracle_decode_window(_ptr(q), _ptr(k), _ptr(v), _ptr(k_ring), _ptr(v_ring),
                                  int(pos), n, dh, int(window), _ptr(y))
+    return y
+
+
+def proj_heads(x, w, H: int, threads: int | None = None) -> np.ndarray:
+    """x [B, L, Dm], w [H*D, Dm] -> y [B, H, L, D] = x W^T split into heads."""
+    x, w = _f64(x), _f64(w)
+    B, L, Dm = x.shape
+    N = w.shape[0]
+    if w.shape[1] != Dm or N % H:
+        raise ValueError("w must be [H*D, Dm]")
+    D = N // H
+    y = np.zeros((B, H, L, D), dtype=np.float64)
+    _load().oracle_proj_heads(_ptr(x), _ptr(w), _ptr(y), B, L, Dm, H, D,
+                              threads or default_threads())
+    return y
+
+
+def baseconv(x, w, bias, h, threads: int | None = None) -> np.ndarray:
+    """x [B, L, D], w [D, D], bias [D], h [D, K] -> y [B, L, D]."""
+    x, w, bias, h = _f64(x), _f64(w), _f64(bias), _f64(h)
+    B, L, D = x.shape
+    if w.shape != (D, D) or bias.shape != (D,) or h.ndim != 2 or h.shape[0] != D:
+        raise ValueError("shapes: w [D, D], bias [D], h [D, K]")
+    K = h.shape[1]
+    y = np.zeros((B, L, D), dtype=np.float64)
+    _load().oracle_baseconv(_ptr(x), _ptr(w), _ptr(bias), _ptr(h), _ptr(y), B, L, D, K,
+                            threads or default_threads())
     return y
