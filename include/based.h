@@ -173,6 +173,34 @@ based_status_t based_decode_step(const void* q, const void* k, const void* v,
                                  based_dtype_t dt, float eps, based_stream_t stream);
 
 /*
+ * Per-head input projection ("Базированная модель, часть 2", the paragraph on
+ * the size of the hidden state: the KV and K states are made smaller by
+ * projections of the layer input):
+ *   y[b][h][t][d] = sum_k x[b][t][k] * w[h*D + d][k]
+ *   x  [B, L, d_model]  bf16      w  [H*D, d_model]  bf16 (one output feature per row)
+ *   y  [B, H, L, D]     bf16 (written)
+ * bf16 only (BASED_ERR_UNSUPPORTED otherwise).  Requires d_model % 64 == 0,
+ * (H*D) % 256 == 0 and D % 8 == 0 (else BASED_ERR_UNSUPPORTED).  Accumulates
+ * in fp32 on the tensor cores and rounds once to bf16.
+ */
+based_status_t based_proj_heads_fwd(const void* x, const void* w, void* y, int B, int L,
+                                    int d_model, int H, int D, based_dtype_t dt,
+                                    based_stream_t stream);
+
+/*
+ * BaseConv block ("Базированная модель, часть 1", section "Кто виноват?":
+ * y = linear(x) (.) conv(h, x)), with a dense D x D map plus bias and a
+ * causal per-channel convolution of K taps:
+ *   y[b][t][c] = (sum_k x[b][t][k] w[c][k] + bias[c])
+ *              * sum_{j=0}^{min(K-1, t)} taps[c][j] x[b][t-j][c]
+ *   x, y  [B, L, D]  bf16      w  [D, D]  bf16      bias [D], taps [D, K]  fp32
+ * bf16 only; requires D % 256 == 0 and 1 <= K <= 8 (else BASED_ERR_UNSUPPORTED).
+ */
+based_status_t based_baseconv_fwd(const void* x, const void* w, const float* bias,
+                                  const float* taps, void* y, int B, int L, int D, int K,
+                                  based_dtype_t dt, based_stream_t stream);
+
+/*
  * Synchronise `stream`, then read and clear the library's device status word
  * on the current device.  Returns BASED_OK, or the first error a kernel
  * recorded since the last call (BASED_ERR_TIMEOUT), or BASED_ERR_CUDA if the

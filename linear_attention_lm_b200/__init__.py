@@ -32,7 +32,7 @@ EXPORTED_SYMBOLS = ("based_abi_version", "based_status_string",
                     "based_linattn_workspace_bytes", "based_linattn_fwd",
                     "based_linattn_fwd_noalloc",
                     "based_window_attn_fwd", "based_window_ring_fill", "based_decode_step",
-                    "based_get_device_error")
+                    "based_proj_heads_fwd", "based_baseconv_fwd", "based_get_device_error")
 
 
 class BasedError(RuntimeError):
@@ -72,9 +72,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.based_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                           _vp, _vp, _ll, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                                           _vp]
+        lib.based_proj_heads_fwd.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
+        lib.based_baseconv_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
         lib.based_get_device_error.argtypes = [_vp]
         for name in ("based_linattn_fwd", "based_linattn_fwd_noalloc", "based_window_attn_fwd",
-                     "based_window_ring_fill", "based_decode_step", "based_get_device_error"):
+                     "based_window_ring_fill", "based_decode_step", "based_proj_heads_fwd",
+                     "based_baseconv_fwd", "based_get_device_error"):
             getattr(lib, name).restype = _i
         _lib = lib
         return lib
@@ -216,6 +219,30 @@ def based_decode_step(q, k, v, state_kv, state_k, out, wq=None, wk=None, wv=None
     _check("based_decode_step", st)
 
 
+def based_proj_heads_fwd(x, w, y, stream=None):
+    """x [B, L, d_model], w [H*D, d_model] -> y [B, H, L, D] (bf16, written)."""
+    B, L, d_model = x.shape
+    _, H, _, D = y.shape
+    dt = _same_dtype(x, w, y)
+    with torch.cuda.device(x.device):
+        st = load_library().based_proj_heads_fwd(_ptr(x), _ptr(w), _ptr(y), B, L, d_model, H, D,
+                                                 dt, _stream(stream))
+    _check("based_proj_heads_fwd", st)
+    return y
+
+
+def based_baseconv_fwd(x, w, bias, taps, y, stream=None):
+    """x, y [B, L, D] bf16; w [D, D] bf16; bias [D], taps [D, K] float32."""
+    B, L, D = x.shape
+    K = taps.shape[-1]
+    dt = _same_dtype(x, w, y)
+    with torch.cuda.device(x.device):
+        st = load_library().based_baseconv_fwd(_ptr(x), _ptr(w), _f32(bias), _f32(taps), _ptr(y),
+                                               B, L, D, K, dt, _stream(stream))
+    _check("based_baseconv_fwd", st)
+    return y
+
+
 def based_get_device_error(stream=None) -> int:
     return load_library().based_get_device_error(_stream(stream))
 
@@ -247,3 +274,16 @@ def window_ring_fill(k, v, window: int = 64, stream=None):
     v_ring = torch.zeros_like(k_ring)
     based_window_ring_fill(k, v, k_ring, v_ring, window, stream=stream)
     return k_ring, v_ring
+
+
+def proj_heads(x, w, H: int, stream=None):
+    """x W^T split into H heads: [B, L, d_model] x [H*D, d_model] -> [B, H, L, D]."""
+    B, L, _ = x.shape
+    y = torch.empty((B, H, L, w.shape[0] // H), dtype=x.dtype, device=x.device)
+    return based_proj_heads_fwd(x, w, y, stream=stream)
+
+
+def baseconv(x, w, bias, taps, stream=None):
+    """linear(x) * conv(taps, x): [B, L, D] -> [B, L, D]."""
+    y = torch.empty_like(x)
+    return based_baseconv_fwd(x, w, bias, taps, y, stream=stream)

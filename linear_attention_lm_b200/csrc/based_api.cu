@@ -17,6 +17,7 @@
 #include "linattn_tc.cuh"
 #include "window_simt.cuh"
 #include "window_tc.cuh"
+#include "proj_tc.cuh"
 
 namespace based {
 
@@ -251,6 +252,18 @@ based_status_t launch_decode(DecodeParams p, cudaStream_t st) {
   return launch_status();
 }
 
+template <int Mode>
+based_status_t launch_proj(const void* x, const void* w, const ProjParams& p, cudaStream_t st) {
+  CUtensorMap xm, wm;
+  if (!make_rows_map(&xm, x, p.Kd, p.M, 1, kPjM) || !make_rows_map(&wm, w, p.Kd, p.N, 1, kPjN))
+    return BASED_ERR_CUDA;
+  auto kern = proj_tc_kernel<Mode>;
+  if (!set_smem(kern, PjLayout::kSmem)) return BASED_ERR_CUDA;
+  const dim3 grid((unsigned)((p.M + kPjM - 1) / kPjM), (unsigned)(p.N / kPjN));
+  kern<<<grid, kPjThreads, PjLayout::kSmem, st>>>(xm, wm, p);
+  return launch_status();
+}
+
 // ---------------------------------------------------------------------------
 // Allocation-free prefill (based_linattn_fwd_noalloc): the segment partials
 // live in this fixed array instead of a caller workspace.  Host code may not
@@ -445,6 +458,45 @@ based_status_t based_decode_step(const void* q, const void* k, const void* v, fl
   if (dt == BASED_F32)
     return wide ? launch_decode<float, 128>(p, st) : launch_decode<float, 64>(p, st);
   return wide ? launch_decode<__nv_bfloat16, 128>(p, st) : launch_decode<__nv_bfloat16, 64>(p, st);
+}
+
+based_status_t based_proj_heads_fwd(const void* x, const void* w, void* y, int B, int L,
+                                    int d_model, int H, int D, based_dtype_t dt,
+                                    based_stream_t stream) {
+  if (B < 0 || L < 0 || d_model <= 0 || H <= 0 || D <= 0) return BASED_ERR_INVALID_ARG;
+  if (dt != BASED_BF16 && dt != BASED_F32) return BASED_ERR_INVALID_ARG;
+  if (dt != BASED_BF16) return BASED_ERR_UNSUPPORTED;
+  if (d_model % kPjK != 0 || ((long long)H * D) % kPjN != 0 || D % 8 != 0)
+    return BASED_ERR_UNSUPPORTED;
+  const long long M = (long long)B * L;
+  if (M > 0x7fffffffLL || (long long)H * D > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
+  if (M == 0) return BASED_OK;
+  if (!x || !w || !y) return BASED_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return BASED_ERR_INVALID_ARG;
+  ProjParams p{};
+  p.y = static_cast<__nv_bfloat16*>(y);
+  p.M = (int)M; p.N = H * D; p.Kd = d_model; p.L = L; p.H = H; p.D = D;
+  return launch_proj<kProjHeads>(x, w, p, static_cast<cudaStream_t>(stream));
+}
+
+based_status_t based_baseconv_fwd(const void* x, const void* w, const float* bias,
+                                  const float* taps, void* y, int B, int L, int D, int K,
+                                  based_dtype_t dt, based_stream_t stream) {
+  if (B < 0 || L < 0 || D <= 0 || K <= 0) return BASED_ERR_INVALID_ARG;
+  if (dt != BASED_BF16 && dt != BASED_F32) return BASED_ERR_INVALID_ARG;
+  if (dt != BASED_BF16) return BASED_ERR_UNSUPPORTED;
+  if (D % kPjN != 0 || K > kPjMaxTaps) return BASED_ERR_UNSUPPORTED;
+  const long long M = (long long)B * L;
+  if (M > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
+  if (M == 0) return BASED_OK;
+  if (!x || !w || !bias || !taps || !y) return BASED_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return BASED_ERR_INVALID_ARG;
+  ProjParams p{};
+  p.x = static_cast<const __nv_bfloat16*>(x);
+  p.y = static_cast<__nv_bfloat16*>(y);
+  p.bias = bias; p.taps = taps;
+  p.M = (int)M; p.N = D; p.Kd = D; p.L = L; p.K = K;
+  return launch_proj<kBaseConv>(x, w, p, static_cast<cudaStream_t>(stream));
 }
 
 based_status_t based_get_device_error(based_stream_t stream) {

@@ -387,21 +387,21 @@ typedef struct {
  * projections of the input).  For sequence b and head hh:
  *     y[b][hh][t][d] = sum_k x[b][t][k] * w[hh*D + d][k]
  * i.e. x W^T split into H heads of D features, heads before positions. */
-static void proj_heads_seq(void* p, int b) {
+static void proj_heads_seq(void* p, int bh) {
     const proj_ctx* c = (const proj_ctx*)p;
-    for (int hh = 0; hh < c->H; ++hh)
-        for (int t = 0; t < c->L; ++t)
-            for (int d = 0; d < c->D; ++d) {
-                const double* xr = c->x + ((size_t)b * c->L + t) * c->Dm;
-                const double* wr = c->w + ((size_t)hh * c->D + d) * c->Dm;
-                c->y[(((size_t)b * c->H + hh) * c->L + t) * c->D + d] = dot(xr, wr, c->Dm);
-            }
+    const int b = bh / c->H, hh = bh % c->H;
+    for (int t = 0; t < c->L; ++t)
+        for (int d = 0; d < c->D; ++d) {
+            const double* xr = c->x + ((size_t)b * c->L + t) * c->Dm;
+            const double* wr = c->w + ((size_t)hh * c->D + d) * c->Dm;
+            c->y[(((size_t)b * c->H + hh) * c->L + t) * c->D + d] = dot(xr, wr, c->Dm);
+        }
 }
 
 void oracle_proj_heads(const double* x, const double* w, double* y, int B, int L, int Dm,
                        int H, int D, int nthreads) {
     proj_ctx c = {x, w, NULL, NULL, y, L, Dm, H, D, 0};
-    parallel_for(B, nthreads, proj_heads_seq, &c);
+    parallel_for(B * H, nthreads, proj_heads_seq, &c);
 }
 
 /* BaseConv ("Базированная модель, часть 1", section "Кто виноват?": the block
@@ -410,22 +410,21 @@ void oracle_proj_heads(const double* x, const double* w, double* y, int B, int L
  * convolution of each channel with its own filter of K taps:
  *     y[b][t][c] = (sum_k x[b][t][k] w[c][k] + bias[c])
  *                * sum_{j=0}^{min(K-1, t)} h[c][j] x[b][t-j][c]. */
-static void baseconv_seq(void* p, int b) {
+static void baseconv_seq(void* p, int bt) {
     const proj_ctx* c = (const proj_ctx*)p;
-    const int D = c->D;
-    for (int t = 0; t < c->L; ++t)
-        for (int ch = 0; ch < D; ++ch) {
-            const double* xr = c->x + ((size_t)b * c->L + t) * D;
-            const double lin = dot(xr, c->w + (size_t)ch * D, D) + c->bias[ch];
-            double conv = 0.0;
-            for (int j = 0; j < c->K && j <= t; ++j)
-                conv += c->h[(size_t)ch * c->K + j] * c->x[((size_t)b * c->L + t - j) * D + ch];
-            c->y[((size_t)b * c->L + t) * D + ch] = lin * conv;
-        }
+    const int D = c->D, t = bt % c->L;
+    for (int ch = 0; ch < D; ++ch) {
+        const double* xr = c->x + (size_t)bt * D;
+        const double lin = dot(xr, c->w + (size_t)ch * D, D) + c->bias[ch];
+        double conv = 0.0;
+        for (int j = 0; j < c->K && j <= t; ++j)
+            conv += c->h[(size_t)ch * c->K + j] * c->x[((size_t)bt - j) * D + ch];
+        c->y[(size_t)bt * D + ch] = lin * conv;
+    }
 }
 
 void oracle_baseconv(const double* x, const double* w, const double* bias, const double* h,
                      double* y, int B, int L, int D, int K, int nthreads) {
     proj_ctx c = {x, w, bias, h, y, L, D, 0, D, K};
-    parallel_for(B, nthreads, baseconv_seq, &c);
+    parallel_for(B * L, nthreads, baseconv_seq, &c);
 }

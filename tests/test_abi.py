@@ -121,6 +121,29 @@ def test_decode_host_validation(lib):
              1e-6, N) == UNSUPPORTED
 
 
+def test_proj_host_validation(lib):
+    f = lib.based_proj_heads_fwd
+    # x, w, y, B, L, d_model, H, D, dt, stream
+    assert f(FAKE, FAKE, FAKE, 1, 8, 1024, 16, 16, 0, None) == UNSUPPORTED   # fp32
+    assert f(FAKE, FAKE, FAKE, 1, 8, 1000, 16, 16, 1, None) == UNSUPPORTED   # d_model % 64
+    assert f(FAKE, FAKE, FAKE, 1, 8, 1024, 3, 16, 1, None) == UNSUPPORTED    # H*D % 256
+    assert f(FAKE, FAKE, FAKE, 1, 8, 1024, 64, 4, 1, None) == UNSUPPORTED    # D % 8
+    assert f(FAKE, FAKE, FAKE, -1, 8, 1024, 16, 16, 1, None) == INVALID
+    assert f(None, FAKE, FAKE, 1, 8, 1024, 16, 16, 1, None) == INVALID
+    assert f(None, None, None, 0, 8, 1024, 16, 16, 1, None) == 0             # nothing to do
+
+
+def test_baseconv_host_validation(lib):
+    f = lib.based_baseconv_fwd
+    # x, w, bias, taps, y, B, L, D, K, dt, stream
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 1024, 3, 0, None) == UNSUPPORTED  # fp32
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 1000, 3, 1, None) == UNSUPPORTED  # D % 256
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 1024, 9, 1, None) == UNSUPPORTED  # > 8 taps
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 1024, 0, 1, None) == INVALID
+    assert f(FAKE, FAKE, None, FAKE, FAKE, 1, 8, 1024, 3, 1, None) == INVALID
+    assert f(None, None, None, None, None, 1, 0, 1024, 3, 1, None) == 0
+
+
 def test_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 1, 8, 16, dtype=torch.bfloat16)
     v = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
