@@ -253,6 +253,10 @@ def run_ours(args, rank, world, dev):
 
     e2e = run_e2e(args, w, lab, dev, world, sets[0][0])
     decode = run_decode(args, lab, dev, world, peaks)
+    try:
+        projections = run_projections(args, lab, dev, world, peaks)
+    except Exception as exc:  # reported in the JSON line, never hidden
+        projections = {"error": f"{type(exc).__name__}: {exc}"}
     clocks = clk.summary()
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
@@ -268,6 +272,7 @@ def run_ours(args, rank, world, dev):
         "roofline": roofline,
         "e2e": e2e,
         "decode": decode,
+        "projections": projections,
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
     }
@@ -315,6 +320,68 @@ def run_e2e(args, w, lab, dev, world, x):
         ms = float(t.item())
     return {"value": round(world * w.B * w.L * n / (ms / 1e3), 1), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n}
+
+
+def run_projections(args, lab, dev, world, peaks):
+    """The step before the attention layers and the third layer type, each on
+    layer_360m's shapes (x [8, 2048, 1024] bf16, synthetic): the six per-head
+    input projections of one linear-attention and one window layer (q, k: 16
+    heads of 16; v and the window's q, k, v: 16 heads of 64) and one BaseConv
+    block (D = 1024, 3 taps).  Four rotating x buffers (128 MB) keep L2 cold."""
+    B, L, dm, H = 8, 2048, 1024, 16
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234)
+    xs = [torch.randn(B, L, dm, device=dev, generator=g).to(torch.bfloat16) for _ in range(4)]
+    heads = [16, 16, 64, 64, 64, 64]
+    ws = [(torch.randn(H * D, dm, device=dev, generator=g) * 0.02).to(torch.bfloat16) for D in heads]
+    ys = [torch.empty(B, H, L, D, device=dev, dtype=torch.bfloat16) for D in heads]
+    wb = (torch.randn(dm, dm, device=dev, generator=g) * 0.03).to(torch.bfloat16)
+    bias = torch.randn(dm, device=dev, generator=g) * 0.1
+    taps = torch.randn(dm, 3, device=dev, generator=g) * 0.5
+    yb = torch.empty(B, L, dm, device=dev, dtype=torch.bfloat16)
+    n = max(10, min(args.steps, 200))
+
+    def timed(fn):
+        for i in range(max(3, args.warmup)):
+            fn(i)
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for i in range(n):
+            fn(i)
+        e.record()
+        torch.cuda.synchronize()
+        ms = s.elapsed_time(e) / n
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    def proj_step(i):
+        x = xs[i % 4]
+        for w, y in zip(ws, ys):
+            lab.based_proj_heads_fwd(x, w, y)
+
+    def conv_step(i):
+        lab.based_baseconv_fwd(xs[i % 4], wb, bias, taps, yb)
+
+    out = {}
+    peak = peaks["bf16_tflops"]
+    for name, fn, flops, launches, what in (
+            ("proj", proj_step, 2.0 * B * L * dm * H * sum(heads), len(heads),
+             "six per-head projections of x [8, 2048, 1024]: q, k 16x16; v 16x64; window q, k, v 16x64"),
+            ("baseconv", conv_step, 2.0 * B * L * dm * dm, 1,
+             "BaseConv block, x [8, 2048, 1024], dense 1024x1024 + bias, 3 causal taps")):
+        ms = timed(fn)
+        tf = flops / (ms / 1e3) / 1e12
+        out[name] = {"workload": what, "ms_per_step": round(ms, 5), "launches_per_step": launches,
+                     "tokens_per_s": round(world * B * L / (ms / 1e3), 1),
+                     "roofline": {"kernel": "proj_tc", "bound": "tensor", "achieved": round(tf, 1),
+                                  "peak": peak, "unit": "TFLOP/s", "frac": round(tf / peak, 4),
+                                  "traffic": None, "peak_source": peaks["source"]}}
+    assert lab.based_get_device_error() == 0
+    return out
 
 
 def run_decode(args, lab, dev, world, peaks):

@@ -253,14 +253,24 @@ based_status_t launch_decode(DecodeParams p, cudaStream_t st) {
 }
 
 template <int Mode>
-based_status_t launch_proj(const void* x, const void* w, const ProjParams& p, cudaStream_t st) {
-  CUtensorMap xm, wm;
+based_status_t launch_proj(const void* x, const void* w, ProjParams p, cudaStream_t st) {
+  CUtensorMap xm, wm, hm;
   if (!make_rows_map(&xm, x, p.Kd, p.M, 1, kPjM) || !make_rows_map(&wm, w, p.Kd, p.N, 1, kPjN))
     return BASED_ERR_CUDA;
+  if (Mode == kBaseConv) {
+    if (!make_rows_map(&hm, x, p.Kd, p.M, 1, kPjHaloRows)) return BASED_ERR_CUDA;
+  } else {
+    hm = xm;  // unused
+  }
   auto kern = proj_tc_kernel<Mode>;
-  if (!set_smem(kern, PjLayout::kSmem)) return BASED_ERR_CUDA;
-  const dim3 grid((unsigned)((p.M + kPjM - 1) / kPjM), (unsigned)(p.N / kPjN));
-  kern<<<grid, kPjThreads, PjLayout::kSmem, st>>>(xm, wm, p);
+  if (!set_smem(kern, PjLayout<Mode>::kSmem)) return BASED_ERR_CUDA;
+  p.n_tiles_n = p.N / kPjN;
+  const long long tiles = (long long)((p.M + kPjM - 1) / kPjM) * p.n_tiles_n;
+  if (tiles > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
+  p.total_tiles = (int)tiles;
+  const long long sms = device_sm_count();
+  const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
+  kern<<<grid, kPjThreads, PjLayout<Mode>::kSmem, st>>>(xm, wm, hm, p);
   return launch_status();
 }
 
