@@ -48,6 +48,24 @@ def load_peaks():
 
 
 # ---------------------------------------------------------------------------
+# replicas: one independent copy of the workload per rank, no data exchange
+# ---------------------------------------------------------------------------
+
+def max_over_ranks(ms: float, dev, world: int) -> float:
+    """The slowest rank's time (every rank gets the same answer)."""
+    if world <= 1:
+        return float(ms)
+    t = torch.tensor([float(ms)], device=dev, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_rate(units_per_rank: float, ms: float, world: int) -> float:
+    """Whole-job throughput: all ranks' units over the slowest rank's time."""
+    return world * units_per_rank / (ms / 1e3)
+
+
+# ---------------------------------------------------------------------------
 # DRAM traffic per launch from the committed ncu captures (profiles/traffic.json),
 # reported only while the headers that define the kernel's code are unchanged
 # since the capture
@@ -230,13 +248,8 @@ def run_ours(args, rank, world, dev):
     t_lin = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
     t_win = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
     assert lab.based_get_device_error() == 0
-    elapsed_max = elapsed_ms
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_max = float(t.item())
-    tokens = world * w.B * w.L * args.steps
-    value = tokens / (elapsed_max / 1e3)
+    elapsed_max = max_over_ranks(elapsed_ms, dev, world)
+    value = replica_rate(w.B * w.L * args.steps, elapsed_max, world)
 
     # roofline of the dominant kernel (both are HBM-bound by algorithmic bytes)
     kern = {"linattn_prefill": (linattn_bytes(w), t_lin), "window_attn": (window_bytes(w), t_win)}
@@ -339,10 +352,7 @@ def run_e2e(args, w, lab, dev, world, x):
     end.record(s_out)  # the last device->host copy waits on everything before it
     torch.cuda.synchronize()
     ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dev, world)
     return {"value": round(world * w.B * w.L * n / (ms / 1e3), 1), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n,
             "pipelined": "h2d(i+1) | kernels(i) | d2h(i-1) on three streams"}
@@ -378,10 +388,7 @@ def run_projections(args, lab, dev, world, peaks):
         e.record()
         torch.cuda.synchronize()
         ms = s.elapsed_time(e) / n
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            ms = float(t.item())
+        ms = max_over_ranks(ms, dev, world)
         return ms
 
     def proj_step(i):
@@ -444,10 +451,7 @@ def run_decode(args, lab, dev, world, peaks):
     e.record()
     torch.cuda.synchronize()
     ms = s.elapsed_time(e) / n
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dev, world)
     b = decode_bytes(w)
     ach = b / (ms / 1e3) / 1e9
     return {"value": round(world * w.B / (ms / 1e3), 1), "unit": "tokens/s",
