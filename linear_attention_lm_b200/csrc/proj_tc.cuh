@@ -46,7 +46,10 @@ struct PjLayout {
   static constexpr int kHalo = kB + kStages * kStageB;            // [4][136 rows][128 B] SW128
   static constexpr int kHaloBlock = kPjHaloRows * 128;
   static constexpr int kHaloBytes = Mode == kBaseConv ? 4 * kHaloBlock : 0;
-  static constexpr int kBar = kHalo + kHaloBytes;
+  // BaseConv: the tile's taps, transposed to [tap][column], and its bias
+  static constexpr int kTaps = kHalo + kHaloBytes;
+  static constexpr int kBias = kTaps + (Mode == kBaseConv ? kPjMaxTaps * kPjN * 4 : 0);
+  static constexpr int kBar = kBias + (Mode == kBaseConv ? kPjN * 4 : 0);
   static constexpr int kBytes = kBar + 256;
   static constexpr size_t kSmem = kBytes + 1024;
   static_assert(kB % 1024 == 0 && kHalo % 1024 == 0 && kHaloBlock % 1024 == 0,
@@ -87,6 +90,8 @@ __global__ void __launch_bounds__(kPjThreads, 1)
   uint64_t* bar_done = bars + 2 * S + 6;   // every MMA issued has completed (commit)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 7);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * S + 8);
+  uint64_t* bar_tready = bars + 2 * S + 9;   // taps and bias of the tile written (epilogue)
+  uint64_t* bar_tfree = bars + 2 * S + 10;   // taps and bias of the tile no longer read
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int first = blockIdx.x, step = gridDim.x;
@@ -105,6 +110,8 @@ __global__ void __launch_bounds__(kPjThreads, 1)
     umma::mbar_init(bar_hfull, 1);
     umma::mbar_init(bar_hempty, kPjM);
     umma::mbar_init(bar_done, 1);
+    umma::mbar_init(bar_tready, kPjM);
+    umma::mbar_init(bar_tfree, kPjM);
     *abort_flag = 0;
     umma::fence_mbar_init();
   }
@@ -199,6 +206,19 @@ __global__ void __launch_bounds__(kPjThreads, 1)
       if (!umma::mbar_wait(bar_afull + a, (k >> 1) & 1)) { fail(); break; }
       if (Mode == kBaseConv && !umma::mbar_wait(bar_hfull, k & 1)) { fail(); break; }
       umma::tc_fence_after();
+      float* tapsT = reinterpret_cast<float*>(sm + Lay::kTaps);
+      float* bias_s = reinterpret_cast<float*>(sm + Lay::kBias);
+      if (Mode == kBaseConv) {
+        // this tile's taps and bias into shared memory, once every epilogue
+        // thread has finished reading the previous tile's
+        if (k >= 1 && !umma::mbar_wait(bar_tfree, (k - 1) & 1)) { fail(); break; }
+        for (int c = r; c < kPjN; c += kPjM) {
+          for (int j = 0; j < p.K; ++j) tapsT[j * kPjN + c] = __ldg(p.taps + (size_t)(n0 + c) * p.K + j);
+          bias_s[c] = __ldg(p.bias + n0 + c);
+        }
+        umma::mbar_arrive(bar_tready);
+        if (!umma::mbar_wait(bar_tready, k & 1)) { fail(); break; }
+      }
       const int m = m0 + r;
       const int b = m / p.L, t = m - (m / p.L) * p.L;
 #pragma unroll 1
@@ -228,16 +248,22 @@ __global__ void __launch_bounds__(kPjThreads, 1)
             for (int j = 0; j < p.K && j <= t; ++j) {
               const int hr = r + kPjMaxTaps - j;
               const uint4 xv = *reinterpret_cast<const uint4*>(hb + hr * 128 + ((chunk ^ (hr & 7)) << 4));
+              const float4 h0 = *reinterpret_cast<const float4*>(tapsT + j * kPjN + cl);
+              const float4 h1 = *reinterpret_cast<const float4*>(tapsT + j * kPjN + cl + 4);
+              const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
               const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[e]));
-                conv[2 * e] = fmaf(__ldg(p.taps + (size_t)(n + 2 * e) * p.K + j), f.x, conv[2 * e]);
-                conv[2 * e + 1] = fmaf(__ldg(p.taps + (size_t)(n + 2 * e + 1) * p.K + j), f.y, conv[2 * e + 1]);
+                conv[2 * e] = fmaf(hv[2 * e], f.x, conv[2 * e]);
+                conv[2 * e + 1] = fmaf(hv[2 * e + 1], f.y, conv[2 * e + 1]);
               }
             }
+            const float4 b0 = *reinterpret_cast<const float4*>(bias_s + cl);
+            const float4 b1 = *reinterpret_cast<const float4*>(bias_s + cl + 4);
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = (v[e] + __ldg(p.bias + n + e)) * conv[e];
+            for (int e = 0; e < 8; ++e) v[e] = (v[e] + bv[e]) * conv[e];
             dst = (size_t)m * p.N + n;
           }
           uint32_t pk[4];
@@ -251,7 +277,10 @@ __global__ void __launch_bounds__(kPjThreads, 1)
       }
       umma::tc_fence_before();
       umma::mbar_arrive(bar_aempty + a);
-      if (Mode == kBaseConv) umma::mbar_arrive(bar_hempty);
+      if (Mode == kBaseConv) {
+        umma::mbar_arrive(bar_hempty);
+        umma::mbar_arrive(bar_tfree);
+      }
     }
   }
   umma::tc_fence_before();
