@@ -17,8 +17,9 @@ def main():
     local_ms = 2.0 + 3.5 * rank  # the ranks finish at different times
     ms = bench.max_over_ranks(local_ms, torch.device("cpu"), world)
     rate = bench.replica_rate(1000, ms, world)
-    print(json.dumps({"rank": rank, "world": world, "local_ms": local_ms, "ms": ms, "rate": rate}),
-          flush=True)
+    # one file per rank: the ranks share stdout, where their lines could interleave
+    with open(os.path.join(os.environ["REPLICA_OUT"], f"rank{rank}.json"), "w") as f:
+        json.dump({"rank": rank, "world": world, "local_ms": local_ms, "ms": ms, "rate": rate}, f)
     torch.distributed.destroy_process_group()
 
 

@@ -16,14 +16,14 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def test_max_over_ranks_and_rate_with_two_gloo_ranks():
+def test_max_over_ranks_and_rate_with_two_gloo_ranks(tmp_path):
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
            "--master-addr", "127.0.0.1", "--master-port", str(_free_port()),
            os.path.join(ROOT, "tests", "_replica_worker.py")]
-    env = dict(os.environ, OMP_NUM_THREADS="1")
+    env = dict(os.environ, OMP_NUM_THREADS="1", REPLICA_OUT=str(tmp_path))
     out = subprocess.run(cmd, capture_output=True, text=True, timeout=300, env=env, cwd=ROOT)
     assert out.returncode == 0, out.stderr[-2000:]
-    lines = [json.loads(l) for l in out.stdout.splitlines() if l.startswith("{")]
+    lines = [json.loads((tmp_path / f"rank{r}.json").read_text()) for r in range(2)]
     assert sorted(d["rank"] for d in lines) == [0, 1]
     slowest = max(d["local_ms"] for d in lines)
     for d in lines:
