@@ -173,6 +173,22 @@ based_status_t based_decode_step(const void* q, const void* k, const void* v,
                                  based_dtype_t dt, float eps, based_stream_t stream);
 
 /*
+ * Gradient of based_linattn_fwd's output (the map the "based/train" README's
+ * training views share; see based_linattn_fwd):
+ *   w_ts = 1 + u + u^2/2, u = q_t.k_s/sqrt(d_feat), s <= t; y_t = sum_s w_ts v_s / (sum_s w_ts + eps)
+ * Given dy = dL/dy returns dq, dk, dv (fp32) on CUDA cores over the quadratic form.
+ *   q, k [B, H, L, d_feat]   v, dy [B, H, L, d_v]   dt (d_feat == 16, d_v in {64, 128})
+ *   dq, dk [B, H, L, d_feat] fp32,  dv [B, H, L, d_v] fp32 (written)
+ *   workspace: device memory of based_linattn_bwd_workspace_bytes() bytes
+ *   (BASED_ERR_WORKSPACE if smaller); its contents are scratch.
+ */
+size_t based_linattn_bwd_workspace_bytes(int B, int H, int L, int d_v);
+based_status_t based_linattn_bwd(const void* q, const void* k, const void* v, const void* dy,
+                                 float* dq, float* dk, float* dv, int B, int H, int L,
+                                 int d_feat, int d_v, based_dtype_t dt, float eps,
+                                 void* workspace, size_t workspace_bytes, based_stream_t stream);
+
+/*
  * Per-head input projection ("Базированная модель, часть 2", the paragraph on
  * the size of the hidden state: the KV and K states are made smaller by
  * projections of the layer input):

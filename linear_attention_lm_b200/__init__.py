@@ -32,7 +32,9 @@ EXPORTED_SYMBOLS = ("based_abi_version", "based_status_string",
                     "based_linattn_workspace_bytes", "based_linattn_fwd",
                     "based_linattn_fwd_noalloc",
                     "based_window_attn_fwd", "based_window_ring_fill", "based_decode_step",
-                    "based_proj_heads_fwd", "based_baseconv_fwd", "based_get_device_error")
+                    "based_proj_heads_fwd", "based_baseconv_fwd",
+                    "based_linattn_bwd_workspace_bytes", "based_linattn_bwd",
+                    "based_get_device_error")
 
 
 class BasedError(RuntimeError):
@@ -72,12 +74,16 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.based_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                           _vp, _vp, _ll, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                                           _vp]
+        lib.based_linattn_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i]
+        lib.based_linattn_bwd_workspace_bytes.restype = _sz
+        lib.based_linattn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                                          _i, _f, _vp, _sz, _vp]
         lib.based_proj_heads_fwd.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
         lib.based_baseconv_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
         lib.based_get_device_error.argtypes = [_vp]
         for name in ("based_linattn_fwd", "based_linattn_fwd_noalloc", "based_window_attn_fwd",
                      "based_window_ring_fill", "based_decode_step", "based_proj_heads_fwd",
-                     "based_baseconv_fwd", "based_get_device_error"):
+                     "based_baseconv_fwd", "based_linattn_bwd", "based_get_device_error"):
             getattr(lib, name).restype = _i
         _lib = lib
         return lib
@@ -219,6 +225,30 @@ def based_decode_step(q, k, v, state_kv, state_k, out, wq=None, wk=None, wv=None
     _check("based_decode_step", st)
 
 
+def based_linattn_bwd_workspace_bytes(B, H, L, d_v) -> int:
+    n = load_library().based_linattn_bwd_workspace_bytes(B, H, L, d_v)
+    if n == ctypes.c_size_t(-1).value:
+        raise BasedError("based_linattn_bwd_workspace_bytes", 1)
+    return n
+
+
+def based_linattn_bwd(q, k, v, dy, dq, dk, dv, eps: float = 1e-6, workspace=None, stream=None):
+    """Gradients dq, dk, dv (float32, written) of based_linattn_fwd given dy."""
+    B, H, L, d = q.shape
+    d_v = v.shape[-1]
+    dt = _same_dtype(q, k, v, dy)
+    if workspace is None:
+        workspace = torch.empty(based_linattn_bwd_workspace_bytes(B, H, L, d_v) or 16,
+                                dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    with torch.cuda.device(q.device):
+        st = load_library().based_linattn_bwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(dy), _f32(dq), _f32(dk), _f32(dv), B, H, L, d, d_v,
+            dt, float(eps), _ptr(workspace), ws_bytes, _stream(stream))
+    _check("based_linattn_bwd", st)
+    return dq, dk, dv
+
+
 def based_proj_heads_fwd(x, w, y, stream=None):
     """x [B, L, d_model], w [H*D, d_model] -> y [B, H, L, D] (bf16, written)."""
     B, L, d_model = x.shape
@@ -287,3 +317,11 @@ def baseconv(x, w, bias, taps, stream=None):
     """linear(x) * conv(taps, x): [B, L, D] -> [B, L, D]."""
     y = torch.empty_like(x)
     return based_baseconv_fwd(x, w, bias, taps, y, stream=stream)
+
+
+def linattn_grad(q, k, v, dy, eps: float = 1e-6, stream=None):
+    """(dq, dk, dv) in float32 for the linear attention's output gradient dy."""
+    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=k.device)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=v.device)
+    return based_linattn_bwd(q, k, v, dy, dq, dk, dv, eps, stream=stream)

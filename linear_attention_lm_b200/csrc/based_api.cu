@@ -15,6 +15,7 @@
 #include "decode.cuh"
 #include "linattn_simt.cuh"
 #include "linattn_tc.cuh"
+#include "linattn_bwd.cuh"
 #include "window_simt.cuh"
 #include "window_tc.cuh"
 #include "proj_tc.cuh"
@@ -274,6 +275,28 @@ based_status_t launch_proj(const void* x, const void* w, ProjParams p, cudaStrea
   return launch_status();
 }
 
+template <typename T, int DV>
+based_status_t launch_linattn_bwd(const void* q, const void* k, const void* v, const void* dy,
+                                  float* dq, float* dk, float* dv, int BH, int L, float eps,
+                                  float* ws, cudaStream_t st) {
+  auto kq = linattn_bwd_q_kernel<T, DV>;
+  auto kkv = linattn_bwd_kv_kernel<T, DV>;
+  const size_t smem = BwLayout<DV>::kSmem;
+  if (!set_smem(kq, smem) || !set_smem(kkv, smem)) return BASED_ERR_CUDA;
+  const long long nblk = (long long)BH * ((L + kBwT - 1) / kBwT);
+  if (nblk > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
+  float* ws_dN = ws;
+  float* ws_dD = ws + (size_t)BH * L * DV;
+  kq<<<(unsigned)nblk, kBwThreads, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
+                                               static_cast<const T*>(v), static_cast<const T*>(dy),
+                                               dq, ws_dN, ws_dD, L, eps);
+  const based_status_t s1 = launch_status();
+  if (s1 != BASED_OK) return s1;
+  kkv<<<(unsigned)nblk, kBwThreads, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
+                                                static_cast<const T*>(v), ws_dN, ws_dD, dk, dv, L);
+  return launch_status();
+}
+
 // ---------------------------------------------------------------------------
 // Allocation-free prefill (based_linattn_fwd_noalloc): the segment partials
 // live in this fixed array instead of a caller workspace.  Host code may not
@@ -468,6 +491,35 @@ based_status_t based_decode_step(const void* q, const void* k, const void* v, fl
   if (dt == BASED_F32)
     return wide ? launch_decode<float, 128>(p, st) : launch_decode<float, 64>(p, st);
   return wide ? launch_decode<__nv_bfloat16, 128>(p, st) : launch_decode<__nv_bfloat16, 64>(p, st);
+}
+
+size_t based_linattn_bwd_workspace_bytes(int B, int H, int L, int d_v) {
+  if (B < 0 || H < 0 || L < 0 || (d_v != 64 && d_v != 128)) return (size_t)-1;
+  return (size_t)B * H * L * (d_v + 1) * sizeof(float);
+}
+
+based_status_t based_linattn_bwd(const void* q, const void* k, const void* v, const void* dy,
+                                 float* dq, float* dk, float* dv, int B, int H, int L,
+                                 int d_feat, int d_v, based_dtype_t dt, float eps,
+                                 void* workspace, size_t workspace_bytes, based_stream_t stream) {
+  if (B < 0 || H < 0 || L < 0) return BASED_ERR_INVALID_ARG;
+  if (dt != BASED_BF16 && dt != BASED_F32) return BASED_ERR_INVALID_ARG;
+  if (d_feat != kD || (d_v != 64 && d_v != 128)) return BASED_ERR_UNSUPPORTED;
+  if (!(eps >= 0.0f)) return BASED_ERR_INVALID_ARG;
+  const long long BH = (long long)B * H;
+  if (BH * L == 0) return BASED_OK;
+  if (BH * L * (d_v + 1) > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !dy || !dq || !dk || !dv) return BASED_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < based_linattn_bwd_workspace_bytes(B, H, L, d_v))
+    return BASED_ERR_WORKSPACE;
+  float* ws = static_cast<float*>(workspace);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dt == BASED_F32)
+    return d_v == 64 ? launch_linattn_bwd<float, 64>(q, k, v, dy, dq, dk, dv, (int)BH, L, eps, ws, st)
+                     : launch_linattn_bwd<float, 128>(q, k, v, dy, dq, dk, dv, (int)BH, L, eps, ws, st);
+  return d_v == 64
+             ? launch_linattn_bwd<__nv_bfloat16, 64>(q, k, v, dy, dq, dk, dv, (int)BH, L, eps, ws, st)
+             : launch_linattn_bwd<__nv_bfloat16, 128>(q, k, v, dy, dq, dk, dv, (int)BH, L, eps, ws, st);
 }
 
 based_status_t based_proj_heads_fwd(const void* x, const void* w, void* y, int B, int L,

@@ -121,6 +121,21 @@ def test_decode_host_validation(lib):
              1e-6, N) == UNSUPPORTED
 
 
+def test_linattn_bwd_host_validation(lib):
+    f = lib.based_linattn_bwd
+    ws = lib.based_linattn_bwd_workspace_bytes
+    assert ws(1, 2, 100, 64) == 1 * 2 * 100 * 65 * 4
+    assert ws(1, 2, 100, 96) == ctypes.c_size_t(-1).value
+    # q, k, v, dy, dq, dk, dv, B, H, L, d_feat, d_v, dt, eps, workspace, bytes, stream
+    A = [FAKE] * 7
+    assert f(*A, 1, 2, 100, 8, 64, 1, 1e-6, FAKE, 1 << 20, None) == UNSUPPORTED   # d_feat
+    assert f(*A, 1, 2, 100, 16, 96, 1, 1e-6, FAKE, 1 << 20, None) == UNSUPPORTED  # d_v
+    assert f(*A, 1, 2, 100, 16, 64, 1, -1.0, FAKE, 1 << 20, None) == INVALID      # eps
+    assert f(*A, 1, 2, 100, 16, 64, 1, 1e-6, FAKE, 16, None) == 5                 # workspace
+    assert f(None, *A[1:], 1, 2, 100, 16, 64, 1, 1e-6, FAKE, 1 << 20, None) == INVALID
+    assert f(*[None] * 7, 1, 2, 0, 16, 64, 1, 1e-6, None, 0, None) == 0           # nothing to do
+
+
 def test_proj_host_validation(lib):
     f = lib.based_proj_heads_fwd
     # x, w, y, B, L, d_model, H, D, dt, stream
