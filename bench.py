@@ -51,6 +51,9 @@ def load_peaks():
 # replicas: one independent copy of the workload per rank, no data exchange
 # ---------------------------------------------------------------------------
 
+FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # 74.4: CUDA-core fp32 peak of a B200
+
+
 def max_over_ranks(ms: float, dev, world: int) -> float:
     """The slowest rank's time (every rank gets the same answer)."""
     if world <= 1:
@@ -359,11 +362,12 @@ def run_e2e(args, w, lab, dev, world, x):
 
 
 def run_projections(args, lab, dev, world, peaks):
-    """The step before the attention layers and the third layer type, each on
-    layer_360m's shapes (x [8, 2048, 1024] bf16, synthetic): the six per-head
-    input projections of one linear-attention and one window layer (q, k: 16
-    heads of 16; v and the window's q, k, v: 16 heads of 64) and one BaseConv
-    block (D = 1024, 3 taps).  Four rotating x buffers (128 MB) keep L2 cold."""
+    """The rows next to the hot path, each on layer_360m's shapes (synthetic):
+    the six per-head input projections of one linear-attention and one window
+    layer (x [8, 2048, 1024] bf16; q, k: 16 heads of 16; v and the window's q,
+    k, v: 16 heads of 64), one BaseConv block (D = 1024, 3 taps), and the
+    linear attention's backward.  Four rotating x buffers (128 MB) keep L2 cold
+    for the projections."""
     B, L, dm, H = 8, 2048, 1024, 16
     g = torch.Generator(device=dev)
     g.manual_seed(1234)
@@ -377,17 +381,17 @@ def run_projections(args, lab, dev, world, peaks):
     yb = torch.empty(B, L, dm, device=dev, dtype=torch.bfloat16)
     n = max(10, min(args.steps, 200))
 
-    def timed(fn):
+    def timed(fn, n_iter):
         for i in range(max(3, args.warmup)):
             fn(i)
         torch.cuda.synchronize()
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s.record()
-        for i in range(n):
+        for i in range(n_iter):
             fn(i)
         e.record()
         torch.cuda.synchronize()
-        ms = s.elapsed_time(e) / n
+        ms = s.elapsed_time(e) / n_iter
         ms = max_over_ranks(ms, dev, world)
         return ms
 
@@ -399,20 +403,41 @@ def run_projections(args, lab, dev, world, peaks):
     def conv_step(i):
         lab.based_baseconv_fwd(xs[i % 4], wb, bias, taps, yb)
 
+    # backward of the linear attention, layer_360m shape, CUDA cores (fp32 FMA)
+    qb = (torch.randn(B, H, L, 16, device=dev, generator=g) * 0.25).to(torch.bfloat16)
+    kb = (torch.randn(B, H, L, 16, device=dev, generator=g) * 0.25).to(torch.bfloat16)
+    vb = torch.randn(B, H, L, 64, device=dev, generator=g).to(torch.bfloat16)
+    dyb = torch.randn(B, H, L, 64, device=dev, generator=g).to(torch.bfloat16)
+    gq, gk = torch.empty(B, H, L, 16, device=dev), torch.empty(B, H, L, 16, device=dev)
+    gv = torch.empty(B, H, L, 64, device=dev)
+    wsb = torch.empty(lab.based_linattn_bwd_workspace_bytes(B, H, L, 64), dtype=torch.uint8,
+                      device=dev)
+
+    def bwd_step(i):
+        lab.based_linattn_bwd(qb, kb, vb, dyb, gq, gk, gv, 1e-6, workspace=wsb)
+
     out = {}
     peak = peaks["bf16_tflops"]
     for name, fn, flops, launches, what in (
             ("proj", proj_step, 2.0 * B * L * dm * H * sum(heads), len(heads),
              "six per-head projections of x [8, 2048, 1024]: q, k 16x16; v 16x64; window q, k, v 16x64"),
             ("baseconv", conv_step, 2.0 * B * L * dm * dm, 1,
-             "BaseConv block, x [8, 2048, 1024], dense 1024x1024 + bias, 3 causal taps")):
-        ms = timed(fn)
+             "BaseConv block, x [8, 2048, 1024], dense 1024x1024 + bias, 3 causal taps"),
+            ("linattn_bwd", bwd_step, 480.0 * B * H * L * (L + 1) / 2, 2,
+             "gradient of the linear attention, B=8 H=16 L=2048 d=16 d_v=64 (quadratic form, "
+             "480 flop per (t, s) pair)")):
+        ms = timed(fn, 10 if name == "linattn_bwd" else n)
         tf = flops / (ms / 1e3) / 1e12
+        if name == "linattn_bwd":
+            # CUDA-core fp32 FMA peak: 148 SMs x 128 FMA/clk x 2 flop x 1.965 GHz
+            kern, bound, pk, src = "linattn_bwd", "alu", FP32_FMA_TFLOPS, "unit counts x max clock"
+        else:
+            kern, bound, pk, src = "proj_tc", "tensor", peak, peaks["source"]
         out[name] = {"workload": what, "ms_per_step": round(ms, 5), "launches_per_step": launches,
                      "tokens_per_s": round(world * B * L / (ms / 1e3), 1),
-                     "roofline": {"kernel": "proj_tc", "bound": "tensor", "achieved": round(tf, 1),
-                                  "peak": peak, "unit": "TFLOP/s", "frac": round(tf / peak, 4),
-                                  "traffic": None, "peak_source": peaks["source"]}}
+                     "roofline": {"kernel": kern, "bound": bound, "achieved": round(tf, 2),
+                                  "peak": pk, "unit": "TFLOP/s", "frac": round(tf / pk, 4),
+                                  "traffic": None, "peak_source": src}}
     assert lab.based_get_device_error() == 0
     return out
 
