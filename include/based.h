@@ -189,6 +189,21 @@ based_status_t based_linattn_bwd(const void* q, const void* k, const void* v, co
                                  void* workspace, size_t workspace_bytes, based_stream_t stream);
 
 /*
+ * Gradient of based_window_attn_fwd's output:
+ *   y_t = sum_{s = max(0, t-window+1)}^{t} softmax_s(q_t . k_s / sqrt(d_head)) v_s
+ * Given dy returns dq, dk, dv (fp32) on CUDA cores.
+ *   q, k, v, dy [B, H, L, d_head] dt (d_head == 64; 1 <= window <= 64)
+ *   dq, dk, dv  [B, H, L, d_head] fp32 (written)
+ *   workspace: based_window_attn_bwd_workspace_bytes() bytes of device memory
+ *   (per query: row max, row sum, dy . y), else BASED_ERR_WORKSPACE.
+ */
+size_t based_window_attn_bwd_workspace_bytes(int B, int H, int L);
+based_status_t based_window_attn_bwd(const void* q, const void* k, const void* v, const void* dy,
+                                     float* dq, float* dk, float* dv, int B, int H, int L,
+                                     int d_head, int window, based_dtype_t dt, void* workspace,
+                                     size_t workspace_bytes, based_stream_t stream);
+
+/*
  * Per-head input projection ("Базированная модель, часть 2", the paragraph on
  * the size of the hidden state: the KV and K states are made smaller by
  * projections of the layer input):

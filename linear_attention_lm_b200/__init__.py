@@ -34,6 +34,7 @@ EXPORTED_SYMBOLS = ("based_abi_version", "based_status_string",
                     "based_window_attn_fwd", "based_window_ring_fill", "based_decode_step",
                     "based_proj_heads_fwd", "based_baseconv_fwd",
                     "based_linattn_bwd_workspace_bytes", "based_linattn_bwd",
+                    "based_window_attn_bwd_workspace_bytes", "based_window_attn_bwd",
                     "based_get_device_error")
 
 
@@ -78,12 +79,17 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.based_linattn_bwd_workspace_bytes.restype = _sz
         lib.based_linattn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                           _i, _f, _vp, _sz, _vp]
+        lib.based_window_attn_bwd_workspace_bytes.argtypes = [_i, _i, _i]
+        lib.based_window_attn_bwd_workspace_bytes.restype = _sz
+        lib.based_window_attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                              _i, _i, _vp, _sz, _vp]
         lib.based_proj_heads_fwd.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
         lib.based_baseconv_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
         lib.based_get_device_error.argtypes = [_vp]
         for name in ("based_linattn_fwd", "based_linattn_fwd_noalloc", "based_window_attn_fwd",
                      "based_window_ring_fill", "based_decode_step", "based_proj_heads_fwd",
-                     "based_baseconv_fwd", "based_linattn_bwd", "based_get_device_error"):
+                     "based_baseconv_fwd", "based_linattn_bwd", "based_window_attn_bwd",
+                     "based_get_device_error"):
             getattr(lib, name).restype = _i
         _lib = lib
         return lib
@@ -249,6 +255,23 @@ def based_linattn_bwd(q, k, v, dy, dq, dk, dv, eps: float = 1e-6, workspace=None
     return dq, dk, dv
 
 
+def based_window_attn_bwd(q, k, v, dy, dq, dk, dv, window: int = 64, workspace=None,
+                          stream=None):
+    """Gradients dq, dk, dv (float32, written) of based_window_attn_fwd given dy."""
+    B, H, L, dh = q.shape
+    dt = _same_dtype(q, k, v, dy)
+    if workspace is None:
+        n = load_library().based_window_attn_bwd_workspace_bytes(B, H, L)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    with torch.cuda.device(q.device):
+        st = load_library().based_window_attn_bwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(dy), _f32(dq), _f32(dk), _f32(dv), B, H, L, dh,
+            int(window), dt, _ptr(workspace), ws_bytes, _stream(stream))
+    _check("based_window_attn_bwd", st)
+    return dq, dk, dv
+
+
 def based_proj_heads_fwd(x, w, y, stream=None):
     """x [B, L, d_model], w [H*D, d_model] -> y [B, H, L, D] (bf16, written)."""
     B, L, d_model = x.shape
@@ -325,3 +348,9 @@ def linattn_grad(q, k, v, dy, eps: float = 1e-6, stream=None):
     dk = torch.empty(k.shape, dtype=torch.float32, device=k.device)
     dv = torch.empty(v.shape, dtype=torch.float32, device=v.device)
     return based_linattn_bwd(q, k, v, dy, dq, dk, dv, eps, stream=stream)
+
+
+def window_grad(q, k, v, dy, window: int = 64, stream=None):
+    """(dq, dk, dv) in float32 for the window attention's output gradient dy."""
+    dq, dk, dv = (torch.empty(t.shape, dtype=torch.float32, device=t.device) for t in (q, k, v))
+    return based_window_attn_bwd(q, k, v, dy, dq, dk, dv, window, stream=stream)

@@ -16,6 +16,7 @@
 #include "linattn_simt.cuh"
 #include "linattn_tc.cuh"
 #include "linattn_bwd.cuh"
+#include "window_bwd.cuh"
 #include "window_simt.cuh"
 #include "window_tc.cuh"
 #include "proj_tc.cuh"
@@ -297,6 +298,26 @@ based_status_t launch_linattn_bwd(const void* q, const void* k, const void* v, c
   return launch_status();
 }
 
+template <typename T>
+based_status_t launch_window_bwd(const void* q, const void* k, const void* v, const void* dy,
+                                 float* dq, float* dk, float* dv, int BH, int L, int W, float* ws,
+                                 cudaStream_t st) {
+  auto kq = window_bwd_q_kernel<T>;
+  auto kkv = window_bwd_kv_kernel<T>;
+  if (!set_smem(kq, WbLayout::kSmem) || !set_smem(kkv, WbLayout::kSmem)) return BASED_ERR_CUDA;
+  const long long nblk = (long long)BH * ((L + kWbT - 1) / kWbT);
+  if (nblk > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
+  kq<<<(unsigned)nblk, kWbThreads, WbLayout::kSmem, st>>>(
+      static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
+      static_cast<const T*>(dy), dq, ws, L, W);
+  const based_status_t s1 = launch_status();
+  if (s1 != BASED_OK) return s1;
+  kkv<<<(unsigned)nblk, kWbThreads, WbLayout::kSmem, st>>>(
+      static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
+      static_cast<const T*>(dy), ws, dk, dv, L, W);
+  return launch_status();
+}
+
 // ---------------------------------------------------------------------------
 // Allocation-free prefill (based_linattn_fwd_noalloc): the segment partials
 // live in this fixed array instead of a caller workspace.  Host code may not
@@ -520,6 +541,31 @@ based_status_t based_linattn_bwd(const void* q, const void* k, const void* v, co
   return d_v == 64
              ? launch_linattn_bwd<__nv_bfloat16, 64>(q, k, v, dy, dq, dk, dv, (int)BH, L, eps, ws, st)
              : launch_linattn_bwd<__nv_bfloat16, 128>(q, k, v, dy, dq, dk, dv, (int)BH, L, eps, ws, st);
+}
+
+size_t based_window_attn_bwd_workspace_bytes(int B, int H, int L) {
+  if (B < 0 || H < 0 || L < 0) return (size_t)-1;
+  return (size_t)B * H * L * 3 * sizeof(float);
+}
+
+based_status_t based_window_attn_bwd(const void* q, const void* k, const void* v, const void* dy,
+                                     float* dq, float* dk, float* dv, int B, int H, int L,
+                                     int d_head, int window, based_dtype_t dt, void* workspace,
+                                     size_t workspace_bytes, based_stream_t stream) {
+  if (B < 0 || H < 0 || L < 0 || window < 1) return BASED_ERR_INVALID_ARG;
+  if (dt != BASED_BF16 && dt != BASED_F32) return BASED_ERR_INVALID_ARG;
+  if (d_head != kWbDh || window > kWbT) return BASED_ERR_UNSUPPORTED;
+  const long long BH = (long long)B * H;
+  if (BH * L == 0) return BASED_OK;
+  if (BH * L * d_head > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !dy || !dq || !dk || !dv) return BASED_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < based_window_attn_bwd_workspace_bytes(B, H, L))
+    return BASED_ERR_WORKSPACE;
+  float* ws = static_cast<float*>(workspace);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dt == BASED_F32)
+    return launch_window_bwd<float>(q, k, v, dy, dq, dk, dv, (int)BH, L, window, ws, st);
+  return launch_window_bwd<__nv_bfloat16>(q, k, v, dy, dq, dk, dv, (int)BH, L, window, ws, st);
 }
 
 based_status_t based_proj_heads_fwd(const void* x, const void* w, void* y, int B, int L,

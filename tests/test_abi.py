@@ -136,6 +136,18 @@ def test_linattn_bwd_host_validation(lib):
     assert f(*[None] * 7, 1, 2, 0, 16, 64, 1, 1e-6, None, 0, None) == 0           # nothing to do
 
 
+def test_window_bwd_host_validation(lib):
+    f = lib.based_window_attn_bwd
+    assert lib.based_window_attn_bwd_workspace_bytes(2, 3, 100) == 2 * 3 * 100 * 3 * 4
+    A = [FAKE] * 7
+    # q, k, v, dy, dq, dk, dv, B, H, L, d_head, window, dt, workspace, bytes, stream
+    assert f(*A, 1, 2, 100, 128, 64, 1, FAKE, 1 << 20, None) == UNSUPPORTED   # d_head
+    assert f(*A, 1, 2, 100, 64, 65, 1, FAKE, 1 << 20, None) == UNSUPPORTED    # window
+    assert f(*A, 1, 2, 100, 64, 0, 1, FAKE, 1 << 20, None) == INVALID
+    assert f(*A, 1, 2, 100, 64, 64, 1, FAKE, 16, None) == 5                   # workspace
+    assert f(*[None] * 7, 1, 2, 0, 64, 64, 1, None, 0, None) == 0
+
+
 def test_proj_host_validation(lib):
     f = lib.based_proj_heads_fwd
     # x, w, y, B, L, d_model, H, D, dt, stream

@@ -75,3 +75,47 @@ def test_linattn_grad_layer_shape_sampled():
         assert head_rel_l2(dq[sl].double().cpu().numpy(), rq) <= REL
         assert head_rel_l2(dk[sl].double().cpu().numpy(), rk) <= REL
         assert head_rel_l2(dvv[sl].double().cpu().numpy(), rv) <= REL
+
+
+# ------------------------------------------------------------------ window attention
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("B,H,L,W", [
+    (1, 2, 100, 64),    # two query tiles, ragged tail
+    (2, 1, 200, 7),     # a short window
+    (1, 1, 1, 64),      # a single token (dq = dk = 0)
+    (1, 3, 64, 64),     # exactly one tile
+    (1, 1, 257, 1),     # window of one: dv = dy, dq = dk = 0
+    (1, 1, 130, 33),
+])
+def test_window_grad_matches_oracle(B, H, L, W, dtype):
+    r = np.random.Generator(np.random.PCG64(L * 11 + W))
+    ts = [torch.from_numpy(r.standard_normal((B, H, L, 64))).to(dtype) for _ in range(4)]
+    q, k, v, dy = ts
+    dq, dk, dv = lab.window_grad(q.cuda(), k.cuda(), v.cuda(), dy.cuda(), W)
+    torch.cuda.synchronize()
+    assert lab.based_get_device_error() == 0
+    rq, rk, rv = grad.window_grad(*(t.double().numpy() for t in ts), W)
+    for got, ref in ((dq, rq), (dk, rk), (dv, rv)):
+        got = got.double().cpu().numpy()
+        scale = max(float(np.linalg.norm(ref)), 1.0)  # dq = dk = 0 exactly for W = 1 or L = 1
+        assert float(np.linalg.norm(got - ref)) <= REL * scale
+        if np.linalg.norm(ref) > 0:
+            assert head_rel_l2(got, ref) <= REL
+
+
+def test_window_grad_layer_shape_sampled():
+    """layer_360m's window shape (B=8, H=16, L=2048, d_h=64, W=64): three
+    whole sequences against the oracle."""
+    B, H, L = 8, 16, 2048
+    r = np.random.Generator(np.random.PCG64(17))
+    ts = [torch.from_numpy(r.standard_normal((B, H, L, 64))).to(torch.bfloat16) for _ in range(4)]
+    dq, dk, dv = lab.window_grad(*(t.cuda() for t in ts), 64)
+    torch.cuda.synchronize()
+    assert lab.based_get_device_error() == 0
+    for b, h in ((0, 0), (4, 9), (7, 15)):
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        rq, rk, rv = grad.window_grad(*(t[sl].double().numpy() for t in ts), 64)
+        assert head_rel_l2(dq[sl].double().cpu().numpy(), rq) <= REL
+        assert head_rel_l2(dk[sl].double().cpu().numpy(), rk) <= REL
+        assert head_rel_l2(dv[sl].double().cpu().numpy(), rv) <= REL
