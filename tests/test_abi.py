@@ -174,8 +174,29 @@ def test_baseconv_host_validation(lib):
 def test_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 1, 8, 16, dtype=torch.bfloat16)
     v = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
-    with pytest.raises(ValueError):
-        lab.based_linattn_fwd(q, q, v, v.clone())
+    g16, g64 = torch.zeros(q.shape), torch.zeros(v.shape)
+    ws = torch.zeros(1 << 16, dtype=torch.uint8)
+    x = torch.zeros(1, 8, 256, dtype=torch.bfloat16)
+    w = torch.zeros(256, 256, dtype=torch.bfloat16)
+    calls = [
+        lambda: lab.based_linattn_fwd(q, q, v, v.clone()),
+        lambda: lab.based_linattn_bwd(q, q, v, v, g16, g16.clone(), g64, workspace=ws),
+        lambda: lab.based_window_attn_bwd(v, v, v, v, g64, g64.clone(), g64.clone(), workspace=ws),
+        lambda: lab.based_proj_heads_fwd(x, w, torch.zeros(1, 16, 8, 16, dtype=torch.bfloat16)),
+        lambda: lab.based_baseconv_fwd(x, w, torch.zeros(256), torch.zeros(256, 3), x.clone()),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError):
+            call()
+
+
+def test_binding_checks_dtypes():
+    q = torch.zeros(1, 1, 8, 16, dtype=torch.bfloat16)
+    v32 = torch.zeros(1, 1, 8, 64, dtype=torch.float32)
+    with pytest.raises(TypeError):  # mixed q/v dtypes
+        lab.based_linattn_fwd(q, q, v32, v32.clone())
+    with pytest.raises(TypeError):  # int tensors
+        lab.based_window_attn_fwd(*(torch.zeros(1, 1, 8, 64, dtype=torch.int32) for _ in range(4)))
 
 
 def test_missing_library_fails_loudly(tmp_path):
