@@ -21,6 +21,10 @@
  *   - the one-token recurrent decode step of both (the recurrent form of the
  *     linear attention over the KV/K states, and a `window`-slot ring cache).
  *
+ * Beside it: the layer's per-head input projections and the BaseConv block
+ * (tensor-core GEMM with fused epilogues), and the gradients of both
+ * attention layers (CUDA cores).
+ *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers, owned by the caller, C-contiguous
  *     in the layouts given below, 16-byte aligned.  The library never keeps a
@@ -35,7 +39,7 @@
  *     with based_get_device_error().
  *   - dtype BASED_BF16: q/k/v/out are bfloat16, arithmetic accumulates in fp32.
  *     dtype BASED_F32: everything is fp32 (fp32 CUDA-core arithmetic).
- *     Recurrent states (state_kv, state_k) are always fp32.
+ *     Recurrent states (state_kv, state_k) and gradients are always fp32.
  *   - Feature order of the 273-row states: row 0 = constant 1; rows 1..16 =
  *     x_i / 2; row 17 + 16 i + j = x_i x_j / (4 sqrt 2)   (d = 16).
  *   - Thread safety: calls on different streams may run concurrently as long
