@@ -79,3 +79,22 @@ def test_window_grad_window_one_is_identity():
     dq, dk, dv = grad.window_grad(q, k, v, dy, 1)
     np.testing.assert_array_equal(dv, dy)
     assert np.all(dq == 0) and np.all(dk == 0)
+
+
+def test_grads_are_per_sequence_over_leading_dims():
+    """Leading [B, H] dims are independent sequences: the batched gradient equals
+    the gradient of each sequence taken alone."""
+    r = rng(21)
+    q, k = r.standard_normal((2, 3, 7, 16)) * 0.3, r.standard_normal((2, 3, 7, 16)) * 0.3
+    v, dy = r.standard_normal((2, 3, 7, 5)), r.standard_normal((2, 3, 7, 5))
+    full = grad.linattn_grad(q, k, v, dy, 1e-6)
+    wq, wk, wv, wdy = (r.standard_normal((2, 3, 9, 8)) for _ in range(4))
+    wfull = grad.window_grad(wq, wk, wv, wdy, 4)
+    for b in range(2):
+        for h in range(3):
+            one = grad.linattn_grad(q[b, h], k[b, h], v[b, h], dy[b, h], 1e-6)
+            wone = grad.window_grad(wq[b, h], wk[b, h], wv[b, h], wdy[b, h], 4)
+            for a, e in zip(full, one):
+                np.testing.assert_array_equal(a[b, h], e)
+            for a, e in zip(wfull, wone):
+                np.testing.assert_array_equal(a[b, h], e)
