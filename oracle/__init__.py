@@ -20,6 +20,9 @@ wrapper names the passage the C routine follows:
 * ``decode_linear`` / ``decode_window`` -- one recurrent generation step
   over the KV / K states (blog post part 2, state-size paragraph) and over a
   ring cache of the last W window keys/values.
+* ``ring_fill`` -- the ring cache a prefill hands to decoding: slot p mod W
+  holds position p for the last min(L, W) positions (the window of the Based
+  README, introduction, item 1, kept as a ring).
 * ``proj_heads`` -- x W^T split into heads (blog post part 2, state-size
   paragraph: the states are made smaller by projections of the input).
 * ``baseconv`` -- y = linear(x) (.) conv(h, x) ("Базированная модель, часть 1",
@@ -229,6 +232,23 @@ def decode_window(q, k, v, k_ring, v_ring, pos: int, window: int = 64):
     _load().oracle_decode_window(_ptr(q), _ptr(k), _ptr(v), _ptr(k_ring), _ptr(v_ring),
                                  int(pos), n, dh, int(window), _ptr(y))
     return y
+
+
+def ring_fill(k, v, window: int = 64):
+    """Rings [..., W, dh] (float64) after a prefill of k, v [..., L, dh]:
+    position p of the last min(L, W) positions sits in slot p mod W; slots
+    that no position reached are zero.  Pure data movement, no arithmetic."""
+    k, v = _f64(k), _f64(v)
+    if k.shape != v.shape:
+        raise ValueError("k, v must share one shape")
+    L, dh = k.shape[-2], k.shape[-1]
+    W = int(window)
+    k_ring = np.zeros(k.shape[:-2] + (W, dh), dtype=np.float64)
+    v_ring = np.zeros_like(k_ring)
+    for p in range(max(0, L - W), L):
+        k_ring[..., p % W, :] = k[..., p, :]
+        v_ring[..., p % W, :] = v[..., p, :]
+    return k_ring, v_ring
 
 
 def proj_heads(x, w, H: int, threads: int | None = None) -> np.ndarray:

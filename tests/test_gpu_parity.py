@@ -28,6 +28,11 @@ def _lib():
     torch.cuda.set_device(0)
 
 
+def test_loaded_device_code_is_sm100():
+    """The CUDA runtime runs the library's sm_100a device code on this GPU."""
+    assert lab.based_binary_version() == 100
+
+
 def head_rel_l2(y, ref):
     """max over leading (b, h) of ||y - ref|| / ||ref|| over the trailing dims."""
     n = ref.shape[0] * ref.shape[1] if ref.ndim >= 3 else 1
@@ -173,7 +178,8 @@ def run_decode(w, steps, sample):
                                            pick(x["v"], lin_idx), w.eps, return_state=True)
     S_o, z_o = np.ascontiguousarray(S_o), np.ascontiguousarray(z_o)
     check(torch.from_numpy(pick(S, lin_idx)), S_o, torch.bfloat16, "prefill state_kv", state=True)
-    kr_o, vr_o = pick(k_ring, win_idx), pick(v_ring, win_idx)
+    # the oracle's ring comes from the prefill inputs, never from the GPU's ring
+    kr_o, vr_o = oracle.ring_fill(pick(x["wk"], win_idx), pick(x["wv"], win_idx), w.window)
     out = torch.empty((w.B, w.H, w.dv), dtype=w.torch_dtype, device=dev)
     wout = torch.empty((w.B, w.Hw, w.dh), dtype=w.torch_dtype, device=dev)
     for step in range(steps):
@@ -191,6 +197,31 @@ def run_decode(w, steps, sample):
     assert lab.based_get_device_error() == 0
     check(torch.from_numpy(pick(S, lin_idx)), S_o, torch.bfloat16, "final state_kv", state=True)
     check(torch.from_numpy(pick(z, lin_idx)), z_o, torch.bfloat16, "final state_k", state=True)
+
+
+@pytest.mark.parametrize("L", [5, 63, 64, 65, 512])
+@pytest.mark.parametrize("W", [7, 64])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_ring_fill_bit_exact(L, W, dtype):
+    """based_window_ring_fill against the oracle's ring (slot p mod W holds
+    position p): bit-exact in the written slots; the other slots keep what the
+    caller put there."""
+    dev = torch.device("cuda:0")
+    w = WORKLOADS["long_16k"].with_(B=2, Hw=3, L=L, window=W, dtype=dtype, name=f"ring{L}_{W}")
+    x = prefill_inputs(w, device=dev)
+    sentinel = 3.5
+    k_ring = torch.full((w.B, w.Hw, W, w.dh), sentinel, dtype=w.torch_dtype, device=dev)
+    v_ring = torch.full_like(k_ring, sentinel)
+    lab.based_window_ring_fill(x["wk"], x["wv"], k_ring, v_ring, W)
+    torch.cuda.synchronize()
+    assert lab.based_get_device_error() == 0
+    kr_o, vr_o = oracle.ring_fill(to_f64(x["wk"]), to_f64(x["wv"]), W)
+    written = sorted({p % W for p in range(max(0, L - W), L)})
+    untouched = [s for s in range(W) if s not in written]
+    for got, ref in ((k_ring, kr_o), (v_ring, vr_o)):
+        g = to_f64(got)
+        assert np.array_equal(g[:, :, written], ref[:, :, written])
+        assert np.all(g[:, :, untouched] == sentinel)
 
 
 def test_decode_small_from_short_prefill():

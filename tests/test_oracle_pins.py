@@ -264,16 +264,38 @@ def test_decode_continues_prefill():
     yw_ref = oracle.window_attn(wq, wk, wv, W)
     _, S, z = oracle.linattn_recurrent(q[:, :L1], k[:, :L1], v[:, :L1], return_state=True)
     S, z = np.ascontiguousarray(S), np.ascontiguousarray(z)
-    k_ring = np.zeros((n_seq, W, dh))
-    v_ring = np.zeros((n_seq, W, dh))
-    for p in range(max(0, L1 - W), L1):
-        k_ring[:, p % W] = wk[:, p]
-        v_ring[:, p % W] = wv[:, p]
+    k_ring, v_ring = oracle.ring_fill(wk[:, :L1], wv[:, :L1], W)
     for t in range(L1, L):
         y = oracle.decode_linear(q[:, t], k[:, t], v[:, t], S, z)
         assert_close(y, y_ref[:, t])
         yw = oracle.decode_window(wq[:, t], wk[:, t], wv[:, t], k_ring, v_ring, t, W)
         assert_close(yw, yw_ref[:, t], rtol=1e-13)
+
+
+@pytest.mark.parametrize("L1,W", [(5, 64), (63, 64), (64, 64), (65, 64), (200, 7), (9, 7)])
+def test_decode_continues_short_and_wrapped_prefill(L1, W):
+    """The ring handed over after prefills shorter than, equal to and longer
+    than the window (wrapped slots) continues the window exactly."""
+    r = rng(100 + L1 + W)
+    n_seq, n, dh = 2, 12, 8
+    L = L1 + n
+    wq, wk, wv = (r.standard_normal((n_seq, L, dh)) for _ in range(3))
+    yw_ref = oracle.window_attn(wq, wk, wv, W)
+    k_ring, v_ring = oracle.ring_fill(wk[:, :L1], wv[:, :L1], W)
+    for t in range(L1, L):
+        yw = oracle.decode_window(wq[:, t], wk[:, t], wv[:, t], k_ring, v_ring, t, W)
+        assert_close(yw, yw_ref[:, t], rtol=1e-13)
+
+
+def test_ring_fill_slots():
+    """Slot p mod W holds position p of the last W positions; the rest is zero."""
+    k = np.arange(1.0, 11.0).reshape(1, 10, 1)
+    kr, vr = oracle.ring_fill(k, -k, 4)
+    # positions 6..9 -> slots 2, 3, 0, 1
+    assert kr[0, :, 0].tolist() == [9.0, 10.0, 7.0, 8.0]
+    assert vr[0, :, 0].tolist() == [-9.0, -10.0, -7.0, -8.0]
+    kr, _ = oracle.ring_fill(k[:, :3], k[:, :3], 8)
+    assert kr[0, :, 0].tolist() == [1.0, 2.0, 3.0, 0, 0, 0, 0, 0]
 
 
 def test_decode_from_empty():
