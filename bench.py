@@ -4,9 +4,13 @@ One step = one pass of the prefill hot path over one batch of the
 360M-layer-shape workload (B=8, L=2048, d_model=1024): causal Taylor linear
 attention over 16 heads (d=16 -> 273 features, d_v=64) with state export, plus
 sliding-window-64 softmax attention over 16 heads of d_head=64.  The metric is
-tokens/s (B*L per step).  The same run also measures the recurrent decode step
-(B=128 sequences x 16 + 16 heads, 273x64 fp32 states, 64-slot rings) and
-reports it under "decode".
+tokens/s (B*L per step).  The same run measures every other workload of the
+path on one GPU and reports each under "workloads": the fp32 check (B=1, H=2,
+L=256), the 1.3B layer shape (d_v = d_head = 128), the 16K-token prefill
+(B=1, 128 chunks carried through one state), and the recurrent decode step
+(B=128 sequences x 16 + 16 heads, 273x64 fp32 states, 64-slot rings).  Each
+carries its kernels' device times, the roofline fraction of each kernel and
+the fp64 oracle's time on the host cores for the same workload.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 For N > 1 launch with torchrun; each rank runs an independent replica (the
@@ -33,6 +37,7 @@ METRIC = "Based attn prefill tokens/s (L=2048) & decode tokens/s; % of roofline"
 UNIT = "tokens/s"
 PREFILL = "layer_360m"
 DECODE = "decode_b128"
+OTHER_PREFILL = ("tiny_fp32", "layer_1b3", "long_16k")
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -99,11 +104,19 @@ def measured_traffic(kernel):
 # algorithmic bytes / flops (per launch)
 # ---------------------------------------------------------------------------
 
-def linattn_bytes(w):
+def linattn_bytes(w, state=True):
     """q, k (d), v, out (d_v) in the input dtype per token-head, + exported states."""
     es = 4 if w.dtype == "f32" else 2
     per_tok = (2 * w.d + 2 * w.dv) * es
-    return w.B * w.H * w.L * per_tok + w.B * w.H * 273 * (w.dv + 1) * 4
+    return w.B * w.H * w.L * per_tok + (w.B * w.H * 273 * (w.dv + 1) * 4 if state else 0)
+
+
+def linattn_flops(w):
+    """Minimum FLOPs of the recurrent form with the full 273 features: per
+    token-head the state update and the read-out of the numerator (2 F d_v
+    each) and of the denominator (2 F each), and the feature maps of q and k."""
+    F = 273
+    return w.B * w.H * w.L * (4.0 * F * w.dv + 4.0 * F + 2 * 2.0 * F)
 
 
 def window_bytes(w):
@@ -116,6 +129,25 @@ def decode_bytes(w):
     lin = w.B * w.H * (2 * 273 * (w.dv + 1) * 4 + (2 * w.d + 2 * w.dv) * es)
     win = w.B * w.Hw * (2 * w.window * w.dh * es + 2 * w.dh * es + 4 * w.dh * es)
     return lin + win
+
+
+def hbm_roofline(kernel, nbytes, ms, peaks, extra=None):
+    ach = nbytes / (ms / 1e3) / 1e9
+    r = {"kernel": kernel, "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
+         "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
+         "traffic": measured_traffic(kernel) if kernel in _KERNEL_SOURCES else None,
+         "algorithmic_bytes": int(nbytes), "ms": round(ms, 5), "peak_source": peaks["source"]}
+    if extra:
+        r.update(extra)
+    return r
+
+
+def tensor_side(w, ms, peaks):
+    """The linear-attention prefill against the bf16 tensor-core peak, by its
+    minimum (algorithmic) FLOPs."""
+    tf = linattn_flops(w) / (ms / 1e3) / 1e12
+    return {"flops_min": linattn_flops(w), "tflops_min": round(tf, 1),
+            "frac_of_bf16_peak_min_flops": round(tf / peaks["bf16_tflops"], 4)}
 
 
 # ---------------------------------------------------------------------------
@@ -187,34 +219,69 @@ class ClockSampler:
                 "samples_in_window": len(inside)}
 
 
+class ClockWarmer:
+    """Keeps the GPU busy for a while right before a timed region, so that the
+    SM clock has left its idle level when timing starts (a short timed region
+    straight after an idle period would otherwise run partly at a low clock).
+    The work is plain writes over a buffer larger than L2, so it also leaves
+    L2 holding none of the timed kernels' data."""
+
+    def __init__(self, dev):
+        self.buf = torch.empty(64 << 20, dtype=torch.float32, device=dev)  # 256 MB
+
+    def __call__(self, ms: float = 150.0):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        spent, i = 0.0, 0
+        while spent < ms:
+            for _ in range(8):
+                self.buf.fill_(float(i))
+                i += 1
+            e.record()
+            e.synchronize()
+            spent = s.elapsed_time(e)
+
+
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
 
-def run_ours(args, rank, world, dev):
-    import linear_attention_lm_b200 as lab
-    from linear_attention_lm_b200 import build as lab_build
-    from linear_attention_lm_b200.inputs import WORKLOADS, decode_step_inputs, prefill_inputs
+def prefill_config(w, world):
+    """The `config` object of a prefill step (shared with the reference arm)."""
+    return {"workload": f"{w.name}: B={w.B} L={w.L}" +
+                        (f" d_model={w.d_model}" if w.d_model else "") +
+                        f"; linear attn {w.H} heads d={w.d}->273 d_v={w.dv} (+state export); "
+                        f"window-{w.window} attn {w.Hw} heads d_h={w.dh}; {w.dtype}",
+            "global_batch": w.B * world, "seq_len": w.L, "parallelism": f"replicas{world}",
+            "l2": "inputs larger than L2: input sets rotate between steps (GPU arm)"}
 
-    if rank == 0:
-        lab_build.build()
-    if world > 1:
-        torch.distributed.barrier()
-    lab.load_library()
-    peaks = load_peaks()
-    w = WORKLOADS[PREFILL]
-    # rotate input sets so that consecutive steps never find their data in L2
+
+def make_sets(w, dev, min_sets=2):
+    """Rotating input/output sets, enough that consecutive steps never find
+    their data in L2."""
+    from linear_attention_lm_b200.inputs import prefill_inputs
     set_bytes = linattn_bytes(w) + window_bytes(w)
-    n_sets = max(2, int(np.ceil(3 * L2_BYTES / set_bytes)))
+    n_sets = max(min_sets, int(np.ceil(3 * L2_BYTES / set_bytes)))
+    n_sets = min(n_sets, 64)
     sets = []
+    base = prefill_inputs(w, device=dev)
     for i in range(n_sets):
-        x = prefill_inputs(w, device=dev) if i == 0 else {k: t.clone() for k, t in sets[0][0].items()}
+        x = base if i == 0 else {k: t.clone() for k, t in base.items()}
         outs = {"y": torch.empty_like(x["v"]), "yw": torch.empty_like(x["wq"]),
                 "S": torch.empty((w.B, w.H, 273, w.dv), dtype=torch.float32, device=dev),
                 "z": torch.empty((w.B, w.H, 273), dtype=torch.float32, device=dev)}
         sets.append((x, outs))
-    ws_bytes = lab.based_linattn_workspace_bytes(w.B, w.H, w.L, w.d, w.dv, lab.BASED_BF16)
+    return sets, set_bytes
+
+
+def time_prefill(lab, w, sets, steps, warmup, warm, dev, world):
+    """Time `steps` prefill steps (linear attention with state export, then
+    window attention), with per-kernel event pairs; returns (total ms,
+    per-step linear ms, per-step window ms, launches per step)."""
+    ws_bytes = lab.based_linattn_workspace_bytes(w.B, w.H, w.L, w.d, w.dv,
+                                                 lab.BASED_BF16 if w.dtype == "bf16" else lab.BASED_F32)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    n_sets = len(sets)
 
     def step(i, ev=None):
         x, o = sets[i % n_sets]
@@ -228,28 +295,50 @@ def run_ours(args, rank, world, dev):
         if ev is not None:
             ev[2].record()
 
-    for i in range(args.warmup):
+    warm()
+    for i in range(warmup):
         step(i)
-    torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for i in range(steps):
+        step(i, evs[i])
+    stop.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    t_lin = sum(e[0].elapsed_time(e[1]) for e in evs) / steps
+    t_win = sum(e[1].elapsed_time(e[2]) for e in evs) / steps
+    launches = 2 + (1 if ws_bytes else 0)  # the split path adds a state-only pass
+    return start.elapsed_time(stop), t_lin, t_win, launches
+
+
+def run_ours(args, rank, world, dev):
+    import linear_attention_lm_b200 as lab
+    from linear_attention_lm_b200 import build as lab_build
+    from linear_attention_lm_b200.inputs import WORKLOADS
+
+    if rank == 0:
+        lab_build.build()
+    if world > 1:
+        torch.distributed.barrier()
+    lab.load_library()
+    peaks = load_peaks()
+    warm = ClockWarmer(dev)
+    w = WORKLOADS[PREFILL]
+    sets, set_bytes = make_sets(w, dev)
     with ClockSampler(dev.index) as clk:
-        time.sleep(0.3)  # let the sampler start
-        if world > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize()
+        time.sleep(0.2)  # let the sampler start
+        # the clock record covers the conditioning burn right before the timed
+        # steps as well: a timed region of a few ms holds at most one sample
         clk.mark("t_start")
-        start.record()
-        for i in range(args.steps):
-            step(i, evs[i])
-        stop.record()
-        torch.cuda.synchronize()
+        warm()
+        elapsed_ms, t_lin, t_win, launches = time_prefill(lab, w, sets, args.steps, args.warmup,
+                                                          lambda: warm(30.0), dev, world)
         clk.mark("t_stop")
-        if world > 1:
-            torch.distributed.barrier()
-    elapsed_ms = start.elapsed_time(stop)
-    t_lin = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
-    t_win = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
     assert lab.based_get_device_error() == 0
     elapsed_max = max_over_ranks(elapsed_ms, dev, world)
     value = replica_rate(w.B * w.L * args.steps, elapsed_max, world)
@@ -258,60 +347,103 @@ def run_ours(args, rank, world, dev):
     kern = {"linattn_prefill": (linattn_bytes(w), t_lin), "window_attn": (window_bytes(w), t_win)}
     dom = max(kern, key=lambda k: kern[k][1])
     b, t_ms = kern[dom]
-    achieved = b / (t_ms / 1e3) / 1e9
-    roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
-                "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": measured_traffic(dom),
-                "algorithmic_bytes": int(b), "peak_source": peaks["source"],
-                "per_kernel_ms": {k: round(v[1], 5) for k, v in kern.items()},
-                "per_kernel_frac": {k: round(v[0] / (v[1] / 1e3) / 1e9 / peaks["hbm_gbs"], 4)
-                                    for k, v in kern.items()}}
+    roofline = hbm_roofline(dom, b, t_ms, peaks)
+    roofline["per_kernel_ms"] = {k: round(v[1], 5) for k, v in kern.items()}
+    roofline["per_kernel_frac"] = {k: round(v[0] / (v[1] / 1e3) / 1e9 / peaks["hbm_gbs"], 4)
+                                   for k, v in kern.items()}
+    roofline["linattn_prefill_tensor"] = tensor_side(w, t_lin, peaks)
+    del sets
 
-    e2e = run_e2e(args, w, lab, dev, world, sets[0][0])
-    decode = run_decode(args, lab, dev, world, peaks)
+    workloads = {PREFILL: {"tokens_per_s": round(value, 1),
+                           "ms_per_step": round(elapsed_max / args.steps, 5),
+                           "kernels": {"linattn_prefill": hbm_roofline(
+                               "linattn_prefill", linattn_bytes(w), t_lin, peaks,
+                               tensor_side(w, t_lin, peaks)),
+                               "window_attn": hbm_roofline("window_attn", window_bytes(w),
+                                                           t_win, peaks)}}}
+    for name in OTHER_PREFILL:
+        workloads[name] = run_other_prefill(args, lab, WORKLOADS[name], dev, world, peaks, warm)
+    decode = run_decode(args, lab, dev, world, peaks, warm)
+    workloads[DECODE] = decode
+    e2e = run_e2e(args, w, lab, dev, world, warm)
     try:
-        projections = run_projections(args, lab, dev, world, peaks)
+        projections = run_projections(args, lab, dev, world, peaks, warm)
     except Exception as exc:  # reported in the JSON line, never hidden
         projections = {"error": f"{type(exc).__name__}: {exc}"}
     clocks = clk.summary()
+    clocks["window"] = "150 ms clock-conditioning burn + warm-up + timed steps"
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(elapsed_max / args.steps, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{PREFILL}: B=8 L=2048 d_model=1024; linear attn 16 heads "
-                               f"d=16->273 d_v=64 (+state export); window-64 attn 16 heads d_h=64",
-                   "global_batch": w.B * world, "seq_len": w.L,
-                   "parallelism": f"replicas{world}",
-                   "l2": f"inputs larger than L2: {n_sets} rotating input sets of "
-                         f"{set_bytes / 1e6:.0f} MB"},
+        "config": prefill_config(w, world),
         "roofline": roofline,
         "e2e": e2e,
-        "decode": decode,
+        "decode": {k: decode[k] for k in ("value", "unit", "ms_per_step", "steps", "roofline")},
+        "workloads": workloads,
         "projections": projections,
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": launches * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1:
         line["cpu_baseline"] = cpu_baseline(w)
+        for name in OTHER_PREFILL:
+            workloads[name]["cpu_baseline"] = cpu_baseline(WORKLOADS[name])
+        workloads[PREFILL]["cpu_baseline"] = line["cpu_baseline"]
+        workloads[DECODE]["cpu_baseline"] = cpu_baseline_decode(WORKLOADS[DECODE])
     return line
 
 
-def run_e2e(args, w, lab, dev, world, x):
-    """Same metric through the public API from pinned host buffers: every step
-    copies its inputs host->device, runs both kernels, and copies both outputs
-    device->host.  Steps are pipelined the way a caller would run them: the
-    inputs of step i+1 travel (copy stream) while step i computes (compute
-    stream) and the outputs of step i-1 come back (a third stream), with two
-    device buffer sets; PCIe carries both directions at once."""
+def run_other_prefill(args, lab, w, dev, world, peaks, warm):
+    """One of the other prefill workloads: K1 (with state export) and K2 timed
+    per kernel over rotating input sets; tokens/s = B L / (K1 + K2)."""
+    sets, _ = make_sets(w, dev)
+    n = max(10, min(args.steps, 200))
+    total_ms, t_lin, t_win, launches = time_prefill(lab, w, sets, n, args.warmup, warm, dev, world)
+    assert lab.based_get_device_error() == 0
+    del sets
+    ms = max_over_ranks(total_ms / n, dev, world)
+    lin = hbm_roofline("linattn_prefill", linattn_bytes(w), t_lin, peaks,
+                       tensor_side(w, t_lin, peaks) if w.dtype == "bf16" else None)
+    win = hbm_roofline("window_attn", window_bytes(w), t_win, peaks)
+    out = {"workload": prefill_config(w, world)["workload"],
+           "tokens_per_s": round(world * w.B * w.L / (ms / 1e3), 1),
+           "ms_per_step": round(ms, 5), "steps": n, "launches_per_step": launches,
+           "kernels": {"linattn_prefill": lin, "window_attn": win}}
+    if w.dtype == "f32":
+        out["note"] = ("fp32 CUDA-core path; a few hundred tokens per head, so the launch "
+                       "latency, not HBM, bounds it")
+    return out
+
+
+def run_e2e(args, w, lab, dev, world, warm):
+    """Same step through the public API from pinned host buffers: every step
+    copies its inputs host->device, runs both kernels (the linear attention
+    with state export, as in the device-timed step), and copies both outputs
+    and the exported states device->host.  Steps are pipelined the way a
+    caller would run them: the inputs of step i+1 travel (copy stream) while
+    step i computes (compute stream) and the outputs of step i-1 come back (a
+    third stream), with two device buffer sets; PCIe carries both directions
+    at once."""
+    from linear_attention_lm_b200.inputs import prefill_inputs
+    x = prefill_inputs(w, device=dev)
     n = max(2, min(args.steps, 30))
     host_in = {k: t.to("cpu").pin_memory() for k, t in x.items()}
-    host_out = [{"y": torch.empty(x["v"].shape, dtype=x["v"].dtype).pin_memory(),
-                 "yw": torch.empty(x["wq"].shape, dtype=x["wq"].dtype).pin_memory()}
-                for _ in range(2)]
+    S_shape, z_shape = (w.B, w.H, 273, w.dv), (w.B, w.H, 273)
+
+    def host_outs():
+        return {"y": torch.empty(x["v"].shape, dtype=x["v"].dtype).pin_memory(),
+                "yw": torch.empty(x["wq"].shape, dtype=x["wq"].dtype).pin_memory(),
+                "S": torch.empty(S_shape, dtype=torch.float32).pin_memory(),
+                "z": torch.empty(z_shape, dtype=torch.float32).pin_memory()}
+
+    host_out = [host_outs() for _ in range(2)]
     dev_in = [{k: torch.empty_like(t, device=dev) for k, t in x.items()} for _ in range(2)]
-    dev_out = [(torch.empty_like(dev_in[0]["v"]), torch.empty_like(dev_in[0]["wq"]))
-               for _ in range(2)]
+    dev_out = [{"y": torch.empty_like(dev_in[0]["v"]), "yw": torch.empty_like(dev_in[0]["wq"]),
+                "S": torch.empty(S_shape, dtype=torch.float32, device=dev),
+                "z": torch.empty(z_shape, dtype=torch.float32, device=dev)} for _ in range(2)]
+    del x
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out[0].values())
     s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
@@ -331,21 +463,22 @@ def run_e2e(args, w, lab, dev, world, x):
             s_run.wait_event(ev_in[b])
             if i >= 2:
                 s_run.wait_event(ev_out[b])  # step i-2's outputs have left dev_out[b]
-            y, yw = dev_out[b]
-            lab.based_linattn_fwd(dev_in[b]["q"], dev_in[b]["k"], dev_in[b]["v"], y, w.eps,
-                                  stream=s_run)
-            lab.based_window_attn_fwd(dev_in[b]["wq"], dev_in[b]["wk"], dev_in[b]["wv"], yw,
+            o = dev_out[b]
+            lab.based_linattn_fwd(dev_in[b]["q"], dev_in[b]["k"], dev_in[b]["v"], o["y"], w.eps,
+                                  o["S"], o["z"], stream=s_run)
+            lab.based_window_attn_fwd(dev_in[b]["wq"], dev_in[b]["wk"], dev_in[b]["wv"], o["yw"],
                                       w.window, stream=s_run)
             ev_run[b].record(s_run)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_run[b])
-            host_out[b]["y"].copy_(dev_out[b][0], non_blocking=True)
-            host_out[b]["yw"].copy_(dev_out[b][1], non_blocking=True)
+            for k in host_out[b]:
+                host_out[b][k].copy_(dev_out[b][k], non_blocking=True)
             ev_out[b].record(s_out)
 
     for i in range(2):
         step(i)
     torch.cuda.synchronize()
+    warm(30.0)
     if world > 1:
         torch.distributed.barrier()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -361,13 +494,13 @@ def run_e2e(args, w, lab, dev, world, x):
             "pipelined": "h2d(i+1) | kernels(i) | d2h(i-1) on three streams"}
 
 
-def run_projections(args, lab, dev, world, peaks):
+def run_projections(args, lab, dev, world, peaks, warm):
     """The rows next to the hot path, each on layer_360m's shapes (synthetic):
     the six per-head input projections of one linear-attention and one window
     layer (x [8, 2048, 1024] bf16; q, k: 16 heads of 16; v and the window's q,
     k, v: 16 heads of 64), one BaseConv block (D = 1024, 3 taps), and the
-    linear attention's backward.  Four rotating x buffers (128 MB) keep L2 cold
-    for the projections."""
+    backward of both attention layers.  Four rotating x buffers (128 MB) keep
+    L2 cold for the projections."""
     B, L, dm, H = 8, 2048, 1024, 16
     g = torch.Generator(device=dev)
     g.manual_seed(1234)
@@ -382,6 +515,7 @@ def run_projections(args, lab, dev, world, peaks):
     n = max(10, min(args.steps, 200))
 
     def timed(fn, n_iter):
+        warm(30.0)
         for i in range(max(3, args.warmup)):
             fn(i)
         torch.cuda.synchronize()
@@ -403,7 +537,7 @@ def run_projections(args, lab, dev, world, peaks):
     def conv_step(i):
         lab.based_baseconv_fwd(xs[i % 4], wb, bias, taps, yb)
 
-    # backward of the linear attention, layer_360m shape, CUDA cores (fp32 FMA)
+    # backward of both attention layers, layer_360m shape, CUDA cores (fp32 FMA)
     qb = (torch.randn(B, H, L, 16, device=dev, generator=g) * 0.25).to(torch.bfloat16)
     kb = (torch.randn(B, H, L, 16, device=dev, generator=g) * 0.25).to(torch.bfloat16)
     vb = torch.randn(B, H, L, 64, device=dev, generator=g).to(torch.bfloat16)
@@ -412,12 +546,23 @@ def run_projections(args, lab, dev, world, peaks):
     gv = torch.empty(B, H, L, 64, device=dev)
     wsb = torch.empty(lab.based_linattn_bwd_workspace_bytes(B, H, L, 64), dtype=torch.uint8,
                       device=dev)
+    wq_, wk_ = (torch.randn(B, H, L, 64, device=dev, generator=g) * 0.25).to(torch.bfloat16), \
+        (torch.randn(B, H, L, 64, device=dev, generator=g) * 0.25).to(torch.bfloat16)
+    gwq, gwk, gwv = (torch.empty(B, H, L, 64, device=dev) for _ in range(3))
+    wsw = torch.empty(lab.based_window_attn_bwd_workspace_bytes(B, H, L), dtype=torch.uint8,
+                      device=dev)
 
     def bwd_step(i):
         lab.based_linattn_bwd(qb, kb, vb, dyb, gq, gk, gv, 1e-6, workspace=wsb)
 
+    def wbwd_step(i):
+        lab.based_window_attn_bwd(wq_, wk_, vb, dyb, gwq, gwk, gwv, 64, workspace=wsw)
+
     out = {}
     peak = peaks["bf16_tflops"]
+    # window backward: per (query, key) pair in the band, S, dP (2 x 2 dh), dq, dk, dv
+    # (3 x 2 dh) -> 10 dh flop; W (W + 1) / 2 + W (L - W) pairs per head
+    w_pairs = 64 * 65 / 2 + 64 * (L - 64)
     for name, fn, flops, launches, what in (
             ("proj", proj_step, 2.0 * B * L * dm * H * sum(heads), len(heads),
              "six per-head projections of x [8, 2048, 1024]: q, k 16x16; v 16x64; window q, k, v 16x64"),
@@ -425,12 +570,15 @@ def run_projections(args, lab, dev, world, peaks):
              "BaseConv block, x [8, 2048, 1024], dense 1024x1024 + bias, 3 causal taps"),
             ("linattn_bwd", bwd_step, 480.0 * B * H * L * (L + 1) / 2, 2,
              "gradient of the linear attention, B=8 H=16 L=2048 d=16 d_v=64 (quadratic form, "
-             "480 flop per (t, s) pair)")):
-        ms = timed(fn, 10 if name == "linattn_bwd" else n)
+             "480 flop per (t, s) pair)"),
+            ("window_bwd", wbwd_step, 10.0 * 64 * B * H * w_pairs, 2,
+             "gradient of the window attention, B=8 H=16 L=2048 d_h=64 W=64 (10 d_h flop per "
+             "(query, key) pair in the band)")):
+        ms = timed(fn, 10 if name.endswith("bwd") else n)
         tf = flops / (ms / 1e3) / 1e12
-        if name == "linattn_bwd":
+        if name.endswith("bwd"):
             # CUDA-core fp32 FMA peak: 148 SMs x 128 FMA/clk x 2 flop x 1.965 GHz
-            kern, bound, pk, src = "linattn_bwd", "alu", FP32_FMA_TFLOPS, "unit counts x max clock"
+            kern, bound, pk, src = name, "alu", FP32_FMA_TFLOPS, "unit counts x max clock"
         else:
             kern, bound, pk, src = "proj_tc", "tensor", peak, peaks["source"]
         out[name] = {"workload": what, "ms_per_step": round(ms, 5), "launches_per_step": launches,
@@ -442,7 +590,7 @@ def run_projections(args, lab, dev, world, peaks):
     return out
 
 
-def run_decode(args, lab, dev, world, peaks):
+def run_decode(args, lab, dev, world, peaks, warm):
     """Recurrent decode: prefill 512 tokens (state export + ring fill), then
     time decode steps; two independent batches alternate so the 176 MB of
     state + ring per batch is never resident in L2 from the previous step."""
@@ -466,6 +614,7 @@ def run_decode(args, lab, dev, world, peaks):
         lab.based_decode_step(d["q"], d["k"], d["v"], S, z, out, d["wq"], d["wk"], d["wv"], kr,
                               vr, wout, pos=w.L + i // 2, window=w.window, eps=w.eps)
 
+    warm()
     for i in range(max(3, args.warmup)):
         one(i)
     torch.cuda.synchronize()
@@ -475,17 +624,16 @@ def run_decode(args, lab, dev, world, peaks):
         one(i)
     e.record()
     torch.cuda.synchronize()
+    assert lab.based_get_device_error() == 0
     ms = s.elapsed_time(e) / n
     ms = max_over_ranks(ms, dev, world)
     b = decode_bytes(w)
-    ach = b / (ms / 1e3) / 1e9
-    return {"value": round(world * w.B / (ms / 1e3), 1), "unit": "tokens/s",
+    return {"workload": f"{w.name}: B={w.B} sequences, {w.H} linear heads (273x{w.dv} fp32 "
+                        f"state) + {w.Hw} window heads ({w.window}-slot bf16 ring, d_h={w.dh}), "
+                        f"after a {w.L}-token prefill",
+            "value": round(world * w.B / (ms / 1e3), 1), "unit": "tokens/s",
             "ms_per_step": round(ms, 5), "steps": n, "batch": w.B, "heads": w.H,
-            "roofline": {"kernel": "decode_step", "bound": "hbm", "achieved": round(ach, 1),
-                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(ach / peaks["hbm_gbs"], 4),
-                         "traffic": measured_traffic("decode_step"),
-                         "algorithmic_bytes": int(b)}}
+            "roofline": hbm_roofline("decode_step", b, ms, peaks)}
 
 
 # ---------------------------------------------------------------------------
@@ -506,54 +654,72 @@ def _oracle_step_sample(w, n_lin, n_win, n_tok, threads):
     qw, kw, vw = (np.concatenate([a] * reps_w)[:n_win] for a in (wq, wk, wv))
     oracle.build()
     t0 = time.perf_counter()
-    oracle.linattn_recurrent(ql, kl, vl, w.eps, threads=threads)
+    oracle.linattn_recurrent(ql, kl, vl, w.eps, threads=threads, return_state=True)
     oracle.window_attn(qw, kw, vw, w.window, threads=threads)
     return time.perf_counter() - t0
 
 
-def cpu_baseline(w):
-    threads = os.cpu_count() or 1
+def cpu_baseline(w, threads=None):
+    threads = threads or os.cpu_count() or 1
     n_seq = w.B * w.H  # one whole step of the workload
-    sec = _oracle_step_sample(w, n_seq, n_seq, w.L, threads)
-    tok_per_s = (n_seq * w.L / w.H) / sec  # tokens through all 16 + 16 heads
-    return {"value": round(tok_per_s, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{n_seq} linear-attention + {n_seq} window sequences of L={w.L} "
-                      f"(fp64 recurrent form and direct window softmax), "
-                      f"= {n_seq / w.H:.2f} batch rows of the {PREFILL} step"}
+    sec = _oracle_step_sample(w, n_seq, w.B * w.Hw, w.L, threads)
+    tok_per_s = w.B * w.L / sec  # tokens through all heads of both layers
+    return {"value": round(tok_per_s, 1), "unit": UNIT, "cores": min(threads, n_seq),
+            "kind": "oracle",
+            "sample": f"one whole step of {w.name}: {n_seq} linear-attention sequences (fp64 "
+                      f"recurrent form, with the final state) + {w.B * w.Hw} window sequences "
+                      f"(direct window softmax) of L={w.L}"}
+
+
+def cpu_baseline_decode(w, n_steps=4):
+    """The oracle's decode steps (single-threaded C, as it stands) over all
+    B x (H + H_w) sequences of the decode workload, for n_steps steps."""
+    import oracle
+    from linear_attention_lm_b200.inputs import decode_step_inputs, to_f64
+    F = 273
+    S = np.zeros((w.B, w.H, F, w.dv))
+    z = np.zeros((w.B, w.H, F))
+    kr = np.zeros((w.B, w.Hw, w.window, w.dh))
+    vr = np.zeros_like(kr)
+    ins = [{k: to_f64(t) for k, t in decode_step_inputs(w, s).items()} for s in range(n_steps)]
+    oracle.build()
+    t0 = time.perf_counter()
+    for s, d in enumerate(ins):
+        oracle.decode_linear(d["q"], d["k"], d["v"], S, z, w.eps)
+        oracle.decode_window(d["wq"], d["wk"], d["wv"], kr, vr, w.L + s, w.window)
+    sec = time.perf_counter() - t0
+    return {"value": round(w.B * n_steps / sec, 1), "unit": "tokens/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"{n_steps} decode steps of all {w.B} sequences x ({w.H} linear + {w.Hw} "
+                      f"window heads) of {w.name}"}
 
 
 def run_reference(args, rank, world):
-    """The fp64 oracle on host cores as the reference arm: each step is one
-    linear-attention + one window sequence of the workload, truncated to a
-    token count that keeps the whole run within a few minutes."""
+    """The fp64 oracle on host cores as the reference arm, on the same
+    workload, config, thread count and sample as the cpu_baseline leg: each
+    step is one whole step of the layer_360m workload (all 128 linear-attention
+    and 128 window sequences of L = 2048), run on all host cores."""
     from linear_attention_lm_b200.inputs import WORKLOADS
     w = WORKLOADS[PREFILL]
-    threads = 1
-    budget_s = 150.0
-    n_tok = w.L
-    probe = _oracle_step_sample(w, 1, 1, 256, threads)
-    per_tok = probe / 256
-    n_tok = int(max(32, min(w.L, budget_s / max(1, args.steps + args.warmup) / per_tok)))
+    threads = os.cpu_count() or 1
+    n_seq = w.B * w.H
     for _ in range(args.warmup):
-        _oracle_step_sample(w, 1, 1, n_tok, threads)
+        _oracle_step_sample(w, n_seq, w.B * w.Hw, w.L, threads)
     t = 0.0
     for _ in range(args.steps):
-        t += _oracle_step_sample(w, 1, 1, n_tok, threads)
-    # one step pushes n_tok tokens through one head of each layer type; a token
-    # of the workload needs 16 + 16 heads
-    value = args.steps * n_tok / w.H / t
-    sample = (f"per step: 1 linear-attention + 1 window sequence of the {PREFILL} workload, "
-              f"first {n_tok} tokens; tokens/s counts a token once all 16+16 heads are done")
+        t += _oracle_step_sample(w, n_seq, w.B * w.Hw, w.L, threads)
+    value = args.steps * w.B * w.L / t
+    sample = (f"one whole step of {w.name}: {n_seq} linear-attention sequences (fp64 "
+              f"recurrent form, with the final state) + {w.B * w.Hw} window sequences "
+              f"(direct window softmax) of L={w.L}")
     return {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(1e3 * t / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": f"{PREFILL}: B=8 L=2048 d_model=1024; linear attn 16 heads "
-                                   f"d=16->273 d_v=64; window-64 attn 16 heads d_h=64",
-                       "global_batch": w.B, "seq_len": w.L, "parallelism": "host cores"},
-            "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": threads,
-                             "kind": "oracle", "sample": sample},
+            "config": prefill_config(w, world),
+            "cpu_baseline": {"value": round(value, 2), "unit": UNIT,
+                             "cores": min(threads, n_seq), "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 

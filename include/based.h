@@ -70,6 +70,14 @@ typedef void* based_stream_t; /* a cudaStream_t */
 /* Version of this ABI (bumped on any incompatible change). */
 int based_abi_version(void);
 
+/*
+ * Architecture of the device code the CUDA runtime loaded for the current
+ * device, as cudaFuncGetAttributes reports it for one of the library's
+ * kernels: major * 10 + minor (100 for the sm_100a build).  Returns -1 when
+ * there is no usable device or the code cannot run on it.
+ */
+int based_binary_version(void);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* based_status_string(based_status_t status);
 
@@ -120,12 +128,13 @@ based_status_t based_linattn_fwd(const void* q, const void* k, const void* v, vo
  * (based_linattn_workspace_bytes) exceeds 16 MiB is refused with
  * BASED_ERR_WORKSPACE before any launch.
  *
- * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  All calls on one device share the array and it
- * keeps the last call's contents (every call writes the parts it reads), so
- * calls whose kernels overlap on the GPU -- concurrent streams, several host
- * threads -- race on it: serialise them.
+ * Every call looks up the array's device address (cudaGetSymbolAddress, no
+ * allocation) on the device that is current, so the address is never stale;
+ * the first call on a device may also load the library's device code, so make
+ * that first call before any stream capture.  All calls on one device share
+ * the array and it keeps the last call's contents (every call writes the parts
+ * it reads), so calls whose kernels overlap on the GPU -- concurrent streams,
+ * several host threads -- race on it: serialise them.
  */
 based_status_t based_linattn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
                                          int B, int H, int L, int d_feat, int d_v,
@@ -185,6 +194,8 @@ based_status_t based_decode_step(const void* q, const void* k, const void* v,
  *   dq, dk [B, H, L, d_feat] fp32,  dv [B, H, L, d_v] fp32 (written)
  *   workspace: device memory of based_linattn_bwd_workspace_bytes() bytes
  *   (BASED_ERR_WORKSPACE if smaller); its contents are scratch.
+ * Arguments are checked as in based_linattn_fwd (16-byte aligned pointers,
+ * finite eps >= 0) before any launch.
  */
 size_t based_linattn_bwd_workspace_bytes(int B, int H, int L, int d_v);
 based_status_t based_linattn_bwd(const void* q, const void* k, const void* v, const void* dy,
@@ -200,6 +211,7 @@ based_status_t based_linattn_bwd(const void* q, const void* k, const void* v, co
  *   dq, dk, dv  [B, H, L, d_head] fp32 (written)
  *   workspace: based_window_attn_bwd_workspace_bytes() bytes of device memory
  *   (per query: row max, row sum, dy . y), else BASED_ERR_WORKSPACE.
+ * Pointers must be 16-byte aligned (BASED_ERR_INVALID_ARG otherwise).
  */
 size_t based_window_attn_bwd_workspace_bytes(int B, int H, int L);
 based_status_t based_window_attn_bwd(const void* q, const void* k, const void* v, const void* dy,

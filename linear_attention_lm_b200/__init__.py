@@ -1,9 +1,10 @@
 """Python binding of the B200 Based attention library (``libbased.so``).
 
 The functions named ``based_*`` mirror the C ABI in ``include/based.h`` one to
-one: they only derive sizes from the tensors' shapes, check dtype, device and
-contiguity, pass raw device pointers and the current CUDA stream through ctypes,
-and turn a non-OK status into ``BasedError``.  Every step of the computation
+one: they only derive sizes from the tensors' shapes, check every tensor's
+shape, dtype, device and contiguity against those sizes (the C ABI cannot see
+them), pass raw device pointers and the CUDA stream through ctypes, and turn a
+non-OK status into ``BasedError``.  Every step of the computation
 runs in the library's CUDA kernels; there is no CPU or PyTorch fallback -- if
 the library is missing or cannot be loaded, every call raises.
 
@@ -28,7 +29,7 @@ D_FEAT = 16
 BASED_F32, BASED_BF16 = 0, 1
 _STATUS = {0: "BASED_OK", 1: "BASED_ERR_INVALID_ARG", 2: "BASED_ERR_UNSUPPORTED",
            3: "BASED_ERR_CUDA", 4: "BASED_ERR_TIMEOUT", 5: "BASED_ERR_WORKSPACE"}
-EXPORTED_SYMBOLS = ("based_abi_version", "based_status_string",
+EXPORTED_SYMBOLS = ("based_abi_version", "based_binary_version", "based_status_string",
                     "based_linattn_workspace_bytes", "based_linattn_fwd",
                     "based_linattn_fwd_noalloc",
                     "based_window_attn_fwd", "based_window_ring_fill", "based_decode_step",
@@ -62,6 +63,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                 "`python -m linear_attention_lm_b200.build` (nvcc, sm_100a)")
         lib = ctypes.CDLL(path)
         lib.based_abi_version.restype = _i
+        lib.based_binary_version.restype = _i
         lib.based_status_string.argtypes = [_i]
         lib.based_status_string.restype = ctypes.c_char_p
         lib.based_linattn_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
@@ -115,12 +117,52 @@ def _ptr(t):
     return t.data_ptr() or None
 
 
-def _stream(stream):
+def _device_of(t) -> torch.device:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    return t.device
+
+
+def _cuda(device: torch.device) -> torch.device:
+    if device.type != "cuda":
+        raise ValueError("tensors must live on a CUDA device")
+    return device
+
+
+def _expect(t, shape, name: str, device: torch.device):
+    """t (if given) must have exactly this shape and sit on this device."""
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _torch_stream(stream, device) -> torch.cuda.Stream:
+    """The caller's stream as a torch stream object (a raw cudaStream_t handle
+    is wrapped, not copied), so that workspaces can be allocated on it."""
     if stream is None:
-        return torch.cuda.current_stream().cuda_stream
+        return torch.cuda.current_stream(device)
     if isinstance(stream, torch.cuda.Stream):
-        return stream.cuda_stream
-    return int(stream)
+        return stream
+    return torch.cuda.ExternalStream(int(stream), device=device)
+
+
+def _workspace(nbytes: int, workspace, device, ts, name: str):
+    """The caller's workspace (checked) or a new one allocated on the launch
+    stream ts, so the caching allocator does not hand it out again while the
+    kernels on ts still use it."""
+    if workspace is None:
+        if not nbytes:
+            return None, 0
+        with torch.cuda.stream(ts):
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    elif workspace.device != device:
+        raise ValueError(f"{name}: workspace is on {workspace.device}, expected {device}")
+    return workspace, workspace.numel() * workspace.element_size()
 
 
 def _check(fn: str, status: int):
@@ -150,6 +192,11 @@ def based_abi_version() -> int:
     return load_library().based_abi_version()
 
 
+def based_binary_version() -> int:
+    """SM version of the loaded device code (100 for sm_100a; -1 without a GPU)."""
+    return load_library().based_binary_version()
+
+
 def based_status_string(status: int) -> str:
     return load_library().based_status_string(int(status)).decode()
 
@@ -161,20 +208,32 @@ def based_linattn_workspace_bytes(B, H, L, d_feat, d_v, dt) -> int:
     return n
 
 
-def based_linattn_fwd(q, k, v, out, eps: float = 1e-6, state_kv=None, state_k=None,
-                      workspace=None, stream=None):
+def _linattn_shapes(q, k, v, out, state_kv, state_k):
+    dev = _device_of(q)
+    if q.dim() != 4 or not isinstance(v, torch.Tensor) or v.dim() != 4:
+        raise ValueError("q, k, v, out must be [B, H, L, d]")
     B, H, L, d = q.shape
     d_v = v.shape[-1]
+    _expect(k, (B, H, L, d), "k", dev)
+    _expect(v, (B, H, L, d_v), "v", dev)
+    _expect(out, (B, H, L, d_v), "out", dev)
+    _expect(state_kv, (B, H, NUM_FEATURES, d_v), "state_kv", dev)
+    _expect(state_k, (B, H, NUM_FEATURES), "state_k", dev)
+    return dev, B, H, L, d, d_v
+
+
+def based_linattn_fwd(q, k, v, out, eps: float = 1e-6, state_kv=None, state_k=None,
+                      workspace=None, stream=None):
+    dev, B, H, L, d, d_v = _linattn_shapes(q, k, v, out, state_kv, state_k)
     dt = _same_dtype(q, k, v, out)
-    if workspace is None:
-        nbytes = based_linattn_workspace_bytes(B, H, L, d, d_v, dt)
-        if nbytes:
-            workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    with torch.cuda.device(q.device):
+    _cuda(dev)
+    ts = _torch_stream(stream, dev)
+    with torch.cuda.device(dev):
+        nbytes = based_linattn_workspace_bytes(B, H, L, d, d_v, dt) if workspace is None else 0
+        workspace, ws_bytes = _workspace(nbytes, workspace, dev, ts, "based_linattn_fwd")
         st = load_library().based_linattn_fwd(
             _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, L, d, d_v, dt, float(eps),
-            _f32(state_kv), _f32(state_k), _ptr(workspace), ws_bytes, _stream(stream))
+            _f32(state_kv), _f32(state_k), _ptr(workspace), ws_bytes, ts.cuda_stream)
     _check("based_linattn_fwd", st)
     return out
 
@@ -184,34 +243,49 @@ def based_linattn_fwd_noalloc(q, k, v, out, eps: float = 1e-6, state_kv=None, st
     """based_linattn_fwd without a workspace: for callers that must not
     allocate device memory (the library's fixed 16 MiB scratch array is used
     instead; calls on one device must not overlap on the GPU)."""
-    B, H, L, d = q.shape
-    d_v = v.shape[-1]
+    dev, B, H, L, d, d_v = _linattn_shapes(q, k, v, out, state_kv, state_k)
     dt = _same_dtype(q, k, v, out)
-    with torch.cuda.device(q.device):
+    _cuda(dev)
+    ts = _torch_stream(stream, dev)
+    with torch.cuda.device(dev):
         st = load_library().based_linattn_fwd_noalloc(
             _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, L, d, d_v, dt, float(eps),
-            _f32(state_kv), _f32(state_k), _stream(stream))
+            _f32(state_kv), _f32(state_k), ts.cuda_stream)
     _check("based_linattn_fwd_noalloc", st)
     return out
 
 
 def based_window_attn_fwd(q, k, v, out, window: int = 64, stream=None):
+    dev = _device_of(q)
+    if q.dim() != 4:
+        raise ValueError("q, k, v, out must be [B, H, L, d_head]")
+    for t, name in ((k, "k"), (v, "v"), (out, "out")):
+        _expect(t, q.shape, name, dev)
     B, H, L, dh = q.shape
     dt = _same_dtype(q, k, v, out)
-    with torch.cuda.device(q.device):
+    _cuda(dev)
+    with torch.cuda.device(dev):
         st = load_library().based_window_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, L,
-                                                  dh, int(window), dt, _stream(stream))
+                                                  dh, int(window), dt,
+                                                  _torch_stream(stream, dev).cuda_stream)
     _check("based_window_attn_fwd", st)
     return out
 
 
 def based_window_ring_fill(k, v, k_ring, v_ring, window: int = 64, stream=None):
+    dev = _device_of(k)
+    if k.dim() != 4:
+        raise ValueError("k, v must be [B, H, L, d_head]")
     B, H, L, dh = k.shape
+    _expect(v, k.shape, "v", dev)
+    _expect(k_ring, (B, H, int(window), dh), "k_ring", dev)
+    _expect(v_ring, (B, H, int(window), dh), "v_ring", dev)
     dt = _same_dtype(k, v, k_ring, v_ring)
-    with torch.cuda.device(k.device):
+    _cuda(dev)
+    with torch.cuda.device(dev):
         st = load_library().based_window_ring_fill(_ptr(k), _ptr(v), B, H, L, dh, int(window),
                                                    _ptr(k_ring), _ptr(v_ring), dt,
-                                                   _stream(stream))
+                                                   _torch_stream(stream, dev).cuda_stream)
     _check("based_window_ring_fill", st)
 
 
@@ -219,15 +293,33 @@ def based_decode_step(q, k, v, state_kv, state_k, out, wq=None, wk=None, wv=None
                       v_ring=None, wout=None, pos: int = 0, window: int = 64,
                       eps: float = 1e-6, stream=None):
     ref = q if q is not None else wq
+    dev = _device_of(ref)
     B = ref.shape[0]
-    H, d_feat, d_v = (q.shape[1], q.shape[2], v.shape[2]) if q is not None else (0, D_FEAT, 64)
+    H, d_feat, d_v = (q.shape[1], q.shape[2], v.shape[-1]) if q is not None else (0, D_FEAT, 64)
     H_w, d_head = (wq.shape[1], wq.shape[2]) if wq is not None else (0, 64)
+    if q is not None:
+        if q.dim() != 3:
+            raise ValueError("q, k must be [B, H, d_feat]")
+        _expect(k, (B, H, d_feat), "k", dev)
+        _expect(v, (B, H, d_v), "v", dev)
+        _expect(out, (B, H, d_v), "out", dev)
+        _expect(state_kv, (B, H, NUM_FEATURES, d_v), "state_kv", dev)
+        _expect(state_k, (B, H, NUM_FEATURES), "state_k", dev)
+    if wq is not None:
+        if wq.dim() != 3:
+            raise ValueError("wq, wk, wv must be [B, H_w, d_head]")
+        for t, name in ((wk, "wk"), (wv, "wv"), (wout, "wout")):
+            _expect(t, (B, H_w, d_head), name, dev)
+        for t, name in ((k_ring, "k_ring"), (v_ring, "v_ring")):
+            _expect(t, (B, H_w, int(window), d_head), name, dev)
     dt = _same_dtype(q, k, v, out, wq, wk, wv, k_ring, v_ring, wout)
-    with torch.cuda.device(ref.device):
+    _cuda(dev)
+    with torch.cuda.device(dev):
         st = load_library().based_decode_step(
             _ptr(q), _ptr(k), _ptr(v), _f32(state_kv), _f32(state_k), _ptr(out), _ptr(wq),
             _ptr(wk), _ptr(wv), _ptr(k_ring), _ptr(v_ring), _ptr(wout), int(pos), B, H,
-            d_feat, d_v, H_w, d_head, int(window), dt, float(eps), _stream(stream))
+            d_feat, d_v, H_w, d_head, int(window), dt, float(eps),
+            _torch_stream(stream, dev).cuda_stream)
     _check("based_decode_step", st)
 
 
@@ -240,17 +332,19 @@ def based_linattn_bwd_workspace_bytes(B, H, L, d_v) -> int:
 
 def based_linattn_bwd(q, k, v, dy, dq, dk, dv, eps: float = 1e-6, workspace=None, stream=None):
     """Gradients dq, dk, dv (float32, written) of based_linattn_fwd given dy."""
-    B, H, L, d = q.shape
-    d_v = v.shape[-1]
+    dev, B, H, L, d, d_v = _linattn_shapes(q, k, v, dy, None, None)
+    _expect(dq, q.shape, "dq", dev)
+    _expect(dk, q.shape, "dk", dev)
+    _expect(dv, v.shape, "dv", dev)
     dt = _same_dtype(q, k, v, dy)
-    if workspace is None:
-        workspace = torch.empty(based_linattn_bwd_workspace_bytes(B, H, L, d_v) or 16,
-                                dtype=torch.uint8, device=q.device)
-    ws_bytes = workspace.numel() * workspace.element_size()
-    with torch.cuda.device(q.device):
+    _cuda(dev)
+    ts = _torch_stream(stream, dev)
+    with torch.cuda.device(dev):
+        nbytes = based_linattn_bwd_workspace_bytes(B, H, L, d_v) if workspace is None else 0
+        workspace, ws_bytes = _workspace(nbytes, workspace, dev, ts, "based_linattn_bwd")
         st = load_library().based_linattn_bwd(
             _ptr(q), _ptr(k), _ptr(v), _ptr(dy), _f32(dq), _f32(dk), _f32(dv), B, H, L, d, d_v,
-            dt, float(eps), _ptr(workspace), ws_bytes, _stream(stream))
+            dt, float(eps), _ptr(workspace), ws_bytes, ts.cuda_stream)
     _check("based_linattn_bwd", st)
     return dq, dk, dv
 
@@ -258,46 +352,73 @@ def based_linattn_bwd(q, k, v, dy, dq, dk, dv, eps: float = 1e-6, workspace=None
 def based_window_attn_bwd(q, k, v, dy, dq, dk, dv, window: int = 64, workspace=None,
                           stream=None):
     """Gradients dq, dk, dv (float32, written) of based_window_attn_fwd given dy."""
+    dev = _device_of(q)
+    if q.dim() != 4:
+        raise ValueError("q, k, v, dy must be [B, H, L, d_head]")
+    for t, name in ((k, "k"), (v, "v"), (dy, "dy"), (dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _expect(t, q.shape, name, dev)
     B, H, L, dh = q.shape
     dt = _same_dtype(q, k, v, dy)
-    if workspace is None:
-        n = load_library().based_window_attn_bwd_workspace_bytes(B, H, L)
-        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
-    ws_bytes = workspace.numel() * workspace.element_size()
-    with torch.cuda.device(q.device):
+    _cuda(dev)
+    ts = _torch_stream(stream, dev)
+    with torch.cuda.device(dev):
+        nbytes = load_library().based_window_attn_bwd_workspace_bytes(B, H, L) \
+            if workspace is None else 0
+        workspace, ws_bytes = _workspace(nbytes, workspace, dev, ts, "based_window_attn_bwd")
         st = load_library().based_window_attn_bwd(
             _ptr(q), _ptr(k), _ptr(v), _ptr(dy), _f32(dq), _f32(dk), _f32(dv), B, H, L, dh,
-            int(window), dt, _ptr(workspace), ws_bytes, _stream(stream))
+            int(window), dt, _ptr(workspace), ws_bytes, ts.cuda_stream)
     _check("based_window_attn_bwd", st)
     return dq, dk, dv
 
 
 def based_proj_heads_fwd(x, w, y, stream=None):
     """x [B, L, d_model], w [H*D, d_model] -> y [B, H, L, D] (bf16, written)."""
+    dev = _device_of(x)
+    if x.dim() != 3 or y.dim() != 4:
+        raise ValueError("x must be [B, L, d_model] and y [B, H, L, D]")
     B, L, d_model = x.shape
-    _, H, _, D = y.shape
+    H, D = y.shape[1], y.shape[3]
+    _expect(w, (H * D, d_model), "w", dev)
+    _expect(y, (B, H, L, D), "y", dev)
     dt = _same_dtype(x, w, y)
-    with torch.cuda.device(x.device):
+    _cuda(dev)
+    with torch.cuda.device(dev):
         st = load_library().based_proj_heads_fwd(_ptr(x), _ptr(w), _ptr(y), B, L, d_model, H, D,
-                                                 dt, _stream(stream))
+                                                 dt, _torch_stream(stream, dev).cuda_stream)
     _check("based_proj_heads_fwd", st)
     return y
 
 
 def based_baseconv_fwd(x, w, bias, taps, y, stream=None):
     """x, y [B, L, D] bf16; w [D, D] bf16; bias [D], taps [D, K] float32."""
+    dev = _device_of(x)
+    if x.dim() != 3 or taps.dim() != 2:
+        raise ValueError("x must be [B, L, D] and taps [D, K]")
     B, L, D = x.shape
     K = taps.shape[-1]
+    _expect(w, (D, D), "w", dev)
+    _expect(bias, (D,), "bias", dev)
+    _expect(taps, (D, K), "taps", dev)
+    _expect(y, (B, L, D), "y", dev)
     dt = _same_dtype(x, w, y)
-    with torch.cuda.device(x.device):
+    _cuda(dev)
+    with torch.cuda.device(dev):
         st = load_library().based_baseconv_fwd(_ptr(x), _ptr(w), _f32(bias), _f32(taps), _ptr(y),
-                                               B, L, D, K, dt, _stream(stream))
+                                               B, L, D, K, dt,
+                                               _torch_stream(stream, dev).cuda_stream)
     _check("based_baseconv_fwd", st)
     return y
 
 
 def based_get_device_error(stream=None) -> int:
-    return load_library().based_get_device_error(_stream(stream))
+    if stream is None:
+        handle = torch.cuda.current_stream().cuda_stream
+    elif isinstance(stream, torch.cuda.Stream):
+        handle = stream.cuda_stream
+    else:
+        handle = int(stream)
+    return load_library().based_get_device_error(handle)
 
 
 # ---------------------------------------------------------------------------

@@ -8,6 +8,7 @@ libcudart the host process loaded first.
 from __future__ import annotations
 
 import glob
+import json
 import os
 import shutil
 import subprocess
@@ -18,6 +19,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(HERE, "libbased.so")
+# the nvcc command line of the last build, written beside the library
+RECORD_PATH = os.path.join(HERE, "libbased.build.json")
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -56,6 +59,9 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if res.returncode != 0:
         raise RuntimeError("nvcc failed building libbased.so")
     os.replace(tmp, LIB_PATH)
+    with open(RECORD_PATH, "w") as f:
+        json.dump({"nvcc": [os.path.basename(cmd[0])] + cmd[1:-3] + cmd[-1:],
+                   "arch_flags": ARCH_FLAGS}, f, indent=1)
     return LIB_PATH
 
 

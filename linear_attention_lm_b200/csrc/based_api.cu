@@ -8,8 +8,6 @@
 #include <math.h>
 #include <stdint.h>
 
-#include <mutex>
-
 #include "based.h"
 #include "common.cuh"
 #include "decode.cuh"
@@ -322,11 +320,9 @@ based_status_t launch_window_bwd(const void* q, const void* k, const void* v, co
 // Allocation-free prefill (based_linattn_fwd_noalloc): the segment partials
 // live in this fixed array instead of a caller workspace.  Host code may not
 // pass the array's name to a kernel (on the host it is only a stand-in); the
-// device address is looked up once per device with cudaGetSymbolAddress.
+// device address is looked up with cudaGetSymbolAddress on every call, with
+// the caller's device current, so it stays right after a device reset.
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
-constexpr int kNoAllocMaxDevices = 64;
-std::mutex g_noalloc_mutex;
-float* g_noalloc_addr[kNoAllocMaxDevices] = {};
 
 }  // namespace
 
@@ -334,20 +330,12 @@ static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / 
 
 namespace {
 
-// Device address of g_noalloc_scratch on the current device (looked up on the
-// first call for that device).
+// Device address of g_noalloc_scratch on the current device.
 based_status_t noalloc_scratch(float** addr) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return BASED_ERR_CUDA;
-  if (dev < 0 || dev >= kNoAllocMaxDevices) return BASED_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-      return BASED_ERR_CUDA;
-    g_noalloc_addr[dev] = static_cast<float*>(p);
-  }
-  *addr = g_noalloc_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+    return BASED_ERR_CUDA;
+  *addr = static_cast<float*>(p);
   return BASED_OK;
 }
 
@@ -356,6 +344,12 @@ based_status_t noalloc_scratch(float** addr) {
 extern "C" {
 
 int based_abi_version(void) { return 1; }
+
+int based_binary_version(void) {
+  cudaFuncAttributes a;
+  if (cudaFuncGetAttributes(&a, linattn_tc_kernel<64, false>) != cudaSuccess) return -1;
+  return a.binaryVersion;
+}
 
 const char* based_status_string(based_status_t status) {
   switch (status) {
@@ -523,16 +517,19 @@ based_status_t based_linattn_bwd(const void* q, const void* k, const void* v, co
                                  float* dq, float* dk, float* dv, int B, int H, int L,
                                  int d_feat, int d_v, based_dtype_t dt, float eps,
                                  void* workspace, size_t workspace_bytes, based_stream_t stream) {
-  if (B < 0 || H < 0 || L < 0) return BASED_ERR_INVALID_ARG;
-  if (dt != BASED_BF16 && dt != BASED_F32) return BASED_ERR_INVALID_ARG;
-  if (d_feat != kD || (d_v != 64 && d_v != 128)) return BASED_ERR_UNSUPPORTED;
-  if (!(eps >= 0.0f)) return BASED_ERR_INVALID_ARG;
+  // the forward's checks of sizes, dtype, eps (finite, >= 0) and of q, k, v, dy
+  based_status_t s = check_linattn(q, k, v, dy, B, H, L, d_feat, d_v, dt, eps, nullptr, nullptr);
+  if (s != BASED_OK) return s;
   const long long BH = (long long)B * H;
-  if (BH * L == 0) return BASED_OK;
+  const bool empty = BH * L == 0;
+  if ((s = check_tensor(dq, empty)) != BASED_OK) return s;
+  if ((s = check_tensor(dk, empty)) != BASED_OK) return s;
+  if ((s = check_tensor(dv, empty)) != BASED_OK) return s;
+  if (empty) return BASED_OK;
   if (BH * L * (d_v + 1) > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
-  if (!q || !k || !v || !dy || !dq || !dk || !dv) return BASED_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < based_linattn_bwd_workspace_bytes(B, H, L, d_v))
     return BASED_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return BASED_ERR_INVALID_ARG;
   float* ws = static_cast<float*>(workspace);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dt == BASED_F32)
@@ -556,11 +553,17 @@ based_status_t based_window_attn_bwd(const void* q, const void* k, const void* v
   if (dt != BASED_BF16 && dt != BASED_F32) return BASED_ERR_INVALID_ARG;
   if (d_head != kWbDh || window > kWbT) return BASED_ERR_UNSUPPORTED;
   const long long BH = (long long)B * H;
-  if (BH * L == 0) return BASED_OK;
+  if (BH > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
+  const bool empty = BH * L == 0;
+  based_status_t s;
+  for (const void* t : {q, k, v, dy, static_cast<const void*>(dq), static_cast<const void*>(dk),
+                        static_cast<const void*>(dv)})
+    if ((s = check_tensor(t, empty)) != BASED_OK) return s;
+  if (empty) return BASED_OK;
   if (BH * L * d_head > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
-  if (!q || !k || !v || !dy || !dq || !dk || !dv) return BASED_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < based_window_attn_bwd_workspace_bytes(B, H, L))
     return BASED_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return BASED_ERR_INVALID_ARG;
   float* ws = static_cast<float*>(workspace);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dt == BASED_F32)

@@ -39,9 +39,15 @@ def test_library_exports_every_declared_symbol(lib):
     assert lib.based_abi_version() == 1
 
 
-def test_built_for_sm100a():
-    out = open(lab_build.LIB_PATH, "rb").read()
-    assert b"sm_100a" in out or b"sm_100" in out
+def test_built_for_sm100a(lib):
+    """The build ran nvcc with the sm_100a target and nothing else (the
+    command line is recorded beside the library at build time; the running
+    device code is checked on a GPU by test_gpu_parity)."""
+    import json
+    rec = json.load(open(lab_build.RECORD_PATH))
+    assert rec["arch_flags"] == ["-gencode", "arch=compute_100a,code=sm_100a"]
+    gencodes = [a for a in rec["nvcc"] if a.startswith("arch=")]
+    assert gencodes == ["arch=compute_100a,code=sm_100a"]
 
 
 def test_status_strings(lib):
@@ -134,6 +140,82 @@ def test_linattn_bwd_host_validation(lib):
     assert f(*A, 1, 2, 100, 16, 64, 1, 1e-6, FAKE, 16, None) == 5                 # workspace
     assert f(None, *A[1:], 1, 2, 100, 16, 64, 1, 1e-6, FAKE, 1 << 20, None) == INVALID
     assert f(*[None] * 7, 1, 2, 0, 16, 64, 1, 1e-6, None, 0, None) == 0           # nothing to do
+
+
+def test_linattn_bwd_checks_like_the_forward(lib):
+    """Alignment and eps are checked as in based_linattn_fwd."""
+    f = lib.based_linattn_bwd
+    A = [FAKE] * 7
+    for i in range(7):  # each of q, k, v, dy, dq, dk, dv misaligned
+        B = list(A)
+        B[i] = FAKE + 4
+        assert f(*B, 1, 2, 100, 16, 64, 1, 1e-6, FAKE, 1 << 20, None) == INVALID
+    assert f(*A, 1, 2, 100, 16, 64, 1, float("inf"), FAKE, 1 << 20, None) == INVALID
+    assert f(*A, 1, 2, 100, 16, 64, 1, float("nan"), FAKE, 1 << 20, None) == INVALID
+    assert f(*A, 1, 2, 100, 16, 64, 1, 1e-6, FAKE + 8, 1 << 20, None) == INVALID  # workspace
+    assert f(*A, 1, 2, 100, 16, 64, 7, 1e-6, FAKE, 1 << 20, None) == INVALID      # dtype
+
+
+def test_window_bwd_checks_alignment(lib):
+    f = lib.based_window_attn_bwd
+    A = [FAKE] * 7
+    for i in range(7):
+        B = list(A)
+        B[i] = FAKE + 2
+        assert f(*B, 1, 2, 100, 64, 64, 1, FAKE, 1 << 20, None) == INVALID
+    assert f(*A, 1, 2, 100, 64, 64, 1, FAKE + 4, 1 << 20, None) == INVALID       # workspace
+
+
+def test_binding_checks_shapes():
+    """Every wrapper checks each tensor's full shape against the sizes it
+    passes to the C ABI (which cannot see them) before anything else."""
+    bf = torch.bfloat16
+
+    def z(*shape, dtype=bf):
+        return torch.zeros(*shape, dtype=dtype)
+
+    q, v = z(1, 2, 8, 16), z(1, 2, 8, 64)
+    bad_calls = [
+        lambda: lab.based_linattn_fwd(q, z(1, 2, 7, 16), v, v.clone()),            # k's L
+        lambda: lab.based_linattn_fwd(q, q, z(1, 2, 7, 64), z(1, 2, 7, 64)),       # v's L
+        lambda: lab.based_linattn_fwd(q, q, v, z(1, 2, 8, 128)),                   # out's d_v
+        lambda: lab.based_linattn_fwd(q, q, v, v.clone(), 1e-6,
+                                      z(1, 2, 272, 64, dtype=torch.float32)),      # state rows
+        lambda: lab.based_linattn_fwd(q, q, v, v.clone(), 1e-6, None,
+                                      z(1, 3, 273, dtype=torch.float32)),          # state_k heads
+        lambda: lab.based_linattn_fwd_noalloc(q, q, v, z(2, 2, 8, 64)),
+        lambda: lab.based_window_attn_fwd(v, v, z(1, 2, 9, 64), v.clone()),
+        lambda: lab.based_window_ring_fill(v, v, z(1, 2, 63, 64), z(1, 2, 64, 64)),
+        lambda: lab.based_decode_step(z(4, 2, 16), z(4, 2, 16), z(4, 2, 64),
+                                      z(4, 2, 273, 64, dtype=torch.float32),
+                                      z(4, 2, 273, dtype=torch.float32), z(4, 2, 32)),
+        lambda: lab.based_decode_step(None, None, None, None, None, None, z(4, 2, 64),
+                                      z(4, 2, 64), z(4, 2, 64), z(4, 2, 32, 64), z(4, 2, 64, 64),
+                                      z(4, 2, 64), window=64),
+        lambda: lab.based_linattn_bwd(q, q, v, v, z(1, 2, 8, 16, dtype=torch.float32),
+                                      z(1, 2, 8, 16, dtype=torch.float32),
+                                      z(1, 2, 8, 32, dtype=torch.float32)),
+        lambda: lab.based_window_attn_bwd(v, v, v, v, *(z(1, 2, 8, 64, dtype=torch.float32)
+                                                        for _ in range(2)),
+                                          z(1, 2, 4, 64, dtype=torch.float32)),
+        lambda: lab.based_proj_heads_fwd(z(1, 8, 256), z(256, 128), z(1, 16, 8, 16)),
+        lambda: lab.based_baseconv_fwd(z(1, 8, 256), z(256, 256), torch.zeros(255),
+                                       torch.zeros(256, 3), z(1, 8, 256)),
+    ]
+    for call in bad_calls:
+        with pytest.raises(ValueError, match="expected shape"):
+            call()
+
+
+def test_binding_checks_devices():
+    """A tensor on another device than q is refused (meta tensors stand in
+    for a second device; nothing is launched)."""
+    q = torch.zeros(1, 2, 8, 16, dtype=torch.bfloat16)
+    v = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="is on meta"):
+        lab.based_linattn_fwd(q, q.to("meta"), v, v.clone())
+    with pytest.raises(ValueError, match="is on meta"):
+        lab.based_window_attn_fwd(v, v, v, v.to("meta"))
 
 
 def test_window_bwd_host_validation(lib):

@@ -36,9 +36,11 @@ def test_noalloc_matches_workspace_entry_point():
     lab.load_library()
     torch.cuda.set_device(0)
     dev = torch.device("cuda:0")
-    # two calls in a row with different problems; both split into segments
+    # calls in a row with different problems; all split into segments, the
+    # last one with d_v = 128 (the other tensor-core layout)
     cases = [WORKLOADS["long_16k"].with_(B=1, H=2, L=3000, name="noalloc_a"),
-             WORKLOADS["long_16k"].with_(B=2, H=1, L=2100, wid=7, name="noalloc_b")]
+             WORKLOADS["long_16k"].with_(B=2, H=1, L=2100, wid=7, name="noalloc_b"),
+             WORKLOADS["long_16k"].with_(B=1, H=3, L=2500, dv=128, wid=8, name="noalloc_c")]
     for w in cases:
         need = lab.based_linattn_workspace_bytes(w.B, w.H, w.L, w.d, w.dv, lab.BASED_BF16)
         assert need > 0, "the case must exercise the scratch path"
@@ -61,3 +63,21 @@ def test_noalloc_matches_workspace_entry_point():
         for got, ref in ((S, S_ref), (z, z_ref)):
             g, r = to_f64(got), to_f64(ref)
             assert np.all(np.isfinite(g)) and head_rel_l2(g, r) <= REL_BF16
+
+
+def test_noalloc_scratch_covers_every_split():
+    """The scratch array (16 MiB) covers the largest workspace any problem
+    asks for on this GPU: the split keeps (segments - 1) x sequences at most
+    one per SM, so the need peaks near SMs x 160 x (d_v + 16) x 4 bytes.
+    Sizes beyond the array would be refused with BASED_ERR_WORKSPACE before
+    any launch; none is reachable here."""
+    lab_build.build()
+    lab.load_library()
+    torch.cuda.set_device(0)
+    worst = 0
+    for dv in (64, 128):
+        for BH in (1, 2, 3, 5, 16, 37, 74):
+            for L in (1024, 4096, 65536, 1 << 20):
+                worst = max(worst, lab.based_linattn_workspace_bytes(1, BH, L, 16, dv,
+                                                                     lab.BASED_BF16))
+    assert 0 < worst <= 16 << 20
