@@ -189,7 +189,10 @@ based_status_t based_decode_step(const void* q, const void* k, const void* v,
  * Gradient of based_linattn_fwd's output (the map the "based/train" README's
  * training views share; see based_linattn_fwd):
  *   w_ts = 1 + u + u^2/2, u = q_t.k_s/sqrt(d_feat), s <= t; y_t = sum_s w_ts v_s / (sum_s w_ts + eps)
- * Given dy = dL/dy returns dq, dk, dv (fp32) on CUDA cores over the quadratic form.
+ * Given dy = dL/dy returns dq, dk, dv (fp32) over the quadratic form: for bf16
+ * inputs on the tensor cores (128 x 128 tiles of the (t, s) triangle, bf16
+ * operands for w, dw (1 + u) and dy / D, fp32 accumulation); for fp32 inputs
+ * on CUDA cores in fp32.
  *   q, k [B, H, L, d_feat]   v, dy [B, H, L, d_v]   dt (d_feat == 16, d_v in {64, 128})
  *   dq, dk [B, H, L, d_feat] fp32,  dv [B, H, L, d_v] fp32 (written)
  *   workspace: device memory of based_linattn_bwd_workspace_bytes() bytes
@@ -246,6 +249,23 @@ based_status_t based_proj_heads_fwd(const void* x, const void* w, void* y, int B
 based_status_t based_baseconv_fwd(const void* x, const void* w, const float* bias,
                                   const float* taps, void* y, int B, int L, int D, int K,
                                   based_dtype_t dt, based_stream_t stream);
+
+/*
+ * Test hook for the failure path of the bounded waits; not for production use.
+ * Synchronises the current device, then sets, for every later launch on it:
+ *   which = 0  normal operation;
+ *   which = 1  the first CTA of the linear-attention prefill (bf16) leaves out
+ *              the V tile load of its second chunk;
+ *   which = 2  the first CTA of the window attention (bf16) leaves out its V
+ *              tile load;
+ * and the time after which every bounded wait gives up, wait_limit_ns > 0
+ * (2e9, two seconds, is the default).  A wait on a load that was left out runs
+ * out: the kernel records BASED_ERR_TIMEOUT (see based_get_device_error),
+ * drains its own loads and stores in flight, releases its tensor memory and
+ * returns; its outputs are then undefined.  Nothing faults and nothing is
+ * left waiting.  BASED_ERR_INVALID_ARG for other values.
+ */
+based_status_t based_debug_stall(int which, long long wait_limit_ns);
 
 /*
  * Synchronise `stream`, then read and clear the library's device status word

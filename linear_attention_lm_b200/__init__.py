@@ -36,7 +36,7 @@ EXPORTED_SYMBOLS = ("based_abi_version", "based_binary_version", "based_status_s
                     "based_proj_heads_fwd", "based_baseconv_fwd",
                     "based_linattn_bwd_workspace_bytes", "based_linattn_bwd",
                     "based_window_attn_bwd_workspace_bytes", "based_window_attn_bwd",
-                    "based_get_device_error")
+                    "based_debug_stall", "based_get_device_error")
 
 
 class BasedError(RuntimeError):
@@ -88,10 +88,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.based_proj_heads_fwd.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
         lib.based_baseconv_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
         lib.based_get_device_error.argtypes = [_vp]
+        lib.based_debug_stall.argtypes = [_i, _ll]
         for name in ("based_linattn_fwd", "based_linattn_fwd_noalloc", "based_window_attn_fwd",
                      "based_window_ring_fill", "based_decode_step", "based_proj_heads_fwd",
                      "based_baseconv_fwd", "based_linattn_bwd", "based_window_attn_bwd",
-                     "based_get_device_error"):
+                     "based_debug_stall", "based_get_device_error"):
             getattr(lib, name).restype = _i
         _lib = lib
         return lib
@@ -409,6 +410,16 @@ def based_baseconv_fwd(x, w, bias, taps, y, stream=None):
                                                _torch_stream(stream, dev).cuda_stream)
     _check("based_baseconv_fwd", st)
     return y
+
+
+STALL_NONE, STALL_LINATTN_V, STALL_WINDOW_V = 0, 1, 2
+
+
+def based_debug_stall(which: int, wait_limit_ns: int = 2_000_000_000):
+    """Test hook: make the first CTA of the chosen kernel leave one load out
+    so its bounded wait runs out after wait_limit_ns (which = 0 restores
+    normal operation)."""
+    _check("based_debug_stall", load_library().based_debug_stall(int(which), int(wait_limit_ns)))
 
 
 def based_get_device_error(stream=None) -> int:

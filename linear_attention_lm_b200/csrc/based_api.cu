@@ -14,9 +14,11 @@
 #include "linattn_simt.cuh"
 #include "linattn_tc.cuh"
 #include "linattn_bwd.cuh"
+#include "linattn_bwd_tc.cuh"
 #include "window_bwd.cuh"
 #include "window_simt.cuh"
 #include "window_tc.cuh"
+#include "window_tcp.cuh"
 #include "proj_tc.cuh"
 
 namespace based {
@@ -215,6 +217,24 @@ based_status_t launch_window_tc(const void* q, const void* k, const void* v, voi
   return launch_status();
 }
 
+// d_head = 64: the persistent kernel, one CTA per SM (or per tile, if fewer)
+based_status_t launch_window_tcp(const void* q, const void* k, const void* v, void* out, int BH,
+                                 int L, int W, cudaStream_t st) {
+  CUtensorMap qm, km, vm, ym;
+  if (!make_rows_map(&qm, q, 64, L, BH, kWtQ) || !make_rows_map(&km, k, 64, L, BH, kWtKeys) ||
+      !make_rows_map(&vm, v, 64, L, BH, kWtKeys) || !make_rows_map(&ym, out, 64, L, BH, kWtQ))
+    return BASED_ERR_CUDA;
+  if (!set_smem(window_tcp_kernel, WpLayout::kSmem)) return BASED_ERR_CUDA;
+  const int tiles_per_seq = (L + kWtQ - 1) / kWtQ;
+  const long long n_total = (long long)tiles_per_seq * BH;
+  if (n_total > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
+  const long long sms = device_sm_count();
+  const unsigned grid = (unsigned)(n_total < sms ? n_total : sms);
+  window_tcp_kernel<<<grid, kWpThreads, WpLayout::kSmem, st>>>(qm, km, vm, ym, L, W,
+                                                               tiles_per_seq, (int)n_total);
+  return launch_status();
+}
+
 template <typename T>
 based_status_t launch_window_simt(const void* q, const void* k, const void* v, void* out,
                                   int BH, int L, int dh, int W, cudaStream_t st) {
@@ -293,6 +313,41 @@ based_status_t launch_linattn_bwd(const void* q, const void* k, const void* v, c
   if (s1 != BASED_OK) return s1;
   kkv<<<(unsigned)nblk, kBwThreads, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
                                                 static_cast<const T*>(v), ws_dN, ws_dD, dk, dv, L);
+  return launch_status();
+}
+
+// bf16 gradient on the tensor cores: workspace = dN (bf16 [BH, L, DV]) then dD
+// (fp32 [BH, L]), well inside based_linattn_bwd_workspace_bytes
+template <int DV>
+based_status_t launch_linattn_bwd_tc(const void* q, const void* k, const void* v, const void* dy,
+                                     float* dq, float* dk, float* dv, int BH, int L, float eps,
+                                     void* ws, cudaStream_t st) {
+  BtParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.dy = static_cast<const __nv_bfloat16*>(dy);
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.ws_dn = static_cast<__nv_bfloat16*>(ws);
+  p.ws_dd = reinterpret_cast<float*>(static_cast<char*>(ws) + (size_t)BH * L * DV * 2);
+  p.L = L;
+  p.n_tiles = (L + kBtT - 1) / kBtT;
+  p.eps = eps;
+  CUtensorMap vmap, dnmap;
+  if (!make_rows_map(&vmap, v, DV, L, BH, kBtT) || !make_rows_map(&dnmap, p.ws_dn, DV, L, BH, kBtT))
+    return BASED_ERR_CUDA;
+  auto kq = linattn_bwd_tc_q_kernel<DV>;
+  auto kkv = linattn_bwd_tc_kv_kernel<DV>;
+  if (!set_smem(kq, BtLayout<DV>::kSmemQ) || !set_smem(kkv, BtLayout<DV>::kSmemK))
+    return BASED_ERR_CUDA;
+  const long long nblk = (long long)BH * p.n_tiles;
+  if (nblk > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
+  kq<<<(unsigned)nblk, kBtThreads, BtLayout<DV>::kSmemQ, st>>>(vmap, p);
+  const based_status_t s1 = launch_status();
+  if (s1 != BASED_OK) return s1;
+  kkv<<<(unsigned)nblk, kBtThreads, BtLayout<DV>::kSmemK, st>>>(vmap, dnmap, p);
   return launch_status();
 }
 
@@ -432,7 +487,7 @@ based_status_t based_window_attn_fwd(const void* q, const void* k, const void* v
   if ((long long)B * H > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dt == BASED_F32) return launch_window_simt<float>(q, k, v, out, B * H, L, d_head, window, st);
-  return d_head == 64 ? launch_window_tc<64>(q, k, v, out, B * H, L, window, st)
+  return d_head == 64 ? launch_window_tcp(q, k, v, out, B * H, L, window, st)
                       : launch_window_tc<128>(q, k, v, out, B * H, L, window, st);
 }
 
@@ -535,9 +590,8 @@ based_status_t based_linattn_bwd(const void* q, const void* k, const void* v, co
   if (dt == BASED_F32)
     return d_v == 64 ? launch_linattn_bwd<float, 64>(q, k, v, dy, dq, dk, dv, (int)BH, L, eps, ws, st)
                      : launch_linattn_bwd<float, 128>(q, k, v, dy, dq, dk, dv, (int)BH, L, eps, ws, st);
-  return d_v == 64
-             ? launch_linattn_bwd<__nv_bfloat16, 64>(q, k, v, dy, dq, dk, dv, (int)BH, L, eps, ws, st)
-             : launch_linattn_bwd<__nv_bfloat16, 128>(q, k, v, dy, dq, dk, dv, (int)BH, L, eps, ws, st);
+  return d_v == 64 ? launch_linattn_bwd_tc<64>(q, k, v, dy, dq, dk, dv, (int)BH, L, eps, workspace, st)
+                   : launch_linattn_bwd_tc<128>(q, k, v, dy, dq, dk, dv, (int)BH, L, eps, workspace, st);
 }
 
 size_t based_window_attn_bwd_workspace_bytes(int B, int H, int L) {
@@ -608,6 +662,18 @@ based_status_t based_baseconv_fwd(const void* x, const void* w, const float* bia
   p.bias = bias; p.taps = taps;
   p.M = (int)M; p.N = D; p.Kd = D; p.L = L; p.K = K;
   return launch_proj<kBaseConv>(x, w, p, static_cast<cudaStream_t>(stream));
+}
+
+based_status_t based_debug_stall(int which, long long wait_limit_ns) {
+  if (which != kStallNone && which != kStallLinattnV && which != kStallWindowV)
+    return BASED_ERR_INVALID_ARG;
+  if (wait_limit_ns <= 0) return BASED_ERR_INVALID_ARG;
+  const uint64_t limit = static_cast<uint64_t>(wait_limit_ns);
+  if (cudaDeviceSynchronize() != cudaSuccess) return BASED_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_stall_test, &which, sizeof(int)) != cudaSuccess ||
+      cudaMemcpyToSymbol(umma::g_wait_limit_ns, &limit, sizeof(uint64_t)) != cudaSuccess)
+    return BASED_ERR_CUDA;
+  return BASED_OK;
 }
 
 based_status_t based_get_device_error(based_stream_t stream) {

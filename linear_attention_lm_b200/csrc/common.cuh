@@ -24,6 +24,17 @@ __device__ __forceinline__ void record_device_error(int code) {
   atomicCAS(&g_device_status, (int)BASED_OK, code);
 }
 
+// Test hook (based_debug_stall): which input load the first CTA of a kernel
+// leaves out, so that the wait for it runs out; 0 = none.
+constexpr int kStallNone = 0;
+constexpr int kStallLinattnV = 1;  // linear-attention prefill: the V tile of its second chunk
+constexpr int kStallWindowV = 2;   // window attention: its V tile
+__device__ int g_stall_test = kStallNone;
+
+__device__ __forceinline__ bool stall_test(int which) {
+  return blockIdx.x == 0 && *const_cast<const volatile int*>(&g_stall_test) == which;
+}
+
 // One Taylor feature of a 16-vector held in shared memory or registers.
 __device__ __forceinline__ float phi_feature(const float* x, int f) {
   if (f == 0) return 1.0f;

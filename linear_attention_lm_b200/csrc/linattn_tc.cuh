@@ -65,6 +65,13 @@
 #include "common.cuh"
 #include "umma.cuh"
 
+// Optional per-chunk event stamps for performance analysis: a build may define
+// BASED_TC_TRACE(event, chunk) to record when each warp passes the points
+// marked below; by default the marks compile to nothing.
+#ifndef BASED_TC_TRACE
+#define BASED_TC_TRACE(event, chunk) ((void)0)
+#endif
+
 namespace based {
 
 constexpr int kTcChunk = 128;          // tokens per chunk (MMA M)
@@ -253,7 +260,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                            ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::kBar);
   uint64_t* bar_tma = bars + 16;     // [kVBuf] V stage landed
-  uint64_t* bar_phi = bars + 2;      // feature maps + Q/K tiles written (group A)
+  uint64_t* bar_qk = bars + 2;       // Q/K tiles and phiK written (group F)
+  uint64_t* bar_phiq = bars + 14;    // phiQ written (group F)
+  uint64_t* bar_fin = bars + 15;     // every MMA of this CTA complete (commit)
   uint64_t* bar_u = bars + 3;        // #1 done (commit)
   uint64_t* bar_p = bars + 4;        // P written (group A)
   uint64_t* bar_m25 = bars + 5;      // #5 and #2 done (commit): feature buffers free
@@ -279,7 +288,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (tid == 0) {
     for (int sidx = 0; sidx < Lay::kVBuf; ++sidx) umma::mbar_init(bar_tma + sidx, 1);
-    umma::mbar_init(bar_phi, kTcGroup);
+    umma::mbar_init(bar_qk, kTcGroup);
+    umma::mbar_init(bar_phiq, kTcGroup);
+    umma::mbar_init(bar_fin, 1);
     umma::mbar_init(bar_u, 1);
     umma::mbar_init(bar_p, kTcGroup);
     umma::mbar_init(bar_m25, 1);
@@ -323,9 +334,70 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   umma::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tm_lane = static_cast<uint32_t>(quad * 32) << 16;
+  BASED_TC_TRACE(15, 0);
   auto fail = [&]() {
     record_device_error(BASED_ERR_TIMEOUT);
     *abort_flag = 1;
+  };
+  // [S|z]^T -> shared memory as [feature][value column | z] (stride DV + 4), then
+  // coalesced rows of the 273-row layout (or of the segment partial).  Called
+  // by the 128 threads of one warp group (t = index in the group, TMEM quadrant
+  // = warp & 3) once the last #5 is complete and the feature-map buffers are no
+  // longer read.
+  auto export_kst = [&](int t) {
+    if constexpr (Lay::kSt) {
+    const bool any_st = has_init || c_begin < c_end;
+    constexpr int kStr = DV + 4;  // keeps each feature row 16-byte aligned
+    float* stage = reinterpret_cast<float*>(sm + Lay::kPhiK);
+    int* rowmap = reinterpret_cast<int*>(stage + kSymFP * kStr);  // [273]: 2 f + (1 if / sqrt 2)
+    static_assert(Lay::kPhiKBuf * 40960 >= (kSymFP * kStr + kF) * 4, "export staging");
+    if (quad < 3) {
+      // two TMEM round trips of 80 features each
+#pragma unroll 1
+      for (int g = 0; g < 2; ++g) {
+        float sv[80];
+        umma::tmem_ld80(tmem + Lay::kTmS0 + tm_lane + g * 80, sv);
+        if (t <= DV) {
+#pragma unroll
+          for (int i = 0; i < 80; ++i) stage[(g * 80 + i) * kStr + t] = any_st ? sv[i] : 0.0f;
+        }
+      }
+    }
+    for (int f = t; f < kSymFP; f += kTcGroup) {
+      int r0 = -1, r1 = -1;
+      float scale = 1.0f;
+      const int nrows = tc_feature_rows(f, &r0, &r1, &scale);
+      const int code = 2 * f + (nrows == 2 ? 1 : 0);
+      if (nrows >= 1) rowmap[r0] = code;
+      if (nrows == 2) rowmap[r1] = code;
+    }
+    umma::named_sync(1, kTcGroup);
+    if (kStateOnly) {
+      float* part = p.partial + ((size_t)bh * (p.n_seg - 1) + seg) * kSymFP * NA;
+      for (int i = t; i < kSymFP * NA; i += kTcGroup) {
+        const int f = i / NA, j = i - f * NA;
+        part[i] = j <= DV ? stage[f * kStr + j] : 0.0f;
+      }
+    } else if (seg == p.n_seg - 1) {
+      if (p.state_kv) {
+        float4* skv = reinterpret_cast<float4*>(p.state_kv + (size_t)bh * kF * DV);
+        for (int i = t; i < kF * (DV / 4); i += kTcGroup) {
+          const int r = i / (DV / 4), j = (i - r * (DV / 4)) * 4;
+          const int code = rowmap[r];
+          const float sc = (code & 1) ? 0.70710678118654752f : 1.0f;
+          const float4 v4 = *reinterpret_cast<const float4*>(stage + (code >> 1) * kStr + j);
+          skv[i] = make_float4(v4.x * sc, v4.y * sc, v4.z * sc, v4.w * sc);
+        }
+      }
+      if (p.state_k) {
+        float* sk = p.state_k + (size_t)bh * kF;
+        for (int r = t; r < kF; r += kTcGroup) {
+          const int code = rowmap[r];
+          sk[r] = stage[(code >> 1) * kStr + DV] * ((code & 1) ? 0.70710678118654752f : 1.0f);
+        }
+      }
+    }
+    }
   };
 
   if (warp == 12) {
@@ -335,12 +407,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                      sP = umma::smem_u32(sm + Lay::kP), sPhiQ = umma::smem_u32(sm + Lay::kPhiQ),
                      sS = umma::smem_u32(sm + Lay::kS);
       constexpr uint32_t kVBytes = DV * kTcChunk * 2;
+      // returns whether a load was issued (the stall test leaves one out)
       auto issue_v = [&](int c, int stage) {
+        if (c == c_begin + 1 && stall_test(kStallLinattnV)) return 0u;
         umma::mbar_arrive_expect_tx(bar_tma + stage, kVBytes);
 #pragma unroll
         for (int blk = 0; blk < DV / 64; ++blk)
           umma::tma_load_3d(sm + Lay::kV + stage * Lay::kVStage + blk * 16384, &vmap,
                             bar_tma + stage, blk * 64, c * kTcChunk, bh);
+        return 1u;
       };
       // descriptors are computed once per buffer and stepped along K by adding
       // the start-address increment (16-byte units) to their low word
@@ -363,10 +438,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // per stage (bit s): a load in flight, and the parity of the phase it completes
       // (bit masks rather than arrays, which would live in local memory)
       uint32_t inflight = 0, vphase = 0;
-      for (int sidx = 0; sidx < Lay::kVBuf && c_begin + sidx < c_end; ++sidx) {
-        issue_v(c_begin + sidx, sidx);
-        inflight |= 1u << sidx;
-      }
+      for (int sidx = 0; sidx < Lay::kVBuf && c_begin + sidx < c_end; ++sidx)
+        inflight |= issue_v(c_begin + sidx, sidx) << sidx;
       int n_done = 0;  // chunks whose MMAs were all issued and committed
       for (int c = c_begin; c < c_end && !*abort_flag; ++c) {
         const int it = c - c_begin;
@@ -382,7 +455,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int kk = has_init ? it : it - 1;
         const uint32_t ph_ss = kk & 1;
         const uint64_t d_s = (kk & 1) ? d_s1 : d_s0;
-        if (!umma::mbar_wait(bar_phi, ph)) { fail(); break; }
+        if (!umma::mbar_wait(bar_qk, ph)) { fail(); break; }
+        BASED_TC_TRACE(0, it);
         // when O shares TMEM with U, #1 may only overwrite it once the epilogue
         // group has read the previous chunk's O
         if (!kStateOnly && !Lay::kEarlyO && has_state) {
@@ -393,7 +467,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           umma::mma_bf16(tmem + Lay::kTmU, d_q, d_k, id_u, 0);
           umma::mma_commit(bar_u);
         }
+        BASED_TC_TRACE(1, it);
         if (!umma::mbar_wait(bar_tma + stage, (vphase >> stage) & 1u)) { fail(); break; }
+        BASED_TC_TRACE(2, it);
         inflight &= ~(1u << stage);
         vphase ^= 1u << stage;
         // #5 overwrites the state: the epilogue group must have read (and copied)
@@ -401,6 +477,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!kStateOnly && Lay::kEarlyO && has_state) {
           if (!umma::mbar_wait(Lay::kTm ? bar_sread : bar_ss, ph_ss)) { fail(); break; }
         }
+        BASED_TC_TRACE(3, it);
         umma::tc_fence_after();
         // K step of 16 tokens: +256 B in the no-swizzle phiK layout (2 core
         // matrices), +2048 B (16 rows of 128 B) in the swizzled V tile
@@ -421,12 +498,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         if (Lay::kTm) {
           umma::mma_commit(bar_m5);
+          BASED_TC_TRACE(4, it);
           // refill the stage of chunk c-1 (its MMAs are done by now) with chunk
           // c + kVBuf - 1
           if (Lay::kVBuf > 1 && it > 0 && c + Lay::kVBuf - 1 < c_end) {
             if (!umma::mbar_wait(bar_o, (it - 1) & 1)) { fail(); break; }
-            issue_v(c + Lay::kVBuf - 1, (it - 1) % Lay::kVBuf);
-            inflight |= 1u << ((it - 1) % Lay::kVBuf);
+            inflight |= issue_v(c + Lay::kVBuf - 1, (it - 1) % Lay::kVBuf)
+                        << ((it - 1) % Lay::kVBuf);
           }
         }
         if (!kStateOnly) {
@@ -434,12 +512,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (!umma::mbar_wait(bar_p, ph)) { fail(); break; }
             umma::tc_fence_after();
           }
+          // phiQ of this chunk is written (waited for even when #2 is skipped, so
+          // that the group's arrivals for chunk c+1 follow this phase's completion)
+          if (!umma::mbar_wait(bar_phiq, ph)) { fail(); break; }
           if (has_state) {
             // #2 overwrites O: the epilogue group must have read the previous O
             if (Lay::kTm) {
               if (!umma::mbar_wait(bar_ss, ph_ss)) { fail(); break; }
-              umma::tc_fence_after();
             }
+            umma::tc_fence_after();
+            BASED_TC_TRACE(5, it);
             // K step of 16 features: +256 B in both no-swizzle layouts, 8 TMEM columns
 #pragma unroll
             for (int ks = 0; ks < kSymFP / 16; ++ks) {
@@ -452,11 +534,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
         umma::mma_commit(bar_m25);
+        BASED_TC_TRACE(6, it);
         if (!kStateOnly) {
           if (Lay::kEarlyO) {
             if (!umma::mbar_wait(bar_p, ph)) { fail(); break; }
             umma::tc_fence_after();
           }
+          BASED_TC_TRACE(7, it);
 #pragma unroll
           for (int ks = 0; ks < kTcChunk / 16; ++ks) {
             const uint32_t acc = has_state || ks > 0;
@@ -467,17 +551,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
         umma::mma_commit(bar_o);
+        BASED_TC_TRACE(8, it);
         ++n_done;
         // refill the stage this chunk used once its MMAs are done
         const int c_next = c + Lay::kVBuf;
         if (!Lay::kTm && c_next < c_end) {
           if (!umma::mbar_wait(bar_o, ph)) { fail(); break; }
-          issue_v(c_next, stage);
-          inflight |= 1u << stage;
+          inflight |= issue_v(c_next, stage) << stage;
         }
       }
       // the last chunk's MMAs must be complete before the state is read out
       if (n_done > 0 && !umma::mbar_wait(bar_o, (n_done - 1) & 1)) fail();
+      // and every MMA this thread issued (an aborted chunk may have left some)
+      // before the TMEM is released
+      umma::mma_commit(bar_fin);
+      if (!umma::mbar_wait(bar_fin, 0)) fail();
       // an aborted run may still have V loads in flight: wait for them (bounded)
       for (int sidx = 0; sidx < Lay::kVBuf; ++sidx)
         if ((inflight >> sidx) & 1u) umma::mbar_wait(bar_tma + sidx, (vphase >> sidx) & 1u);
@@ -491,6 +579,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // ---- scores: P = mask(1 + u/4 + u^2/32) * sc ------------------------------------
       if (!umma::mbar_wait(bar_u, it & 1)) { fail(); break; }
       if (!Lay::kTm && it > 0 && !umma::mbar_wait(bar_o, (it - 1) & 1)) { fail(); break; }
+      BASED_TC_TRACE(0, it);
       umma::tc_fence_after();
       const float sc = tc_chunk_scale((long long)t0 + kTcChunk);
       const float c0 = sc, c1 = 0.25f * sc, c2 = 0.03125f * sc;
@@ -511,22 +600,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // P (bf16 pairs) of key block b (32 keys) goes to U columns [16b, 16b + 16),
         // which this thread has read already (they belong to block b / 2 <= b);
         // one loop body for every block keeps the code small
+        // blocks are taken two at a time (one TMEM load of 64 columns) while two
+        // remain, so a warp pays at most two load round trips
         const int row = lane + 32 * quad;  // this thread's token within the chunk
 #pragma unroll 1
-        for (int b = 0; b <= quad; ++b) {
-          float u[32];
-          umma::tmem_ld32(tmem + Lay::kTmU + tm_lane + 32 * b, u);
+        for (int b = 0; b <= quad; b += 2) {
+          const bool two = b + 1 <= quad;  // warp-uniform
+          float u[64];
+          if (two) umma::tmem_ld64(tmem + Lay::kTmU + tm_lane + 32 * b, u);
+          else umma::tmem_ld32(tmem + Lay::kTmU + tm_lane + 32 * b, u);
           const int lim = row - 32 * b;  // keys 32b + j with j > lim lie in the future
-          uint32_t pk[16];
+          uint32_t pk[32];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
+          for (int e = 0; e < 32; ++e) {
             float w0 = fmaf(u[2 * e], fmaf(u[2 * e], c2, c1), c0);
             float w1 = fmaf(u[2 * e + 1], fmaf(u[2 * e + 1], c2, c1), c0);
             if (2 * e > lim) w0 = 0.0f;
             if (2 * e + 1 > lim) w1 = 0.0f;
             pk[e] = as_u32(__floats2bfloat162_rn(w0, w1));
           }
-          umma::tmem_st16_nowait(tmem + Lay::kTmU + tm_lane + 16 * b, pk);
+          if (two) umma::tmem_st32_nowait(tmem + Lay::kTmU + tm_lane + 16 * b, pk);
+          else umma::tmem_st16_nowait(tmem + Lay::kTmU + tm_lane + 16 * b, pk);
         }
         uint32_t zero[16];
 #pragma unroll
@@ -557,7 +651,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         umma::fence_async_smem();
         umma::tc_fence_before();
       }
+      BASED_TC_TRACE(1, it);
       umma::mbar_arrive(bar_p);
+    }
+    if constexpr (Lay::kSt && !kStateOnly) {
+      // the final state (or nothing, for an empty segment) is exported here, as
+      // soon as the last #5 completes, while #2, #4 and the last output still run
+      if (c_begin < c_end) {
+        const bool ok = !*abort_flag && umma::mbar_wait(bar_m5, (c_end - 1 - c_begin) & 1);
+        if (umma::named_sync_all(1, kTcGroup, ok)) {
+          umma::tc_fence_after();
+          export_kst(t);
+        } else if (!*abort_flag) {
+          fail();
+        }
+      }
     }
   } else if (warp < 8) {
     // ================= group F: feature maps and Q/K tiles of chunk c =================
@@ -594,9 +702,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // With a single phiK buffer (and for the smem phiQ tile) wait until the
       // previous chunk's #5 and #2 are done.  With two phiK buffers, this chunk's
       // buffer was released by the wait of the previous iteration.
+      BASED_TC_TRACE(0, it);
       if (!Lay::kTm && it > 0 && !umma::mbar_wait(bar_m25, (it - 1) & 1)) { fail(); break; }
       // the Q/K tiles are rewritten once #1 of the previous chunk has read them
       if (!kStateOnly && it > 0 && !umma::mbar_wait(bar_u, (it - 1) & 1)) { fail(); break; }
+      BASED_TC_TRACE(1, it);
       // ---- phiK and Q/K tiles -------------------------------------------------------
       {
         __nv_bfloat162 XK[8], YK[8];
@@ -618,7 +728,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           *reinterpret_cast<uint4*>(krow + 128) = kr[1];
         }
       }
-      if (Lay::kTm && it > 0 && !umma::mbar_wait(bar_m25, (it - 1) & 1)) { fail(); break; }
+      umma::fence_async_smem();
+      BASED_TC_TRACE(2, it);
+      // An arrival for chunk c must follow the completion of the phase of chunk
+      // c-1 (arrivals carry no phase, and the four warps run at their own pace).
+      // The main pass has that through its wait for #1 of chunk c-1; the
+      // state-only pass waits for the MMAs of chunk c-1 before arriving.
+      if (kStateOnly && Lay::kTm && it > 0 && !umma::mbar_wait(bar_m25, (it - 1) & 1)) {
+        fail();
+        break;
+      }
+      umma::mbar_arrive(bar_qk);
+      if (!kStateOnly && Lay::kTm && it > 0 && !umma::mbar_wait(bar_m25, (it - 1) & 1)) {
+        fail();
+        break;
+      }
+      BASED_TC_TRACE(3, it);
       // ---- phiQ (TMEM operand, or smem) ------------------------------------------------
       if (!kStateOnly) {
         __half2 XQ[8], YQ[8];
@@ -650,9 +775,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       qr[0] = qn[0]; qr[1] = qn[1]; kr[0] = kn[0]; kr[1] = kn[1];
       load_qk(c + 2, qn, kn);
-      umma::fence_async_smem();
-      umma::tc_fence_before();
-      umma::mbar_arrive(bar_phi);
+      if (!kStateOnly) {
+        umma::fence_async_smem();
+        umma::tc_fence_before();
+        BASED_TC_TRACE(4, it);
+        umma::mbar_arrive(bar_phiq);
+      }
     }
   } else if (!kStateOnly) {
     // ================= group E: epilogue of chunk c (output, fp16 state copy) =================
@@ -679,15 +807,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         };
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
-          float sv[64];
-          umma::tmem_ld64(base + 64 * h, sv);
+          float sv[80];
+          umma::tmem_ld80(base + 80 * h, sv);
 #pragma unroll
-          for (int g = 0; g < 8; ++g) put8(sv + 8 * g, 8 * h + g);
+          for (int g = 0; g < 10; ++g) put8(sv + 8 * g, 10 * h + g);
         }
-        float sv[32];
-        umma::tmem_ld32(base + 128, sv);
-#pragma unroll
-        for (int g = 0; g < 4; ++g) put8(sv + 8 * g, 16 + g);
         return;
       }
       for (int tile = 0; tile < 2; ++tile) {
@@ -783,13 +907,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (Lay::kTm && c + 1 < c_end) {
         // the state after #5 of this chunk, copied while #2 and #4 still run
         if (!umma::mbar_wait(bar_m5, it & 1)) { fail(); break; }
+        BASED_TC_TRACE(0, it);
         umma::tc_fence_after();
         copy_state(tc_chunk_scale((long long)t0 + 2 * kTcChunk));
         umma::fence_async_smem();
         umma::tc_fence_before();
+        BASED_TC_TRACE(1, it);
         umma::mbar_arrive(bar_sread);
       }
       if (!umma::mbar_wait(bar_o, it & 1)) { fail(); break; }
+      BASED_TC_TRACE(2, it);
       umma::tc_fence_after();
       if constexpr (Lay::kTm) {
         float o[64], den;
@@ -800,6 +927,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           umma::mbar_arrive(bar_ss);
           ++kk;
         }
+        BASED_TC_TRACE(3, it);
         // y row t into the swizzled staging tile; one TMA store per chunk
         uint8_t* ybuf = sm + Lay::kY;
         if (t == 0) {  // the store of chunk c-1 has finished reading ybuf
@@ -845,6 +973,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ++kk;
       }
       if constexpr (Lay::kTm) {
+        BASED_TC_TRACE(4, it);
         umma::mbar_arrive(bar_yfull);
         if (t == 0) {
           if (!umma::mbar_wait(bar_yfull, it & 1)) { fail(); break; }
@@ -864,59 +993,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int t = tid - 2 * kTcGroup;
     const bool any_st = has_init || c_begin < c_end;
     if constexpr (Lay::kSt) {
-      // [S|z]^T -> shared memory as [feature][value column | z] (stride DV + 4),
-      // then coalesced rows of the 273-row layout (or of the segment partial).
-      // The feature-map buffers are free: every MMA has completed.
-      constexpr int kStr = DV + 4;  // keeps each feature row 16-byte aligned
-      float* stage = reinterpret_cast<float*>(sm + Lay::kPhiK);
-      int* rowmap = reinterpret_cast<int*>(stage + kSymFP * kStr);  // [273]: 2 f + (1 if / sqrt 2)
-      static_assert(Lay::kPhiKBuf * 40960 >= (kSymFP * kStr + kF) * 4, "export staging");
-      if (quad < 3) {
-        // two TMEM round trips of 80 features each
-#pragma unroll 1
-        for (int g = 0; g < 2; ++g) {
-          float sv[80];
-          umma::tmem_ld80(tmem + Lay::kTmS0 + tm_lane + g * 80, sv);
-          if (t <= DV) {
-#pragma unroll
-            for (int i = 0; i < 80; ++i) stage[(g * 80 + i) * kStr + t] = any_st ? sv[i] : 0.0f;
-          }
-        }
-      }
-      for (int f = t; f < kSymFP; f += kTcGroup) {
-        int r0 = -1, r1 = -1;
-        float scale = 1.0f;
-        const int nrows = tc_feature_rows(f, &r0, &r1, &scale);
-        const int code = 2 * f + (nrows == 2 ? 1 : 0);
-        if (nrows >= 1) rowmap[r0] = code;
-        if (nrows == 2) rowmap[r1] = code;
-      }
-      umma::named_sync(1, kTcGroup);
-      if (kStateOnly) {
-        float* part = p.partial + ((size_t)bh * (p.n_seg - 1) + seg) * kSymFP * NA;
-        for (int i = t; i < kSymFP * NA; i += kTcGroup) {
-          const int f = i / NA, j = i - f * NA;
-          part[i] = j <= DV ? stage[f * kStr + j] : 0.0f;
-        }
-      } else if (seg == p.n_seg - 1) {
-        if (p.state_kv) {
-          float4* skv = reinterpret_cast<float4*>(p.state_kv + (size_t)bh * kF * DV);
-          for (int i = t; i < kF * (DV / 4); i += kTcGroup) {
-            const int r = i / (DV / 4), j = (i - r * (DV / 4)) * 4;
-            const int code = rowmap[r];
-            const float sc = (code & 1) ? 0.70710678118654752f : 1.0f;
-            const float4 v4 = *reinterpret_cast<const float4*>(stage + (code >> 1) * kStr + j);
-            skv[i] = make_float4(v4.x * sc, v4.y * sc, v4.z * sc, v4.w * sc);
-          }
-        }
-        if (p.state_k) {
-          float* sk = p.state_k + (size_t)bh * kF;
-          for (int r = t; r < kF; r += kTcGroup) {
-            const int code = rowmap[r];
-            sk[r] = stage[(code >> 1) * kStr + DV] * ((code & 1) ? 0.70710678118654752f : 1.0f);
-          }
-        }
-      }
+      // the main pass exported from group P already (right after its last #5)
+      if (kStateOnly || c_begin == c_end) export_kst(t);
     }
     for (int tile = 0; tile < 2 && !Lay::kSt; ++tile) {
       if (tile == 1 && quad > 1) break;
@@ -964,6 +1042,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   umma::tc_fence_before();
   __syncthreads();
+  BASED_TC_TRACE(14, 0);
   if (warp == 0) umma::tmem_dealloc(tmem, kTcTmemCols);
 }
 

@@ -24,8 +24,9 @@ namespace umma {
 
 constexpr uint32_t kLayoutNone = 0;
 constexpr uint32_t kLayoutSW128 = 2;
-// Bounded waits give up after this many nanoseconds of %globaltimer.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Bounded waits give up after this many nanoseconds of %globaltimer (2 s by
+// default; a test may shorten it with based_debug_stall).
+__device__ uint64_t g_wait_limit_ns = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -68,13 +69,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // warp-specialised kernel stay small in the instruction cache.
 __device__ __noinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = global_timer_ns();
+  const uint64_t limit = *const_cast<const volatile uint64_t*>(&g_wait_limit_ns);
   while (true) {
     for (int i = 0; i < 256; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    if (global_timer_ns() - t0 > limit) return false;
   }
 }
-// Wait for the phase with the given parity to complete; false after kWaitLimitNs.
+// Wait for the phase with the given parity to complete; false after g_wait_limit_ns.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   return mbar_wait_spin(bar, parity);
@@ -332,6 +334,20 @@ __device__ __forceinline__ void bulk_wait() {
 // Named barrier over `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// Named barrier that also returns, to every participant, whether `pred` held
+// for all of them (so a group takes a decision together).
+__device__ __forceinline__ bool named_sync_all(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
 }
 
 // ---------------------------------------------------------------- MMA

@@ -52,30 +52,48 @@ __global__ void __launch_bounds__(kWtThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
-  uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + Lay::kBar);
+  uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + Lay::kBar);  // Q and K landed
   uint64_t* bar_s = bar_tma + 1;
   uint64_t* bar_o = bar_tma + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_tma + 3);
   int* abort_flag = reinterpret_cast<int*>(bar_tma + 4);
+  uint64_t* bar_v = bar_tma + 5;                                      // V landed
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tile = blockIdx.x % n_tiles;
   const int bh = blockIdx.x / n_tiles;
   const int t0 = tile * kWtQ;
 
+  // Q and K first (S needs them), V on its own barrier (only P V needs it)
   if (tid == 0) {
     umma::mbar_init(bar_tma, 1);
+    umma::mbar_init(bar_v, 1);
     umma::mbar_init(bar_s, 1);
     umma::mbar_init(bar_o, 1);
     *abort_flag = 0;
     umma::fence_mbar_init();
-    constexpr uint32_t bytes = (kWtQ + 2 * kWtKeys) * DH * 2;
-    umma::mbar_arrive_expect_tx(bar_tma, bytes);
+    umma::mbar_arrive_expect_tx(bar_tma, (kWtQ + kWtKeys) * DH * 2);
 #pragma unroll
     for (int b = 0; b < DH / 64; ++b) {
       umma::tma_load_3d(sm + Lay::kQ + b * kWtQ * 128, &qmap, bar_tma, b * 64, t0, bh);
       umma::tma_load_3d(sm + Lay::kK + b * kWtKeys * 128, &kmap, bar_tma, b * 64, t0 - 64, bh);
-      umma::tma_load_3d(sm + Lay::kV + b * kWtKeys * 128, &vmap, bar_tma, b * 64, t0 - 64, bh);
+    }
+    if (!stall_test(kStallWindowV)) {  // the stall test leaves the V tile out
+      umma::mbar_arrive_expect_tx(bar_v, kWtKeys * DH * 2);
+#pragma unroll
+      for (int b = 0; b < DH / 64; ++b)
+        umma::tma_load_3d(sm + Lay::kV + b * kWtKeys * 128, &vmap, bar_v, b * 64, t0 - 64, bh);
+    }
+  }
+  __syncthreads();  // barrier initialisation visible to every thread
+  // TMEM is taken only once Q and K have landed: a CTA that still waits for
+  // its loads holds none, so the TMEM of the SM serves the CTAs that compute
+  // while further CTAs' loads are in flight
+  {
+    const bool ok = umma::mbar_wait(bar_tma, 0);
+    if (!ok && tid == 0) {
+      record_device_error(BASED_ERR_TIMEOUT);
+      *abort_flag = 1;
     }
   }
   if (warp == 0) {
@@ -92,10 +110,7 @@ __global__ void __launch_bounds__(kWtThreads, 1)
 
   // ---- S = Q K^T ----------------------------------------------------------------
   if (tid == 0) {
-    if (!umma::mbar_wait(bar_tma, 0)) {
-      record_device_error(BASED_ERR_TIMEOUT);
-      *abort_flag = 1;
-    } else {
+    if (!*abort_flag) {
       umma::tc_fence_after();
       const uint32_t id = umma::idesc_bf16(kWtQ, kWtKeys, false, false);
 #pragma unroll
@@ -183,6 +198,14 @@ __global__ void __launch_bounds__(kWtThreads, 1)
 
   // ---- O = P V --------------------------------------------------------------------------
   if (tid == 0) {
+    if (!umma::mbar_wait(bar_v, 0)) {
+      record_device_error(BASED_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+  }
+  __syncthreads();
+  if (*abort_flag) goto done;
+  if (tid == 0) {
     const uint32_t id = umma::idesc_bf16(kWtQ, DH, false, true);
 #pragma unroll
     for (int k0 = 0; k0 < kWtKeys; k0 += 16)
@@ -231,7 +254,10 @@ __global__ void __launch_bounds__(kWtThreads, 1)
   }
 done:
   // an aborted tile may still have its loads in flight: wait for them (bounded)
-  if (tid == 0 && *abort_flag) umma::mbar_wait(bar_tma, 0);
+  if (tid == 0 && *abort_flag) {
+    umma::mbar_wait(bar_tma, 0);
+    if (!stall_test(kStallWindowV)) umma::mbar_wait(bar_v, 0);
+  }
   umma::tc_fence_before();
   __syncthreads();
   if (warp == 0) umma::tmem_dealloc(tmem, Lay::kTmemCols);
