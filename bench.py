@@ -569,14 +569,16 @@ def run_projections(args, lab, dev, world, peaks, warm):
             ("baseconv", conv_step, 2.0 * B * L * dm * dm, 1,
              "BaseConv block, x [8, 2048, 1024], dense 1024x1024 + bias, 3 causal taps"),
             ("linattn_bwd", bwd_step, 480.0 * B * H * L * (L + 1) / 2, 2,
-             "gradient of the linear attention, B=8 H=16 L=2048 d=16 d_v=64 (quadratic form, "
-             "480 flop per (t, s) pair)"),
+             "gradient of the linear attention, bf16, B=8 H=16 L=2048 d=16 d_v=64 (quadratic "
+             "form on the tensor cores; 480 flop per (t, s) pair counted)"),
             ("window_bwd", wbwd_step, 10.0 * 64 * B * H * w_pairs, 2,
              "gradient of the window attention, B=8 H=16 L=2048 d_h=64 W=64 (10 d_h flop per "
              "(query, key) pair in the band)")):
         ms = timed(fn, 10 if name.endswith("bwd") else n)
         tf = flops / (ms / 1e3) / 1e12
-        if name.endswith("bwd"):
+        if name == "linattn_bwd":
+            kern, bound, pk, src = "linattn_bwd_tc", "tensor", peak, peaks["source"]
+        elif name.endswith("bwd"):
             # CUDA-core fp32 FMA peak: 148 SMs x 128 FMA/clk x 2 flop x 1.965 GHz
             kern, bound, pk, src = name, "alu", FP32_FMA_TFLOPS, "unit counts x max clock"
         else:

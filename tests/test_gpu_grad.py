@@ -1,9 +1,16 @@
-"""GPU parity of the linear-attention gradient (based_linattn_bwd) against the
-fp64 gradient oracle (oracle/grad.py) on the same seeded inputs.
+"""GPU parity of the attention gradients (based_linattn_bwd,
+based_window_attn_bwd) against the fp64 gradient oracle (oracle/grad.py) on
+the same seeded inputs.
 
-The kernels compute in fp32 from inputs that widen exactly (bf16 or fp32), so
-the per-(b, h) relative L2 error of each gradient is bounded by fp32
-accumulation over at most L terms: 2e-4 here.
+fp32 inputs, and the window attention's gradient in both dtypes, are computed
+in fp32 on CUDA cores: the per-(b, h) relative L2 error is bounded by fp32
+accumulation over at most L terms, 2e-4 here.  The linear attention's bf16
+gradient runs on the tensor cores with bf16 operands for three intermediates
+(w, e = dw (1 + u'), dN): each rounding is at most 2^-9 relative, a product term
+carries at most two of them, and the terms of each sum are independent, so the
+relative L2 error of a gradient is about 2 x 2^-9 / sqrt(3) ~ 2.3e-3 for terms
+of random sign; 1e-2 leaves room for the partial cancellation in dq and dk
+(their terms sum to nearly zero for every query).
 """
 import numpy as np
 import pytest
@@ -15,6 +22,11 @@ from oracle import grad
 
 pytestmark = pytest.mark.gpu
 REL = 2e-4
+REL_LIN_BF16 = 1e-2  # linear attention, bf16 inputs, tensor-core path
+
+
+def lin_rel(dtype):
+    return REL_LIN_BF16 if dtype == torch.bfloat16 else REL
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -56,9 +68,10 @@ def test_linattn_grad_matches_oracle(B, H, L, dv, eps, dtype):
     torch.cuda.synchronize()
     assert lab.based_get_device_error() == 0
     rq, rk, rv = grad.linattn_grad(q64, k64, v64, dy64, eps)
-    assert head_rel_l2(dq.double().cpu().numpy(), rq) <= REL
-    assert head_rel_l2(dk.double().cpu().numpy(), rk) <= REL
-    assert head_rel_l2(dvv.double().cpu().numpy(), rv) <= REL
+    errs = [head_rel_l2(g.double().cpu().numpy(), r) for g, r in ((dq, rq), (dk, rk), (dvv, rv))]
+    print(f"linattn grad {dtype} B={B} H={H} L={L} dv={dv}: rel L2 dq {errs[0]:.2e} "
+          f"dk {errs[1]:.2e} dv {errs[2]:.2e}")
+    assert max(errs) <= lin_rel(dtype), errs
 
 
 def test_linattn_grad_layer_shape_sampled():
@@ -72,9 +85,11 @@ def test_linattn_grad_layer_shape_sampled():
     for b, h in ((0, 0), (3, 7), (7, 15)):
         sl = (slice(b, b + 1), slice(h, h + 1))
         rq, rk, rv = grad.linattn_grad(*(t[sl].double().numpy() for t in (q, k, v, dy)), 1e-6)
-        assert head_rel_l2(dq[sl].double().cpu().numpy(), rq) <= REL
-        assert head_rel_l2(dk[sl].double().cpu().numpy(), rk) <= REL
-        assert head_rel_l2(dvv[sl].double().cpu().numpy(), rv) <= REL
+        errs = [head_rel_l2(g[sl].double().cpu().numpy(), r)
+                for g, r in ((dq, rq), (dk, rk), (dvv, rv))]
+        print(f"linattn grad layer_360m ({b}, {h}): rel L2 dq {errs[0]:.2e} dk {errs[1]:.2e} "
+              f"dv {errs[2]:.2e}")
+        assert max(errs) <= REL_LIN_BF16, errs
 
 
 # ------------------------------------------------------------------ window attention
