@@ -350,6 +350,13 @@ def based_linattn_bwd(q, k, v, dy, dq, dk, dv, eps: float = 1e-6, workspace=None
     return dq, dk, dv
 
 
+def based_window_attn_bwd_workspace_bytes(B, H, L) -> int:
+    n = load_library().based_window_attn_bwd_workspace_bytes(B, H, L)
+    if n == ctypes.c_size_t(-1).value:
+        raise BasedError("based_window_attn_bwd_workspace_bytes", 1)
+    return n
+
+
 def based_window_attn_bwd(q, k, v, dy, dq, dk, dv, window: int = 64, workspace=None,
                           stream=None):
     """Gradients dq, dk, dv (float32, written) of based_window_attn_fwd given dy."""
@@ -363,8 +370,7 @@ def based_window_attn_bwd(q, k, v, dy, dq, dk, dv, window: int = 64, workspace=N
     _cuda(dev)
     ts = _torch_stream(stream, dev)
     with torch.cuda.device(dev):
-        nbytes = load_library().based_window_attn_bwd_workspace_bytes(B, H, L) \
-            if workspace is None else 0
+        nbytes = based_window_attn_bwd_workspace_bytes(B, H, L) if workspace is None else 0
         workspace, ws_bytes = _workspace(nbytes, workspace, dev, ts, "based_window_attn_bwd")
         st = load_library().based_window_attn_bwd(
             _ptr(q), _ptr(k), _ptr(v), _ptr(dy), _f32(dq), _f32(dk), _f32(dv), B, H, L, dh,

@@ -33,6 +33,11 @@ def test_header_declares_binding_symbols():
     assert declared_functions() == sorted(lab.EXPORTED_SYMBOLS)
 
 
+def test_binding_wraps_every_symbol():
+    for name in lab.EXPORTED_SYMBOLS:
+        assert callable(getattr(lab, name, None)), name
+
+
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
