@@ -186,6 +186,26 @@ based_status_t based_decode_step(const void* q, const void* k, const void* v,
                                  based_dtype_t dt, float eps, based_stream_t stream);
 
 /*
+ * based_decode_step for a batch whose sequences sit at different positions
+ * (prompts of different lengths; the Based README's generation example decodes
+ * a batch of prompts): identical arguments, except that `pos` is a DEVICE
+ * array of B int64 positions (8-byte aligned; read on the GPU; may be NULL
+ * when the window part is skipped).  Only the window part uses positions:
+ * sequence b's new window k/v go to slot pos[b] mod window and its softmax
+ * covers the slots holding positions max(0, pos[b]-window+1) .. pos[b].  A
+ * negative entry cannot be checked on the host: the kernel leaves that
+ * sequence's window heads untouched (ring and wout) and records
+ * BASED_ERR_INVALID_ARG, read with based_get_device_error().
+ */
+based_status_t based_decode_step_at(const void* q, const void* k, const void* v,
+                                    float* state_kv, float* state_k, void* out,
+                                    const void* wq, const void* wk, const void* wv,
+                                    void* k_ring, void* v_ring, void* wout,
+                                    const long long* pos, int B, int H, int d_feat, int d_v,
+                                    int H_w, int d_head, int window,
+                                    based_dtype_t dt, float eps, based_stream_t stream);
+
+/*
  * Gradient of based_linattn_fwd's output (the map the "based/train" README's
  * training views share; see based_linattn_fwd):
  *   w_ts = 1 + u + u^2/2, u = q_t.k_s/sqrt(d_feat), s <= t; y_t = sum_s w_ts v_s / (sum_s w_ts + eps)
@@ -270,7 +290,8 @@ based_status_t based_debug_stall(int which, long long wait_limit_ns);
 /*
  * Synchronise `stream`, then read and clear the library's device status word
  * on the current device.  Returns BASED_OK, or the first error a kernel
- * recorded since the last call (BASED_ERR_TIMEOUT), or BASED_ERR_CUDA if the
+ * recorded since the last call (BASED_ERR_TIMEOUT; BASED_ERR_INVALID_ARG for a
+ * negative position given to based_decode_step_at), or BASED_ERR_CUDA if the
  * synchronisation itself failed.
  */
 based_status_t based_get_device_error(based_stream_t stream);

@@ -33,6 +33,7 @@ EXPORTED_SYMBOLS = ("based_abi_version", "based_binary_version", "based_status_s
                     "based_linattn_workspace_bytes", "based_linattn_fwd",
                     "based_linattn_fwd_noalloc",
                     "based_window_attn_fwd", "based_window_ring_fill", "based_decode_step",
+                    "based_decode_step_at",
                     "based_proj_heads_fwd", "based_baseconv_fwd",
                     "based_linattn_bwd_workspace_bytes", "based_linattn_bwd",
                     "based_window_attn_bwd_workspace_bytes", "based_window_attn_bwd",
@@ -77,6 +78,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.based_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                           _vp, _vp, _ll, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                                           _vp]
+        lib.based_decode_step_at.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                             _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
+                                             _f, _vp]
         lib.based_linattn_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i]
         lib.based_linattn_bwd_workspace_bytes.restype = _sz
         lib.based_linattn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
@@ -90,7 +94,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.based_get_device_error.argtypes = [_vp]
         lib.based_debug_stall.argtypes = [_i, _ll]
         for name in ("based_linattn_fwd", "based_linattn_fwd_noalloc", "based_window_attn_fwd",
-                     "based_window_ring_fill", "based_decode_step", "based_proj_heads_fwd",
+                     "based_window_ring_fill", "based_decode_step", "based_decode_step_at",
+                     "based_proj_heads_fwd",
                      "based_baseconv_fwd", "based_linattn_bwd", "based_window_attn_bwd",
                      "based_debug_stall", "based_get_device_error"):
             getattr(lib, name).restype = _i
@@ -291,8 +296,10 @@ def based_window_ring_fill(k, v, k_ring, v_ring, window: int = 64, stream=None):
 
 
 def based_decode_step(q, k, v, state_kv, state_k, out, wq=None, wk=None, wv=None, k_ring=None,
-                      v_ring=None, wout=None, pos: int = 0, window: int = 64,
+                      v_ring=None, wout=None, pos=0, window: int = 64,
                       eps: float = 1e-6, stream=None):
+    """One decode step.  `pos` is an int (every sequence at that position) or
+    an int64 CUDA tensor of B per-sequence positions (based_decode_step_at)."""
     ref = q if q is not None else wq
     dev = _device_of(ref)
     B = ref.shape[0]
@@ -313,15 +320,35 @@ def based_decode_step(q, k, v, state_kv, state_k, out, wq=None, wk=None, wv=None
             _expect(t, (B, H_w, d_head), name, dev)
         for t, name in ((k_ring, "k_ring"), (v_ring, "v_ring")):
             _expect(t, (B, H_w, int(window), d_head), name, dev)
+    per_seq = isinstance(pos, torch.Tensor)
+    if per_seq:
+        _expect(pos, (B,), "pos", dev)
+        if pos.dtype != torch.int64:
+            raise TypeError("pos must be an int64 tensor of B positions")
     dt = _same_dtype(q, k, v, out, wq, wk, wv, k_ring, v_ring, wout)
     _cuda(dev)
+    lib = load_library()
+    args = (_ptr(q), _ptr(k), _ptr(v), _f32(state_kv), _f32(state_k), _ptr(out), _ptr(wq),
+            _ptr(wk), _ptr(wv), _ptr(k_ring), _ptr(v_ring), _ptr(wout))
+    tail = (B, H, d_feat, d_v, H_w, d_head, int(window), dt, float(eps))
     with torch.cuda.device(dev):
-        st = load_library().based_decode_step(
-            _ptr(q), _ptr(k), _ptr(v), _f32(state_kv), _f32(state_k), _ptr(out), _ptr(wq),
-            _ptr(wk), _ptr(wv), _ptr(k_ring), _ptr(v_ring), _ptr(wout), int(pos), B, H,
-            d_feat, d_v, H_w, d_head, int(window), dt, float(eps),
-            _torch_stream(stream, dev).cuda_stream)
-    _check("based_decode_step", st)
+        if per_seq:
+            st = lib.based_decode_step_at(*args, _ptr(pos), *tail,
+                                          _torch_stream(stream, dev).cuda_stream)
+        else:
+            st = lib.based_decode_step(*args, int(pos), *tail,
+                                       _torch_stream(stream, dev).cuda_stream)
+    _check("based_decode_step_at" if per_seq else "based_decode_step", st)
+
+
+def based_decode_step_at(q, k, v, state_kv, state_k, out, wq, wk, wv, k_ring, v_ring, wout,
+                         pos, window: int = 64, eps: float = 1e-6, stream=None):
+    """based_decode_step with per-sequence positions: pos is an int64 CUDA
+    tensor [B]."""
+    if not isinstance(pos, torch.Tensor):
+        raise TypeError("pos must be an int64 tensor of B positions")
+    based_decode_step(q, k, v, state_kv, state_k, out, wq, wk, wv, k_ring, v_ring, wout, pos,
+                      window, eps, stream)
 
 
 def based_linattn_bwd_workspace_bytes(B, H, L, d_v) -> int:

@@ -519,12 +519,17 @@ based_status_t based_window_ring_fill(const void* k, const void* v, int B, int H
   return launch_status();
 }
 
-based_status_t based_decode_step(const void* q, const void* k, const void* v, float* state_kv,
-                                 float* state_k, void* out, const void* wq, const void* wk,
-                                 const void* wv, void* k_ring, void* v_ring, void* wout,
-                                 long long pos, int B, int H, int d_feat, int d_v, int H_w,
-                                 int d_head, int window, based_dtype_t dt, float eps,
-                                 based_stream_t stream) {
+}  // extern "C"
+
+namespace {
+// Shared body of based_decode_step (one position, pos_arr == null) and
+// based_decode_step_at (per-sequence positions in device memory).
+based_status_t decode_step_impl(const void* q, const void* k, const void* v, float* state_kv,
+                                float* state_k, void* out, const void* wq, const void* wk,
+                                const void* wv, void* k_ring, void* v_ring, void* wout,
+                                long long pos, const long long* pos_arr, int B, int H,
+                                int d_feat, int d_v, int H_w, int d_head, int window,
+                                based_dtype_t dt, float eps, based_stream_t stream) {
   if (B < 0 || H < 0 || H_w < 0 || pos < 0) return BASED_ERR_INVALID_ARG;
   if (dt != BASED_F32 && dt != BASED_BF16) return BASED_ERR_INVALID_ARG;
   const bool lin = q != nullptr || H > 0;
@@ -554,13 +559,41 @@ based_status_t based_decode_step(const void* q, const void* k, const void* v, fl
   DecodeParams p;
   p.q = q; p.k = k; p.v = v; p.S = state_kv; p.z = state_k; p.out = out;
   p.wq = wq; p.wk = wk; p.wv = wv; p.k_ring = k_ring; p.v_ring = v_ring; p.wout = wout;
-  p.pos = pos; p.n_lin = (int)n_lin; p.n_win = (int)n_win;
+  p.pos = pos; p.pos_arr = pos_arr; p.H_w = H_w > 0 ? H_w : 1;
+  p.n_lin = (int)n_lin; p.n_win = (int)n_win;
   p.dh = d_head; p.W = window; p.eps = eps;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool wide = lin && d_v == 128;
   if (dt == BASED_F32)
     return wide ? launch_decode<float, 128>(p, st) : launch_decode<float, 64>(p, st);
   return wide ? launch_decode<__nv_bfloat16, 128>(p, st) : launch_decode<__nv_bfloat16, 64>(p, st);
+}
+}  // namespace
+
+extern "C" {
+
+based_status_t based_decode_step(const void* q, const void* k, const void* v, float* state_kv,
+                                 float* state_k, void* out, const void* wq, const void* wk,
+                                 const void* wv, void* k_ring, void* v_ring, void* wout,
+                                 long long pos, int B, int H, int d_feat, int d_v, int H_w,
+                                 int d_head, int window, based_dtype_t dt, float eps,
+                                 based_stream_t stream) {
+  return decode_step_impl(q, k, v, state_kv, state_k, out, wq, wk, wv, k_ring, v_ring, wout, pos,
+                          nullptr, B, H, d_feat, d_v, H_w, d_head, window, dt, eps, stream);
+}
+
+based_status_t based_decode_step_at(const void* q, const void* k, const void* v,
+                                    float* state_kv, float* state_k, void* out, const void* wq,
+                                    const void* wk, const void* wv, void* k_ring, void* v_ring,
+                                    void* wout, const long long* pos, int B, int H, int d_feat,
+                                    int d_v, int H_w, int d_head, int window, based_dtype_t dt,
+                                    float eps, based_stream_t stream) {
+  const bool win = wq != nullptr || H_w > 0;
+  if (win && B > 0 && (pos == nullptr || (reinterpret_cast<uintptr_t>(pos) & 7u) != 0))
+    return BASED_ERR_INVALID_ARG;
+  return decode_step_impl(q, k, v, state_kv, state_k, out, wq, wk, wv, k_ring, v_ring, wout, 0,
+                          win ? pos : nullptr, B, H, d_feat, d_v, H_w, d_head, window, dt, eps,
+                          stream);
 }
 
 size_t based_linattn_bwd_workspace_bytes(int B, int H, int L, int d_v) {

@@ -31,6 +31,8 @@ struct DecodeParams {
   const void *wq, *wk, *wv;
   void *k_ring, *v_ring, *wout;
   long long pos;
+  const long long* pos_arr;  // [B] per-sequence positions (device), or null: pos for all
+  int H_w;     // window heads per sequence (window item i belongs to sequence i / H_w)
   int n_lin;   // B * H   (one CTA each)
   int n_win;   // B * H_w window heads
   int n_wblk;  // window CTAs, each serving up to wg heads
@@ -194,10 +196,10 @@ __device__ __forceinline__ void decode_window_block(const DecodeParams& p, int w
   T* kvn = reinterpret_cast<T*>(sm + lay.kvn);
   float* pr = reinterpret_cast<float*>(sm + lay.pr);
   float* red = reinterpret_cast<float*>(sm + lay.red);
-  const long long pos = p.pos;
-  const int slot = (int)(pos % W);
-  const int nvalid = pos + 1 < W ? (int)(pos + 1) : W;  // valid slots are 0..nvalid-1
-  const uint32_t load_bytes = (uint32_t)(nvalid * dh * sizeof(T));
+  // position of window item i: its sequence's entry of pos_arr, or the shared pos
+  auto pos_of = [&](int i) -> long long {
+    return p.pos_arr != nullptr ? p.pos_arr[(w0 + i) / p.H_w] : p.pos;
+  };
   T* kring = static_cast<T*>(p.k_ring);
   T* vring = static_cast<T*>(p.v_ring);
 
@@ -205,6 +207,14 @@ __device__ __forceinline__ void decode_window_block(const DecodeParams& p, int w
     for (int g = 0; g < n_items; ++g) umma::mbar_init(bar + g, 1);
     umma::fence_mbar_init();
     for (int g = 0; g < n_items; ++g) {
+      const long long pg = pos_of(g);
+      if (pg < 0) {  // a negative position is refused: nothing of this item is touched
+        record_device_error(BASED_ERR_INVALID_ARG);
+        umma::mbar_arrive(bar + g);
+        continue;
+      }
+      const int nv = pg + 1 < W ? (int)(pg + 1) : W;  // valid slots are 0..nv-1
+      const uint32_t load_bytes = (uint32_t)(nv * dh * sizeof(T));
       const size_t ro = (size_t)(w0 + g) * W * dh;
       T* dst = rings + (size_t)g * 2 * W * dh;
       umma::mbar_arrive_expect_tx(bar + g, 2 * load_bytes);
@@ -221,7 +231,10 @@ __device__ __forceinline__ void decode_window_block(const DecodeParams& p, int w
   __syncthreads();
 
   const int g = tid >> 6, s = tid & 63;  // head and slot / column of this thread
-  const bool active = g < n_items;
+  const long long pos = g < n_items ? pos_of(g) : 0;
+  const bool active = g < n_items && pos >= 0;
+  const int slot = active ? (int)(pos % W) : 0;
+  const int nvalid = !active ? 0 : (pos + 1 < W ? (int)(pos + 1) : W);  // valid slots 0..nvalid-1
   T* K = rings + (size_t)g * 2 * W * dh;
   T* V = K + W * dh;
   bool ok = true;

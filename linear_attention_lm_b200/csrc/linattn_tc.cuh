@@ -212,6 +212,22 @@ template <> __device__ __forceinline__ __nv_bfloat162 pack2<__nv_bfloat162>(floa
   return __floats2bfloat162_rn(a, b);
 }
 
+// Two fp32 values as one packed pair, and c0 + u (c1 + c2 u) for a pair of u
+// with two packed fp32 FMAs (each lane of fma.rn.f32x2 rounds like fmaf).
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void poly2(float u0, float u1, uint64_t c0, uint64_t c1, uint64_t c2,
+                                      float* w0, float* w1) {
+  const uint64_t u = f32x2(u0, u1);
+  uint64_t t, w;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(t) : "l"(u), "l"(c2), "l"(c1));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(w) : "l"(u), "l"(t), "l"(c0));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(*w0), "=f"(*w1) : "l"(w));
+}
+
 // Feature chunk ch (8 features) of one token from its packed pairs X[8] (x/2),
 // the shifted pairs Y[8], and its raw bf16 input pairs (the diagonal features are
 // formed in fp32 and rounded once).  ch must be a compile-time constant.
@@ -583,6 +599,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       umma::tc_fence_after();
       const float sc = tc_chunk_scale((long long)t0 + kTcChunk);
       const float c0 = sc, c1 = 0.25f * sc, c2 = 0.03125f * sc;
+      const uint64_t c0x2 = f32x2(c0, c0), c1x2 = f32x2(c1, c1), c2x2 = f32x2(c2, c2);
       auto poly_pack = [&](const float* u, int c32, uint32_t* pk) {
         const bool diag = c32 == quad;
 #pragma unroll
@@ -611,13 +628,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           else umma::tmem_ld32(tmem + Lay::kTmU + tm_lane + 32 * b, u);
           const int lim = row - 32 * b;  // keys 32b + j with j > lim lie in the future
           uint32_t pk[32];
+          if (b + 1 >= quad) {  // the pair holds the diagonal block: causal mask
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            float w0 = fmaf(u[2 * e], fmaf(u[2 * e], c2, c1), c0);
-            float w1 = fmaf(u[2 * e + 1], fmaf(u[2 * e + 1], c2, c1), c0);
-            if (2 * e > lim) w0 = 0.0f;
-            if (2 * e + 1 > lim) w1 = 0.0f;
-            pk[e] = as_u32(__floats2bfloat162_rn(w0, w1));
+            for (int e = 0; e < 32; ++e) {
+              float w0, w1;
+              poly2(u[2 * e], u[2 * e + 1], c0x2, c1x2, c2x2, &w0, &w1);
+              if (2 * e > lim) w0 = 0.0f;
+              if (2 * e + 1 > lim) w1 = 0.0f;
+              pk[e] = as_u32(__floats2bfloat162_rn(w0, w1));
+            }
+          } else {  // entirely below the diagonal
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              float w0, w1;
+              poly2(u[2 * e], u[2 * e + 1], c0x2, c1x2, c2x2, &w0, &w1);
+              pk[e] = as_u32(__floats2bfloat162_rn(w0, w1));
+            }
           }
           if (two) umma::tmem_st32_nowait(tmem + Lay::kTmU + tm_lane + 16 * b, pk);
           else umma::tmem_st16_nowait(tmem + Lay::kTmU + tm_lane + 16 * b, pk);
@@ -672,8 +698,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int t = tid - kTcGroup;  // token row of the chunk; also the TMEM lane (quadrant = warp & 3)
     const __nv_bfloat16* q = p.q + (size_t)bh * L * kD;
     const __nv_bfloat16* k = p.k + (size_t)bh * L * kD;
-    // q/k rows of this thread's token, loaded two chunks ahead of their use
-    uint4 qr[2], kr[2], qn[2], kn[2];
+    // q/k rows of this thread's token, loaded three chunks ahead of their use
+    // (the loads of cold inputs take a few microseconds under load)
+    uint4 qr[2], kr[2], qn[2], kn[2], qm[2], km[2];
     auto load_qk = [&](int c, uint4* qd, uint4* kd) {
       const long long tt = (long long)c * kTcChunk + t;
       if (c < c_end && tt < L) {
@@ -691,6 +718,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     };
     load_qk(c_begin, qr, kr);
     load_qk(c_begin + 1, qn, kn);
+    load_qk(c_begin + 2, qm, km);
     for (int c = c_begin; c < c_end && !*abort_flag; ++c) {
       const int it = c - c_begin;
       const int t0 = c * kTcChunk;
@@ -774,7 +802,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
       qr[0] = qn[0]; qr[1] = qn[1]; kr[0] = kn[0]; kr[1] = kn[1];
-      load_qk(c + 2, qn, kn);
+      qn[0] = qm[0]; qn[1] = qm[1]; kn[0] = km[0]; kn[1] = km[1];
+      load_qk(c + 3, qm, km);
       if (!kStateOnly) {
         umma::fence_async_smem();
         umma::tc_fence_before();

@@ -9,6 +9,9 @@
 // each with its own 256-column TMEM slot (S: 192 columns, O: 64) and its own y
 // staging tile.  The MMA thread issues S of tile k+1 before P V of tile k, so
 // the tensor core works on one tile while a softmax group works on the other.
+// Q/K and V of a stage are loaded and released separately (two producer
+// warps): Q/K of tile k+3 are loaded as soon as S of tile k has read them, V
+// once P V of tile k has, so each load has about three tile periods to land.
 #pragma once
 
 #include "common.cuh"
@@ -23,7 +26,7 @@
 namespace based {
 
 constexpr int kWpStages = 3;
-constexpr int kWpThreads = 320;  // softmax groups: warps 0-3, 4-7; TMA warp 8; MMA warp 9
+constexpr int kWpThreads = 352;  // softmax groups: warps 0-3, 4-7; MMA warp 8; Q/K, V TMA warps 9, 10
 
 struct WpLayout {
   static constexpr int kQ = 0;                        // per stage: Q [128 x 64] K-major SW128
@@ -34,7 +37,8 @@ struct WpLayout {
   static constexpr int kBar = kY + 2 * 16384;
   static constexpr int kBytes = kBar + 256;
   static constexpr size_t kSmem = kBytes + 1024;
-  static constexpr uint32_t kTxBytes = (128 + 2 * 192) * 64 * 2;
+  static constexpr uint32_t kTxQK = (128 + 192) * 64 * 2;
+  static constexpr uint32_t kTxV = 192 * 64 * 2;
 };
 static_assert(WpLayout::kSmem <= 232448, "shared memory budget");
 
@@ -49,8 +53,8 @@ __global__ void __launch_bounds__(kWpThreads, 1)
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::kBar);
-  uint64_t* full = bars;          // [3] stage loaded (TMA)
-  uint64_t* empty = bars + 3;     // [3] stage consumed (commit after P V)
+  uint64_t* full = bars;          // [3] Q/K of a stage loaded (TMA)
+  uint64_t* empty = bars + 3;     // [3] Q/K of a stage read (commit after S)
   uint64_t* sfull = bars + 6;     // [2] S ready in slot (commit)
   uint64_t* pfull = bars + 8;     // [2] P written to slot (softmax group)
   uint64_t* ofull = bars + 10;    // [2] O ready in slot (commit)
@@ -58,7 +62,10 @@ __global__ void __launch_bounds__(kWpThreads, 1)
   uint64_t* bar_fin = bars + 14;  // every MMA complete (commit)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 16);
-  volatile int* consumed = reinterpret_cast<volatile int*>(bars + 17);
+  volatile int* consumed = reinterpret_cast<volatile int*>(bars + 17);     // Q/K loads waited
+  uint64_t* vfull = bars + 18;    // [3] V of a stage loaded (TMA)
+  uint64_t* vempty = bars + 21;   // [3] V of a stage read (commit after P V)
+  volatile int* consumed_v = reinterpret_cast<volatile int*>(bars + 24);  // V loads waited
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x;
@@ -77,6 +84,8 @@ __global__ void __launch_bounds__(kWpThreads, 1)
     for (int i = 0; i < kWpStages; ++i) {
       umma::mbar_init(full + i, 1);
       umma::mbar_init(empty + i, 1);
+      umma::mbar_init(vfull + i, 1);
+      umma::mbar_init(vempty + i, 1);
     }
     for (int j = 0; j < 2; ++j) {
       umma::mbar_init(sfull + j, 1);
@@ -87,9 +96,10 @@ __global__ void __launch_bounds__(kWpThreads, 1)
     umma::mbar_init(bar_fin, 1);
     *abort_flag = 0;
     *consumed = 0;
+    *consumed_v = 0;
     umma::fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == 8) {
     umma::tmem_alloc(tmem_slot, 512);
     umma::tmem_relinquish();
   }
@@ -99,15 +109,16 @@ __global__ void __launch_bounds__(kWpThreads, 1)
   const uint32_t tmem = *tmem_slot;
   int issued = 0;  // loads issued (TMA thread)
 
-  if (warp == 8) {
-    // ================= TMA producer =================
+  if (warp == 9 || warp == 10) {
+    // ================= TMA producers: Q/K (warp 9) and V (warp 10) =================
+    const bool is_v = warp == 10;
     if (lane == 0) {
-      umma::tma_prefetch_desc(&qmap);
-      umma::tma_prefetch_desc(&kmap);
-      umma::tma_prefetch_desc(&vmap);
+      umma::tma_prefetch_desc(is_v ? &vmap : &qmap);
+      if (!is_v) umma::tma_prefetch_desc(&kmap);
       for (int k = 0; k < n_mine && !*abort_flag; ++k) {
         const int stage = k % kWpStages;
-        if (k >= kWpStages && !umma::mbar_wait(empty + stage, ((k / kWpStages) - 1) & 1)) {
+        if (k >= kWpStages &&
+            !umma::mbar_wait((is_v ? vempty : empty) + stage, ((k / kWpStages) - 1) & 1)) {
           fail();
           break;
         }
@@ -115,16 +126,18 @@ __global__ void __launch_bounds__(kWpThreads, 1)
         int bh, t0;
         tile_of(k, &bh, &t0);
         uint8_t* st = sm + stage * Lay::kStage;
-        umma::mbar_arrive_expect_tx(full + stage, Lay::kTxBytes);
-        umma::tma_load_3d(st + Lay::kQ, &qmap, full + stage, 0, t0, bh);
-        umma::tma_load_3d(st + Lay::kK, &kmap, full + stage, 0, t0 - 64, bh);
-        // the stall test leaves the first V tile out: its stage never completes
-        if (k > 0 || !stall_test(kStallWindowV))
-          umma::tma_load_3d(st + Lay::kV, &vmap, full + stage, 0, t0 - 64, bh);
+        if (!is_v) {
+          umma::mbar_arrive_expect_tx(full + stage, Lay::kTxQK);
+          umma::tma_load_3d(st + Lay::kQ, &qmap, full + stage, 0, t0, bh);
+          umma::tma_load_3d(st + Lay::kK, &kmap, full + stage, 0, t0 - 64, bh);
+        } else if (k > 0 || !stall_test(kStallWindowV)) {  // the stall test leaves V(0) out
+          umma::mbar_arrive_expect_tx(vfull + stage, Lay::kTxV);
+          umma::tma_load_3d(st + Lay::kV, &vmap, vfull + stage, 0, t0 - 64, bh);
+        }
         ++issued;
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 8) {
     // ================= MMA issuer =================
     if (lane == 0) {
       const uint32_t id_s = umma::idesc_bf16(128, 192, false, false);
@@ -143,6 +156,7 @@ __global__ void __launch_bounds__(kWpThreads, 1)
           umma::mma_bf16(tmem + slot * 256, umma::desc_kmajor_sw128(sQ, k0, 128),
                          umma::desc_kmajor_sw128(sK, k0, 192), id_s, k0 > 0);
         umma::mma_commit(sfull + slot);
+        umma::mma_commit(empty + stage);  // Q/K of this stage may be refilled
         BASED_WP_TRACE(1, k);
         return true;
       };
@@ -151,6 +165,8 @@ __global__ void __launch_bounds__(kWpThreads, 1)
         const int stage = k % kWpStages, slot = k & 1;
         if (k + 1 < n_mine && !issue_s(k + 1)) { ok = false; break; }
         if (!umma::mbar_wait(pfull + slot, (k >> 1) & 1)) { ok = false; break; }
+        if (!umma::mbar_wait(vfull + stage, (k / kWpStages) & 1)) { ok = false; break; }
+        *consumed_v = k + 1;
         BASED_WP_TRACE(2, k);
         umma::tc_fence_after();
         const uint32_t sV = umma::smem_u32(sm + stage * Lay::kStage + Lay::kV);
@@ -159,7 +175,7 @@ __global__ void __launch_bounds__(kWpThreads, 1)
           umma::mma_ts(tmem + slot * 256 + 192, tmem + slot * 256 + k0 / 2,
                        umma::desc_mnmajor_sw128(sV, k0, 192), id_o, k0 > 0);
         umma::mma_commit(ofull + slot);
-        umma::mma_commit(empty + stage);
+        umma::mma_commit(vempty + stage);  // V of this stage may be refilled
         BASED_WP_TRACE(3, k);
       }
       if (!ok) fail();
@@ -272,12 +288,15 @@ __global__ void __launch_bounds__(kWpThreads, 1)
   umma::tc_fence_before();
   __syncthreads();
   // loads the MMA thread never consumed (an aborted run) are waited for (bounded)
-  if (warp == 8 && lane == 0) {
-    for (int k = *consumed; k < issued; ++k)
-      umma::mbar_wait(full + k % kWpStages, (k / kWpStages) & 1);
+  if ((warp == 9 || warp == 10) && lane == 0) {
+    const bool is_v = warp == 10;
+    for (int k = is_v ? *consumed_v : *consumed; k < issued; ++k) {
+      if (is_v && k == 0 && stall_test(kStallWindowV)) continue;  // never issued
+      umma::mbar_wait((is_v ? vfull : full) + k % kWpStages, (k / kWpStages) & 1);
+    }
   }
   __syncthreads();
-  if (warp == 9) umma::tmem_dealloc(tmem, 512);
+  if (warp == 8) umma::tmem_dealloc(tmem, 512);
 }
 
 }  // namespace based

@@ -132,6 +132,31 @@ def test_decode_host_validation(lib):
              1e-6, N) == UNSUPPORTED
 
 
+def test_decode_at_host_validation(lib):
+    f = lib.based_decode_step_at
+    N = None
+    # window part with no position array, or a misaligned one
+    assert f(N, N, N, N, N, N, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, N, 2, 0, 16, 64, 1, 64, 64, 1,
+             1e-6, N) == INVALID
+    assert f(N, N, N, N, N, N, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 4, 2, 0, 16, 64, 1, 64,
+             64, 1, 1e-6, N) == INVALID
+    # the linear part alone needs no positions; its checks are based_decode_step's
+    assert f(FAKE, FAKE, FAKE, N, FAKE, FAKE, N, N, N, N, N, N, N, 1, 1, 16, 64, 0, 64, 64, 1,
+             1e-6, N) == INVALID  # missing state
+
+
+def test_binding_decode_positions_checked():
+    z = torch.zeros
+    wq = z(3, 2, 64, dtype=torch.bfloat16)
+    ring = z(3, 2, 64, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="expected shape"):
+        lab.based_decode_step(None, None, None, None, None, None, wq, wq, wq, ring, ring, wq,
+                              pos=z(2, dtype=torch.int64))
+    with pytest.raises(TypeError):
+        lab.based_decode_step(None, None, None, None, None, None, wq, wq, wq, ring, ring, wq,
+                              pos=z(3, dtype=torch.int32))
+
+
 def test_linattn_bwd_host_validation(lib):
     f = lib.based_linattn_bwd
     ws = lib.based_linattn_bwd_workspace_bytes

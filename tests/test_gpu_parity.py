@@ -267,3 +267,80 @@ def test_decode_zero_state_matches_prefill():
     torch.cuda.synchronize()
     check(torch.stack(ys, 2), to_f64(y), torch.bfloat16, "decode vs prefill")
     check(torch.stack(yws, 2), to_f64(yw), torch.bfloat16, "decode window vs prefill")
+
+
+# --------------------------------------------------------------------------
+# decode with per-sequence positions (prompts of different lengths)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("W", [64, 7])
+def test_decode_per_sequence_positions(W):
+    """Window decode for a batch whose sequences start at different positions
+    (prefill lengths 5, 63, 64 and 200): each sequence's ring is built by the
+    oracle from its own prefill, every step is compared with the oracle
+    stepping that sequence at its own position."""
+    dev = torch.device("cuda:0")
+    lens = [5, 63, 64, 200]
+    B, Hw, dh, steps = len(lens), 2, 64, 70
+    w = WORKLOADS["decode_b128"].with_(B=B, H=2, Hw=Hw, L=max(lens), window=W, name="dec_ragged")
+    x = prefill_inputs(w, device=dev)
+    wk, wv = to_f64(x["wk"]), to_f64(x["wv"])
+    kr_o = np.zeros((B, Hw, W, dh))
+    vr_o = np.zeros_like(kr_o)
+    for b, Lb in enumerate(lens):
+        kr_o[b], vr_o[b] = oracle.ring_fill(wk[b, :, :Lb], wv[b, :, :Lb], W)
+    k_ring = torch.from_numpy(kr_o).to(torch.bfloat16).to(dev)
+    v_ring = torch.from_numpy(vr_o).to(torch.bfloat16).to(dev)
+    wout = torch.empty((B, Hw, dh), dtype=torch.bfloat16, device=dev)
+    for step in range(steps):
+        d = decode_step_inputs(w, step, device=dev)
+        pos = torch.tensor([Lb + step for Lb in lens], dtype=torch.int64, device=dev)
+        lab.based_decode_step(None, None, None, None, None, None, d["wq"], d["wk"], d["wv"],
+                              k_ring, v_ring, wout, pos=pos, window=W)
+        ref = np.stack([oracle.decode_window(to_f64(d["wq"])[b], to_f64(d["wk"])[b],
+                                             to_f64(d["wv"])[b], kr_o[b], vr_o[b],
+                                             lens[b] + step, W) for b in range(B)])
+        check(wout, ref, torch.bfloat16, f"per-sequence decode step {step}")
+    assert lab.based_get_device_error() == 0
+
+
+def test_decode_positions_equal_match_scalar_entry_point():
+    """All positions equal: based_decode_step_at and based_decode_step give
+    bit-identical outputs and rings."""
+    dev = torch.device("cuda:0")
+    w = WORKLOADS["decode_b128"].with_(B=3, H=2, Hw=2, L=90, name="dec_eq")
+    x = prefill_inputs(w, device=dev)
+    _, S, z = lab.linattn(x["q"], x["k"], x["v"], w.eps, return_state=True)
+    kr, vr = lab.window_ring_fill(x["wk"], x["wv"], w.window)
+    state = [(S.clone(), z.clone(), kr.clone(), vr.clone()) for _ in range(2)]
+    outs = []
+    for use_array, (S_, z_, kr_, vr_) in zip((False, True), state):
+        o = torch.empty((3, 2, 64), dtype=torch.bfloat16, device=dev)
+        wo = torch.empty_like(o)
+        for step in range(5):
+            d = decode_step_inputs(w, step, device=dev)
+            pos = w.L + step
+            if use_array:
+                pos = torch.full((3,), pos, dtype=torch.int64, device=dev)
+            lab.based_decode_step(d["q"], d["k"], d["v"], S_, z_, o, d["wq"], d["wk"], d["wv"],
+                                  kr_, vr_, wo, pos=pos, window=w.window, eps=w.eps)
+        torch.cuda.synchronize()
+        outs.append((o, wo, S_, kr_, vr_))
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+
+
+def test_decode_negative_position_is_refused_on_the_device():
+    dev = torch.device("cuda:0")
+    B, Hw, W, dh = 2, 2, 64, 64
+    ring = torch.randn(B, Hw, W, dh, device=dev).to(torch.bfloat16)
+    k_ring, v_ring = ring.clone(), ring.clone()
+    wq = torch.randn(B, Hw, dh, device=dev).to(torch.bfloat16)
+    wout = torch.full((B, Hw, dh), 7.0, dtype=torch.bfloat16, device=dev)
+    pos = torch.tensor([100, -3], dtype=torch.int64, device=dev)
+    lab.based_decode_step(None, None, None, None, None, None, wq, wq, wq, k_ring, v_ring, wout,
+                          pos=pos, window=W)
+    assert lab.based_get_device_error() == 1  # BASED_ERR_INVALID_ARG
+    assert torch.equal(k_ring[1], ring[1]) and torch.equal(v_ring[1], ring[1])
+    assert torch.all(wout[1] == 7.0)
+    assert not torch.equal(k_ring[0], ring[0])  # sequence 0 was served
