@@ -529,10 +529,19 @@ def run_projections(args, lab, dev, world, peaks, warm):
         ms = max_over_ranks(ms, dev, world)
         return ms
 
+    w_cat = torch.cat(ws, 0).contiguous()
+
     def proj_step(i):
-        x = xs[i % 4]
-        for w, y in zip(ws, ys):
-            lab.based_proj_heads_fwd(x, w, y)
+        # the six projections of a layer pair in one launch (x streamed once)
+        lab.based_proj_heads_multi_fwd(xs[i % 4], w_cat, ys)
+
+    def torch_proj_step(i):
+        # the same product by torch's matmul (cuBLAS), row-major [B*L, 4608]
+        # output, no split into heads: a lower bound on the library's time
+        torch.matmul(xs[i % 4].view(B * L, dm), w_cat.t())
+
+    def torch_conv_gemm(i):
+        torch.matmul(xs[i % 4].view(B * L, dm), wb.t())
 
     def conv_step(i):
         lab.based_baseconv_fwd(xs[i % 4], wb, bias, taps, yb)
@@ -564,8 +573,9 @@ def run_projections(args, lab, dev, world, peaks, warm):
     # (3 x 2 dh) -> 10 dh flop; W (W + 1) / 2 + W (L - W) pairs per head
     w_pairs = 64 * 65 / 2 + 64 * (L - 64)
     for name, fn, flops, launches, what in (
-            ("proj", proj_step, 2.0 * B * L * dm * H * sum(heads), len(heads),
-             "six per-head projections of x [8, 2048, 1024]: q, k 16x16; v 16x64; window q, k, v 16x64"),
+            ("proj", proj_step, 2.0 * B * L * dm * H * sum(heads), 1,
+             "six per-head projections of x [8, 2048, 1024] in one launch: q, k 16x16; v 16x64; "
+             "window q, k, v 16x64"),
             ("baseconv", conv_step, 2.0 * B * L * dm * dm, 1,
              "BaseConv block, x [8, 2048, 1024], dense 1024x1024 + bias, 3 causal taps"),
             ("linattn_bwd", bwd_step, 480.0 * B * H * L * (L + 1) / 2, 2,
@@ -588,6 +598,11 @@ def run_projections(args, lab, dev, world, peaks, warm):
                      "roofline": {"kernel": kern, "bound": bound, "achieved": round(tf, 2),
                                   "peak": pk, "unit": "TFLOP/s", "frac": round(tf / pk, 4),
                                   "traffic": None, "peak_source": src}}
+        if name in ("proj", "baseconv"):
+            # library context: torch.matmul of the same GEMM (no epilogue, no head split)
+            tms = timed(torch_proj_step if name == "proj" else torch_conv_gemm, n)
+            out[name]["torch_matmul"] = {"ms": round(tms, 5),
+                                         "tflops": round(flops / (tms / 1e3) / 1e12, 2)}
     assert lab.based_get_device_error() == 0
     return out
 

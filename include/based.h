@@ -258,6 +258,26 @@ based_status_t based_proj_heads_fwd(const void* x, const void* w, void* y, int B
                                     based_stream_t stream);
 
 /*
+ * Several per-head projections of the same input in one launch (for instance
+ * the q, k and v projections of a linear-attention layer and of a window
+ * layer): x is streamed once for all of them.
+ *   w     [sum_g H*D[g], d_model]  bf16: the n_out weight matrices stacked
+ *         row-wise, projection g taking H*D[g] rows in order
+ *   D     host array [n_out]: features per head of each projection
+ *   y     host array [n_out] of device pointers; y[g] is [B, H, L, D[g]] bf16
+ *   y[g][b][h][t][d] = sum_k x[b][t][k] * w[off_g + h*D[g] + d][k],
+ *   off_g = H * (D[0] + ... + D[g-1]).
+ * Requires 1 <= n_out <= 8 (BASED_ERR_INVALID_ARG otherwise), bf16,
+ * d_model % 64 == 0, (H*D[g]) % 256 == 0 and D[g] % 8 == 0 for every g (else
+ * BASED_ERR_UNSUPPORTED); every pointer 16-byte aligned.  The outputs must not
+ * overlap each other or x.  based_proj_heads_fwd is this call with n_out = 1.
+ * Runs on pairs of CTAs (thread-block clusters of two).
+ */
+based_status_t based_proj_heads_multi_fwd(const void* x, const void* w, int n_out, const int* D,
+                                          void* const* y, int B, int L, int d_model, int H,
+                                          based_dtype_t dt, based_stream_t stream);
+
+/*
  * BaseConv block ("Базированная модель, часть 1", section "Кто виноват?":
  * y = linear(x) (.) conv(h, x)), with a dense D x D map plus bias and a
  * causal per-channel convolution of K taps:

@@ -34,7 +34,7 @@ EXPORTED_SYMBOLS = ("based_abi_version", "based_binary_version", "based_status_s
                     "based_linattn_fwd_noalloc",
                     "based_window_attn_fwd", "based_window_ring_fill", "based_decode_step",
                     "based_decode_step_at",
-                    "based_proj_heads_fwd", "based_baseconv_fwd",
+                    "based_proj_heads_fwd", "based_proj_heads_multi_fwd", "based_baseconv_fwd",
                     "based_linattn_bwd_workspace_bytes", "based_linattn_bwd",
                     "based_window_attn_bwd_workspace_bytes", "based_window_attn_bwd",
                     "based_debug_stall", "based_get_device_error")
@@ -90,12 +90,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.based_window_attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                               _i, _i, _vp, _sz, _vp]
         lib.based_proj_heads_fwd.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
+        lib.based_proj_heads_multi_fwd.argtypes = [_vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i,
+                                                   _vp]
         lib.based_baseconv_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
         lib.based_get_device_error.argtypes = [_vp]
         lib.based_debug_stall.argtypes = [_i, _ll]
         for name in ("based_linattn_fwd", "based_linattn_fwd_noalloc", "based_window_attn_fwd",
                      "based_window_ring_fill", "based_decode_step", "based_decode_step_at",
-                     "based_proj_heads_fwd",
+                     "based_proj_heads_fwd", "based_proj_heads_multi_fwd",
                      "based_baseconv_fwd", "based_linattn_bwd", "based_window_attn_bwd",
                      "based_debug_stall", "based_get_device_error"):
             getattr(lib, name).restype = _i
@@ -424,6 +426,32 @@ def based_proj_heads_fwd(x, w, y, stream=None):
     return y
 
 
+def based_proj_heads_multi_fwd(x, w, ys, stream=None):
+    """x [B, L, d_model], w [H*(D_0+...+D_{n-1}), d_model] -> ys[g] [B, H, L, D_g]
+    (bf16, written), every projection in one launch."""
+    dev = _device_of(x)
+    ys = list(ys)
+    if x.dim() != 3 or not ys or any(y.dim() != 4 for y in ys):
+        raise ValueError("x must be [B, L, d_model] and every y [B, H, L, D]")
+    B, L, d_model = x.shape
+    H = ys[0].shape[1]
+    Ds = [int(y.shape[3]) for y in ys]
+    _expect(w, (H * sum(Ds), d_model), "w", dev)
+    for g, y in enumerate(ys):
+        _expect(y, (B, H, L, Ds[g]), f"ys[{g}]", dev)
+    dt = _same_dtype(x, w, *ys)
+    _cuda(dev)
+    d_arr = (ctypes.c_int * len(ys))(*Ds)
+    y_arr = (ctypes.c_void_p * len(ys))(*[_ptr(y) for y in ys])
+    with torch.cuda.device(dev):
+        st = load_library().based_proj_heads_multi_fwd(
+            _ptr(x), _ptr(w), len(ys), ctypes.cast(d_arr, ctypes.c_void_p),
+            ctypes.cast(y_arr, ctypes.c_void_p), B, L, d_model, H, dt,
+            _torch_stream(stream, dev).cuda_stream)
+    _check("based_proj_heads_multi_fwd", st)
+    return ys
+
+
 def based_baseconv_fwd(x, w, bias, taps, y, stream=None):
     """x, y [B, L, D] bf16; w [D, D] bf16; bias [D], taps [D, K] float32."""
     dev = _device_of(x)
@@ -499,6 +527,14 @@ def proj_heads(x, w, H: int, stream=None):
     B, L, _ = x.shape
     y = torch.empty((B, H, L, w.shape[0] // H), dtype=x.dtype, device=x.device)
     return based_proj_heads_fwd(x, w, y, stream=stream)
+
+
+def proj_heads_multi(x, w, H: int, Ds, stream=None):
+    """Several per-head projections of x in one launch: w stacks H*D_g rows per
+    projection; returns the list of [B, H, L, D_g] outputs."""
+    B, L, _ = x.shape
+    ys = [torch.empty((B, H, L, D), dtype=x.dtype, device=x.device) for D in Ds]
+    return based_proj_heads_multi_fwd(x, w, ys, stream=stream)
 
 
 def baseconv(x, w, bias, taps, stream=None):

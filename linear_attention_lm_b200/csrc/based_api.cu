@@ -275,7 +275,7 @@ based_status_t launch_decode(DecodeParams p, cudaStream_t st) {
 template <int Mode>
 based_status_t launch_proj(const void* x, const void* w, ProjParams p, cudaStream_t st) {
   CUtensorMap xm, wm, hm;
-  if (!make_rows_map(&xm, x, p.Kd, p.M, 1, kPjM) || !make_rows_map(&wm, w, p.Kd, p.N, 1, kPjN))
+  if (!make_rows_map(&xm, x, p.Kd, p.M, 1, kPjM) || !make_rows_map(&wm, w, p.Kd, p.N, 1, kPjNHalf))
     return BASED_ERR_CUDA;
   if (Mode == kBaseConv) {
     if (!make_rows_map(&hm, x, p.Kd, p.M, 1, kPjHaloRows)) return BASED_ERR_CUDA;
@@ -285,12 +285,28 @@ based_status_t launch_proj(const void* x, const void* w, ProjParams p, cudaStrea
   auto kern = proj_tc_kernel<Mode>;
   if (!set_smem(kern, PjLayout<Mode>::kSmem)) return BASED_ERR_CUDA;
   p.n_tiles_n = p.N / kPjN;
-  const long long tiles = (long long)((p.M + kPjM - 1) / kPjM) * p.n_tiles_n;
+  const long long tiles = (long long)((p.M + 2 * kPjM - 1) / (2 * kPjM)) * p.n_tiles_n;
   if (tiles > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
   p.total_tiles = (int)tiles;
-  const long long sms = device_sm_count();
-  const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
-  kern<<<grid, kPjThreads, PjLayout<Mode>::kSmem, st>>>(xm, wm, hm, p);
+  // CTA pairs: clusters of two, as many as fit at once (one CTA per SM)
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kPjThreads, 1, 1);
+  cfg.dynamicSmemBytes = PjLayout<Mode>::kSmem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.gridDim = dim3(2 * (unsigned)((device_sm_count() + 1) / 2), 1, 1);
+  int max_clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg) != cudaSuccess || max_clusters <= 0)
+    return BASED_ERR_CUDA;
+  const long long pairs = tiles < max_clusters ? tiles : max_clusters;
+  cfg.gridDim = dim3(2 * (unsigned)pairs, 1, 1);
+  if (cudaLaunchKernelEx(&cfg, kern, xm, wm, hm, p) != cudaSuccess) return BASED_ERR_CUDA;
   return launch_status();
 }
 
@@ -658,23 +674,48 @@ based_status_t based_window_attn_bwd(const void* q, const void* k, const void* v
   return launch_window_bwd<__nv_bfloat16>(q, k, v, dy, dq, dk, dv, (int)BH, L, window, ws, st);
 }
 
+based_status_t based_proj_heads_multi_fwd(const void* x, const void* w, int n_out, const int* D,
+                                          void* const* y, int B, int L, int d_model, int H,
+                                          based_dtype_t dt, based_stream_t stream) {
+  if (B < 0 || L < 0 || d_model <= 0 || H <= 0 || n_out < 1 || n_out > kPjMaxOut || !D || !y)
+    return BASED_ERR_INVALID_ARG;
+  if (dt != BASED_BF16 && dt != BASED_F32) return BASED_ERR_INVALID_ARG;
+  for (int g = 0; g < n_out; ++g)
+    if (D[g] <= 0) return BASED_ERR_INVALID_ARG;
+  if (dt != BASED_BF16) return BASED_ERR_UNSUPPORTED;
+  if (d_model % kPjK != 0) return BASED_ERR_UNSUPPORTED;
+  long long N = 0;
+  for (int g = 0; g < n_out; ++g) {
+    if (((long long)H * D[g]) % kPjN != 0 || D[g] % 8 != 0) return BASED_ERR_UNSUPPORTED;
+    N += (long long)H * D[g];
+  }
+  const long long M = (long long)B * L;
+  if (M > 0x7fffffffLL || N > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
+  if (M == 0) return BASED_OK;
+  if (!x || !w || !aligned16(x) || !aligned16(w)) return BASED_ERR_INVALID_ARG;
+  for (int g = 0; g < n_out; ++g)
+    if (!y[g] || !aligned16(y[g])) return BASED_ERR_INVALID_ARG;
+  ProjParams p{};
+  p.n_out = n_out;
+  int col = 0;
+  for (int g = 0; g < n_out; ++g) {
+    p.y[g] = static_cast<__nv_bfloat16*>(y[g]);
+    p.D[g] = D[g];
+    p.col_begin[g] = col;
+    col += H * D[g];
+  }
+  p.col_begin[n_out] = col;
+  p.M = (int)M; p.N = (int)N; p.Kd = d_model; p.L = L; p.H = H;
+  return launch_proj<kProjHeads>(x, w, p, static_cast<cudaStream_t>(stream));
+}
+
 based_status_t based_proj_heads_fwd(const void* x, const void* w, void* y, int B, int L,
                                     int d_model, int H, int D, based_dtype_t dt,
                                     based_stream_t stream) {
-  if (B < 0 || L < 0 || d_model <= 0 || H <= 0 || D <= 0) return BASED_ERR_INVALID_ARG;
-  if (dt != BASED_BF16 && dt != BASED_F32) return BASED_ERR_INVALID_ARG;
-  if (dt != BASED_BF16) return BASED_ERR_UNSUPPORTED;
-  if (d_model % kPjK != 0 || ((long long)H * D) % kPjN != 0 || D % 8 != 0)
-    return BASED_ERR_UNSUPPORTED;
-  const long long M = (long long)B * L;
-  if (M > 0x7fffffffLL || (long long)H * D > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
-  if (M == 0) return BASED_OK;
-  if (!x || !w || !y) return BASED_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return BASED_ERR_INVALID_ARG;
-  ProjParams p{};
-  p.y = static_cast<__nv_bfloat16*>(y);
-  p.M = (int)M; p.N = H * D; p.Kd = d_model; p.L = L; p.H = H; p.D = D;
-  return launch_proj<kProjHeads>(x, w, p, static_cast<cudaStream_t>(stream));
+  void* ys[1] = {y};
+  const int Ds[1] = {D};
+  if (D <= 0) return BASED_ERR_INVALID_ARG;
+  return based_proj_heads_multi_fwd(x, w, 1, Ds, ys, B, L, d_model, H, dt, stream);
 }
 
 based_status_t based_baseconv_fwd(const void* x, const void* w, const float* bias,
@@ -691,7 +732,8 @@ based_status_t based_baseconv_fwd(const void* x, const void* w, const float* bia
   if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return BASED_ERR_INVALID_ARG;
   ProjParams p{};
   p.x = static_cast<const __nv_bfloat16*>(x);
-  p.y = static_cast<__nv_bfloat16*>(y);
+  p.n_out = 1;
+  p.y[0] = static_cast<__nv_bfloat16*>(y);
   p.bias = bias; p.taps = taps;
   p.M = (int)M; p.N = D; p.Kd = D; p.L = L; p.K = K;
   return launch_proj<kBaseConv>(x, w, p, static_cast<cudaStream_t>(stream));

@@ -578,6 +578,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       // the last chunk's MMAs must be complete before the state is read out
       if (n_done > 0 && !umma::mbar_wait(bar_o, (n_done - 1) & 1)) fail();
+      BASED_TC_TRACE(9, 0);
       // and every MMA this thread issued (an aborted chunk may have left some)
       // before the TMEM is released
       umma::mma_commit(bar_fin);
@@ -684,10 +685,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // the final state (or nothing, for an empty segment) is exported here, as
       // soon as the last #5 completes, while #2, #4 and the last output still run
       if (c_begin < c_end) {
+        BASED_TC_TRACE(2, 0);
         const bool ok = !*abort_flag && umma::mbar_wait(bar_m5, (c_end - 1 - c_begin) & 1);
         if (umma::named_sync_all(1, kTcGroup, ok)) {
           umma::tc_fence_after();
+          BASED_TC_TRACE(3, 0);
           export_kst(t);
+          BASED_TC_TRACE(4, 0);
         } else if (!*abort_flag) {
           fail();
         }
@@ -1011,7 +1015,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
     }
-    if (Lay::kTm && t == 0) umma::bulk_wait<0>();
+    BASED_TC_TRACE(5, 0);
+    // the last output store has read its staging tile (its global writes
+    // complete with the grid)
+    if (Lay::kTm && t == 0) umma::bulk_wait_read<0>();
+    BASED_TC_TRACE(6, 0);
   }
 
   umma::tc_fence_before();

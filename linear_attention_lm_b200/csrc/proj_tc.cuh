@@ -3,21 +3,31 @@
 // Y = X W^T for X [M, Kd] (M = B*L tokens, row-major) and W [N, Kd] (one output
 // feature per row), bf16 in, fp32 accumulation in TMEM, with one of two epilogues:
 //
-//  * kProjHeads -- the per-head projection that feeds the attention layers
+//  * kProjHeads -- the per-head projections that feed the attention layers
 //    ("Базированная модель, часть 2", the paragraph on the size of the hidden
-//    state: the KV and K states are made smaller by projections of the input):
-//    column n = h*D + d of token m = b*L + t goes to y[b][h][t][d] (bf16).
+//    state: the KV and K states are made smaller by projections of the input).
+//    W stacks up to kPjMaxOut projections of the same x (rows [col_begin[g],
+//    col_begin[g+1]) are projection g, H heads of D[g] features); column
+//    n = col_begin[g] + h*D[g] + d of token m = b*L + t goes to
+//    y_g[b][h][t][d] (bf16).  One launch serves every projection of a layer,
+//    so x is streamed once for all of them.
 //  * kBaseConv -- the BaseConv block ("Базированная модель, часть 1", section
 //    "Кто виноват?": y = linear(x) (.) conv(h, x)): N = Kd = D channels, and
 //    y[m][c] = (Y[m][c] + bias[c]) * sum_{j <= min(K-1, t)} h[c][j] x[m-j][c].
 //
-// Persistent: one CTA per SM walks the 128 x 256 output tiles (tiles sharing an
-// X row block are adjacent, so X is read from DRAM about once).  Warp 0 (one
-// thread) streams 64-wide K blocks of X and W by TMA through a ring of stages
-// (128B swizzle, K-major); warp 1 (one thread) issues four M=128/N=256/K=16 MMAs
-// per block into one of two TMEM accumulators, so the epilogue of tile k
-// overlaps the main loop of tile k+1; warps 2-5 (one per TMEM lane quadrant)
-// run the epilogue.  For BaseConv the producer also loads the tile's input rows
+// CTA pairs: a cluster of two CTAs (one TPC) owns a 256 x 256 output tile and
+// runs it as M = 256 tcgen05 MMAs (.cta_group::2).  Each CTA loads its own 128
+// rows of X and 128 of the tile's 256 rows of W, so a pair reads 64 KiB per
+// 64-deep K block for 2 x 256 x 256 x 64 flop -- half the L2 traffic per flop of
+// a one-CTA 128 x 256 tile, which the L2 -> SM bandwidth could not feed.
+// Persistent: the pairs walk the tiles (tiles sharing an X row block are
+// adjacent, so X is read from DRAM about once).  Per CTA: warp 0 (one thread)
+// streams K blocks by TMA through a ring of stages (128B swizzle, K-major),
+// counting the bytes of both CTAs on the even CTA's barrier; warp 1 of the even
+// CTA (one thread) issues four M=256/N=256/K=16 MMAs per block into one of two
+// TMEM accumulators, so the epilogue of tile k overlaps the main loop of tile
+// k+1; warps 2-5 (one per TMEM lane quadrant) run the epilogue on the CTA's own
+// 128 rows.  For BaseConv the producer also loads the CTA's input rows
 // [m0-8, m0+128) x [n0, n0+256) (the convolution's reach) into shared memory,
 // once the previous tile's epilogue has released them.
 #pragma once
@@ -27,20 +37,23 @@
 
 namespace based {
 
-constexpr int kPjM = 128;       // rows (tokens) per tile
+constexpr int kPjM = 128;       // rows (tokens) per CTA; a pair covers 256
 constexpr int kPjN = 256;       // columns per tile
+constexpr int kPjNHalf = 128;   // rows of W loaded by each CTA of the pair
 constexpr int kPjK = 64;        // K block per stage (one 128-byte swizzle atom)
 constexpr int kPjThreads = 192;
 constexpr int kPjMaxTaps = 8;
 constexpr int kPjHaloRows = kPjM + kPjMaxTaps;  // rows [m0 - 8, m0 + 128)
+constexpr int kPjMaxOut = 8;    // projections per launch
 
 enum ProjMode { kProjHeads = 0, kBaseConv = 1 };
 
 template <int Mode>
 struct PjLayout {
-  static constexpr int kStages = Mode == kBaseConv ? 3 : 4;
+  static constexpr int kStages = Mode == kBaseConv ? 4 : 6;
   static constexpr int kStageA = kPjM * kPjK * 2;                 // 16 KiB
-  static constexpr int kStageB = kPjN * kPjK * 2;                 // 32 KiB
+  static constexpr int kStageB = kPjNHalf * kPjK * 2;             // 16 KiB
+  static constexpr uint32_t kTxPair = 2u * (kStageA + kStageB);   // both CTAs' bytes
   static constexpr int kA = 0;
   static constexpr int kB = kStages * kStageA;
   static constexpr int kHalo = kB + kStages * kStageB;            // [4][136 rows][128 B] SW128
@@ -59,15 +72,18 @@ struct PjLayout {
 
 struct ProjParams {
   const __nv_bfloat16* x;  // kBaseConv: the layer input (for the convolution's taps)
-  __nv_bfloat16* y;
+  __nv_bfloat16* y[kPjMaxOut];
+  int D[kPjMaxOut];        // kProjHeads: features per head of each projection
+  int col_begin[kPjMaxOut + 1];
+  int n_out;
   const float* bias;       // kBaseConv: [N]
   const float* taps;       // kBaseConv: [N][K]
   int M, N, Kd;
   int L;                   // tokens per sequence
-  int H, D;                // kProjHeads: heads and features per head (N = H * D)
+  int H;                   // kProjHeads: heads of every projection
   int K;                   // kBaseConv: filter taps
   int n_tiles_n;           // N / 256
-  int total_tiles;
+  int total_tiles;         // 256 x 256 tiles
 };
 
 template <int Mode>
@@ -81,10 +97,10 @@ __global__ void __launch_bounds__(kPjThreads, 1)
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::kBar);
-  uint64_t* bar_full = bars;               // [S] stage landed
-  uint64_t* bar_empty = bars + S;          // [S] stage read by the MMAs (commit)
-  uint64_t* bar_afull = bars + 2 * S;      // [2] accumulator complete (commit)
-  uint64_t* bar_aempty = bars + 2 * S + 2; // [2] accumulator read (epilogue)
+  uint64_t* bar_full = bars;               // [S] both CTAs' stage landed (even CTA's copy used)
+  uint64_t* bar_empty = bars + S;          // [S] stage read by the MMAs (commit, both CTAs)
+  uint64_t* bar_afull = bars + 2 * S;      // [2] accumulator complete (commit, both CTAs)
+  uint64_t* bar_aempty = bars + 2 * S + 2; // [2] accumulator read by both epilogues (even CTA)
   uint64_t* bar_hfull = bars + 2 * S + 4;  // input rows of the tile landed
   uint64_t* bar_hempty = bars + 2 * S + 5; // input rows read (epilogue)
   uint64_t* bar_done = bars + 2 * S + 6;   // every MMA issued has completed (commit)
@@ -94,7 +110,8 @@ __global__ void __launch_bounds__(kPjThreads, 1)
   uint64_t* bar_tfree = bars + 2 * S + 10;   // taps and bias of the tile no longer read
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int first = blockIdx.x, step = gridDim.x;
+  const uint32_t rank = umma::cluster_ctarank();  // 0: issues the pair's MMAs
+  const int first = (int)umma::cluster_id_x(), step = (int)umma::cluster_count_x();
   const int n_mine = p.total_tiles > first ? (p.total_tiles - first + step - 1) / step : 0;
   const int nkb = p.Kd / kPjK;
 
@@ -105,7 +122,7 @@ __global__ void __launch_bounds__(kPjThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       umma::mbar_init(bar_afull + a, 1);
-      umma::mbar_init(bar_aempty + a, kPjM);
+      umma::mbar_init(bar_aempty + a, 8);  // one arrival per epilogue warp of both CTAs
     }
     umma::mbar_init(bar_hfull, 1);
     umma::mbar_init(bar_hempty, kPjM);
@@ -116,28 +133,31 @@ __global__ void __launch_bounds__(kPjThreads, 1)
     umma::fence_mbar_init();
   }
   if (warp == 1) {
-    umma::tmem_alloc(tmem_slot, 2 * kPjN);
-    umma::tmem_relinquish();
+    umma::tmem_alloc_pair(tmem_slot, 2 * kPjN);
+    umma::tmem_relinquish_pair();
   }
   umma::tc_fence_before();
-  __syncthreads();
+  // both CTAs' barriers are initialised and their TMEM allocated before any
+  // load, MMA or arrival reaches the other CTA
+  umma::cluster_sync();
   umma::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   auto fail = [&]() {
     record_device_error(BASED_ERR_TIMEOUT);
     *abort_flag = 1;
   };
+  // this CTA's rows of the pair tile k, and the tile's first column
   auto tile_at = [&](int k, int* m0, int* n0) {
     const int i = first + k * step;
     const int mt = i / p.n_tiles_n;
-    *m0 = mt * kPjM;
+    *m0 = mt * (2 * kPjM) + (int)rank * kPjM;
     *n0 = (i - mt * p.n_tiles_n) * kPjN;
   };
 
   if (warp == 0) {
-    // ================= producer =================
+    // ================= producer (both CTAs) =================
     if (lane == 0) {
-      constexpr uint32_t bytes = (kPjM + kPjN) * kPjK * 2;
+      const uint32_t full0 = umma::cluster_addr(bar_full, 0);  // the even CTA's barriers
       int g = 0, halo_issued = 0;
       for (int k = 0; k < n_mine && !*abort_flag; ++k) {
         int m0, n0;
@@ -145,13 +165,15 @@ __global__ void __launch_bounds__(kPjThreads, 1)
         for (int kb = 0; kb < nkb; ++kb, ++g) {
           const int s = g % S;
           if (g >= S && !umma::mbar_wait(bar_empty + s, ((g - S) / S) & 1)) { fail(); break; }
-          umma::mbar_arrive_expect_tx(bar_full + s, bytes);
-          umma::tma_load_3d(sm + Lay::kA + s * Lay::kStageA, &xmap, bar_full + s, kb * kPjK, m0, 0);
-          umma::tma_load_3d(sm + Lay::kB + s * Lay::kStageB, &wmap, bar_full + s, kb * kPjK, n0, 0);
+          if (rank == 0) umma::mbar_arrive_expect_tx(bar_full + s, Lay::kTxPair);
+          umma::tma_load_3d_pair(sm + Lay::kA + s * Lay::kStageA, &xmap, full0 + 8u * s,
+                                 kb * kPjK, m0, 0);
+          umma::tma_load_3d_pair(sm + Lay::kB + s * Lay::kStageB, &wmap, full0 + 8u * s,
+                                 kb * kPjK, n0 + (int)rank * kPjNHalf, 0);
         }
         if (*abort_flag) break;
         if (Mode == kBaseConv) {
-          // this tile's input rows, once the previous tile's epilogue has read its own
+          // this CTA's input rows, once the previous tile's epilogue has read its own
           if (k >= 1 && !umma::mbar_wait(bar_hempty, (k - 1) & 1)) { fail(); break; }
           umma::mbar_arrive_expect_tx(bar_hfull, 4 * Lay::kHaloBlock);
 #pragma unroll
@@ -161,21 +183,35 @@ __global__ void __launch_bounds__(kPjThreads, 1)
           halo_issued = k + 1;
         }
       }
-      // loads that nobody consumed (after an abort) must land before the CTA exits
+      // Loads that nobody consumed (after an abort) must land before the CTAs
+      // exit.  The even CTA's barrier counts both CTAs' bytes of a stage; the odd
+      // CTA cannot see it, so it waits long enough for any load in flight.
       if (*abort_flag) {
-        for (int gg = g - S > 0 ? g - S : 0; gg < g; ++gg)
-          umma::mbar_wait(bar_full + gg % S, (gg / S) & 1);
+        if (rank == 0) {
+          for (int gg = g - S > 0 ? g - S : 0; gg < g; ++gg)
+            umma::mbar_wait(bar_full + gg % S, (gg / S) & 1);
+        } else {
+          const uint64_t t0 = umma::global_timer_ns();
+          while (umma::global_timer_ns() - t0 < 200000ull) {
+          }
+        }
         if (halo_issued > 0) umma::mbar_wait(bar_hfull, (halo_issued - 1) & 1);
       }
     }
   } else if (warp == 1) {
-    // ================= MMA issue =================
-    if (lane == 0) {
-      const uint32_t id = umma::idesc_bf16(kPjM, kPjN, false, false);
+    // ================= MMA issue (even CTA) =================
+    if (lane == 0 && rank == 0) {
+      const uint32_t id = umma::idesc_bf16(2 * kPjM, kPjN, false, false);
+      const uint32_t empty1 = umma::cluster_addr(bar_empty, 1);
+      const uint32_t afull1 = umma::cluster_addr(bar_afull, 1);
       int g = 0;
       for (int k = 0; k < n_mine && !*abort_flag; ++k) {
         const int a = k & 1;
-        if (k >= 2 && !umma::mbar_wait(bar_aempty + a, ((k - 2) >> 1) & 1)) { fail(); break; }
+        // both epilogues have read accumulator a (tile k-2)
+        if (k >= 2 && !umma::mbar_wait_cluster(bar_aempty + a, ((k - 2) >> 1) & 1)) {
+          fail();
+          break;
+        }
         umma::tc_fence_after();
         bool okk = true;
         for (int kb = 0; kb < nkb; ++kb, ++g) {
@@ -186,19 +222,22 @@ __global__ void __launch_bounds__(kPjThreads, 1)
           const uint32_t sb = umma::smem_u32(sm + Lay::kB + s * Lay::kStageB);
 #pragma unroll
           for (int k0 = 0; k0 < kPjK; k0 += 16)
-            umma::mma_bf16(tmem + a * kPjN, umma::desc_kmajor_sw128(sa, k0, kPjM),
-                           umma::desc_kmajor_sw128(sb, k0, kPjN), id, (kb | k0) != 0);
-          umma::mma_commit(bar_empty + s);
+            umma::mma_bf16_pair(tmem + a * kPjN, umma::desc_kmajor_sw128(sa, k0, kPjM),
+                                umma::desc_kmajor_sw128(sb, k0, kPjNHalf), id, (kb | k0) != 0);
+          umma::mma_commit_pair(umma::smem_u32(bar_empty + s));
+          umma::mma_commit_pair(empty1 + 8u * s);
         }
         if (!okk) { fail(); break; }
-        umma::mma_commit(bar_afull + a);
+        umma::mma_commit_pair(umma::smem_u32(bar_afull + a));
+        umma::mma_commit_pair(afull1 + 8u * a);
       }
-      umma::mma_commit(bar_done);
+      umma::mma_commit_pair(umma::smem_u32(bar_done));
     }
   } else {
     // ================= epilogue: warps 2-5, TMEM lane quadrant = warp mod 4 =================
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
+    const uint32_t aempty0 = umma::cluster_addr(bar_aempty, 0);
     for (int k = 0; k < n_mine && !*abort_flag; ++k) {
       const int a = k & 1;
       int m0, n0;
@@ -219,6 +258,13 @@ __global__ void __launch_bounds__(kPjThreads, 1)
         umma::mbar_arrive(bar_tready);
         if (!umma::mbar_wait(bar_tready, k & 1)) { fail(); break; }
       }
+      // the projection this tile belongs to (every projection is whole tiles wide)
+      int og = 0;
+      if (Mode == kProjHeads)
+        while (og + 1 < p.n_out && n0 >= p.col_begin[og + 1]) ++og;
+      __nv_bfloat16* yo = p.y[og];
+      const int Dg = p.D[og];
+      const int nb = n0 - p.col_begin[og];
       const int m = m0 + r;
       const int b = m / p.L, t = m - (m / p.L) * p.L;
 #pragma unroll 1
@@ -229,14 +275,14 @@ __global__ void __launch_bounds__(kPjThreads, 1)
 #pragma unroll
         for (int g = 0; g < 4; ++g) {  // 8 columns = one 16-byte store
           const int cl = c32 * 32 + g * 8;  // column within the tile
-          const int n = n0 + cl;
           float v[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) v[e] = acc[g * 8 + e];
           size_t dst;
           if (Mode == kProjHeads) {
-            const int hh = n / p.D, d = n - hh * p.D;
-            dst = (((size_t)b * p.H + hh) * p.L + t) * p.D + d;
+            const int n = nb + cl;
+            const int hh = n / Dg, d = n - hh * Dg;
+            dst = (((size_t)b * p.H + hh) * p.L + t) * Dg + d;
           } else {
             // input rows m - j of this tile's columns: row r + 8 - j of the staged
             // block cl / 64, 16-byte chunk (cl mod 64) / 8, swizzled by row mod 8
@@ -264,7 +310,7 @@ __global__ void __launch_bounds__(kPjThreads, 1)
             const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
             for (int e = 0; e < 8; ++e) v[e] = (v[e] + bv[e]) * conv[e];
-            dst = (size_t)m * p.N + n;
+            dst = (size_t)m * p.N + n0 + cl;
           }
           uint32_t pk[4];
 #pragma unroll
@@ -272,11 +318,13 @@ __global__ void __launch_bounds__(kPjThreads, 1)
             const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
             pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
           }
-          *reinterpret_cast<uint4*>(p.y + dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(yo + dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
       }
+      // accumulator a is read: one arrival per warp on the even CTA's barrier
       umma::tc_fence_before();
-      umma::mbar_arrive(bar_aempty + a);
+      __syncwarp();
+      if (lane == 0) umma::mbar_arrive_cluster(aempty0 + 8u * a);
       if (Mode == kBaseConv) {
         umma::mbar_arrive(bar_hempty);
         umma::mbar_arrive(bar_tfree);
@@ -285,12 +333,14 @@ __global__ void __launch_bounds__(kPjThreads, 1)
   }
   umma::tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
-    // TMEM is released only after every MMA issued here has completed
+  // every MMA of the pair has completed before either CTA releases its TMEM
+  if (warp == 1 && rank == 0) {
     if (lane == 0) umma::mbar_wait(bar_done, 0);
     __syncwarp();
-    umma::tmem_dealloc(tmem, 2 * kPjN);
   }
+  umma::cluster_sync();
+  umma::tc_fence_after();
+  if (warp == 1) umma::tmem_dealloc_pair(tmem, 2 * kPjN);
 }
 
 }  // namespace based

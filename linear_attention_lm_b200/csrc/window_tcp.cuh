@@ -283,7 +283,8 @@ __global__ void __launch_bounds__(kWpThreads, 1)
         umma::bulk_commit();
       }
     }
-    if (r == 0) umma::bulk_wait<0>();
+    // the last store has read its staging tile (its global writes complete with the grid)
+    if (r == 0) umma::bulk_wait_read<0>();
   }
   umma::tc_fence_before();
   __syncthreads();

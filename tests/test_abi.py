@@ -272,6 +272,24 @@ def test_proj_host_validation(lib):
     assert f(None, None, None, 0, 8, 1024, 16, 16, 1, None) == 0             # nothing to do
 
 
+def test_proj_multi_host_validation(lib):
+    f = lib.based_proj_heads_multi_fwd
+    D = (ctypes.c_int * 3)(16, 64, 64)
+    Y = (ctypes.c_void_p * 3)(FAKE, FAKE, FAKE)
+    Yn = (ctypes.c_void_p * 3)(FAKE, None, FAKE)
+    d, y, yn = (ctypes.cast(a, ctypes.c_void_p) for a in (D, Y, Yn))
+    # x, w, n_out, D, y, B, L, d_model, H, dt, stream
+    assert f(FAKE, FAKE, 0, d, y, 1, 8, 1024, 16, 1, None) == INVALID     # no projection
+    assert f(FAKE, FAKE, 9, d, y, 1, 8, 1024, 16, 1, None) == INVALID     # more than 8
+    assert f(FAKE, FAKE, 3, None, y, 1, 8, 1024, 16, 1, None) == INVALID  # no D array
+    assert f(FAKE, FAKE, 3, d, y, 1, 8, 1024, 16, 0, None) == UNSUPPORTED # fp32
+    assert f(FAKE, FAKE, 3, d, y, 1, 8, 1024, 3, 1, None) == UNSUPPORTED  # H*D % 256
+    assert f(FAKE, FAKE, 3, d, y, 1, 8, 1000, 16, 1, None) == UNSUPPORTED # d_model % 64
+    assert f(FAKE, FAKE, 3, d, yn, 1, 8, 1024, 16, 1, None) == INVALID    # a null output
+    assert f(None, FAKE, 3, d, y, 1, 8, 1024, 16, 1, None) == INVALID
+    assert f(None, None, 3, d, yn, 0, 8, 1024, 16, 1, None) == 0          # nothing to do
+
+
 def test_baseconv_host_validation(lib):
     f = lib.based_baseconv_fwd
     # x, w, bias, taps, y, B, L, D, K, dt, stream

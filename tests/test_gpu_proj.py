@@ -80,6 +80,45 @@ def test_proj_heads_full_size_sampled():
     assert lab.based_get_device_error() == 0
 
 
+@pytest.mark.parametrize("B,L,d_model,H,Ds", [
+    (1, 100, 256, 16, (16, 16, 64, 64, 64, 64)),  # one pair tile, the odd CTA's rows all past M
+    (3, 257, 192, 32, (8, 64)),                    # ragged M over several pair tiles
+    (2, 300, 1024, 16, (64, 16, 64, 16)),          # projections of different widths interleaved
+])
+def test_proj_heads_multi_matches_oracle(B, L, d_model, H, Ds):
+    """Every output of one multi-projection launch against the oracle's
+    projection with that output's rows of the stacked weights."""
+    x = gen(600 + L, (B, L, d_model))
+    w = gen(700 + d_model, (H * sum(Ds), d_model), 0.02)
+    ys = lab.proj_heads_multi(x.cuda(), w.cuda(), H, Ds)
+    torch.cuda.synchronize()
+    assert lab.based_get_device_error() == 0
+    off = 0
+    for D, y in zip(Ds, ys):
+        check_close(y, oracle.proj_heads(f64(x), f64(w[off:off + H * D]), H))
+        off += H * D
+
+
+def test_proj_heads_multi_full_size_sampled():
+    """layer_360m's six projections (q, k: 16 heads of 16; v and the window
+    layer's q, k, v: 16 heads of 64) of x [8, 2048, 1024] in one launch, checked
+    on two whole sequences and a ragged time slice of all of them."""
+    B, L, dm, H = 8, 2048, 1024, 16
+    Ds = (16, 16, 64, 64, 64, 64)
+    x = gen(21, (B, L, dm))
+    w = gen(22, (H * sum(Ds), dm), 0.02)
+    ys = [y.cpu() for y in lab.proj_heads_multi(x.cuda(), w.cuda(), H, Ds)]
+    torch.cuda.synchronize()
+    assert lab.based_get_device_error() == 0
+    off = 0
+    for D, y in zip(Ds, ys):
+        wd = f64(w[off:off + H * D])
+        for b in (2, 7):
+            check_close(y[b:b + 1], oracle.proj_heads(f64(x[b:b + 1]), wd, H))
+        check_close(y[:, :, 1500:1533], oracle.proj_heads(f64(x[:, 1500:1533]), wd, H))
+        off += H * D
+
+
 # ------------------------------------------------------------------ BaseConv
 
 @pytest.mark.parametrize("B,L,D,K", [
