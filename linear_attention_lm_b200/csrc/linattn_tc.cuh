@@ -355,65 +355,79 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     record_device_error(BASED_ERR_TIMEOUT);
     *abort_flag = 1;
   };
-  // [S|z]^T -> shared memory as [feature][value column | z] (stride DV + 4), then
-  // coalesced rows of the 273-row layout (or of the segment partial).  Called
-  // by the 128 threads of one warp group (t = index in the group, TMEM quadrant
-  // = warp & 3) once the last #5 is complete and the feature-map buffers are no
-  // longer read.
-  auto export_kst = [&](int t) {
+  // Export of [S|z]^T in two steps.  export_stage: TMEM -> shared memory as
+  // [feature][value column | z] (stride DV + 4) and the map from the 273 output
+  // rows to features; run by the 128 threads of one warp group (t = index in
+  // the group, TMEM quadrant = warp & 3) once the last #5 is complete and the
+  // feature-map buffers are no longer read.  export_store: coalesced rows of the
+  // 273-row layout (or of the segment partial) by n threads (u = 0..n-1), after
+  // a barrier that orders them behind export_stage.
+  constexpr int kStr = DV + 4;  // keeps each feature row 16-byte aligned
+  auto export_stage = [&](int t) {
     if constexpr (Lay::kSt) {
-    const bool any_st = has_init || c_begin < c_end;
-    constexpr int kStr = DV + 4;  // keeps each feature row 16-byte aligned
-    float* stage = reinterpret_cast<float*>(sm + Lay::kPhiK);
-    int* rowmap = reinterpret_cast<int*>(stage + kSymFP * kStr);  // [273]: 2 f + (1 if / sqrt 2)
-    static_assert(Lay::kPhiKBuf * 40960 >= (kSymFP * kStr + kF) * 4, "export staging");
-    if (quad < 3) {
-      // two TMEM round trips of 80 features each
+      const bool any_st = has_init || c_begin < c_end;
+      float* stage = reinterpret_cast<float*>(sm + Lay::kPhiK);
+      int* rowmap = reinterpret_cast<int*>(stage + kSymFP * kStr);  // [273]: 2 f + (1 if / sqrt 2)
+      static_assert(Lay::kPhiKBuf * 40960 >= (kSymFP * kStr + kF) * 4, "export staging");
+      if (quad < 3) {
+        // two TMEM round trips of 80 features each
 #pragma unroll 1
-      for (int g = 0; g < 2; ++g) {
-        float sv[80];
-        umma::tmem_ld80(tmem + Lay::kTmS0 + tm_lane + g * 80, sv);
-        if (t <= DV) {
+        for (int g = 0; g < 2; ++g) {
+          float sv[80];
+          umma::tmem_ld80(tmem + Lay::kTmS0 + tm_lane + g * 80, sv);
+          if (t <= DV) {
 #pragma unroll
-          for (int i = 0; i < 80; ++i) stage[(g * 80 + i) * kStr + t] = any_st ? sv[i] : 0.0f;
+            for (int i = 0; i < 80; ++i) stage[(g * 80 + i) * kStr + t] = any_st ? sv[i] : 0.0f;
+          }
+        }
+      }
+      for (int f = t; f < kSymFP; f += kTcGroup) {
+        int r0 = -1, r1 = -1;
+        float scale = 1.0f;
+        const int nrows = tc_feature_rows(f, &r0, &r1, &scale);
+        const int code = 2 * f + (nrows == 2 ? 1 : 0);
+        if (nrows >= 1) rowmap[r0] = code;
+        if (nrows == 2) rowmap[r1] = code;
+      }
+    }
+  };
+  auto export_store = [&](int u, int n) {
+    if constexpr (Lay::kSt) {
+      const float* stage = reinterpret_cast<const float*>(sm + Lay::kPhiK);
+      const int* rowmap = reinterpret_cast<const int*>(stage + kSymFP * kStr);
+      if (kStateOnly) {
+        float* part = p.partial + ((size_t)bh * (p.n_seg - 1) + seg) * kSymFP * NA;
+        for (int i = u; i < kSymFP * NA; i += n) {
+          const int f = i / NA, j = i - f * NA;
+          part[i] = j <= DV ? stage[f * kStr + j] : 0.0f;
+        }
+      } else if (seg == p.n_seg - 1) {
+        if (p.state_kv) {
+          float4* skv = reinterpret_cast<float4*>(p.state_kv + (size_t)bh * kF * DV);
+#pragma unroll 4
+          for (int i = u; i < kF * (DV / 4); i += n) {
+            const int r = i / (DV / 4), j = (i - r * (DV / 4)) * 4;
+            const int code = rowmap[r];
+            const float sc = (code & 1) ? 0.70710678118654752f : 1.0f;
+            const float4 v4 = *reinterpret_cast<const float4*>(stage + (code >> 1) * kStr + j);
+            skv[i] = make_float4(v4.x * sc, v4.y * sc, v4.z * sc, v4.w * sc);
+          }
+        }
+        if (p.state_k) {
+          float* sk = p.state_k + (size_t)bh * kF;
+          for (int r = u; r < kF; r += n) {
+            const int code = rowmap[r];
+            sk[r] = stage[(code >> 1) * kStr + DV] * ((code & 1) ? 0.70710678118654752f : 1.0f);
+          }
         }
       }
     }
-    for (int f = t; f < kSymFP; f += kTcGroup) {
-      int r0 = -1, r1 = -1;
-      float scale = 1.0f;
-      const int nrows = tc_feature_rows(f, &r0, &r1, &scale);
-      const int code = 2 * f + (nrows == 2 ? 1 : 0);
-      if (nrows >= 1) rowmap[r0] = code;
-      if (nrows == 2) rowmap[r1] = code;
-    }
+  };
+  // the whole export by one warp group (segment partials, empty segments)
+  auto export_kst = [&](int t) {
+    export_stage(t);
     umma::named_sync(1, kTcGroup);
-    if (kStateOnly) {
-      float* part = p.partial + ((size_t)bh * (p.n_seg - 1) + seg) * kSymFP * NA;
-      for (int i = t; i < kSymFP * NA; i += kTcGroup) {
-        const int f = i / NA, j = i - f * NA;
-        part[i] = j <= DV ? stage[f * kStr + j] : 0.0f;
-      }
-    } else if (seg == p.n_seg - 1) {
-      if (p.state_kv) {
-        float4* skv = reinterpret_cast<float4*>(p.state_kv + (size_t)bh * kF * DV);
-        for (int i = t; i < kF * (DV / 4); i += kTcGroup) {
-          const int r = i / (DV / 4), j = (i - r * (DV / 4)) * 4;
-          const int code = rowmap[r];
-          const float sc = (code & 1) ? 0.70710678118654752f : 1.0f;
-          const float4 v4 = *reinterpret_cast<const float4*>(stage + (code >> 1) * kStr + j);
-          skv[i] = make_float4(v4.x * sc, v4.y * sc, v4.z * sc, v4.w * sc);
-        }
-      }
-      if (p.state_k) {
-        float* sk = p.state_k + (size_t)bh * kF;
-        for (int r = t; r < kF; r += kTcGroup) {
-          const int code = rowmap[r];
-          sk[r] = stage[(code >> 1) * kStr + DV] * ((code & 1) ? 0.70710678118654752f : 1.0f);
-        }
-      }
-    }
-    }
+    export_store(t, kTcGroup);
   };
 
   if (warp == 12) {
@@ -682,15 +696,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       umma::mbar_arrive(bar_p);
     }
     if constexpr (Lay::kSt && !kStateOnly) {
-      // the final state (or nothing, for an empty segment) is exported here, as
-      // soon as the last #5 completes, while #2, #4 and the last output still run
+      // the final state is exported here, as soon as the last #5 completes,
+      // while #2, #4 and the last output still run: this group stages it, then
+      // this group and group F (idle by then) write it out.  Both groups take
+      // the decision together (barrier 2, 256 threads).
       if (c_begin < c_end) {
         BASED_TC_TRACE(2, 0);
         const bool ok = !*abort_flag && umma::mbar_wait(bar_m5, (c_end - 1 - c_begin) & 1);
-        if (umma::named_sync_all(1, kTcGroup, ok)) {
+        if (umma::named_sync_all(2, 2 * kTcGroup, ok)) {
           umma::tc_fence_after();
           BASED_TC_TRACE(3, 0);
-          export_kst(t);
+          export_stage(t);
+          umma::named_sync(3, 2 * kTcGroup);
+          export_store(t, 2 * kTcGroup);
           BASED_TC_TRACE(4, 0);
         } else if (!*abort_flag) {
           fail();
@@ -813,6 +831,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         umma::tc_fence_before();
         BASED_TC_TRACE(4, it);
         umma::mbar_arrive(bar_phiq);
+      }
+    }
+    if constexpr (Lay::kSt && !kStateOnly) {
+      // second half of the export writers (group P decides and stages)
+      if (c_begin < c_end && umma::named_sync_all(2, 2 * kTcGroup, true)) {
+        umma::named_sync(3, 2 * kTcGroup);
+        export_store(kTcGroup + t, 2 * kTcGroup);
       }
     }
   } else if (!kStateOnly) {
