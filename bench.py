@@ -56,7 +56,6 @@ def load_peaks():
 # replicas: one independent copy of the workload per rank, no data exchange
 # ---------------------------------------------------------------------------
 
-FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # 74.4: CUDA-core fp32 peak of a B200
 
 
 def max_over_ranks(ms: float, dev, world: int) -> float:
@@ -582,22 +581,29 @@ def run_projections(args, lab, dev, world, peaks, warm):
              "gradient of the linear attention, bf16, B=8 H=16 L=2048 d=16 d_v=64 (quadratic "
              "form on the tensor cores; 480 flop per (t, s) pair counted)"),
             ("window_bwd", wbwd_step, 10.0 * 64 * B * H * w_pairs, 2,
-             "gradient of the window attention, B=8 H=16 L=2048 d_h=64 W=64 (10 d_h flop per "
-             "(query, key) pair in the band)")):
-        ms = timed(fn, 10 if name.endswith("bwd") else n)
+             "gradient of the window attention, bf16, B=8 H=16 L=2048 d_h=64 W=64 on the "
+             "tensor cores (q, k, v, dy read in bf16, dq, dk, dv written in fp32, 3 fp32 "
+             "statistics per query written and read; 10 d_h flop per (query, key) pair in "
+             "the band)")):
+        ms = timed(fn, 10 if name == "linattn_bwd" else n)
         tf = flops / (ms / 1e3) / 1e12
         if name == "linattn_bwd":
             kern, bound, pk, src = "linattn_bwd_tc", "tensor", peak, peaks["source"]
-        elif name.endswith("bwd"):
-            # CUDA-core fp32 FMA peak: 148 SMs x 128 FMA/clk x 2 flop x 1.965 GHz
-            kern, bound, pk, src = name, "alu", FP32_FMA_TFLOPS, "unit counts x max clock"
+        elif name == "window_bwd":
+            kern, bound = "window_bwd_tc", "hbm"
         else:
             kern, bound, pk, src = "proj_tc", "tensor", peak, peaks["source"]
         out[name] = {"workload": what, "ms_per_step": round(ms, 5), "launches_per_step": launches,
-                     "tokens_per_s": round(world * B * L / (ms / 1e3), 1),
-                     "roofline": {"kernel": kern, "bound": bound, "achieved": round(tf, 2),
-                                  "peak": pk, "unit": "TFLOP/s", "frac": round(tf / pk, 4),
-                                  "traffic": None, "peak_source": src}}
+                     "tokens_per_s": round(world * B * L / (ms / 1e3), 1)}
+        if bound == "hbm":
+            # bytes per token-head: 4 x 2 d_h (bf16 in) + 3 x 4 d_h (fp32 out) + 3 x 4 x 2
+            nbytes = B * H * L * (4 * 2 * 64 + 3 * 4 * 64 + 24)
+            out[name]["roofline"] = hbm_roofline(kern, nbytes, ms, peaks)
+            out[name]["tflops"] = round(tf, 2)
+        else:
+            out[name]["roofline"] = {"kernel": kern, "bound": bound, "achieved": round(tf, 2),
+                                     "peak": pk, "unit": "TFLOP/s", "frac": round(tf / pk, 4),
+                                     "traffic": None, "peak_source": src}
         if name in ("proj", "baseconv"):
             # library context: torch.matmul of the same GEMM (no epilogue, no head split)
             tms = timed(torch_proj_step if name == "proj" else torch_conv_gemm, n)

@@ -229,12 +229,16 @@ based_status_t based_linattn_bwd(const void* q, const void* k, const void* v, co
 /*
  * Gradient of based_window_attn_fwd's output:
  *   y_t = sum_{s = max(0, t-window+1)}^{t} softmax_s(q_t . k_s / sqrt(d_head)) v_s
- * Given dy returns dq, dk, dv (fp32) on CUDA cores.
- *   q, k, v, dy [B, H, L, d_head] dt (d_head == 64; 1 <= window <= 64)
+ * Given dy returns dq, dk, dv (fp32).  bf16 inputs run on the tensor cores
+ * (d_head 64 or 128): the scores and dP = dy v^T by tcgen05, P and
+ * dS = P (dP - delta) rounded to bf16 as the operands of dq, dk, dv, fp32
+ * accumulation.  fp32 inputs run on CUDA cores in fp32 (d_head 64).
+ *   q, k, v, dy [B, H, L, d_head] dt (1 <= window <= 64)
  *   dq, dk, dv  [B, H, L, d_head] fp32 (written)
  *   workspace: based_window_attn_bwd_workspace_bytes() bytes of device memory
  *   (per query: row max, row sum, dy . y), else BASED_ERR_WORKSPACE.
- * Pointers must be 16-byte aligned (BASED_ERR_INVALID_ARG otherwise).
+ * Other d_head values: BASED_ERR_UNSUPPORTED.  Pointers must be 16-byte
+ * aligned (BASED_ERR_INVALID_ARG otherwise).
  */
 size_t based_window_attn_bwd_workspace_bytes(int B, int H, int L);
 based_status_t based_window_attn_bwd(const void* q, const void* k, const void* v, const void* dy,

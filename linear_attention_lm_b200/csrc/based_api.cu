@@ -20,6 +20,7 @@
 #include "window_tc.cuh"
 #include "window_tcp.cuh"
 #include "proj_tc.cuh"
+#include "window_bwd_tc.cuh"
 
 namespace based {
 
@@ -387,6 +388,34 @@ based_status_t launch_window_bwd(const void* q, const void* k, const void* v, co
   return launch_status();
 }
 
+// bf16 window gradient on the tensor cores (d_h = 64 or 128)
+template <int DH>
+based_status_t launch_window_bwd_tc(const void* q, const void* k, const void* v, const void* dy,
+                                    float* dq, float* dk, float* dv, int BH, int L, int W,
+                                    float* ws, cudaStream_t st) {
+  CUtensorMap q128, dy128, k192, v192, k128, v128, q192, dy192;
+  if (!make_rows_map(&q128, q, DH, L, BH, kWgT) || !make_rows_map(&dy128, dy, DH, L, BH, kWgT) ||
+      !make_rows_map(&k192, k, DH, L, BH, kWgN) || !make_rows_map(&v192, v, DH, L, BH, kWgN) ||
+      !make_rows_map(&k128, k, DH, L, BH, kWgT) || !make_rows_map(&v128, v, DH, L, BH, kWgT) ||
+      !make_rows_map(&q192, q, DH, L, BH, kWgN) || !make_rows_map(&dy192, dy, DH, L, BH, kWgN))
+    return BASED_ERR_CUDA;
+  auto kq = window_bwd_tc_q_kernel<DH>;
+  auto kkv = window_bwd_tc_kv_kernel<DH>;
+  const size_t smem = WgLayout<DH>::kSmem;
+  if (!set_smem(kq, smem) || !set_smem(kkv, smem)) return BASED_ERR_CUDA;
+  WgParams p;
+  p.dq = dq; p.dk = dk; p.dv = dv; p.ws = ws;
+  p.L = L; p.W = W; p.BH = BH;
+  p.n_tiles = (L + kWgT - 1) / kWgT;
+  const long long nblk = (long long)BH * p.n_tiles;
+  if (nblk > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
+  kq<<<(unsigned)nblk, kWgThreads, smem, st>>>(q128, dy128, k192, v192, p);
+  const based_status_t s1 = launch_status();
+  if (s1 != BASED_OK) return s1;
+  kkv<<<(unsigned)nblk, kWgThreads, smem, st>>>(k128, v128, q192, dy192, p);
+  return launch_status();
+}
+
 // ---------------------------------------------------------------------------
 // Allocation-free prefill (based_linattn_fwd_noalloc): the segment partials
 // live in this fixed array instead of a caller workspace.  Host code may not
@@ -654,7 +683,9 @@ based_status_t based_window_attn_bwd(const void* q, const void* k, const void* v
                                      size_t workspace_bytes, based_stream_t stream) {
   if (B < 0 || H < 0 || L < 0 || window < 1) return BASED_ERR_INVALID_ARG;
   if (dt != BASED_BF16 && dt != BASED_F32) return BASED_ERR_INVALID_ARG;
-  if (d_head != kWbDh || window > kWbT) return BASED_ERR_UNSUPPORTED;
+  // bf16: tensor cores, d_h 64 or 128; fp32: CUDA cores, d_h 64
+  if (window > kWbT || (dt == BASED_F32 ? d_head != kWbDh : (d_head != 64 && d_head != 128)))
+    return BASED_ERR_UNSUPPORTED;
   const long long BH = (long long)B * H;
   if (BH > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
   const bool empty = BH * L == 0;
@@ -671,7 +702,9 @@ based_status_t based_window_attn_bwd(const void* q, const void* k, const void* v
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dt == BASED_F32)
     return launch_window_bwd<float>(q, k, v, dy, dq, dk, dv, (int)BH, L, window, ws, st);
-  return launch_window_bwd<__nv_bfloat16>(q, k, v, dy, dq, dk, dv, (int)BH, L, window, ws, st);
+  if (d_head == 128)
+    return launch_window_bwd_tc<128>(q, k, v, dy, dq, dk, dv, (int)BH, L, window, ws, st);
+  return launch_window_bwd_tc<64>(q, k, v, dy, dq, dk, dv, (int)BH, L, window, ws, st);
 }
 
 based_status_t based_proj_heads_multi_fwd(const void* x, const void* w, int n_out, const int* D,

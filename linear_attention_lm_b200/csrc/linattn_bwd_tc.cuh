@@ -184,14 +184,17 @@ __global__ void __launch_bounds__(kBtThreads, 1)
   float dsum = 0.0f;  // D_t (pass 1), then dD_t (pass 2), for query t0 + tid
   const int row = tid;  // compute threads: query row = TMEM lane
   const uint32_t sQ = umma::smem_u32(sm + Lay::kQ);
+  // K rows of the next step, loaded one step ahead of their use
+  uint4 klo = make_uint4(0, 0, 0, 0), khi = klo;
+  if (!issuer) bt_load_row16(kb, (long long)tid, L, &klo, &khi);
   for (int step = 0; step < n_steps; ++step) {
     const int pass = step / (i + 1), j = step % (i + 1), b = step & 1;
     const bool diag = j == i;
-    if (!issuer) {  // K_j rows, both layouts
-      uint4 lo, hi;
-      bt_load_row16(kb, (long long)j * kBtT + tid, L, &lo, &hi);
-      bt_put_row16(sm + Lay::kK + b * 4096, sm + Lay::kKm + b * 4096, tid, lo, hi);
+    if (!issuer) {  // K_j rows, both layouts; then the next step's rows
+      bt_put_row16(sm + Lay::kK + b * 4096, sm + Lay::kKm + b * 4096, tid, klo, khi);
       umma::fence_async_smem();
+      if (step + 1 < n_steps)
+        bt_load_row16(kb, (long long)((step + 1) % (i + 1)) * kBtT + tid, L, &klo, &khi);
     }
     if (__syncthreads_or(failed)) break;
     if (issuer && lane == 0) {
@@ -213,6 +216,12 @@ __global__ void __launch_bounds__(kBtThreads, 1)
                            umma::idesc_bf16(128, 128, false, false), k0 > 0);
         }
         umma::mma_commit(bar_m1);
+        // the next step's V tile goes to the other buffer, whose MMAs (those of
+        // the previous step) are complete
+        if (step + 1 < n_steps) {
+          issue_v(step + 1);
+          ++v_inflight;
+        }
       }
     }
     // ---- CUDA cores: W (pass 1) or E (pass 2) of this lane's query row ----
@@ -274,11 +283,6 @@ __global__ void __launch_bounds__(kBtThreads, 1)
                        umma::idesc_bf16(128, 16, false, true), (j > 0 || ks > 0) ? 1u : 0u);
       }
       umma::mma_commit(bar_m2);
-      // the next step's V tile goes to the other buffer, whose MMAs are complete
-      if (step + 1 < n_steps) {
-        issue_v(step + 1);
-        ++v_inflight;
-      }
     }
     if (!umma::mbar_wait(bar_m2, step & 1)) fail();
     umma::tc_fence_after();
@@ -442,16 +446,23 @@ __global__ void __launch_bounds__(kBtThreads, 1)
   const int row = tid;  // compute threads: key row = TMEM lane
   const uint32_t sK = umma::smem_u32(sm + Lay::kKk);
   const uint32_t sV = umma::smem_u32(sm + Lay::kVk);
+  // Q rows and dD of the next step, loaded one step ahead of their use
+  uint4 qlo = make_uint4(0, 0, 0, 0), qhi = qlo;
+  float ddn = 0.0f;
+  auto load_q = [&](int ti) {
+    const long long t = (long long)ti * kBtT + tid;
+    bt_load_row16(qb, t, L, &qlo, &qhi);
+    ddn = t < L ? p.ws_dd[bh * L + t] : 0.0f;
+  };
+  if (!issuer) load_q(j);
   for (int step = 0; step < n_steps; ++step) {
     const int ti = j + step, b = step & 1;
     const bool diag = ti == j;
-    if (!issuer) {  // Q_i rows (both layouts) and dD_i
-      uint4 lo, hi;
-      const long long t = (long long)ti * kBtT + tid;
-      bt_load_row16(qb, t, L, &lo, &hi);
-      bt_put_row16(sm + Lay::kQk + b * 4096, sm + Lay::kQm + b * 4096, tid, lo, hi);
-      reinterpret_cast<float*>(sm + Lay::kDD + b * 512)[tid] = t < L ? p.ws_dd[bh * L + t] : 0.0f;
+    if (!issuer) {  // Q_i rows (both layouts) and dD_i; then the next step's
+      bt_put_row16(sm + Lay::kQk + b * 4096, sm + Lay::kQm + b * 4096, tid, qlo, qhi);
+      reinterpret_cast<float*>(sm + Lay::kDD + b * 512)[tid] = ddn;
       umma::fence_async_smem();
+      if (step + 1 < n_steps) load_q(ti + 1);
     }
     if (__syncthreads_or(failed)) break;
     if (issuer && lane == 0) {
@@ -470,6 +481,12 @@ __global__ void __launch_bounds__(kBtThreads, 1)
                          umma::desc_kmajor_sw128(sD, k0, kBtT),
                          umma::idesc_bf16(128, 128, false, false), k0 > 0);
         umma::mma_commit(bar_m1);
+        // the next step's dN tile goes to the other buffer (the previous step's
+        // MMAs are complete)
+        if (step + 1 < n_steps) {
+          issue_dn(step + 1);
+          ++inflight;
+        }
       }
     }
     if (!issuer) {
@@ -523,10 +540,6 @@ __global__ void __launch_bounds__(kBtThreads, 1)
                      umma::idesc_bf16(128, 16, false, true), acc);  // dK += E^T Q_i
       }
       umma::mma_commit(bar_m2);
-      if (step + 1 < n_steps) {
-        issue_dn(step + 1);
-        ++inflight;
-      }
     }
     if (!umma::mbar_wait(bar_m2, step & 1)) fail();
     umma::tc_fence_after();

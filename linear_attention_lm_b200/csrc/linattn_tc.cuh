@@ -1053,7 +1053,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (!*abort_flag && warp >= 8 && warp < 12) {
     // ---- state out of TMEM (group E lanes): segment partials or the final export ----
     const int t = tid - 2 * kTcGroup;
-    const bool any_st = has_init || c_begin < c_end;
     if constexpr (Lay::kSt) {
       // the main pass exported from group P already (right after its last #5)
       if (kStateOnly || c_begin == c_end) export_kst(t);

@@ -253,7 +253,8 @@ def test_window_bwd_host_validation(lib):
     assert lib.based_window_attn_bwd_workspace_bytes(2, 3, 100) == 2 * 3 * 100 * 3 * 4
     A = [FAKE] * 7
     # q, k, v, dy, dq, dk, dv, B, H, L, d_head, window, dt, workspace, bytes, stream
-    assert f(*A, 1, 2, 100, 128, 64, 1, FAKE, 1 << 20, None) == UNSUPPORTED   # d_head
+    assert f(*A, 1, 2, 100, 96, 64, 1, FAKE, 1 << 20, None) == UNSUPPORTED    # d_head (bf16: 64, 128)
+    assert f(*A, 1, 2, 100, 128, 64, 0, FAKE, 1 << 20, None) == UNSUPPORTED   # d_head (fp32: 64)
     assert f(*A, 1, 2, 100, 64, 65, 1, FAKE, 1 << 20, None) == UNSUPPORTED    # window
     assert f(*A, 1, 2, 100, 64, 0, 1, FAKE, 1 << 20, None) == INVALID
     assert f(*A, 1, 2, 100, 64, 64, 1, FAKE, 16, None) == 5                   # workspace
