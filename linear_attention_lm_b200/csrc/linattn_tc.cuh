@@ -45,8 +45,8 @@
 //            still works on chunk c;
 //   group E (warps 8-11): epilogue of chunk c -- y from O, and the fp16 copy of the
 //            state for chunk c+1;
-//   issue warp (warp 12, one thread): V tiles by TMA (double-buffered when shared
-//            memory allows) and the MMAs in the order #1, #5, #2, (P), #4.
+//   issue warp (warp 12, one thread): V tiles by TMA (three stages at d_v = 64,
+//            one at d_v = 128) and the MMAs in the order #1, #5, #2, (P), #4.
 // Warps w, w+4 and w+8 share TMEM lane quadrant w, so each group reads and writes
 // the TMEM rows of its own 32 tokens.
 // The second state tile (features 128..191, of which 128..159 are used) is an
@@ -290,6 +290,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* bar_yfull = bars + 11;   // y staging tile written (group E)
   uint64_t* bar_m5 = bars + 12;      // #5 done (commit): the state can be read
   uint64_t* bar_sread = bars + 13;   // state read and its fp16 copy written (group E)
+  constexpr int kThreads = kTcThreads;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quad = warp & 3;
@@ -327,7 +328,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // ones block of every V stage: column DV of the augmented V is 1 for every token
   for (int b = 0; b < Lay::kNOnes; ++b) {
     uint8_t* ones = sm + Lay::kV + Lay::ones_off(b);
-    for (int i = tid; i < 16384 / 16; i += kTcThreads)
+    for (int i = tid; i < 16384 / 16; i += kThreads)
       reinterpret_cast<uint4*>(ones)[i] = make_uint4(0, 0, 0, 0);
   }
   __syncthreads();
@@ -340,7 +341,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // rows DV..NA-1 of the transposed fp16 state copies: row DV (z) is rewritten
     // for every chunk, the rows after it stay zero
     for (int b = 0; b < Lay::kSBuf; ++b)
-      for (int i = tid; i < (NA - DV) * kSymFP * 2 / 16; i += kTcThreads)
+      for (int i = tid; i < (NA - DV) * kSymFP * 2 / 16; i += kThreads)
         reinterpret_cast<uint4*>(sm + Lay::kS + b * Lay::kSBytes + DV * kSymFP * 2)[i] =
             make_uint4(0, 0, 0, 0);
   }
@@ -423,11 +424,52 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     }
   };
+  // Final state of the main pass straight from TMEM: the thread on TMEM lane j
+  // (j < DV: value column j; j = DV: z) loads 80 features (half h of the 160)
+  // and writes its column of every output row they map to; the 32 lanes of a
+  // warp write 32 consecutive floats of a row.  Run by warps of quadrants 0-2
+  // of one group per half, once the last #5 is complete.
+  auto export_direct = [&](int h) {
+    if constexpr (Lay::kSt) {
+      if (quad < 3 && seg == p.n_seg - 1) {
+        float sv[80];
+        umma::tmem_ld80(tmem + Lay::kTmS0 + tm_lane + h * 80, sv);
+        const int j = quad * 32 + lane;
+        float* skv = p.state_kv ? p.state_kv + (size_t)bh * kF * DV + j : nullptr;
+        float* sk = p.state_k ? p.state_k + (size_t)bh * kF : nullptr;
+        float* dst = j < DV ? skv : (j == DV ? sk : nullptr);
+        const int stride = j < DV ? DV : 1;
+        if (dst != nullptr) {
+#pragma unroll
+          for (int i = 0; i < 80; ++i) {
+            int r0 = -1, r1 = -1;
+            float scale = 1.0f;
+            const int nrows = tc_feature_rows(h * 80 + i, &r0, &r1, &scale);
+            const float v = sv[i] * scale;
+            if (nrows >= 1) dst[(size_t)r0 * stride] = v;
+            if (nrows == 2) dst[(size_t)r1 * stride] = v;
+          }
+        }
+      }
+    }
+  };
   // the whole export by one warp group (segment partials, empty segments)
   auto export_kst = [&](int t) {
     export_stage(t);
     umma::named_sync(1, kTcGroup);
     export_store(t, kTcGroup);
+  };
+
+  // V tile of chunk c into a stage; returns whether a load was issued (the stall
+  // test leaves one out)
+  auto issue_v = [&](int c, int stage) {
+    if (c == c_begin + 1 && stall_test(kStallLinattnV)) return 0u;
+    umma::mbar_arrive_expect_tx(bar_tma + stage, DV * kTcChunk * 2);
+#pragma unroll
+    for (int blk = 0; blk < DV / 64; ++blk)
+      umma::tma_load_3d(sm + Lay::kV + stage * Lay::kVStage + blk * 16384, &vmap,
+                        bar_tma + stage, blk * 64, c * kTcChunk, bh);
+    return 1u;
   };
 
   if (warp == 12) {
@@ -436,17 +478,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint32_t sQ = umma::smem_u32(sm + Lay::kQ), sK = umma::smem_u32(sm + Lay::kK),
                      sP = umma::smem_u32(sm + Lay::kP), sPhiQ = umma::smem_u32(sm + Lay::kPhiQ),
                      sS = umma::smem_u32(sm + Lay::kS);
-      constexpr uint32_t kVBytes = DV * kTcChunk * 2;
-      // returns whether a load was issued (the stall test leaves one out)
-      auto issue_v = [&](int c, int stage) {
-        if (c == c_begin + 1 && stall_test(kStallLinattnV)) return 0u;
-        umma::mbar_arrive_expect_tx(bar_tma + stage, kVBytes);
-#pragma unroll
-        for (int blk = 0; blk < DV / 64; ++blk)
-          umma::tma_load_3d(sm + Lay::kV + stage * Lay::kVStage + blk * 16384, &vmap,
-                            bar_tma + stage, blk * 64, c * kTcChunk, bh);
-        return 1u;
-      };
       // descriptors are computed once per buffer and stepped along K by adding
       // the start-address increment (16-byte units) to their low word
       const uint64_t d_q = umma::desc_kmajor_none(sQ, 0, 16), d_k = umma::desc_kmajor_none(sK, 0, 16);
@@ -502,6 +533,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         BASED_TC_TRACE(2, it);
         inflight &= ~(1u << stage);
         vphase ^= 1u << stage;
+
         // #5 overwrites the state: the epilogue group must have read (and copied)
         // the previous chunk's state out of TMEM
         if (!kStateOnly && Lay::kEarlyO && has_state) {
@@ -697,18 +729,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     if constexpr (Lay::kSt && !kStateOnly) {
       // the final state is exported here, as soon as the last #5 completes,
-      // while #2, #4 and the last output still run: this group stages it, then
-      // this group and group F (idle by then) write it out.  Both groups take
-      // the decision together (barrier 2, 256 threads).
+      // while #2, #4 and the last output still run: this group writes features
+      // 0-79, group F (idle by then) features 80-159.  Both groups take the
+      // decision together (barrier 2, 256 threads).
       if (c_begin < c_end) {
         BASED_TC_TRACE(2, 0);
         const bool ok = !*abort_flag && umma::mbar_wait(bar_m5, (c_end - 1 - c_begin) & 1);
         if (umma::named_sync_all(2, 2 * kTcGroup, ok)) {
           umma::tc_fence_after();
           BASED_TC_TRACE(3, 0);
-          export_stage(t);
-          umma::named_sync(3, 2 * kTcGroup);
-          export_store(t, 2 * kTcGroup);
+          export_direct(0);
           BASED_TC_TRACE(4, 0);
         } else if (!*abort_flag) {
           fail();
@@ -741,6 +771,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     load_qk(c_begin, qr, kr);
     load_qk(c_begin + 1, qn, kn);
     load_qk(c_begin + 2, qm, km);
+    BASED_TC_TRACE(5, 0);
     for (int c = c_begin; c < c_end && !*abort_flag; ++c) {
       const int it = c - c_begin;
       const int t0 = c * kTcChunk;
@@ -769,6 +800,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int ch = 0; ch < 20; ++ch)
           *reinterpret_cast<uint4*>(phik + (ch * 16 + (t >> 3)) * 128 + (t & 7) * 16) =
               live ? tc_feature_chunk(XK, YK, k2, ch) : make_uint4(0, 0, 0, 0);
+
         if (!kStateOnly) {
           uint8_t* qrow = sm + Lay::kQ + ((t >> 3) * 2) * 128 + (t & 7) * 16;
           uint8_t* krow = sm + Lay::kK + ((t >> 3) * 2) * 128 + (t & 7) * 16;
@@ -834,10 +866,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     }
     if constexpr (Lay::kSt && !kStateOnly) {
-      // second half of the export writers (group P decides and stages)
+      // second half of the export (group P waits for the last #5 and decides)
       if (c_begin < c_end && umma::named_sync_all(2, 2 * kTcGroup, true)) {
-        umma::named_sync(3, 2 * kTcGroup);
-        export_store(kTcGroup + t, 2 * kTcGroup);
+        umma::tc_fence_after();
+        export_direct(1);
       }
     }
   } else if (!kStateOnly) {

@@ -26,8 +26,8 @@
 // counting the bytes of both CTAs on the even CTA's barrier; warp 1 of the even
 // CTA (one thread) issues four M=256/N=256/K=16 MMAs per block into one of two
 // TMEM accumulators, so the epilogue of tile k overlaps the main loop of tile
-// k+1; warps 2-5 (one per TMEM lane quadrant) run the epilogue on the CTA's own
-// 128 rows.  For BaseConv the producer also loads the CTA's input rows
+// k+1; warps 2-9 run the epilogue on the CTA's own 128 rows (warps w and w+4
+// share TMEM lane quadrant w mod 4 and take one half of the 256 columns each).  For BaseConv the producer also loads the CTA's input rows
 // [m0-8, m0+128) x [n0, n0+256) (the convolution's reach) into shared memory,
 // once the previous tile's epilogue has released them.
 #pragma once
@@ -41,7 +41,9 @@ constexpr int kPjM = 128;       // rows (tokens) per CTA; a pair covers 256
 constexpr int kPjN = 256;       // columns per tile
 constexpr int kPjNHalf = 128;   // rows of W loaded by each CTA of the pair
 constexpr int kPjK = 64;        // K block per stage (one 128-byte swizzle atom)
-constexpr int kPjThreads = 192;
+constexpr int kPjEpiWarps = 8;  // two per TMEM lane quadrant, each on half the columns
+constexpr int kPjEpiThreads = kPjEpiWarps * 32;
+constexpr int kPjThreads = 64 + kPjEpiThreads;
 constexpr int kPjMaxTaps = 8;
 constexpr int kPjHaloRows = kPjM + kPjMaxTaps;  // rows [m0 - 8, m0 + 128)
 constexpr int kPjMaxOut = 8;    // projections per launch
@@ -122,13 +124,13 @@ __global__ void __launch_bounds__(kPjThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       umma::mbar_init(bar_afull + a, 1);
-      umma::mbar_init(bar_aempty + a, 8);  // one arrival per epilogue warp of both CTAs
+      umma::mbar_init(bar_aempty + a, 2 * kPjEpiWarps);  // one per epilogue warp, both CTAs
     }
     umma::mbar_init(bar_hfull, 1);
-    umma::mbar_init(bar_hempty, kPjM);
+    umma::mbar_init(bar_hempty, kPjEpiThreads);
     umma::mbar_init(bar_done, 1);
-    umma::mbar_init(bar_tready, kPjM);
-    umma::mbar_init(bar_tfree, kPjM);
+    umma::mbar_init(bar_tready, kPjEpiThreads);
+    umma::mbar_init(bar_tfree, kPjEpiThreads);
     *abort_flag = 0;
     umma::fence_mbar_init();
   }
@@ -234,9 +236,11 @@ __global__ void __launch_bounds__(kPjThreads, 1)
       umma::mma_commit_pair(umma::smem_u32(bar_done));
     }
   } else {
-    // ================= epilogue: warps 2-5, TMEM lane quadrant = warp mod 4 =================
+    // ================= epilogue: warps 2-9, TMEM lane quadrant = warp mod 4 =================
     const int quad = warp & 3;
-    const int r = quad * 32 + lane;
+    const int r = quad * 32 + lane;          // row of the CTA's 128
+    const int half = (warp - 2) >> 2;        // columns [128 half, 128 half + 128)
+    const int et = (warp - 2) * 32 + lane;   // index among the epilogue threads
     const uint32_t aempty0 = umma::cluster_addr(bar_aempty, 0);
     for (int k = 0; k < n_mine && !*abort_flag; ++k) {
       const int a = k & 1;
@@ -251,7 +255,7 @@ __global__ void __launch_bounds__(kPjThreads, 1)
         // this tile's taps and bias into shared memory, once every epilogue
         // thread has finished reading the previous tile's
         if (k >= 1 && !umma::mbar_wait(bar_tfree, (k - 1) & 1)) { fail(); break; }
-        for (int c = r; c < kPjN; c += kPjM) {
+        for (int c = et; c < kPjN; c += kPjEpiThreads) {
           for (int j = 0; j < p.K; ++j) tapsT[j * kPjN + c] = __ldg(p.taps + (size_t)(n0 + c) * p.K + j);
           bias_s[c] = __ldg(p.bias + n0 + c);
         }
@@ -268,7 +272,7 @@ __global__ void __launch_bounds__(kPjThreads, 1)
       const int m = m0 + r;
       const int b = m / p.L, t = m - (m / p.L) * p.L;
 #pragma unroll 1
-      for (int c32 = 0; c32 < kPjN / 32; ++c32) {
+      for (int c32 = 4 * half; c32 < 4 * half + 4; ++c32) {
         float acc[32];
         umma::tmem_ld32(tmem + a * kPjN + (static_cast<uint32_t>(quad * 32) << 16) + c32 * 32, acc);
         if (m >= p.M) continue;

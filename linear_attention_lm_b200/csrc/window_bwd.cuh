@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(kWbThreads)
   using Lay = WbLayout;
   extern __shared__ float wsm[];
   float *qs = wsm + Lay::kA, *dys = wsm + Lay::kA2, *ks = wsm + Lay::kB, *vs = wsm + Lay::kB2;
-  float *pt = wsm + Lay::kP, *st = wsm + Lay::kR;
+  float* pt = wsm + Lay::kP;
   const int n_t = (L + kWbT - 1) / kWbT;
   const int bh = blockIdx.x / n_t, qt = blockIdx.x - bh * n_t;
   const int t0 = qt * kWbT, s_base = t0 - kWbT;  // staged key row c is key s_base + c
