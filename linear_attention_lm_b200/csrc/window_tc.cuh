@@ -15,8 +15,11 @@
 //                    S in its own TMEM lane
 //   O = P V          tcgen05, A = P from TMEM, M=128, N=dh, K=192 -> TMEM (fp32)
 //   y = O / l        CUDA cores: TMEM -> 128B-swizzled staging tile -> TMA store.
-// Keeping P in TMEM leaves shared memory to the Q, K, V tiles (the y staging tile
-// reuses Q's once O is complete) and spares the tensor core the P reads.
+// Keeping P in TMEM spares the tensor core the P reads.  Two CTAs share an SM:
+// V is loaded over Q and K once S is complete (its load overlaps the softmax,
+// and the other CTA's work), the y staging tile goes over V once O is complete,
+// and O takes the TMEM columns of S that P no longer needs, so a CTA holds
+// 32 + 48 KiB of shared memory and 256 TMEM columns at d_h = 128.
 #pragma once
 
 #include "common.cuh"
@@ -32,14 +35,17 @@ template <int DH>
 struct WtLayout {
   static constexpr int kQ = 0;                              // Q [128 x DH] K-major SW128
   static constexpr int kK = kQ + kWtQ * DH * 2;             // K [192 x DH] K-major SW128
-  static constexpr int kY = 0;                              // y [128 x DH] bf16 SW128 (over Q)
-  static constexpr int kV = kK + kWtKeys * DH * 2;          // V [192 x DH] MN-major SW128
-  static constexpr int kBar = kV + kWtKeys * DH * 2;
+  static constexpr int kV = 0;                              // V [192 x DH] MN-major SW128 (over Q, K)
+  static constexpr int kY = 0;                              // y [128 x DH] bf16 SW128 (over V)
+  static constexpr int kBar = kK + kWtKeys * DH * 2;
   static constexpr int kBytes = kBar + 64;
   static constexpr size_t kSmem = kBytes + 1024;
+  static_assert(kWtKeys * DH * 2 <= kBar, "V fits over Q and K");
+  // S in columns [0, 192); P (bf16 pairs) in [0, 96); O over the rest of S
   static constexpr int kTmS = 0;
-  static constexpr int kTmO = kWtKeys;
-  static constexpr int kTmemCols = (kTmO + DH <= 256) ? 256 : 512;
+  static constexpr int kTmO = kWtKeys / 2;
+  static constexpr int kTmemCols = 256;
+  static_assert(kTmO + DH <= kTmemCols, "TMEM budget");
 };
 
 template <int DH>
@@ -64,7 +70,8 @@ __global__ void __launch_bounds__(kWtThreads, 1)
   const int bh = blockIdx.x / n_tiles;
   const int t0 = tile * kWtQ;
 
-  // Q and K first (S needs them), V on its own barrier (only P V needs it)
+  // Q and K first (S needs them); V over them once S is complete
+  bool v_issued = false;  // thread 0
   if (tid == 0) {
     umma::mbar_init(bar_tma, 1);
     umma::mbar_init(bar_v, 1);
@@ -77,12 +84,6 @@ __global__ void __launch_bounds__(kWtThreads, 1)
     for (int b = 0; b < DH / 64; ++b) {
       umma::tma_load_3d(sm + Lay::kQ + b * kWtQ * 128, &qmap, bar_tma, b * 64, t0, bh);
       umma::tma_load_3d(sm + Lay::kK + b * kWtKeys * 128, &kmap, bar_tma, b * 64, t0 - 64, bh);
-    }
-    if (!stall_test(kStallWindowV)) {  // the stall test leaves the V tile out
-      umma::mbar_arrive_expect_tx(bar_v, kWtKeys * DH * 2);
-#pragma unroll
-      for (int b = 0; b < DH / 64; ++b)
-        umma::tma_load_3d(sm + Lay::kV + b * kWtKeys * 128, &vmap, bar_v, b * 64, t0 - 64, bh);
     }
   }
   __syncthreads();  // barrier initialisation visible to every thread
@@ -127,6 +128,15 @@ __global__ void __launch_bounds__(kWtThreads, 1)
     *abort_flag = 1;
   }
   umma::tc_fence_after();
+  // S is complete, so its operands are no longer read: V goes over Q and K
+  // (the stall test leaves the V tile out)
+  if (tid == 0 && !*abort_flag && !stall_test(kStallWindowV)) {
+    umma::mbar_arrive_expect_tx(bar_v, kWtKeys * DH * 2);
+#pragma unroll
+    for (int b = 0; b < DH / 64; ++b)
+      umma::tma_load_3d(sm + Lay::kV + b * kWtKeys * 128, &vmap, bar_v, b * 64, t0 - 64, bh);
+    v_issued = true;
+  }
 
   // ---- P = exp(S - m) over each row's band ---------------------------------------------
   // Row r = 32 w + lane (w = warp) reads the 96 staged columns [32 w, 32 w + 96);
@@ -256,7 +266,7 @@ done:
   // an aborted tile may still have its loads in flight: wait for them (bounded)
   if (tid == 0 && *abort_flag) {
     umma::mbar_wait(bar_tma, 0);
-    if (!stall_test(kStallWindowV)) umma::mbar_wait(bar_v, 0);
+    if (v_issued) umma::mbar_wait(bar_v, 0);
   }
   umma::tc_fence_before();
   __syncthreads();
