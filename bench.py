@@ -78,16 +78,20 @@ def replica_rate(units_per_rank: float, ms: float, world: int) -> float:
 # since the capture
 # ---------------------------------------------------------------------------
 
-_KERNEL_SOURCES = {"linattn_prefill": "linattn_tc.cuh", "window_attn": "window_tc.cuh",
+_KERNEL_SOURCES = {"linattn_prefill": "linattn_tc.cuh", "window_attn": "window_tcp.cuh",
                    "decode_step": "decode.cuh"}
 
 
-def measured_traffic(kernel):
+def measured_traffic(kernel, workload):
+    """DRAM bytes of one launch from the ncu capture of this kernel on this
+    workload, or None (no capture of it, or the code changed since)."""
     import hashlib
     csrc = os.path.join(ROOT, "linear_attention_lm_b200", "csrc")
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             entry = json.load(f)[kernel]
+        if entry["workload"] != workload:
+            return None
         h = hashlib.sha256()
         for name in (_KERNEL_SOURCES[kernel], "umma.cuh", "common.cuh"):
             with open(os.path.join(csrc, name), "rb") as f:
@@ -130,11 +134,11 @@ def decode_bytes(w):
     return lin + win
 
 
-def hbm_roofline(kernel, nbytes, ms, peaks, extra=None):
+def hbm_roofline(kernel, nbytes, ms, peaks, extra=None, workload=None):
     ach = nbytes / (ms / 1e3) / 1e9
     r = {"kernel": kernel, "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
          "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
-         "traffic": measured_traffic(kernel) if kernel in _KERNEL_SOURCES else None,
+         "traffic": measured_traffic(kernel, workload) if kernel in _KERNEL_SOURCES else None,
          "algorithmic_bytes": int(nbytes), "ms": round(ms, 5), "peak_source": peaks["source"]}
     if extra:
         r.update(extra)
@@ -346,7 +350,7 @@ def run_ours(args, rank, world, dev):
     kern = {"linattn_prefill": (linattn_bytes(w), t_lin), "window_attn": (window_bytes(w), t_win)}
     dom = max(kern, key=lambda k: kern[k][1])
     b, t_ms = kern[dom]
-    roofline = hbm_roofline(dom, b, t_ms, peaks)
+    roofline = hbm_roofline(dom, b, t_ms, peaks, workload=w.name)
     roofline["per_kernel_ms"] = {k: round(v[1], 5) for k, v in kern.items()}
     roofline["per_kernel_frac"] = {k: round(v[0] / (v[1] / 1e3) / 1e9 / peaks["hbm_gbs"], 4)
                                    for k, v in kern.items()}
@@ -357,9 +361,9 @@ def run_ours(args, rank, world, dev):
                            "ms_per_step": round(elapsed_max / args.steps, 5),
                            "kernels": {"linattn_prefill": hbm_roofline(
                                "linattn_prefill", linattn_bytes(w), t_lin, peaks,
-                               tensor_side(w, t_lin, peaks)),
+                               tensor_side(w, t_lin, peaks), workload=w.name),
                                "window_attn": hbm_roofline("window_attn", window_bytes(w),
-                                                           t_win, peaks)}}}
+                                                           t_win, peaks, workload=w.name)}}}
     for name in OTHER_PREFILL:
         workloads[name] = run_other_prefill(args, lab, WORKLOADS[name], dev, world, peaks, warm)
     decode = run_decode(args, lab, dev, world, peaks, warm)
@@ -404,8 +408,9 @@ def run_other_prefill(args, lab, w, dev, world, peaks, warm):
     del sets
     ms = max_over_ranks(total_ms / n, dev, world)
     lin = hbm_roofline("linattn_prefill", linattn_bytes(w), t_lin, peaks,
-                       tensor_side(w, t_lin, peaks) if w.dtype == "bf16" else None)
-    win = hbm_roofline("window_attn", window_bytes(w), t_win, peaks)
+                       tensor_side(w, t_lin, peaks) if w.dtype == "bf16" else None,
+                       workload=w.name)
+    win = hbm_roofline("window_attn", window_bytes(w), t_win, peaks, workload=w.name)
     out = {"workload": prefill_config(w, world)["workload"],
            "tokens_per_s": round(world * w.B * w.L / (ms / 1e3), 1),
            "ms_per_step": round(ms, 5), "steps": n, "launches_per_step": launches,
@@ -656,7 +661,7 @@ def run_decode(args, lab, dev, world, peaks, warm):
                         f"after a {w.L}-token prefill",
             "value": round(world * w.B / (ms / 1e3), 1), "unit": "tokens/s",
             "ms_per_step": round(ms, 5), "steps": n, "batch": w.B, "heads": w.H,
-            "roofline": hbm_roofline("decode_step", b, ms, peaks)}
+            "roofline": hbm_roofline("decode_step", b, ms, peaks, workload=w.name)}
 
 
 # ---------------------------------------------------------------------------
