@@ -161,18 +161,28 @@ TcPlan plan_linattn_tc(long long BH, int L, int d_v) {
   return pl;
 }
 
+// BH sequences of v_split * DV value columns; the kernel runs each DV-wide
+// column slice of a sequence as its own CTA (bh * v_split + slice)
+// bf16 inputs: every d_v runs on the d_v = 64 kernel, one CTA per 64-column slice
+TcPlan plan_linattn_bf16(long long BH, int L, int d_v) {
+  return plan_linattn_tc(BH * (d_v / 64), L, 64);
+}
+
 template <int DV>
 based_status_t launch_linattn_tc(const void* q, const void* k, const void* v, void* out, int BH,
                                  int L, float eps, float* state_kv, float* state_k,
-                                 void* workspace, size_t workspace_bytes, cudaStream_t st) {
-  const TcPlan pl = plan_linattn_tc(BH, L, DV);
+                                 void* workspace, size_t workspace_bytes, cudaStream_t st,
+                                 int v_split = 1) {
+  const long long BHv = (long long)BH * v_split;
+  if (BHv > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
+  const TcPlan pl = plan_linattn_tc(BHv, L, DV);
   if (pl.workspace > 0 && (workspace == nullptr || workspace_bytes < pl.workspace))
     return BASED_ERR_WORKSPACE;
   if (pl.workspace > 0 && (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0)
     return BASED_ERR_INVALID_ARG;
   CUtensorMap vmap, ymap;
-  if (!make_rows_map(&vmap, v, DV, L, BH, kTcChunk)) return BASED_ERR_CUDA;
-  if (!make_rows_map(&ymap, out, DV, L, BH, kTcChunk)) return BASED_ERR_CUDA;
+  if (!make_rows_map(&vmap, v, DV * v_split, L, BH, kTcChunk)) return BASED_ERR_CUDA;
+  if (!make_rows_map(&ymap, out, DV * v_split, L, BH, kTcChunk)) return BASED_ERR_CUDA;
   TcParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k = static_cast<const __nv_bfloat16*>(k);
@@ -184,18 +194,20 @@ based_status_t launch_linattn_tc(const void* q, const void* k, const void* v, vo
   p.seg_chunks = pl.seg_chunks;
   p.n_seg = pl.n_seg;
   p.eps = eps;
+  p.v_split = v_split;
+  p.ld_v = DV * v_split;
   const size_t smem = TcLayout<DV>::kSmem;
   if (pl.n_seg > 1) {
     auto kst = linattn_tc_kernel<DV, true>;
     if (!set_smem(kst, smem)) return BASED_ERR_CUDA;
-    const long long nblk = (long long)BH * (pl.n_seg - 1);
+    const long long nblk = BHv * (pl.n_seg - 1);
     if (nblk > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
     kst<<<(unsigned)nblk, kTcThreads, smem, st>>>(vmap, ymap, p);
     if (cudaGetLastError() != cudaSuccess) return BASED_ERR_CUDA;
   }
   auto kern = linattn_tc_kernel<DV, false>;
   if (!set_smem(kern, smem)) return BASED_ERR_CUDA;
-  const long long nblk = (long long)BH * pl.n_seg;
+  const long long nblk = BHv * pl.n_seg;
   if (nblk > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
   kern<<<(unsigned)nblk, kTcThreads, smem, st>>>(vmap, ymap, p);
   return launch_status();
@@ -469,7 +481,7 @@ size_t based_linattn_workspace_bytes(int B, int H, int L, int d_feat, int d_v,
       (d_v != 64 && d_v != 128))
     return (size_t)-1;
   if (dt == BASED_F32) return 0;
-  return plan_linattn_tc((long long)B * H, L, d_v).workspace;
+  return plan_linattn_bf16((long long)B * H, L, d_v).workspace;
 }
 
 based_status_t based_linattn_fwd(const void* q, const void* k, const void* v, void* out,
@@ -485,10 +497,8 @@ based_status_t based_linattn_fwd(const void* q, const void* k, const void* v, vo
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dt == BASED_F32)
     return launch_linattn_simt<float>(q, k, v, out, BH, L, d_v, eps, state_kv, state_k, st);
-  return d_v == 64 ? launch_linattn_tc<64>(q, k, v, out, BH, L, eps, state_kv, state_k,
-                                            workspace, workspace_bytes, st)
-                   : launch_linattn_tc<128>(q, k, v, out, BH, L, eps, state_kv, state_k,
-                                            workspace, workspace_bytes, st);
+  return launch_linattn_tc<64>(q, k, v, out, BH, L, eps, state_kv, state_k, workspace,
+                               workspace_bytes, st, d_v / 64);
 }
 
 based_status_t based_linattn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
@@ -504,14 +514,12 @@ based_status_t based_linattn_fwd_noalloc(const void* q, const void* k, const voi
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dt == BASED_F32)  // the fp32 path needs no scratch
     return launch_linattn_simt<float>(q, k, v, out, BH, L, d_v, eps, state_kv, state_k, st);
-  const size_t need = plan_linattn_tc(BH, L, d_v).workspace;
+  const size_t need = plan_linattn_bf16(BH, L, d_v).workspace;
   if (need > kNoAllocScratchBytes) return BASED_ERR_WORKSPACE;
   float* scratch = nullptr;
   if (need > 0 && (s = noalloc_scratch(&scratch)) != BASED_OK) return s;
-  return d_v == 64 ? launch_linattn_tc<64>(q, k, v, out, BH, L, eps, state_kv, state_k, scratch,
-                                           kNoAllocScratchBytes, st)
-                   : launch_linattn_tc<128>(q, k, v, out, BH, L, eps, state_kv, state_k, scratch,
-                                            kNoAllocScratchBytes, st);
+  return launch_linattn_tc<64>(q, k, v, out, BH, L, eps, state_kv, state_k, scratch,
+                               kNoAllocScratchBytes, st, d_v / 64);
 }
 
 based_status_t based_window_attn_fwd(const void* q, const void* k, const void* v, void* out,

@@ -152,6 +152,12 @@ struct TcParams {
   int seg_chunks;    // chunks per segment
   int n_seg;         // segments per sequence (1 = no split)
   float eps;
+  // A sequence with ld_v value columns runs as v_split = ld_v / DV independent
+  // CTAs (blocks bh * v_split + h), each on value columns [h DV, h DV + DV): the
+  // denominator does not depend on v, so every slice is exact on its own.  v, out
+  // and state_kv have ld_v columns; q, k and state_k are per sequence.
+  int v_split;
+  int ld_v;
 };
 
 // Power-of-two scale applied to the fp16 state copy (and to P) for the chunk
@@ -290,6 +296,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* bar_yfull = bars + 11;   // y staging tile written (group E)
   uint64_t* bar_m5 = bars + 12;      // #5 done (commit): the state can be read
   uint64_t* bar_sread = bars + 13;   // state read and its fp16 copy written (group E)
+  uint64_t* bar_done = bars + 19;    // [2] state-only pass, d_v = 64: #5 of the chunk that
+                                     // used phiK buffer b complete (commit)
   constexpr int kThreads = kTcThreads;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -297,8 +305,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int L = p.L;
   const int n_chunks = (L + kTcChunk - 1) / kTcChunk;
   const int segs_here = kStateOnly ? p.n_seg - 1 : p.n_seg;
-  const int bh = blockIdx.x / segs_here;
+  const int bh = blockIdx.x / segs_here;  // the CTA's (sequence, column slice)
   const int seg = blockIdx.x - bh * segs_here;
+  const int bh_seq = bh / p.v_split;        // the sequence
+  const int col0 = (bh - bh_seq * p.v_split) * DV;
   const int c_begin = seg * p.seg_chunks;
   const int c_end = min(c_begin + p.seg_chunks, n_chunks);
   const bool has_init = !kStateOnly && seg > 0;
@@ -317,6 +327,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     umma::mbar_init(bar_yfull, kTcGroup);
     umma::mbar_init(bar_m5, 1);
     umma::mbar_init(bar_sread, kTcGroup);
+    umma::mbar_init(bar_done, 1);
+    umma::mbar_init(bar_done + 1, 1);
     *abort_flag = 0;
     umma::fence_mbar_init();
     umma::tma_prefetch_desc(&vmap);
@@ -404,18 +416,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       } else if (seg == p.n_seg - 1) {
         if (p.state_kv) {
-          float4* skv = reinterpret_cast<float4*>(p.state_kv + (size_t)bh * kF * DV);
+          float* skv = p.state_kv + (size_t)bh_seq * kF * p.ld_v + col0;
 #pragma unroll 4
           for (int i = u; i < kF * (DV / 4); i += n) {
             const int r = i / (DV / 4), j = (i - r * (DV / 4)) * 4;
             const int code = rowmap[r];
             const float sc = (code & 1) ? 0.70710678118654752f : 1.0f;
             const float4 v4 = *reinterpret_cast<const float4*>(stage + (code >> 1) * kStr + j);
-            skv[i] = make_float4(v4.x * sc, v4.y * sc, v4.z * sc, v4.w * sc);
+            *reinterpret_cast<float4*>(skv + (size_t)r * p.ld_v + j) =
+                make_float4(v4.x * sc, v4.y * sc, v4.z * sc, v4.w * sc);
           }
         }
-        if (p.state_k) {
-          float* sk = p.state_k + (size_t)bh * kF;
+        if (p.state_k && col0 == 0) {
+          float* sk = p.state_k + (size_t)bh_seq * kF;
           for (int r = u; r < kF; r += n) {
             const int code = rowmap[r];
             sk[r] = stage[(code >> 1) * kStr + DV] * ((code & 1) ? 0.70710678118654752f : 1.0f);
@@ -435,10 +448,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         float sv[80];
         umma::tmem_ld80(tmem + Lay::kTmS0 + tm_lane + h * 80, sv);
         const int j = quad * 32 + lane;
-        float* skv = p.state_kv ? p.state_kv + (size_t)bh * kF * DV + j : nullptr;
-        float* sk = p.state_k ? p.state_k + (size_t)bh * kF : nullptr;
+        float* skv = p.state_kv ? p.state_kv + (size_t)bh_seq * kF * p.ld_v + col0 + j : nullptr;
+        float* sk = p.state_k && col0 == 0 ? p.state_k + (size_t)bh_seq * kF : nullptr;
         float* dst = j < DV ? skv : (j == DV ? sk : nullptr);
-        const int stride = j < DV ? DV : 1;
+        const int stride = j < DV ? p.ld_v : 1;
         if (dst != nullptr) {
 #pragma unroll
           for (int i = 0; i < 80; ++i) {
@@ -468,7 +481,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
     for (int blk = 0; blk < DV / 64; ++blk)
       umma::tma_load_3d(sm + Lay::kV + stage * Lay::kVStage + blk * 16384, &vmap,
-                        bar_tma + stage, blk * 64, c * kTcChunk, bh);
+                        bar_tma + stage, col0 + blk * 64, c * kTcChunk, bh_seq);
     return 1u;
   };
 
@@ -559,7 +572,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
         if (Lay::kTm) {
-          umma::mma_commit(bar_m5);
+          // the state-only pass releases this chunk's phiK buffer to group F
+          umma::mma_commit(kStateOnly ? bar_done + (it & 1) : bar_m5);
           BASED_TC_TRACE(4, it);
           // refill the stage of chunk c-1 (its MMAs are done by now) with chunk
           // c + kVBuf - 1
@@ -595,7 +609,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
           }
         }
-        umma::mma_commit(bar_m25);
+        if (!(kStateOnly && Lay::kTm)) umma::mma_commit(bar_m25);
         BASED_TC_TRACE(6, it);
         if (!kStateOnly) {
           if (Lay::kEarlyO) {
@@ -748,8 +762,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (warp < 8) {
     // ================= group F: feature maps and Q/K tiles of chunk c =================
     const int t = tid - kTcGroup;  // token row of the chunk; also the TMEM lane (quadrant = warp & 3)
-    const __nv_bfloat16* q = p.q + (size_t)bh * L * kD;
-    const __nv_bfloat16* k = p.k + (size_t)bh * L * kD;
+    const __nv_bfloat16* q = p.q + (size_t)bh_seq * L * kD;
+    const __nv_bfloat16* k = p.k + (size_t)bh_seq * L * kD;
     // q/k rows of this thread's token, loaded three chunks ahead of their use
     // (the loads of cold inputs take a few microseconds under load)
     uint4 qr[2], kr[2], qn[2], kn[2], qm[2], km[2];
@@ -768,15 +782,42 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         qd[0] = qd[1] = kd[0] = kd[1] = make_uint4(0, 0, 0, 0);
       }
     };
-    load_qk(c_begin, qr, kr);
-    load_qk(c_begin + 1, qn, kn);
-    load_qk(c_begin + 2, qm, km);
+    // The state-only pass runs a chunk in about 1,000 cycles, less than a load
+    // under load takes: its k rows stream through a ring in the (otherwise
+    // unused) state-copy buffer by cp.async, kAhead chunks ahead, so no register
+    // waits for them early.
+    constexpr int kRing = 8, kAhead = 6;
+    static_assert(kRing * kTcChunk * 32 <= Lay::kSBuf * Lay::kSBytes, "k-row ring");
+    uint8_t* ring = sm + Lay::kS;
+    auto ring_fetch = [&](int c) {  // one commit group per call, empty rows zero-filled
+      const long long tt = (long long)c * kTcChunk + t;
+      const bool in = c < c_end && tt < L;
+      uint8_t* dst = ring + ((c - c_begin) % kRing) * (kTcChunk * 32) + t * 32;
+      const __nv_bfloat16* src = k + (in ? tt : 0) * kD;
+      umma::cp_async16(dst, src, in);
+      umma::cp_async16(dst + 16, src + 8, in);
+      umma::cp_async_commit();
+    };
+    if constexpr (kStateOnly) {
+      for (int j = 0; j < kAhead; ++j) ring_fetch(c_begin + j);
+    } else {
+      load_qk(c_begin, qr, kr);
+      load_qk(c_begin + 1, qn, kn);
+      load_qk(c_begin + 2, qm, km);
+    }
     BASED_TC_TRACE(5, 0);
     for (int c = c_begin; c < c_end && !*abort_flag; ++c) {
       const int it = c - c_begin;
       const int t0 = c * kTcChunk;
       const int n = min(kTcChunk, L - t0);
       const bool live = t < n;
+      if constexpr (kStateOnly) {  // this chunk's k row (this thread's own copy)
+        umma::cp_async_wait<kAhead - 1>();
+        const uint4* src = reinterpret_cast<const uint4*>(ring + (it % kRing) * (kTcChunk * 32) + t * 32);
+        kr[0] = src[0];
+        kr[1] = src[1];
+        ring_fetch(c + kAhead);
+      }
       const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(qr);
       const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(kr);
       uint8_t* phik = sm + Lay::kPhiK + (it % Lay::kPhiKBuf) * 40960;
@@ -785,6 +826,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // buffer was released by the wait of the previous iteration.
       BASED_TC_TRACE(0, it);
       if (!Lay::kTm && it > 0 && !umma::mbar_wait(bar_m25, (it - 1) & 1)) { fail(); break; }
+
       // the Q/K tiles are rewritten once #1 of the previous chunk has read them
       if (!kStateOnly && it > 0 && !umma::mbar_wait(bar_u, (it - 1) & 1)) { fail(); break; }
       BASED_TC_TRACE(1, it);
@@ -813,10 +855,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       umma::fence_async_smem();
       BASED_TC_TRACE(2, it);
       // An arrival for chunk c must follow the completion of the phase of chunk
-      // c-1 (arrivals carry no phase, and the four warps run at their own pace).
-      // The main pass has that through its wait for #1 of chunk c-1; the
-      // state-only pass waits for the MMAs of chunk c-1 before arriving.
-      if (kStateOnly && Lay::kTm && it > 0 && !umma::mbar_wait(bar_m25, (it - 1) & 1)) {
+      // c-1 (arrivals carry no phase, and the four warps run at their own pace),
+      // and the issue thread must have seen that phase (else bar_qk could
+      // complete two phases before it looks).  The main pass has both through its
+      // wait for #1 of chunk c-1.  The state-only pass (d_v = 64) waits for #5 of
+      // chunk c-1 (bar_done of its buffer), which also frees that buffer for
+      // chunk c+1; bar_done cannot run ahead of this wait (its next phase needs
+      // chunk c+1's #5, after this arrival).
+      if (kStateOnly && Lay::kTm && it > 0 &&
+          !umma::mbar_wait(bar_done + ((it - 1) & 1), ((it - 1) >> 1) & 1)) {
         fail();
         break;
       }
@@ -855,9 +902,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tc_feature_chunk(XQ, YQ, q2, ch);
         }
       }
-      qr[0] = qn[0]; qr[1] = qn[1]; kr[0] = kn[0]; kr[1] = kn[1];
-      qn[0] = qm[0]; qn[1] = qm[1]; kn[0] = km[0]; kn[1] = km[1];
-      load_qk(c + 3, qm, km);
+      if constexpr (!kStateOnly) {
+        qr[0] = qn[0]; qr[1] = qn[1]; kr[0] = kn[0]; kr[1] = kn[1];
+        qn[0] = qm[0]; qn[1] = qm[1]; kn[0] = km[0]; kn[1] = km[1];
+        load_qk(c + 3, qm, km);
+      }
       if (!kStateOnly) {
         umma::fence_async_smem();
         umma::tc_fence_before();
@@ -865,6 +914,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         umma::mbar_arrive(bar_phiq);
       }
     }
+    // the ring's copies still in flight (rows past the segment) land before exit
+    if constexpr (kStateOnly) umma::cp_async_wait<0>();
     if constexpr (Lay::kSt && !kStateOnly) {
       // second half of the export (group P waits for the last #5 and decides)
       if (c_begin < c_end && umma::named_sync_all(2, 2 * kTcGroup, true)) {
@@ -875,7 +926,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (!kStateOnly) {
     // ================= group E: epilogue of chunk c (output, fp16 state copy) =================
     const int t = tid - 2 * kTcGroup;  // TMEM lane of this thread (quadrant = warp - 8)
-    __nv_bfloat16* out = p.out + (size_t)bh * L * DV;
+    __nv_bfloat16* out = p.out + (size_t)bh_seq * L * DV;  // (v_split = 1 here)
     // fp16 copy (scaled by sn) of the state rows this thread holds, as #2's B operand:
     // tile 0 row t = feature t; tile 1 (M=64) lanes 0..15 of quadrants 0, 1 = features
     // 128 + 16 * quad + lane
@@ -1067,7 +1118,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         umma::mbar_arrive(bar_yfull);
         if (t == 0) {
           if (!umma::mbar_wait(bar_yfull, it & 1)) { fail(); break; }
-          umma::tma_store_3d(&ymap, sm + Lay::kY, 0, t0, bh);
+          umma::tma_store_3d(&ymap, sm + Lay::kY, col0, t0, bh_seq);
           umma::bulk_commit();
         }
       }
@@ -1113,8 +1164,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int i = 0; i < 32; ++i)
             if (g * 32 + i < NA) row[i] = s[i];
         } else if (seg == p.n_seg - 1) {
-          float* skv = p.state_kv ? p.state_kv + (size_t)bh * kF * DV : nullptr;
-          float* sk = p.state_k ? p.state_k + (size_t)bh * kF : nullptr;
+          float* skv = p.state_kv ? p.state_kv + (size_t)bh_seq * kF * DV : nullptr;
+          float* sk = p.state_k ? p.state_k + (size_t)bh_seq * kF : nullptr;
           for (int r = 0; r < nrows; ++r) {
             const int row = r == 0 ? r0 : r1;
             if (skv) {

@@ -68,7 +68,8 @@ def test_noalloc_matches_workspace_entry_point():
 def test_noalloc_scratch_covers_every_split():
     """The scratch array (16 MiB) covers the largest workspace any problem
     asks for on this GPU: the split keeps (segments - 1) x sequences at most
-    one per SM, so the need peaks near SMs x 160 x (d_v + 16) x 4 bytes.
+    one per SM, so the need peaks near SMs x 160 x 80 x 4 bytes (every d_v runs
+    as 64-column slices).
     Sizes beyond the array would be refused with BASED_ERR_WORKSPACE before
     any launch; none is reachable here."""
     lab_build.build()
