@@ -32,6 +32,9 @@ __global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
     T* __restrict__ out, float* __restrict__ state_kv, float* __restrict__ state_k, int L,
     int DV, float eps) {
   constexpr int C = kSimtChunk, NC = kSimtCols, NT = kSimtThreads;
+  constexpr int G = NT / NC;   // row groups
+  constexpr int RPT = C / G;   // rows per thread in the numerator
+  static_assert(NT % NC == 0 && C % G == 0, "thread layout");
   extern __shared__ __align__(16) float smem[];
   float* S = smem;                 // [273][64]
   float* z = S + kF * NC;          // [273] (+pad)
@@ -53,7 +56,7 @@ __global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
   for (int i = tid; i < kF * NC; i += NT) S[i] = 0.0f;
   for (int i = tid; i < 276; i += NT) z[i] = 0.0f;
 
-  const int j = tid % NC, grp = tid / NC;  // output column, row group (0..3)
+  const int j = tid % NC, grp = tid / NC;  // output column, row group (0..G-1)
   for (int t0 = 0; t0 < L; t0 += C) {
     const int n = min(C, L - t0);
     __syncthreads();  // previous chunk's state update is complete
@@ -73,14 +76,21 @@ __global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
       fk[i] = phi_feature(xk + r * kD, f);
     }
     __syncthreads();
-    // intra-chunk scores, causal mask s <= t
+    // intra-chunk scores, causal mask s <= t (four partial sums: the loop is
+    // latency-bound on one chain)
     for (int i = tid; i < C * C; i += NT) {
       const int t = i / C, s = i - t * C;
       float a = 0.0f;
       if (s <= t) {
         const float* a_row = fq + t * kF;
         const float* b_row = fk + s * kF;
-        for (int f = 0; f < kF; ++f) a = fmaf(a_row[f], b_row[f], a);
+        float a4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 4
+        for (int f = 0; f < kF - 1; f += 4) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) a4[e] = fmaf(a_row[f + e], b_row[f + e], a4[e]);
+        }
+        a = fmaf(a_row[kF - 1], b_row[kF - 1], (a4[0] + a4[1]) + (a4[2] + a4[3]));
       }
       A[t * 33 + s] = a;
     }
@@ -93,36 +103,39 @@ __global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
       for (int s = 0; s < C; ++s) d += A[tid * 33 + s];
       den[tid] = d;
     }
-    // numerators for rows grp, grp+4, ..., column j
-    float acc[C / 4];
+    // numerators for rows grp, grp+G, ..., column j
+    float acc[RPT];
 #pragma unroll
-    for (int i = 0; i < C / 4; ++i) acc[i] = 0.0f;
+    for (int i = 0; i < RPT; ++i) acc[i] = 0.0f;
     for (int f = 0; f < kF; ++f) {
       const float sf = S[f * NC + j];
 #pragma unroll
-      for (int i = 0; i < C / 4; ++i) acc[i] = fmaf(fq[(grp + 4 * i) * kF + f], sf, acc[i]);
+      for (int i = 0; i < RPT; ++i) acc[i] = fmaf(fq[(grp + G * i) * kF + f], sf, acc[i]);
     }
     for (int s = 0; s < C; ++s) {
       const float vj = vs[s * NC + j];
 #pragma unroll
-      for (int i = 0; i < C / 4; ++i) acc[i] = fmaf(A[(grp + 4 * i) * 33 + s], vj, acc[i]);
+      for (int i = 0; i < RPT; ++i) acc[i] = fmaf(A[(grp + G * i) * 33 + s], vj, acc[i]);
     }
     __syncthreads();  // den ready; all reads of S and z for this chunk done
 #pragma unroll
-    for (int i = 0; i < C / 4; ++i) {
-      const int t = grp + 4 * i;
+    for (int i = 0; i < RPT; ++i) {
+      const int t = grp + G * i;
       if (t < n) out[(size_t)(t0 + t) * DV + j] = from_f32<T>(acc[i] / (den[t] + eps));
     }
-    // state update
-    for (int f = grp; f < kF; f += 4) {
-      float s_acc = S[f * NC + j];
-      for (int s = 0; s < n; ++s) s_acc = fmaf(fk[s * kF + f], vs[s * NC + j], s_acc);
-      S[f * NC + j] = s_acc;
+    // state update over the chunk's 32 rows (rows past the end have v = 0;
+    // z skips them), four partial sums per entry
+    for (int f = grp; f < kF; f += G) {
+      float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int s = 0; s < C; ++s) s4[s & 3] = fmaf(fk[s * kF + f], vs[s * NC + j], s4[s & 3]);
+      S[f * NC + j] += (s4[0] + s4[1]) + (s4[2] + s4[3]);
     }
     for (int f = tid; f < kF; f += NT) {
-      float z_acc = z[f];
-      for (int s = 0; s < n; ++s) z_acc += fk[s * kF + f];
-      z[f] = z_acc;
+      float z4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int s = 0; s < C; ++s) z4[s & 3] += s < n ? fk[s * kF + f] : 0.0f;
+      z[f] += (z4[0] + z4[1]) + (z4[2] + z4[3]);
     }
   }
   __syncthreads();

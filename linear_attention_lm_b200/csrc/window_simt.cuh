@@ -64,15 +64,16 @@ __global__ void __launch_bounds__(kWinQ) window_simt_kernel(const T* __restrict_
     float a = -INFINITY;
     if (s >= lo) {
       const float4* k4 = reinterpret_cast<const float4*>(ks + (tid + j) * ld);
-      float acc = 0.0f;
+      // four independent chains: the loop is latency-bound on one
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int c = 0; c < dh / 4; ++c) {
         const float4 x = q4[c], y = k4[c];
-        acc = fmaf(x.x, y.x, acc);
-        acc = fmaf(x.y, y.y, acc);
-        acc = fmaf(x.z, y.z, acc);
-        acc = fmaf(x.w, y.w, acc);
+        acc.x = fmaf(x.x, y.x, acc.x);
+        acc.y = fmaf(x.y, y.y, acc.y);
+        acc.z = fmaf(x.z, y.z, acc.z);
+        acc.w = fmaf(x.w, y.w, acc.w);
       }
-      a = acc * scale;
+      a = ((acc.x + acc.y) + (acc.z + acc.w)) * scale;
     }
     sc[j] = a;
     m = fmaxf(m, a);
