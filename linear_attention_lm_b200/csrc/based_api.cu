@@ -363,6 +363,7 @@ based_status_t launch_linattn_bwd_tc(const void* q, const void* k, const void* v
   p.ws_dd = reinterpret_cast<float*>(static_cast<char*>(ws) + (size_t)BH * L * DV * 2);
   p.L = L;
   p.n_tiles = (L + kBtT - 1) / kBtT;
+  p.BH = BH;
   p.eps = eps;
   CUtensorMap vmap, dnmap;
   if (!make_rows_map(&vmap, v, DV, L, BH, kBtT) || !make_rows_map(&dnmap, p.ws_dn, DV, L, BH, kBtT))

@@ -80,6 +80,7 @@ struct BtParams {
   float* ws_dd;          // [BH, L]
   int L;
   int n_tiles;
+  int BH;
   float eps;
 };
 
@@ -132,8 +133,10 @@ __global__ void __launch_bounds__(kBtThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool issuer = warp == 4;
-  const int i = blockIdx.x % p.n_tiles;
-  const long long bh = blockIdx.x / p.n_tiles;
+  // the CTAs with the most key tiles (the last query tiles) are launched first,
+  // so the short ones fill the end of the grid
+  const int i = p.n_tiles - 1 - (int)(blockIdx.x / p.BH);
+  const long long bh = blockIdx.x % p.BH;
   const int L = p.L;
   const int t0 = i * kBtT;
   const int n_steps = 2 * (i + 1);
@@ -387,8 +390,9 @@ __global__ void __launch_bounds__(kBtThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool issuer = warp == 4;
-  const int j = blockIdx.x % p.n_tiles;
-  const long long bh = blockIdx.x / p.n_tiles;
+  // the CTAs with the most query tiles (the first key tiles) are launched first
+  const int j = (int)(blockIdx.x / p.BH);
+  const long long bh = blockIdx.x % p.BH;
   const int L = p.L;
   const int s0 = j * kBtT;
   const int n_steps = p.n_tiles - j;  // query tiles j .. n_tiles - 1
