@@ -59,6 +59,25 @@ inline bool set_smem(K kernel, size_t bytes) {
                               (int)bytes) == cudaSuccess;
 }
 
+// Launch as a programmatic dependent of the previous kernel in the stream: the
+// kernel's CTAs may start (and run their set-up) while that kernel finishes;
+// the kernel waits for it (griddepcontrol.wait) before touching global memory.
+template <typename... KArgs, typename... Args>
+bool launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) == cudaSuccess;
+}
+
 // Shared argument checks of the prefill entry points.  Null tensor pointers
 // are accepted only when the tensors are empty.
 inline based_status_t check_tensor(const void* p, bool empty) {
@@ -202,14 +221,15 @@ based_status_t launch_linattn_tc(const void* q, const void* k, const void* v, vo
     if (!set_smem(kst, smem)) return BASED_ERR_CUDA;
     const long long nblk = BHv * (pl.n_seg - 1);
     if (nblk > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
-    kst<<<(unsigned)nblk, kTcThreads, smem, st>>>(vmap, ymap, p);
-    if (cudaGetLastError() != cudaSuccess) return BASED_ERR_CUDA;
+    if (!launch_dependent(kst, dim3((unsigned)nblk), dim3(kTcThreads), smem, st, vmap, ymap, p))
+      return BASED_ERR_CUDA;
   }
   auto kern = linattn_tc_kernel<DV, false>;
   if (!set_smem(kern, smem)) return BASED_ERR_CUDA;
   const long long nblk = BHv * pl.n_seg;
   if (nblk > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
-  kern<<<(unsigned)nblk, kTcThreads, smem, st>>>(vmap, ymap, p);
+  if (!launch_dependent(kern, dim3((unsigned)nblk), dim3(kTcThreads), smem, st, vmap, ymap, p))
+    return BASED_ERR_CUDA;
   return launch_status();
 }
 
@@ -226,7 +246,9 @@ based_status_t launch_window_tc(const void* q, const void* k, const void* v, voi
   const int n_tiles = (L + kWtQ - 1) / kWtQ;
   const long long nblk = (long long)n_tiles * BH;
   if (nblk > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
-  kern<<<(unsigned)nblk, kWtThreads, smem, st>>>(qm, km, vm, ym, L, W, n_tiles);
+  if (!launch_dependent(kern, dim3((unsigned)nblk), dim3(kWtThreads), smem, st, qm, km, vm, ym, L,
+                        W, n_tiles))
+    return BASED_ERR_CUDA;
   return launch_status();
 }
 
@@ -243,8 +265,9 @@ based_status_t launch_window_tcp(const void* q, const void* k, const void* v, vo
   if (n_total > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
   const long long sms = device_sm_count();
   const unsigned grid = (unsigned)(n_total < sms ? n_total : sms);
-  window_tcp_kernel<<<grid, kWpThreads, WpLayout::kSmem, st>>>(qm, km, vm, ym, L, W,
-                                                               tiles_per_seq, (int)n_total);
+  if (!launch_dependent(window_tcp_kernel, dim3(grid), dim3(kWpThreads), WpLayout::kSmem, st, qm,
+                        km, vm, ym, L, W, tiles_per_seq, (int)n_total))
+    return BASED_ERR_CUDA;
   return launch_status();
 }
 
@@ -281,7 +304,8 @@ based_status_t launch_decode(DecodeParams p, cudaStream_t st) {
   if (!set_smem(kern, smem)) return BASED_ERR_CUDA;
   const long long nblk = (long long)p.n_lin + p.n_wblk;
   p.wstride = p.n_wblk > 0 ? (int)(nblk / p.n_wblk) : 1;
-  kern<<<(unsigned)nblk, kThreads, smem, st>>>(p);
+  if (!launch_dependent(kern, dim3((unsigned)nblk), dim3(kThreads), smem, st, p))
+    return BASED_ERR_CUDA;
   return launch_status();
 }
 

@@ -302,6 +302,10 @@ __device__ __forceinline__ void decode_window_block(const DecodeParams& p, int w
 template <typename T, int DV>
 __global__ void __launch_bounds__(4 * DV, 1) decode_step_kernel(const DecodeParams p) {
   extern __shared__ __align__(16) uint8_t dec_smem[];
+  // a dependent launch: the previous step's kernel has finished (and its state
+  // and ring writes are visible) before this one reads them
+  umma::grid_dep_wait();
+  umma::grid_dep_launch();
   // window CTAs are interleaved evenly: with stride = n / n_wblk, CTA b is a
   // window CTA iff b mod stride = stride - 1 and b / stride < n_wblk
   const int b = blockIdx.x, q = b / p.wstride, r = b - q * p.wstride;

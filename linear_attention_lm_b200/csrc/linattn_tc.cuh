@@ -361,6 +361,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   umma::tc_fence_before();
   __syncthreads();
   umma::tc_fence_after();
+  // the set-up above touched no global memory: it overlaps the previous kernel
+  umma::grid_dep_wait();
+  umma::grid_dep_launch();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tm_lane = static_cast<uint32_t>(quad * 32) << 16;
   BASED_TC_TRACE(15, 0);

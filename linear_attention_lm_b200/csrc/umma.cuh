@@ -82,6 +82,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return mbar_wait_spin(bar, parity);
 }
 
+// ---------------------------------------------------------------- dependent launches
+// A kernel launched as a programmatic dependent of the previous kernel in its
+// stream may start while that kernel still runs; grid_dep_wait blocks until it
+// has completed and its memory is visible (a no-op for an ordinary launch), so
+// it goes before a kernel's first global-memory access.  grid_dep_launch lets
+// the next such launch start its CTAs as SMs free up.
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -66,6 +66,9 @@ __global__ void __launch_bounds__(kWtThreads, 1)
   uint64_t* bar_v = bar_tma + 5;                                      // V landed
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // a dependent launch: the previous kernel has finished before any load
+  umma::grid_dep_wait();
+  umma::grid_dep_launch();
   const int tile = blockIdx.x % n_tiles;
   const int bh = blockIdx.x / n_tiles;
   const int t0 = tile * kWtQ;

@@ -106,6 +106,9 @@ __global__ void __launch_bounds__(kWpThreads, 1)
   umma::tc_fence_before();
   __syncthreads();
   umma::tc_fence_after();
+  // the set-up above touched no global memory: it overlaps the previous kernel
+  umma::grid_dep_wait();
+  umma::grid_dep_launch();
   const uint32_t tmem = *tmem_slot;
   int issued = 0;  // loads issued (TMA thread)
 
