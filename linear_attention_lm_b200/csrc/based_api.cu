@@ -327,22 +327,25 @@ based_status_t launch_proj(const void* x, const void* w, ProjParams p, cudaStrea
   p.total_tiles = (int)tiles;
   // CTA pairs: clusters of two, as many as fit at once (one CTA per SM)
   cudaLaunchConfig_t cfg{};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // a dependent launch
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(kPjThreads, 1, 1);
   cfg.dynamicSmemBytes = PjLayout<Mode>::kSmem;
   cfg.stream = st;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 1;  // the occupancy query below takes the cluster shape only
   cfg.gridDim = dim3(2 * (unsigned)((device_sm_count() + 1) / 2), 1, 1);
   int max_clusters = 0;
   if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg) != cudaSuccess || max_clusters <= 0)
     return BASED_ERR_CUDA;
   const long long pairs = tiles < max_clusters ? tiles : max_clusters;
   cfg.gridDim = dim3(2 * (unsigned)pairs, 1, 1);
+  cfg.numAttrs = 2;
   if (cudaLaunchKernelEx(&cfg, kern, xm, wm, hm, p) != cudaSuccess) return BASED_ERR_CUDA;
   return launch_status();
 }
@@ -398,10 +401,14 @@ based_status_t launch_linattn_bwd_tc(const void* q, const void* k, const void* v
     return BASED_ERR_CUDA;
   const long long nblk = (long long)BH * p.n_tiles;
   if (nblk > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
-  kq<<<(unsigned)nblk, kBtThreads, BtLayout<DV>::kSmemQ, st>>>(vmap, p);
+  if (!launch_dependent(kq, dim3((unsigned)nblk), dim3(kBtThreads), BtLayout<DV>::kSmemQ, st, vmap,
+                        p))
+    return BASED_ERR_CUDA;
   const based_status_t s1 = launch_status();
   if (s1 != BASED_OK) return s1;
-  kkv<<<(unsigned)nblk, kBtThreads, BtLayout<DV>::kSmemK, st>>>(vmap, dnmap, p);
+  if (!launch_dependent(kkv, dim3((unsigned)nblk), dim3(kBtThreads), BtLayout<DV>::kSmemK, st,
+                        vmap, dnmap, p))
+    return BASED_ERR_CUDA;
   return launch_status();
 }
 
@@ -446,10 +453,14 @@ based_status_t launch_window_bwd_tc(const void* q, const void* k, const void* v,
   p.n_tiles = (L + kWgT - 1) / kWgT;
   const long long nblk = (long long)BH * p.n_tiles;
   if (nblk > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
-  kq<<<(unsigned)nblk, kWgThreads, smem, st>>>(q128, dy128, k192, v192, p);
+  if (!launch_dependent(kq, dim3((unsigned)nblk), dim3(kWgThreads), smem, st, q128, dy128, k192,
+                        v192, p))
+    return BASED_ERR_CUDA;
   const based_status_t s1 = launch_status();
   if (s1 != BASED_OK) return s1;
-  kkv<<<(unsigned)nblk, kWgThreads, smem, st>>>(k128, v128, q192, dy192, p);
+  if (!launch_dependent(kkv, dim3((unsigned)nblk), dim3(kWgThreads), smem, st, k128, v128, q192,
+                        dy192, p))
+    return BASED_ERR_CUDA;
   return launch_status();
 }
 

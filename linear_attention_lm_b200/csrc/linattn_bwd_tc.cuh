@@ -133,6 +133,9 @@ __global__ void __launch_bounds__(kBtThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool issuer = warp == 4;
+  // a dependent launch: the previous kernel has finished before any global access
+  umma::grid_dep_wait();
+  umma::grid_dep_launch();
   // the CTAs with the most key tiles (the last query tiles) are launched first,
   // so the short ones fill the end of the grid
   const int i = p.n_tiles - 1 - (int)(blockIdx.x / p.BH);
@@ -390,6 +393,9 @@ __global__ void __launch_bounds__(kBtThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool issuer = warp == 4;
+  // a dependent launch: the previous kernel has finished before any global access
+  umma::grid_dep_wait();
+  umma::grid_dep_launch();
   // the CTAs with the most query tiles (the first key tiles) are launched first
   const int j = (int)(blockIdx.x / p.BH);
   const long long bh = blockIdx.x % p.BH;

@@ -143,6 +143,9 @@ __global__ void __launch_bounds__(kPjThreads, 1)
   // load, MMA or arrival reaches the other CTA
   umma::cluster_sync();
   umma::tc_fence_after();
+  // a dependent launch: the set-up above overlaps the previous kernel
+  umma::grid_dep_wait();
+  umma::grid_dep_launch();
   const uint32_t tmem = *tmem_slot;
   auto fail = [&]() {
     record_device_error(BASED_ERR_TIMEOUT);

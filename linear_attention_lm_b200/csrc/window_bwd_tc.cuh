@@ -144,6 +144,9 @@ __global__ void __launch_bounds__(kWgThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ld + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // a dependent launch: the previous kernel has finished before any global access
+  umma::grid_dep_wait();
+  umma::grid_dep_launch();
   const int tile = blockIdx.x % p.n_tiles;
   const int bh = blockIdx.x / p.n_tiles;
   const int t0 = tile * kWgT;
@@ -297,6 +300,9 @@ __global__ void __launch_bounds__(kWgThreads, 1)
   float* st_d = st_l + kWgN;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // a dependent launch: the previous kernel has finished before any global access
+  umma::grid_dep_wait();
+  umma::grid_dep_launch();
   const int tile = blockIdx.x % p.n_tiles;
   const int bh = blockIdx.x / p.n_tiles;
   const int s0 = tile * kWgT;
