@@ -322,7 +322,10 @@ def time_prefill(lab, w, sets, steps, warmup, warm, dev, world):
         torch.distributed.barrier()
     t_lin = sum(e[0].elapsed_time(e[1]) for e in evs) / steps
     t_win = sum(e[1].elapsed_time(e[2]) for e in evs) / steps
-    launches = 2 + (1 if ws_bytes else 0)  # the split path adds a state-only pass
+    # the split path adds a state-only pass, and with more than two segments a
+    # running sum over their partials (160 x 80 fp32 per 64-column slice)
+    n_part = ws_bytes // (w.B * w.H * (w.dv // 64) * 160 * 80 * 4) if ws_bytes else 0
+    launches = 2 + (1 if n_part >= 1 else 0) + (1 if n_part >= 2 else 0)
     return start.elapsed_time(stop), t_lin, t_win, launches
 
 

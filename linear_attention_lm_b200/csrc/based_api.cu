@@ -223,6 +223,14 @@ based_status_t launch_linattn_tc(const void* q, const void* k, const void* v, vo
     if (nblk > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
     if (!launch_dependent(kst, dim3((unsigned)nblk), dim3(kTcThreads), smem, st, vmap, ymap, p))
       return BASED_ERR_CUDA;
+    // running sums over the segments, so each main-pass CTA reads one partial
+    if (pl.n_seg > 2) {
+      const int elems = kSymFP * TcLayout<DV>::NA;
+      const long long threads = BHv * (elems / 4);
+      if (!launch_dependent(linattn_partial_prefix_kernel, dim3((unsigned)((threads + 255) / 256)),
+                            dim3(256), 0, st, p.partial, (int)BHv, pl.n_seg - 1, elems))
+        return BASED_ERR_CUDA;
+    }
   }
   auto kern = linattn_tc_kernel<DV, false>;
   if (!set_smem(kern, smem)) return BASED_ERR_CUDA;

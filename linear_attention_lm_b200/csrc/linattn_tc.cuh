@@ -998,21 +998,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     };
     if (has_init) {
-      // seed the TMEM state of a later segment with the sum of the earlier partials
+      // seed the TMEM state of a later segment with the sum of the earlier
+      // partials: after linattn_partial_prefix_kernel, partial seg-1 holds it
       const float* part = p.partial + (size_t)bh * (p.n_seg - 1) * kSymFP * NA;
       if (Lay::kSt && quad < 3) {
         // partials are [feature][value column]; this lane seeds row t of [S|z]^T
+        const float* col0 = part + (size_t)(seg - 1) * kSymFP * NA + t;
+#pragma unroll 1
         for (int g = 0; g < kSymFP / 32; ++g) {
           float acc[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
-          if (t <= DV) {
-            for (int sp = 0; sp < seg; ++sp) {
-              const float* col = part + ((size_t)sp * kSymFP + g * 32) * NA + t;
-#pragma unroll
-              for (int i = 0; i < 32; ++i) acc[i] += col[(size_t)i * NA];
-            }
-          }
+          for (int i = 0; i < 32; ++i) acc[i] = t <= DV ? col0[(size_t)(g * 32 + i) * NA] : 0.0f;
           umma::tmem_st32(tmem + Lay::kTmS0 + tm_lane + g * 32, acc);
         }
       }
@@ -1026,12 +1022,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
           if (tile == 0 || lane < 16) {
-            for (int sp = 0; sp < seg; ++sp) {
-              const float* row = part + ((size_t)sp * kSymFP + f) * NA + g * 32;
+            const float* row = part + ((size_t)(seg - 1) * kSymFP + f) * NA + g * 32;
 #pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (g * 32 + i < NA) acc[i] += row[i];
-            }
+            for (int i = 0; i < 32; ++i)
+              if (g * 32 + i < NA) acc[i] += row[i];
           }
           umma::tmem_st32(base + g * 32, acc);
         }
@@ -1191,6 +1185,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   BASED_TC_TRACE(14, 0);
   if (warp == 0) umma::tmem_dealloc(tmem, kTcTmemCols);
+}
+
+// In-place running sum over the segment partials of each sequence (between
+// the state-only pass and the main pass): partial g becomes the sum of
+// partials 0..g, the state a segment g+1 starts from.  partial is
+// [n_seq][n_part][elems] fp32, elems a multiple of 4; one thread per float4
+// column of one sequence.
+__global__ void __launch_bounds__(256) linattn_partial_prefix_kernel(float* partial, int n_seq,
+                                                                     int n_part, int elems) {
+  umma::grid_dep_wait();
+  umma::grid_dep_launch();
+  const long long cols = (long long)elems / 4;
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)n_seq * cols) return;
+  const long long sq = i / cols, c = i - sq * cols;
+  float4* p4 = reinterpret_cast<float4*>(partial) + sq * n_part * cols + c;
+  float4 acc = p4[0];
+  for (int g = 1; g < n_part; ++g) {
+    const float4 v = p4[(long long)g * cols];
+    acc = make_float4(acc.x + v.x, acc.y + v.y, acc.z + v.z, acc.w + v.w);
+    p4[(long long)g * cols] = acc;
+  }
 }
 
 }  // namespace based
