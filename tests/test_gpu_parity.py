@@ -107,9 +107,19 @@ def test_linattn_head_dims(dv, dtype):
 @pytest.mark.parametrize("L", [3000, 1025])
 def test_linattn_split_segments(L):
     """Few sequences, long L: the prefill splits each sequence into segments
-    (state-only pass + seeded main pass); ragged last chunk, state export."""
+    (state-only pass, running sums of the partials, seeded main pass); ragged
+    last chunk, state export."""
     w = WORKLOADS["long_16k"].with_(B=1, H=2, L=L, name=f"split{L}")
     assert lab.based_linattn_workspace_bytes(1, 2, L, 16, 64, lab.BASED_BF16) > 0
+    run_linattn(w)
+
+
+@pytest.mark.parametrize("H,L,dv", [(64, 1024, 64), (20, 1500, 64), (5, 900, 128)])
+def test_linattn_split_segment_counts(H, L, dv):
+    """Two segments (one partial: no running sum), several segments, and d_v =
+    128 split into 64-column slices that are split into segments themselves."""
+    w = WORKLOADS["long_16k"].with_(B=1, H=H, L=L, dv=dv, name=f"seg{H}_{L}_{dv}")
+    assert lab.based_linattn_workspace_bytes(1, H, L, 16, dv, lab.BASED_BF16) > 0
     run_linattn(w)
 
 
