@@ -64,6 +64,11 @@ struct BtLayout {
   static constexpr size_t kSmemK = kBarK + 128 + 1024;
   // TMEM columns (both kernels): U / W, G / E, the d_v accumulator, the 16-wide one
   static constexpr int kTmU = 0, kTmG = 128, kTmAcc = 256, kTmAcc16 = 384;
+  // kernel Q takes 256 columns, so two of its CTAs share an SM: pass 1's N
+  // accumulates over G's columns (G is only used in pass 2, after N is read),
+  // and each pass-2 step's dQ contribution lands in U's columns [64, 80) (free
+  // once E is packed into [0, 64)) and is added up in registers
+  static constexpr int kQCols = 256, kQTmN = 128, kQTmDq = 64;
   static_assert(kV % 1024 == 0 && kDN % 1024 == 0 && kVk % 1024 == 0 && kDNk % 1024 == 0,
                 "swizzled tiles need 1024-byte alignment");
 };
@@ -119,7 +124,7 @@ __device__ __forceinline__ uint32_t bt_pack(float a, float b) {
 // kernel Q: D, N -> dN, dD (workspace) -> dq
 // ---------------------------------------------------------------------------
 template <int DV>
-__global__ void __launch_bounds__(kBtThreads, 1)
+__global__ void __launch_bounds__(kBtThreads, DV == 64 ? 2 : 1)
     linattn_bwd_tc_q_kernel(const __grid_constant__ CUtensorMap vmap, const BtParams p) {
   using Lay = BtLayout<DV>;
   extern __shared__ uint8_t smem_raw[];
@@ -154,7 +159,7 @@ __global__ void __launch_bounds__(kBtThreads, 1)
     umma::fence_mbar_init();
   }
   if (warp == 0) {
-    umma::tmem_alloc(tmem_slot, 512);
+    umma::tmem_alloc(tmem_slot, Lay::kQCols);
     umma::tmem_relinquish();
   }
   if (!issuer) {  // Q_i rows
@@ -188,6 +193,9 @@ __global__ void __launch_bounds__(kBtThreads, 1)
   int v_inflight = issuer && lane == 0 ? 1 : 0;  // loads issued and not yet waited for (issuer)
 
   float dsum = 0.0f;  // D_t (pass 1), then dD_t (pass 2), for query t0 + tid
+  float dq_acc[16];   // dQ of this lane's query (pass 2)
+#pragma unroll
+  for (int c = 0; c < 16; ++c) dq_acc[c] = 0.0f;
   const int row = tid;  // compute threads: query row = TMEM lane
   const uint32_t sQ = umma::smem_u32(sm + Lay::kQ);
   // K rows of the next step, loaded one step ahead of their use
@@ -277,62 +285,73 @@ __global__ void __launch_bounds__(kBtThreads, 1)
         const uint32_t sV = umma::smem_u32(sm + Lay::kV + b * Lay::kVTile);
 #pragma unroll
         for (int ks = 0; ks < kBtT / 16; ++ks)
-          umma::mma_ts(tmem + Lay::kTmAcc, tmem + Lay::kTmU + ks * 8,
+          umma::mma_ts(tmem + Lay::kQTmN, tmem + Lay::kTmU + ks * 8,
                        umma::desc_mnmajor_sw128(sV, ks * 16, kBtT),
                        umma::idesc_bf16(128, DV, false, true), (j > 0 || ks > 0) ? 1u : 0u);
-      } else {  // dQ += E K_j
+      } else {  // this step's E K_j (added to dQ in registers)
         const uint32_t sKm = umma::smem_u32(sm + Lay::kKm + b * 4096);
 #pragma unroll
         for (int ks = 0; ks < kBtT / 16; ++ks)
-          umma::mma_ts(tmem + Lay::kTmAcc16, tmem + Lay::kTmU + ks * 8,
+          umma::mma_ts(tmem + Lay::kQTmDq, tmem + Lay::kTmU + ks * 8,
                        umma::desc_mnmajor_none(sKm, ks * 16, kBtT),
-                       umma::idesc_bf16(128, 16, false, true), (j > 0 || ks > 0) ? 1u : 0u);
+                       umma::idesc_bf16(128, 16, false, true), ks > 0 ? 1u : 0u);
       }
       umma::mma_commit(bar_m2);
     }
     if (!umma::mbar_wait(bar_m2, step & 1)) fail();
     umma::tc_fence_after();
+    // this step's dQ contribution (read before the next step's U overwrites it;
+    // warp-collective load, so the whole warp decides)
+    if (pass == 1 && !issuer && __all_sync(0xffffffffu, !failed)) {
+      float tmp[32];
+      umma::tmem_ld32(tmem + Lay::kQTmDq + tm_lane, tmp);  // columns 64..95 (16 used)
+#pragma unroll
+      for (int c = 0; c < 16; ++c) dq_acc[c] += tmp[c];
+    }
+    umma::tc_fence_before();
     if (__syncthreads_or(failed)) break;
     // ---- end of pass 1: dN and dD of this lane's query ----
     if (pass == 0 && j == i && !issuer) {
       const long long t = (long long)t0 + row;
       const float D = dsum + p.eps;
-      float dy[DV];
-      if (t < L) {
-        const uint4* src = reinterpret_cast<const uint4*>(p.dy + (bh * L + t) * DV);
+      // dy row in 8-column pieces (read twice: for dy . N, then for dN), so few
+      // registers are live at a time
+      const uint4* src = reinterpret_cast<const uint4*>(p.dy + (bh * L + (t < L ? t : 0)) * DV);
+      auto dy8 = [&](int c8, float* f8) {
+        const uint4 w4 = t < L ? src[c8] : make_uint4(0, 0, 0, 0);
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w4);
 #pragma unroll
-        for (int c8 = 0; c8 < DV / 8; ++c8) {
-          const uint4 w4 = src[c8];
-          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w4);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(h[e]);
-            dy[c8 * 8 + 2 * e] = f.x;
-            dy[c8 * 8 + 2 * e + 1] = f.y;
-          }
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(h[e]);
+          f8[2 * e] = f.x;
+          f8[2 * e + 1] = f.y;
         }
-      } else {
-#pragma unroll
-        for (int c = 0; c < DV; ++c) dy[c] = 0.0f;
-      }
+      };
       float dot = 0.0f;
-#pragma unroll
+#pragma unroll 1
       for (int blk = 0; blk < DV / 64; ++blk) {
         float n[64];
-        umma::tmem_ld64(tmem + Lay::kTmAcc + tm_lane + 64 * blk, n);
+        umma::tmem_ld64(tmem + Lay::kQTmN + tm_lane + 64 * blk, n);
 #pragma unroll
-        for (int c = 0; c < 64; ++c) dot = fmaf(dy[64 * blk + c], n[c], dot);
+        for (int c8 = 0; c8 < 8; ++c8) {
+          float f8[8];
+          dy8(blk * 8 + c8, f8);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) dot = fmaf(f8[e], n[c8 * 8 + e], dot);
+        }
       }
       const float invD = 1.0f / D;
       dsum = -dot * invD * invD;  // dD_t
       __nv_bfloat16* wdn = p.ws_dn + (bh * L + t) * DV;
 #pragma unroll
       for (int c8 = 0; c8 < DV / 8; ++c8) {
+        float f8[8];
+        dy8(c8, f8);
         uint4 w4;
-        w4.x = bt_pack(dy[c8 * 8 + 0] * invD, dy[c8 * 8 + 1] * invD);
-        w4.y = bt_pack(dy[c8 * 8 + 2] * invD, dy[c8 * 8 + 3] * invD);
-        w4.z = bt_pack(dy[c8 * 8 + 4] * invD, dy[c8 * 8 + 5] * invD);
-        w4.w = bt_pack(dy[c8 * 8 + 6] * invD, dy[c8 * 8 + 7] * invD);
+        w4.x = bt_pack(f8[0] * invD, f8[1] * invD);
+        w4.y = bt_pack(f8[2] * invD, f8[3] * invD);
+        w4.z = bt_pack(f8[4] * invD, f8[5] * invD);
+        w4.w = bt_pack(f8[6] * invD, f8[7] * invD);
         // K-major, 128-byte swizzle: 64-column blocks of 128 rows x 128 B
         const int blk = c8 >> 3, ch = c8 & 7;
         *reinterpret_cast<uint4*>(sm + Lay::kDN + blk * (kBtT * 128) + row * 128 +
@@ -347,13 +366,7 @@ __global__ void __launch_bounds__(kBtThreads, 1)
   // ---- dq of this lane's query ----
   if (!issuer && !any_failed) {
     const long long t = (long long)t0 + row;
-    float g[16];
-    {
-      float tmp[32];
-      umma::tmem_ld32(tmem + Lay::kTmAcc16 + tm_lane, tmp);  // columns 384..415 (16 used)
-#pragma unroll
-      for (int c = 0; c < 16; ++c) g[c] = tmp[c];
-    }
+    const float* g = dq_acc;
     if (t < L) {
       float4* dst = reinterpret_cast<float4*>(p.dq + (bh * L + t) * kD);
 #pragma unroll
@@ -370,7 +383,7 @@ __global__ void __launch_bounds__(kBtThreads, 1)
     umma::mbar_wait(bar_v + 1, 0);
   }
   __syncthreads();
-  if (warp == 0) umma::tmem_dealloc(tmem, 512);
+  if (warp == 0) umma::tmem_dealloc(tmem, Lay::kQCols);
 }
 
 // ---------------------------------------------------------------------------
