@@ -39,19 +39,23 @@
 // scaled by the same power so the ratio is unchanged).  All accumulation is fp32
 // in TMEM; the master state never leaves TMEM until the export.
 //
-// Schedule (warp-specialised, chunks pipelined):
-//   group P (warps 0-3):  P of chunk c from U;
-//   group F (warps 4-7):  feature maps and Q/K tiles of chunk c+1, while group P
-//            still works on chunk c;
+// Schedule (warp-specialised, chunks pipelined), 64 value columns per CTA (a
+// sequence with d_v = 128 runs as two CTAs, one per 64-column slice of v: the
+// denominator does not depend on v):
+//   group P (warps 0-3):  P of chunk c from U, written back over U in TMEM;
+//   group F (warps 4-7):  Q/K tiles and phiK of chunk c+1 (shared memory) and its
+//            phiQ (TMEM), while group P still works on chunk c;
 //   group E (warps 8-11): epilogue of chunk c -- y from O, and the fp16 copy of the
-//            state for chunk c+1;
-//   issue warp (warp 12, one thread): V tiles by TMA (three stages at d_v = 64,
-//            one at d_v = 128) and the MMAs in the order #1, #5, #2, (P), #4.
-// Warps w, w+4 and w+8 share TMEM lane quadrant w, so each group reads and writes
-// the TMEM rows of its own 32 tokens.
-// The second state tile (features 128..191, of which 128..159 are used) is an
-// M=64 MMA.  Hand-offs are mbarriers (128 arrivals from a warp group, or a
-// tcgen05.commit); every wait is bounded.
+//            state for chunk c+1; once chunk c's MMAs are done, the V tile of
+//            chunk c+3 into its stage (TMA);
+//   issue warp (warp 12, one thread): the first three V tiles, then the MMAs in
+//            the order #1, #5, #2, (P), #4 -- and nothing else, since every
+//            instruction it runs between two MMA groups leaves the tensor pipe idle.
+// The state is kept transposed in TMEM, [S|z]^T: lane j holds value column j
+// (lane DV holds z), column f holds feature f, so #5 is one N = 160 MMA per K
+// step.  Warps w, w+4 and w+8 share TMEM lane quadrant w, so each group reads and
+// writes the TMEM rows of its own 32 tokens.  Hand-offs are mbarriers (arrivals
+// from warp groups, or a tcgen05.commit); every wait is bounded.
 //
 // Long sequences are split into n_seg segments of seg_chunks chunks so that
 // B*H*n_seg CTAs fill the GPU: a state-only pass (kStateOnly) runs #5 alone
@@ -82,62 +86,39 @@ constexpr int kTcTmemCols = 512;
 
 template <int DV>
 struct TcLayout {
+  static_assert(DV == 64, "the kernel runs 64 value columns per CTA");
   static constexpr int NA = DV + 16;                       // [V | 1 | 0..] columns
-  static constexpr int NG = (NA + 31) / 32;                // 32-column groups of a state tile
-  static constexpr int kTileCols = NG * 32;                // TMEM columns per state tile
-  // d_v = 64 fits phiQ and P in TMEM as A operands (and frees the shared memory
-  // for a second phiK buffer and a y staging tile stored by TMA); d_v = 128
-  // keeps them in shared memory
-  static constexpr bool kTm = DV == 64;
-  static constexpr int kVBuf = DV == 64 ? 3 : 1;           // V stages
-  static constexpr int kPhiKBuf = kTm ? 2 : 1;             // phiK buffers
-  // d_v = 64: three V stages share one ones block placed after them (each stage's
-  // descriptor reaches it through its own block stride); d_v = 128: one stage
-  // holding its V blocks and its ones block
-  static constexpr int kVStage = DV == 64 ? 16384 : (DV / 64 + 1) * 16384;
-  static constexpr int kNOnes = DV == 64 ? 1 : kVBuf;
-  static constexpr int kVBytes = DV == 64 ? (kVBuf + 1) * 16384 : kVBuf * kVStage;
-  // ones block used by V stage s, and the stride from the stage's first V block
-  // to it (the descriptor's block stride), relative to kV
-  static __host__ __device__ constexpr int ones_off(int s) {
-    return DV == 64 ? kVBuf * 16384 : s * kVStage + (DV / 64) * 16384;
-  }
-  static __host__ __device__ constexpr int v_lbo(int s) { return DV == 64 ? (kVBuf - s) * 16384 : 16384; }
+  static constexpr int kTileCols = 96;                     // TMEM columns of O (NA, 32-aligned)
+  static constexpr int kVBuf = 3;                          // V stages
+  static constexpr int kPhiKBuf = 2;                       // phiK buffers
+  // the three V stages share one ones block placed after them; each stage's
+  // descriptor reaches it through its own block stride (v_lbo)
+  static constexpr int kVStage = 16384;
+  static constexpr int kVBytes = (kVBuf + 1) * kVStage;
+  static constexpr int kOnes = kVBuf * kVStage;
+  static __host__ __device__ constexpr int v_lbo(int s) { return (kVBuf - s) * kVStage; }
   // shared memory (byte offsets from a 1024-aligned base)
   static constexpr int kQ = 0;                             // Q tile  [128 x 16] bf16, K-major
   static constexpr int kK = kQ + 4096;                     // K tile  [128 x 16] bf16, K-major
   static constexpr int kV = kK + 4096;                     // [V | ones] MN-major SW128 stages
   static constexpr int kPhiK = kV + kVBytes;               // phiK [160 x 128] bf16, MN-major
-  static constexpr int kP = kPhiK + kPhiKBuf * 40960;      // P [128 x 128] bf16 (smem path)
-  static constexpr int kPhiQ = kP + (kTm ? 0 : 32768);     // phiQ [128 x 160] fp16 (smem path)
-  static constexpr int kSBuf = kTm ? 2 : 1;                // fp16 state copies
+  static constexpr int kSBuf = 2;                          // fp16 state copies
   static constexpr int kSBytes = NA * kSymFP * 2;
-  static constexpr int kS = kPhiQ + (kTm ? 0 : 40960);     // [S|z] copies [160 x NA] fp16, MN-major
+  static constexpr int kS = kPhiK + kPhiKBuf * 40960;      // [S|z]^T copies [NA x 160] fp16, K-major
   static constexpr int kY = kS + kSBuf * kSBytes;          // y staging [128 x 64] bf16 SW128
-  static constexpr int kBar = kY + (kTm ? 16384 : 0);      // mbarriers + TMEM address
+  static constexpr int kBar = kY + 16384;                  // mbarriers + TMEM address
   static constexpr int kBytes = kBar + 256;
   static constexpr size_t kSmem = kBytes + 1024;           // + alignment slack
-  // TMEM: state tile 0 (features 0..127, M=128), state tile 1 (features
-  // 128..191, M=64: row r in lane r%16 + 32*(r/16)), the score tile U (P is
-  // written over it), the output accumulator O -- separate from U when the
-  // columns allow it -- and phiQ (80 columns of fp16 pairs)
-  // d_v = 64 keeps the state transposed, [S|z]^T: TMEM lane = value column (64
-  // columns, then z in lane 64), TMEM column = feature; #5 is then one N=160 MMA
-  // per K step.  d_v = 128 keeps features on the lanes (tile 0: features
-  // 0..127, M=128; tile 1: features 128..191, M=64).
-  static constexpr bool kSt = DV == 64;
+  // TMEM: the transposed state [S|z]^T (160 feature columns), the score tile U
+  // (P is written over it as bf16 pairs), the output accumulator O, and phiQ
+  // (80 columns of fp16 pairs)
   static constexpr int kTmS0 = 0;
-  static constexpr int kTmS1 = kSt ? 0 : kTileCols;
-  static constexpr int kTmU = kSt ? kSymFP : 2 * kTileCols;
-  static constexpr bool kEarlyO = kTmU + 128 + kTileCols <= kTcTmemCols;
-  static constexpr int kTmO = kEarlyO ? kTmU + 128 : kTmU;
-  static_assert(kTmU % 32 == 0, "TMEM region alignment");
+  static constexpr int kTmU = kSymFP;
+  static constexpr int kTmO = kTmU + 128;
   static constexpr int kTmQ = kTmO + kTileCols;
-  static_assert(kTmO + kTileCols + (kTm ? kSymFP / 2 : 0) <= kTcTmemCols, "TMEM budget");
-  static_assert(!kTm || kEarlyO, "TMEM operands need a separate O");
+  static_assert(kTmU % 32 == 0 && kTileCols >= NA, "TMEM regions");
+  static_assert(kTmQ + kSymFP / 2 <= kTcTmemCols, "TMEM budget");
   static_assert(kY % 1024 == 0, "TMA staging alignment");
-  // the M=64 state MMA reads feature groups 16..23 (8 past the 160 written)
-  static_assert(kPhiK + (kPhiKBuf - 1) * 40960 + 49152 <= kBytes, "phiK over-read window");
   static_assert(kSmem <= 232448, "shared memory budget");
 };
 
@@ -276,26 +257,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                       const __grid_constant__ CUtensorMap ymap, const TcParams p) {
   using Lay = TcLayout<DV>;
   constexpr int NA = Lay::NA;
-  constexpr int NG = Lay::NG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::kBar);
   uint64_t* bar_tma = bars + 16;     // [kVBuf] V stage landed
   uint64_t* bar_qk = bars + 2;       // Q/K tiles and phiK written (group F)
-  uint64_t* bar_phiq = bars + 14;    // phiQ written (group F)
+  uint64_t* bar_go = bars + 14;      // phiQ of chunk c written (group F); O, the state and its
+                                     // fp16 copy of chunk c-1 read and written (group E)
   uint64_t* bar_fin = bars + 15;     // every MMA of this CTA complete (commit)
   uint64_t* bar_u = bars + 3;        // #1 done (commit)
   uint64_t* bar_p = bars + 4;        // P written (group A)
   uint64_t* bar_m25 = bars + 5;      // #5 and #2 done (commit): feature buffers free
   uint64_t* bar_o = bars + 6;        // every MMA of the chunk done (commit)
-  uint64_t* bar_ss = bars + 7;       // state read + fp16 copy written, O read (group E)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 9);
   uint64_t* bar_yfree = bars + 10;   // y staging tile free again (TMA store read it)
   uint64_t* bar_yfull = bars + 11;   // y staging tile written (group E)
   uint64_t* bar_m5 = bars + 12;      // #5 done (commit): the state can be read
-  uint64_t* bar_sread = bars + 13;   // state read and its fp16 copy written (group E)
   uint64_t* bar_done = bars + 19;    // [2] state-only pass, d_v = 64: #5 of the chunk that
                                      // used phiK buffer b complete (commit)
   constexpr int kThreads = kTcThreads;
@@ -316,17 +295,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (tid == 0) {
     for (int sidx = 0; sidx < Lay::kVBuf; ++sidx) umma::mbar_init(bar_tma + sidx, 1);
     umma::mbar_init(bar_qk, kTcGroup);
-    umma::mbar_init(bar_phiq, kTcGroup);
+    umma::mbar_init(bar_go, 2 * kTcGroup);
     umma::mbar_init(bar_fin, 1);
     umma::mbar_init(bar_u, 1);
     umma::mbar_init(bar_p, kTcGroup);
     umma::mbar_init(bar_m25, 1);
     umma::mbar_init(bar_o, 1);
-    umma::mbar_init(bar_ss, kTcGroup);
     umma::mbar_init(bar_yfree, 1);
     umma::mbar_init(bar_yfull, kTcGroup);
     umma::mbar_init(bar_m5, 1);
-    umma::mbar_init(bar_sread, kTcGroup);
     umma::mbar_init(bar_done, 1);
     umma::mbar_init(bar_done + 1, 1);
     *abort_flag = 0;
@@ -337,26 +314,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     umma::tmem_alloc(tmem_slot, kTcTmemCols);
     umma::tmem_relinquish();
   }
-  // ones block of every V stage: column DV of the augmented V is 1 for every token
-  for (int b = 0; b < Lay::kNOnes; ++b) {
-    uint8_t* ones = sm + Lay::kV + Lay::ones_off(b);
-    for (int i = tid; i < 16384 / 16; i += kThreads)
-      reinterpret_cast<uint4*>(ones)[i] = make_uint4(0, 0, 0, 0);
-  }
+  // the ones block of the V stages: column DV of the augmented V is 1 for every token
+  for (int i = tid; i < Lay::kVStage / 16; i += kThreads)
+    reinterpret_cast<uint4*>(sm + Lay::kV + Lay::kOnes)[i] = make_uint4(0, 0, 0, 0);
   __syncthreads();
-  for (int b = 0; b < Lay::kNOnes; ++b)
-    if (tid < kTcChunk)
-      *reinterpret_cast<__nv_bfloat16*>(sm + Lay::kV + Lay::ones_off(b) +
-                                        umma::off_mnmajor_sw128(0, tid, kTcChunk)) =
-          __float2bfloat16(1.0f);
-  if constexpr (Lay::kSt) {
-    // rows DV..NA-1 of the transposed fp16 state copies: row DV (z) is rewritten
-    // for every chunk, the rows after it stay zero
-    for (int b = 0; b < Lay::kSBuf; ++b)
-      for (int i = tid; i < (NA - DV) * kSymFP * 2 / 16; i += kThreads)
-        reinterpret_cast<uint4*>(sm + Lay::kS + b * Lay::kSBytes + DV * kSymFP * 2)[i] =
-            make_uint4(0, 0, 0, 0);
-  }
+  if (tid < kTcChunk)
+    *reinterpret_cast<__nv_bfloat16*>(sm + Lay::kV + Lay::kOnes +
+                                      umma::off_mnmajor_sw128(0, tid, kTcChunk)) =
+        __float2bfloat16(1.0f);
+  // rows DV..NA-1 of the transposed fp16 state copies: row DV (z) is rewritten
+  // for every chunk, the rows after it stay zero
+  for (int b = 0; b < Lay::kSBuf; ++b)
+    for (int i = tid; i < (NA - DV) * kSymFP * 2 / 16; i += kThreads)
+      reinterpret_cast<uint4*>(sm + Lay::kS + b * Lay::kSBytes + DV * kSymFP * 2)[i] =
+          make_uint4(0, 0, 0, 0);
   umma::fence_async_smem();
   umma::tc_fence_before();
   __syncthreads();
@@ -380,62 +351,58 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // a barrier that orders them behind export_stage.
   constexpr int kStr = DV + 4;  // keeps each feature row 16-byte aligned
   auto export_stage = [&](int t) {
-    if constexpr (Lay::kSt) {
-      const bool any_st = has_init || c_begin < c_end;
-      float* stage = reinterpret_cast<float*>(sm + Lay::kPhiK);
-      int* rowmap = reinterpret_cast<int*>(stage + kSymFP * kStr);  // [273]: 2 f + (1 if / sqrt 2)
-      static_assert(Lay::kPhiKBuf * 40960 >= (kSymFP * kStr + kF) * 4, "export staging");
-      if (quad < 3) {
-        // two TMEM round trips of 80 features each
+    const bool any_st = has_init || c_begin < c_end;
+    float* stage = reinterpret_cast<float*>(sm + Lay::kPhiK);
+    int* rowmap = reinterpret_cast<int*>(stage + kSymFP * kStr);  // [273]: 2 f + (1 if / sqrt 2)
+    static_assert(Lay::kPhiKBuf * 40960 >= (kSymFP * kStr + kF) * 4, "export staging");
+    if (quad < 3) {
+      // two TMEM round trips of 80 features each
 #pragma unroll 1
-        for (int g = 0; g < 2; ++g) {
-          float sv[80];
-          umma::tmem_ld80(tmem + Lay::kTmS0 + tm_lane + g * 80, sv);
-          if (t <= DV) {
+      for (int g = 0; g < 2; ++g) {
+        float sv[80];
+        umma::tmem_ld80(tmem + Lay::kTmS0 + tm_lane + g * 80, sv);
+        if (t <= DV) {
 #pragma unroll
-            for (int i = 0; i < 80; ++i) stage[(g * 80 + i) * kStr + t] = any_st ? sv[i] : 0.0f;
-          }
+          for (int i = 0; i < 80; ++i) stage[(g * 80 + i) * kStr + t] = any_st ? sv[i] : 0.0f;
         }
       }
-      for (int f = t; f < kSymFP; f += kTcGroup) {
-        int r0 = -1, r1 = -1;
-        float scale = 1.0f;
-        const int nrows = tc_feature_rows(f, &r0, &r1, &scale);
-        const int code = 2 * f + (nrows == 2 ? 1 : 0);
-        if (nrows >= 1) rowmap[r0] = code;
-        if (nrows == 2) rowmap[r1] = code;
-      }
+    }
+    for (int f = t; f < kSymFP; f += kTcGroup) {
+      int r0 = -1, r1 = -1;
+      float scale = 1.0f;
+      const int nrows = tc_feature_rows(f, &r0, &r1, &scale);
+      const int code = 2 * f + (nrows == 2 ? 1 : 0);
+      if (nrows >= 1) rowmap[r0] = code;
+      if (nrows == 2) rowmap[r1] = code;
     }
   };
   auto export_store = [&](int u, int n) {
-    if constexpr (Lay::kSt) {
-      const float* stage = reinterpret_cast<const float*>(sm + Lay::kPhiK);
-      const int* rowmap = reinterpret_cast<const int*>(stage + kSymFP * kStr);
-      if (kStateOnly) {
-        float* part = p.partial + ((size_t)bh * (p.n_seg - 1) + seg) * kSymFP * NA;
-        for (int i = u; i < kSymFP * NA; i += n) {
-          const int f = i / NA, j = i - f * NA;
-          part[i] = j <= DV ? stage[f * kStr + j] : 0.0f;
-        }
-      } else if (seg == p.n_seg - 1) {
-        if (p.state_kv) {
-          float* skv = p.state_kv + (size_t)bh_seq * kF * p.ld_v + col0;
+    const float* stage = reinterpret_cast<const float*>(sm + Lay::kPhiK);
+    const int* rowmap = reinterpret_cast<const int*>(stage + kSymFP * kStr);
+    if (kStateOnly) {
+      float* part = p.partial + ((size_t)bh * (p.n_seg - 1) + seg) * kSymFP * NA;
+      for (int i = u; i < kSymFP * NA; i += n) {
+        const int f = i / NA, j = i - f * NA;
+        part[i] = j <= DV ? stage[f * kStr + j] : 0.0f;
+      }
+    } else if (seg == p.n_seg - 1) {
+      if (p.state_kv) {
+        float* skv = p.state_kv + (size_t)bh_seq * kF * p.ld_v + col0;
 #pragma unroll 4
-          for (int i = u; i < kF * (DV / 4); i += n) {
-            const int r = i / (DV / 4), j = (i - r * (DV / 4)) * 4;
-            const int code = rowmap[r];
-            const float sc = (code & 1) ? 0.70710678118654752f : 1.0f;
-            const float4 v4 = *reinterpret_cast<const float4*>(stage + (code >> 1) * kStr + j);
-            *reinterpret_cast<float4*>(skv + (size_t)r * p.ld_v + j) =
-                make_float4(v4.x * sc, v4.y * sc, v4.z * sc, v4.w * sc);
-          }
+        for (int i = u; i < kF * (DV / 4); i += n) {
+          const int r = i / (DV / 4), j = (i - r * (DV / 4)) * 4;
+          const int code = rowmap[r];
+          const float sc = (code & 1) ? 0.70710678118654752f : 1.0f;
+          const float4 v4 = *reinterpret_cast<const float4*>(stage + (code >> 1) * kStr + j);
+          *reinterpret_cast<float4*>(skv + (size_t)r * p.ld_v + j) =
+              make_float4(v4.x * sc, v4.y * sc, v4.z * sc, v4.w * sc);
         }
-        if (p.state_k && col0 == 0) {
-          float* sk = p.state_k + (size_t)bh_seq * kF;
-          for (int r = u; r < kF; r += n) {
-            const int code = rowmap[r];
-            sk[r] = stage[(code >> 1) * kStr + DV] * ((code & 1) ? 0.70710678118654752f : 1.0f);
-          }
+      }
+      if (p.state_k && col0 == 0) {
+        float* sk = p.state_k + (size_t)bh_seq * kF;
+        for (int r = u; r < kF; r += n) {
+          const int code = rowmap[r];
+          sk[r] = stage[(code >> 1) * kStr + DV] * ((code & 1) ? 0.70710678118654752f : 1.0f);
         }
       }
     }
@@ -446,25 +413,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // warp write 32 consecutive floats of a row.  Run by warps of quadrants 0-2
   // of one group per half, once the last #5 is complete.
   auto export_direct = [&](int h) {
-    if constexpr (Lay::kSt) {
-      if (quad < 3 && seg == p.n_seg - 1) {
-        float sv[80];
-        umma::tmem_ld80(tmem + Lay::kTmS0 + tm_lane + h * 80, sv);
-        const int j = quad * 32 + lane;
-        float* skv = p.state_kv ? p.state_kv + (size_t)bh_seq * kF * p.ld_v + col0 + j : nullptr;
-        float* sk = p.state_k && col0 == 0 ? p.state_k + (size_t)bh_seq * kF : nullptr;
-        float* dst = j < DV ? skv : (j == DV ? sk : nullptr);
-        const int stride = j < DV ? p.ld_v : 1;
-        if (dst != nullptr) {
+    if (quad < 3 && seg == p.n_seg - 1) {
+      float sv[80];
+      umma::tmem_ld80(tmem + Lay::kTmS0 + tm_lane + h * 80, sv);
+      const int j = quad * 32 + lane;
+      float* skv = p.state_kv ? p.state_kv + (size_t)bh_seq * kF * p.ld_v + col0 + j : nullptr;
+      float* sk = p.state_k && col0 == 0 ? p.state_k + (size_t)bh_seq * kF : nullptr;
+      float* dst = j < DV ? skv : (j == DV ? sk : nullptr);
+      const int stride = j < DV ? p.ld_v : 1;
+      if (dst != nullptr) {
 #pragma unroll
-          for (int i = 0; i < 80; ++i) {
-            int r0 = -1, r1 = -1;
-            float scale = 1.0f;
-            const int nrows = tc_feature_rows(h * 80 + i, &r0, &r1, &scale);
-            const float v = sv[i] * scale;
-            if (nrows >= 1) dst[(size_t)r0 * stride] = v;
-            if (nrows == 2) dst[(size_t)r1 * stride] = v;
-          }
+        for (int i = 0; i < 80; ++i) {
+          int r0 = -1, r1 = -1;
+          float scale = 1.0f;
+          const int nrows = tc_feature_rows(h * 80 + i, &r0, &r1, &scale);
+          const float v = sv[i] * scale;
+          if (nrows >= 1) dst[(size_t)r0 * stride] = v;
+          if (nrows == 2) dst[(size_t)r1 * stride] = v;
         }
       }
     }
@@ -492,25 +457,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ================= issue warp: lane 0 drives TMA and the tensor cores =================
     if (lane == 0) {
       const uint32_t sQ = umma::smem_u32(sm + Lay::kQ), sK = umma::smem_u32(sm + Lay::kK),
-                     sP = umma::smem_u32(sm + Lay::kP), sPhiQ = umma::smem_u32(sm + Lay::kPhiQ),
-                     sS = umma::smem_u32(sm + Lay::kS);
+                     sS = umma::smem_u32(sm + Lay::kS), sPhiK = umma::smem_u32(sm + Lay::kPhiK);
       // descriptors are computed once per buffer and stepped along K by adding
       // the start-address increment (16-byte units) to their low word
       const uint64_t d_q = umma::desc_kmajor_none(sQ, 0, 16), d_k = umma::desc_kmajor_none(sK, 0, 16);
-      // fp16 state copy: [value column x feature] K-major (transposed state) or
-      // [feature x value column] MN-major
-      const uint32_t sS1 = sS + (Lay::kSBuf - 1) * Lay::kSBytes;
-      const uint64_t d_s0 = Lay::kSt ? umma::desc_kmajor_none(sS, 0, kSymFP)
-                                     : umma::desc_mnmajor_none(sS, 0, kSymFP);
-      const uint64_t d_s1 = Lay::kSt ? umma::desc_kmajor_none(sS1, 0, kSymFP)
-                                     : umma::desc_mnmajor_none(sS1, 0, kSymFP);
-      const uint64_t d_p = umma::desc_kmajor_none(sP, 0, kTcChunk);
-      const uint64_t d_phiq = umma::desc_kmajor_none(sPhiQ, 0, kSymFP);
+      // fp16 state copies, [value column x feature] K-major
+      const uint64_t d_s0 = umma::desc_kmajor_none(sS, 0, kSymFP);
+      const uint64_t d_s1 = umma::desc_kmajor_none(sS + Lay::kSBytes, 0, kSymFP);
+      // V stages (MN-major, 128B swizzle; the block stride reaches the ones block)
+      auto v_desc = [&](int st) {
+        return umma::smem_desc(umma::smem_u32(sm + Lay::kV + st * Lay::kVStage), Lay::v_lbo(st),
+                               1024, umma::kLayoutSW128);
+      };
+      const uint64_t d_v0 = v_desc(0), d_v1 = v_desc(1), d_v2 = v_desc(2);
+      static_assert(Lay::kVBuf == 3, "three V stages");
+      // phiK buffers (MN-major, no swizzle)
+      const uint64_t d_k0 = umma::desc_mnmajor_none(sPhiK, 0, kTcChunk);
+      const uint64_t d_k1 = umma::desc_mnmajor_none(sPhiK + 40960, 0, kTcChunk);
       const uint32_t id_u = umma::idesc_bf16(128, 128, false, false);
-      const uint32_t id_o2 = umma::idesc_f16(128, NA, false, !Lay::kSt);
+      const uint32_t id_o2 = umma::idesc_f16(128, NA, false, false);
       const uint32_t id_o4 = umma::idesc_bf16(128, NA, false, true);
-      const uint32_t id_s0 = umma::idesc_bf16(128, NA, true, true);
-      const uint32_t id_s1 = umma::idesc_bf16(64, NA, true, true);
       const uint32_t id_st = umma::idesc_bf16(128, kSymFP, true, true);
       // per stage (bit s): a load in flight, and the parity of the phase it completes
       // (bit masks rather than arrays, which would live in local memory)
@@ -518,27 +484,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int sidx = 0; sidx < Lay::kVBuf && c_begin + sidx < c_end; ++sidx)
         inflight |= issue_v(c_begin + sidx, sidx) << sidx;
       int n_done = 0;  // chunks whose MMAs were all issued and committed
-      for (int c = c_begin; c < c_end && !*abort_flag; ++c) {
+      int stage = 0;   // V stage of chunk c
+      // (no abort check per chunk: a group that gave up stops arriving, and the
+      // bounded waits below then end this loop too)
+      for (int c = c_begin; c < c_end; ++c) {
         const int it = c - c_begin;
         const uint32_t ph = it & 1;
-        const int stage = it % Lay::kVBuf;
-        const uint64_t d_v = umma::smem_desc(umma::smem_u32(sm + Lay::kV + stage * Lay::kVStage),
-                                             Lay::v_lbo(stage), 1024, umma::kLayoutSW128);
-        const uint32_t sPhiK = umma::smem_u32(sm + Lay::kPhiK + (it % Lay::kPhiKBuf) * 40960);
-        const uint64_t d_k0 = umma::desc_mnmajor_none(sPhiK, 0, kTcChunk);
-        const uint64_t d_k1 = umma::desc_mnmajor_none(sPhiK + 16 * 2048, 0, kTcChunk);
+        const uint64_t d_v = stage == 0 ? d_v0 : (stage == 1 ? d_v1 : d_v2);
+        const uint64_t d_phik = (it & 1) ? d_k1 : d_k0;
         const bool has_state = has_init || it > 0;
-        // index of the epilogue hand-off (state copy) of chunk c-1
-        const int kk = has_init ? it : it - 1;
-        const uint32_t ph_ss = kk & 1;
-        const uint64_t d_s = (kk & 1) ? d_s1 : d_s0;
+        // the fp16 copy of the state before chunk c (group E's copy number it - 1,
+        // or it with a seeded state)
+        const uint64_t d_s = ((has_init ? it : it - 1) & 1) ? d_s1 : d_s0;
+        BASED_TC_TRACE(10, it);
         if (!umma::mbar_wait(bar_qk, ph)) { fail(); break; }
         BASED_TC_TRACE(0, it);
-        // when O shares TMEM with U, #1 may only overwrite it once the epilogue
-        // group has read the previous chunk's O
-        if (!kStateOnly && !Lay::kEarlyO && has_state) {
-          if (!umma::mbar_wait(bar_ss, ph_ss)) { fail(); break; }
-        }
         umma::tc_fence_after();
         if (!kStateOnly) {
           umma::mma_bf16(tmem + Lay::kTmU, d_q, d_k, id_u, 0);
@@ -549,95 +509,59 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         BASED_TC_TRACE(2, it);
         inflight &= ~(1u << stage);
         vphase ^= 1u << stage;
-
-        // #5 overwrites the state: the epilogue group must have read (and copied)
-        // the previous chunk's state out of TMEM
-        if (!kStateOnly && Lay::kEarlyO && has_state) {
-          if (!umma::mbar_wait(Lay::kTm ? bar_sread : bar_ss, ph_ss)) { fail(); break; }
-        }
+        // #5 overwrites the state in TMEM, #2 reads its fp16 copy and overwrites O:
+        // group E must have read the previous chunk's state and O and written the
+        // copy, and group F this chunk's phiQ (one barrier for all three, which
+        // are ready well before #5 comes up)
+        if (!kStateOnly && !umma::mbar_wait(bar_go, ph)) { fail(); break; }
         BASED_TC_TRACE(3, it);
         umma::tc_fence_after();
-        // K step of 16 tokens: +256 B in the no-swizzle phiK layout (2 core
-        // matrices), +2048 B (16 rows of 128 B) in the swizzled V tile
-        if constexpr (Lay::kSt) {
-          // [S|z]^T += [V|1]^T phiK: A = the V stage (value columns x tokens,
-          // MN-major; the ones block supplies row DV), B = phiK (N = 160 features)
+        // #5 [S|z]^T += [V|1]^T phiK: A = the V stage (value columns x tokens,
+        // MN-major; the ones block supplies row DV), B = phiK (N = 160 features).
+        // K step of 16 tokens: +2048 B (16 rows of 128 B) in the swizzled V tile,
+        // +256 B (2 core matrices) in the no-swizzle phiK layout
+#pragma unroll
+        for (int ks = 0; ks < kTcChunk / 16; ++ks)
+          umma::mma_bf16(tmem + Lay::kTmS0, d_v + ks * 128, d_phik + ks * 16, id_st,
+                         has_state || ks > 0);
+        // the state-only pass releases this chunk's phiK buffer to group F
+        umma::mma_commit(kStateOnly ? bar_done + (it & 1) : bar_m5);
+        BASED_TC_TRACE(4, it);
+        // state-only pass: refill the stage of chunk c-1 (its MMAs are done by
+        // now) with chunk c + kVBuf - 1 (in the main pass group E refills a stage
+        // once every MMA of its chunk is done)
+        if (kStateOnly && it > 0 && c + Lay::kVBuf - 1 < c_end) {
+          const int s_prev = stage == 0 ? Lay::kVBuf - 1 : stage - 1;
+          if (!umma::mbar_wait(bar_o, (it - 1) & 1)) { fail(); break; }
+          BASED_TC_TRACE(11, it);
+          inflight |= issue_v(c + Lay::kVBuf - 1, s_prev) << s_prev;
+          BASED_TC_TRACE(12, it);
+        }
+        if (!kStateOnly) {
+          if (has_state) {
+            BASED_TC_TRACE(5, it);
+            // #2 O = phiQ [S|z]_{c-1}: A = phiQ from TMEM, B = the fp16 state copy.
+            // K step of 16 features: 8 TMEM columns, +256 B in the copy
+#pragma unroll
+            for (int ks = 0; ks < kSymFP / 16; ++ks)
+              umma::mma_ts(tmem + Lay::kTmO, tmem + Lay::kTmQ + ks * 8, d_s + ks * 16, id_o2,
+                           ks > 0);
+          }
+          umma::mma_commit(bar_m25);
+          BASED_TC_TRACE(6, it);
+          if (!umma::mbar_wait(bar_p, ph)) { fail(); break; }
+          umma::tc_fence_after();
+          BASED_TC_TRACE(7, it);
+          // #4 O += P [V|1]: A = P from TMEM (bf16 pairs over U), B = the V stage
 #pragma unroll
           for (int ks = 0; ks < kTcChunk / 16; ++ks)
-            umma::mma_bf16(tmem + Lay::kTmS0, d_v + ks * 128, d_k0 + ks * 16, id_st,
-                           has_state || ks > 0);
-        } else {
-#pragma unroll
-          for (int ks = 0; ks < kTcChunk / 16; ++ks) {
-            const uint32_t acc = has_state || ks > 0;
-            umma::mma_bf16(tmem + Lay::kTmS0, d_k0 + ks * 16, d_v + ks * 128, id_s0, acc);
-            umma::mma_bf16(tmem + Lay::kTmS1, d_k1 + ks * 16, d_v + ks * 128, id_s1, acc);
-          }
-        }
-        if (Lay::kTm) {
-          // the state-only pass releases this chunk's phiK buffer to group F
-          umma::mma_commit(kStateOnly ? bar_done + (it & 1) : bar_m5);
-          BASED_TC_TRACE(4, it);
-          // refill the stage of chunk c-1 (its MMAs are done by now) with chunk
-          // c + kVBuf - 1
-          if (Lay::kVBuf > 1 && it > 0 && c + Lay::kVBuf - 1 < c_end) {
-            if (!umma::mbar_wait(bar_o, (it - 1) & 1)) { fail(); break; }
-            inflight |= issue_v(c + Lay::kVBuf - 1, (it - 1) % Lay::kVBuf)
-                        << ((it - 1) % Lay::kVBuf);
-          }
-        }
-        if (!kStateOnly) {
-          if (!Lay::kEarlyO) {  // O shares TMEM with U: wait until P has been read out
-            if (!umma::mbar_wait(bar_p, ph)) { fail(); break; }
-            umma::tc_fence_after();
-          }
-          // phiQ of this chunk is written (waited for even when #2 is skipped, so
-          // that the group's arrivals for chunk c+1 follow this phase's completion)
-          if (!umma::mbar_wait(bar_phiq, ph)) { fail(); break; }
-          if (has_state) {
-            // #2 overwrites O: the epilogue group must have read the previous O
-            if (Lay::kTm) {
-              if (!umma::mbar_wait(bar_ss, ph_ss)) { fail(); break; }
-            }
-            umma::tc_fence_after();
-            BASED_TC_TRACE(5, it);
-            // K step of 16 features: +256 B in both no-swizzle layouts, 8 TMEM columns
-#pragma unroll
-            for (int ks = 0; ks < kSymFP / 16; ++ks) {
-              if constexpr (Lay::kTm)
-                umma::mma_ts(tmem + Lay::kTmO, tmem + Lay::kTmQ + ks * 8, d_s + ks * 16, id_o2,
-                             ks > 0);
-              else
-                umma::mma_f16(tmem + Lay::kTmO, d_phiq + ks * 16, d_s + ks * 16, id_o2, ks > 0);
-            }
-          }
-        }
-        if (!(kStateOnly && Lay::kTm)) umma::mma_commit(bar_m25);
-        BASED_TC_TRACE(6, it);
-        if (!kStateOnly) {
-          if (Lay::kEarlyO) {
-            if (!umma::mbar_wait(bar_p, ph)) { fail(); break; }
-            umma::tc_fence_after();
-          }
-          BASED_TC_TRACE(7, it);
-#pragma unroll
-          for (int ks = 0; ks < kTcChunk / 16; ++ks) {
-            const uint32_t acc = has_state || ks > 0;
-            if constexpr (Lay::kTm)
-              umma::mma_ts(tmem + Lay::kTmO, tmem + Lay::kTmU + ks * 8, d_v + ks * 128, id_o4, acc);
-            else
-              umma::mma_bf16(tmem + Lay::kTmO, d_p + ks * 16, d_v + ks * 128, id_o4, acc);
-          }
+            umma::mma_ts(tmem + Lay::kTmO, tmem + Lay::kTmU + ks * 8, d_v + ks * 128, id_o4,
+                         has_state || ks > 0);
         }
         umma::mma_commit(bar_o);
         BASED_TC_TRACE(8, it);
         ++n_done;
-        // refill the stage this chunk used once its MMAs are done
-        const int c_next = c + Lay::kVBuf;
-        if (!Lay::kTm && c_next < c_end) {
-          if (!umma::mbar_wait(bar_o, ph)) { fail(); break; }
-          inflight |= issue_v(c_next, stage) << stage;
-        }
+        stage = stage == Lay::kVBuf - 1 ? 0 : stage + 1;
       }
       // the last chunk's MMAs must be complete before the state is read out
       if (n_done > 0 && !umma::mbar_wait(bar_o, (n_done - 1) & 1)) fail();
@@ -658,93 +582,56 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int t0 = c * kTcChunk;
       // ---- scores: P = mask(1 + u/4 + u^2/32) * sc ------------------------------------
       if (!umma::mbar_wait(bar_u, it & 1)) { fail(); break; }
-      if (!Lay::kTm && it > 0 && !umma::mbar_wait(bar_o, (it - 1) & 1)) { fail(); break; }
       BASED_TC_TRACE(0, it);
       umma::tc_fence_after();
       const float sc = tc_chunk_scale((long long)t0 + kTcChunk);
       const float c0 = sc, c1 = 0.25f * sc, c2 = 0.03125f * sc;
       const uint64_t c0x2 = f32x2(c0, c0), c1x2 = f32x2(c1, c1), c2x2 = f32x2(c2, c2);
-      auto poly_pack = [&](const float* u, int c32, uint32_t* pk) {
-        const bool diag = c32 == quad;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float w0 = fmaf(u[2 * e], fmaf(u[2 * e], c2, c1), c0);
-          float w1 = fmaf(u[2 * e + 1], fmaf(u[2 * e + 1], c2, c1), c0);
-          if (diag) {
-            if (2 * e > lane) w0 = 0.0f;
-            if (2 * e + 1 > lane) w1 = 0.0f;
-          }
-          pk[e] = as_u32(__floats2bfloat162_rn(w0, w1));
-        }
-      };
-      if constexpr (Lay::kTm) {
-        // P (bf16 pairs) of key block b (32 keys) goes to U columns [16b, 16b + 16),
-        // which this thread has read already (they belong to block b / 2 <= b);
-        // one loop body for every block keeps the code small
-        // blocks are taken two at a time (one TMEM load of 64 columns) while two
-        // remain, so a warp pays at most two load round trips
-        const int row = lane + 32 * quad;  // this thread's token within the chunk
+      // P (bf16 pairs) of key block b (32 keys) goes to U columns [16b, 16b + 16),
+      // which this thread has read already (they belong to block b / 2 <= b);
+      // one loop body for every block keeps the code small
+      // blocks are taken two at a time (one TMEM load of 64 columns) while two
+      // remain, so a warp pays at most two load round trips
+      const int row = lane + 32 * quad;  // this thread's token within the chunk
 #pragma unroll 1
-        for (int b = 0; b <= quad; b += 2) {
-          const bool two = b + 1 <= quad;  // warp-uniform
-          float u[64];
-          if (two) umma::tmem_ld64(tmem + Lay::kTmU + tm_lane + 32 * b, u);
-          else umma::tmem_ld32(tmem + Lay::kTmU + tm_lane + 32 * b, u);
-          const int lim = row - 32 * b;  // keys 32b + j with j > lim lie in the future
-          uint32_t pk[32];
-          if (b + 1 >= quad) {  // the pair holds the diagonal block: causal mask
+      for (int b = 0; b <= quad; b += 2) {
+        const bool two = b + 1 <= quad;  // warp-uniform
+        float u[64];
+        if (two) umma::tmem_ld64(tmem + Lay::kTmU + tm_lane + 32 * b, u);
+        else umma::tmem_ld32(tmem + Lay::kTmU + tm_lane + 32 * b, u);
+        const int lim = row - 32 * b;  // keys 32b + j with j > lim lie in the future
+        uint32_t pk[32];
+        if (b + 1 >= quad) {  // the pair holds the diagonal block: causal mask
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              float w0, w1;
-              poly2(u[2 * e], u[2 * e + 1], c0x2, c1x2, c2x2, &w0, &w1);
-              if (2 * e > lim) w0 = 0.0f;
-              if (2 * e + 1 > lim) w1 = 0.0f;
-              pk[e] = as_u32(__floats2bfloat162_rn(w0, w1));
-            }
-          } else {  // entirely below the diagonal
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              float w0, w1;
-              poly2(u[2 * e], u[2 * e + 1], c0x2, c1x2, c2x2, &w0, &w1);
-              pk[e] = as_u32(__floats2bfloat162_rn(w0, w1));
-            }
+          for (int e = 0; e < 32; ++e) {
+            float w0, w1;
+            poly2(u[2 * e], u[2 * e + 1], c0x2, c1x2, c2x2, &w0, &w1);
+            if (2 * e > lim) w0 = 0.0f;
+            if (2 * e + 1 > lim) w1 = 0.0f;
+            pk[e] = as_u32(__floats2bfloat162_rn(w0, w1));
           }
-          if (two) umma::tmem_st32_nowait(tmem + Lay::kTmU + tm_lane + 16 * b, pk);
-          else umma::tmem_st16_nowait(tmem + Lay::kTmU + tm_lane + 16 * b, pk);
-        }
-        uint32_t zero[16];
+        } else {  // entirely below the diagonal
 #pragma unroll
-        for (int e = 0; e < 16; ++e) zero[e] = 0u;
-#pragma unroll 1
-        for (int b = quad + 1; b < 4; ++b) umma::tmem_st16_nowait(tmem + Lay::kTmU + tm_lane + 16 * b, zero);
-        umma::tmem_wait_st();
-        umma::tc_fence_before();
-      } else {
-#pragma unroll
-        for (int c32 = 0; c32 < 4; ++c32) {
-          if (c32 > quad) {  // strictly above the diagonal: zeros (warp-uniform)
-#pragma unroll
-            for (int g = 0; g < 4; ++g)
-              *reinterpret_cast<uint4*>(sm + Lay::kP + ((t >> 3) * 16 + c32 * 4 + g) * 128 + (t & 7) * 16) =
-                  make_uint4(0, 0, 0, 0);
-            continue;
+          for (int e = 0; e < 32; ++e) {
+            float w0, w1;
+            poly2(u[2 * e], u[2 * e + 1], c0x2, c1x2, c2x2, &w0, &w1);
+            pk[e] = as_u32(__floats2bfloat162_rn(w0, w1));
           }
-          float u[32];
-          umma::tmem_ld32(tmem + Lay::kTmU + tm_lane + c32 * 32, u);
-          uint32_t pk[16];
-          poly_pack(u, c32, pk);
-#pragma unroll
-          for (int g = 0; g < 4; ++g)
-            *reinterpret_cast<uint4*>(sm + Lay::kP + ((t >> 3) * 16 + c32 * 4 + g) * 128 + (t & 7) * 16) =
-                make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
         }
-        umma::fence_async_smem();
-        umma::tc_fence_before();
+        if (two) umma::tmem_st32_nowait(tmem + Lay::kTmU + tm_lane + 16 * b, pk);
+        else umma::tmem_st16_nowait(tmem + Lay::kTmU + tm_lane + 16 * b, pk);
       }
+      uint32_t zero[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) zero[e] = 0u;
+#pragma unroll 1
+      for (int b = quad + 1; b < 4; ++b) umma::tmem_st16_nowait(tmem + Lay::kTmU + tm_lane + 16 * b, zero);
+      umma::tmem_wait_st();
+      umma::tc_fence_before();
       BASED_TC_TRACE(1, it);
       umma::mbar_arrive(bar_p);
     }
-    if constexpr (Lay::kSt && !kStateOnly) {
+    if constexpr (!kStateOnly) {
       // the final state is exported here, as soon as the last #5 completes,
       // while #2, #4 and the last output still run: this group writes features
       // 0-79, group F (idle by then) features 80-159.  Both groups take the
@@ -824,11 +711,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(qr);
       const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(kr);
       uint8_t* phik = sm + Lay::kPhiK + (it % Lay::kPhiKBuf) * 40960;
-      // With a single phiK buffer (and for the smem phiQ tile) wait until the
-      // previous chunk's #5 and #2 are done.  With two phiK buffers, this chunk's
-      // buffer was released by the wait of the previous iteration.
+      // phiK goes to buffer it % 2, last read by #5 of chunk c-2: complete before
+      // #1 of chunk c-1 (main pass, the wait below) or released by the bar_done
+      // wait of the previous iteration (state-only pass)
       BASED_TC_TRACE(0, it);
-      if (!Lay::kTm && it > 0 && !umma::mbar_wait(bar_m25, (it - 1) & 1)) { fail(); break; }
 
       // the Q/K tiles are rewritten once #1 of the previous chunk has read them
       if (!kStateOnly && it > 0 && !umma::mbar_wait(bar_u, (it - 1) & 1)) { fail(); break; }
@@ -865,18 +751,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // chunk c-1 (bar_done of its buffer), which also frees that buffer for
       // chunk c+1; bar_done cannot run ahead of this wait (its next phase needs
       // chunk c+1's #5, after this arrival).
-      if (kStateOnly && Lay::kTm && it > 0 &&
+      if (kStateOnly && it > 0 &&
           !umma::mbar_wait(bar_done + ((it - 1) & 1), ((it - 1) >> 1) & 1)) {
         fail();
         break;
       }
       umma::mbar_arrive(bar_qk);
-      if (!kStateOnly && Lay::kTm && it > 0 && !umma::mbar_wait(bar_m25, (it - 1) & 1)) {
+      if (!kStateOnly && it > 0 && !umma::mbar_wait(bar_m25, (it - 1) & 1)) {
         fail();
         break;
       }
       BASED_TC_TRACE(3, it);
-      // ---- phiQ (TMEM operand, or smem) ------------------------------------------------
+      // ---- phiQ (TMEM, the A operand of #2) ----------------------------------------------
       if (!kStateOnly) {
         __half2 XQ[8], YQ[8];
 #pragma unroll
@@ -886,24 +772,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
 #pragma unroll
         for (int m = 0; m < 8; ++m) YQ[m] = H2Ops::shift(XQ[m], XQ[(m + 1) & 7]);
-        if constexpr (Lay::kTm) {
-          umma::tc_fence_after();
-          uint32_t buf[32];
+        umma::tc_fence_after();
+        uint32_t buf[32];
 #pragma unroll
-          for (int ch = 0; ch < 20; ++ch) {
-            const uint4 v = tc_feature_chunk(XQ, YQ, q2, ch);
-            const int s4 = (ch * 4) & 31;
-            buf[s4] = v.x; buf[s4 + 1] = v.y; buf[s4 + 2] = v.z; buf[s4 + 3] = v.w;
-            if (ch == 7 || ch == 15) umma::tmem_st32_nowait(tmem + Lay::kTmQ + tm_lane + (ch - 7) * 4, buf);
-            if (ch == 19) umma::tmem_st16_nowait(tmem + Lay::kTmQ + tm_lane + 64, buf);
-          }
-          umma::tmem_wait_st();
-        } else {
-#pragma unroll
-          for (int ch = 0; ch < 20; ++ch)
-            *reinterpret_cast<uint4*>(sm + Lay::kPhiQ + ((t >> 3) * 20 + ch) * 128 + (t & 7) * 16) =
-                tc_feature_chunk(XQ, YQ, q2, ch);
+        for (int ch = 0; ch < 20; ++ch) {
+          const uint4 v = tc_feature_chunk(XQ, YQ, q2, ch);
+          const int s4 = (ch * 4) & 31;
+          buf[s4] = v.x; buf[s4 + 1] = v.y; buf[s4 + 2] = v.z; buf[s4 + 3] = v.w;
+          if (ch == 7 || ch == 15) umma::tmem_st32_nowait(tmem + Lay::kTmQ + tm_lane + (ch - 7) * 4, buf);
+          if (ch == 19) umma::tmem_st16_nowait(tmem + Lay::kTmQ + tm_lane + 64, buf);
         }
+        umma::tmem_wait_st();
       }
       if constexpr (!kStateOnly) {
         qr[0] = qn[0]; qr[1] = qn[1]; kr[0] = kn[0]; kr[1] = kn[1];
@@ -914,12 +793,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         umma::fence_async_smem();
         umma::tc_fence_before();
         BASED_TC_TRACE(4, it);
-        umma::mbar_arrive(bar_phiq);
+        umma::mbar_arrive(bar_go);
       }
     }
     // the ring's copies still in flight (rows past the segment) land before exit
     if constexpr (kStateOnly) umma::cp_async_wait<0>();
-    if constexpr (Lay::kSt && !kStateOnly) {
+    if constexpr (!kStateOnly) {
       // second half of the export (group P waits for the last #5 and decides)
       if (c_begin < c_end && umma::named_sync_all(2, 2 * kTcGroup, true)) {
         umma::tc_fence_after();
@@ -929,79 +808,35 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (!kStateOnly) {
     // ================= group E: epilogue of chunk c (output, fp16 state copy) =================
     const int t = tid - 2 * kTcGroup;  // TMEM lane of this thread (quadrant = warp - 8)
-    __nv_bfloat16* out = p.out + (size_t)bh_seq * L * DV;  // (v_split = 1 here)
-    // fp16 copy (scaled by sn) of the state rows this thread holds, as #2's B operand:
-    // tile 0 row t = feature t; tile 1 (M=64) lanes 0..15 of quadrants 0, 1 = features
-    // 128 + 16 * quad + lane
+    // fp16 copy (scaled by sn) of the state row this thread holds, as #2's B operand:
+    // row t of [S|z]^T (value column t, or z for t = DV) -> row t of the K-major
+    // copy; lanes past DV hold nothing (quadrant 3 skips the loads)
     int kk = 0;  // number of state copies handed off so far (buffer kk % kSBuf)
     auto copy_state = [&](float sn) {
       uint8_t* sbuf = sm + Lay::kS + (kk % Lay::kSBuf) * Lay::kSBytes;
-      if constexpr (Lay::kSt) {
-        // row t of [S|z]^T (value column t, or z for t = DV) -> row t of the
-        // K-major copy; lanes past DV hold nothing (quadrant 3 skips the loads)
-        if (quad == 3) return;
-        uint8_t* dst = sbuf + (t >> 3) * (kSymFP * 16) + (t & 7) * 16;
-        const uint32_t base = tmem + Lay::kTmS0 + tm_lane;
-        auto put8 = [&](const float* sv, int fg) {
-          uint32_t pk[4];
+      if (quad == 3) return;
+      uint8_t* dst = sbuf + (t >> 3) * (kSymFP * 16) + (t & 7) * 16;
+      const uint32_t base = tmem + Lay::kTmS0 + tm_lane;
+      auto put8 = [&](const float* sv, int fg) {
+        uint32_t pk[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            pk[e] = as_u32(__floats2half2_rn(sv[2 * e] * sn, sv[2 * e + 1] * sn));
-          if (t <= DV) *reinterpret_cast<uint4*>(dst + fg * 128) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        };
+        for (int e = 0; e < 4; ++e)
+          pk[e] = as_u32(__floats2half2_rn(sv[2 * e] * sn, sv[2 * e + 1] * sn));
+        if (t <= DV) *reinterpret_cast<uint4*>(dst + fg * 128) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      };
 #pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
-          float sv[80];
-          umma::tmem_ld80(base + 80 * h, sv);
+      for (int h = 0; h < 2; ++h) {
+        float sv[80];
+        umma::tmem_ld80(base + 80 * h, sv);
 #pragma unroll
-          for (int g = 0; g < 10; ++g) put8(sv + 8 * g, 10 * h + g);
-        }
-        return;
-      }
-      for (int tile = 0; tile < 2; ++tile) {
-        if (tile == 1 && (quad > 1)) break;
-        const int f = tile == 0 ? t : 128 + quad * 16 + lane;
-        const uint32_t base = tmem + (tile == 0 ? Lay::kTmS0 : Lay::kTmS1) + tm_lane;
-        auto put = [&](const float* sv, int j0) {
-          uint32_t pk[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            pk[e] = as_u32(__floats2half2_rn(sv[2 * e] * sn, sv[2 * e + 1] * sn));
-          *reinterpret_cast<uint4*>(sbuf + ((j0 >> 3) * 20 + (f >> 3)) * 128 + (f & 7) * 16) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        };
-        if constexpr (NG == 3) {
-          {
-            float sv[64];
-            umma::tmem_ld64(base, sv);
-            if (tile == 0 || lane < 16) {
-#pragma unroll
-              for (int j0 = 0; j0 < 64; j0 += 8) put(sv + j0, j0);
-            }
-          }
-          float sv[32];
-          umma::tmem_ld32(base + 64, sv);
-          if (tile == 1 && lane >= 16) continue;
-#pragma unroll
-          for (int j0 = 64; j0 < NA; j0 += 8) put(sv + j0 - 64, j0);
-        } else {
-#pragma unroll
-          for (int g = 0; g < NG; ++g) {
-            float sv[32];
-            umma::tmem_ld32(base + g * 32, sv);
-            if (tile == 1 && lane >= 16) continue;
-#pragma unroll
-            for (int h = 0; h < 4; ++h)
-              if (g * 32 + h * 8 < NA) put(sv + h * 8, g * 32 + h * 8);
-          }
-        }
+        for (int g = 0; g < 10; ++g) put8(sv + 8 * g, 10 * h + g);
       }
     };
     if (has_init) {
       // seed the TMEM state of a later segment with the sum of the earlier
       // partials: after linattn_partial_prefix_kernel, partial seg-1 holds it
       const float* part = p.partial + (size_t)bh * (p.n_seg - 1) * kSymFP * NA;
-      if (Lay::kSt && quad < 3) {
+      if (quad < 3) {
         // partials are [feature][value column]; this lane seeds row t of [S|z]^T
         const float* col0 = part + (size_t)(seg - 1) * kSymFP * NA + t;
 #pragma unroll 1
@@ -1012,118 +847,86 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           umma::tmem_st32(tmem + Lay::kTmS0 + tm_lane + g * 32, acc);
         }
       }
-      for (int tile = 0; tile < 2 && !Lay::kSt; ++tile) {
-        if (tile == 1 && quad > 1) break;
-        const int f = tile == 0 ? t : 128 + quad * 16 + (lane & 15);
-        const uint32_t base = tmem + (tile == 0 ? Lay::kTmS0 : Lay::kTmS1) + tm_lane;
-#pragma unroll
-        for (int g = 0; g < NG; ++g) {
-          float acc[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
-          if (tile == 0 || lane < 16) {
-            const float* row = part + ((size_t)(seg - 1) * kSymFP + f) * NA + g * 32;
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (g * 32 + i < NA) acc[i] += row[i];
-          }
-          umma::tmem_st32(base + g * 32, acc);
-        }
-      }
       copy_state(tc_chunk_scale((long long)c_begin * kTcChunk + kTcChunk));
       umma::fence_async_smem();
-      umma::tc_fence_before();
-      if (Lay::kTm) umma::mbar_arrive(bar_sread);
-      umma::mbar_arrive(bar_ss);
       ++kk;
     }
+    // The hand-off of chunk c-1 to #5 and #2 of chunk c (bar_go): before the first
+    // chunk it carries the seeded state and its copy, or nothing.
+    umma::tc_fence_before();
+    umma::mbar_arrive(bar_go);
+    // (thread 0) V loads this group issued, per stage: one issued (bit s) and the
+    // parity of the phase it completes
+    uint32_t v_issued = 0, v_par = 0;
+    int vstage = 0;  // V stage of chunk c
     for (int c = c_begin; c < c_end && !*abort_flag; ++c) {
       const int it = c - c_begin;
       const int t0 = c * kTcChunk;
-      const int n = min(kTcChunk, L - t0);
       const float sc = tc_chunk_scale((long long)t0 + kTcChunk);
-      if (Lay::kTm && c + 1 < c_end) {
+      if (c + 1 < c_end) {
         // the state after #5 of this chunk, copied while #2 and #4 still run
         if (!umma::mbar_wait(bar_m5, it & 1)) { fail(); break; }
         BASED_TC_TRACE(0, it);
         umma::tc_fence_after();
         copy_state(tc_chunk_scale((long long)t0 + 2 * kTcChunk));
         umma::fence_async_smem();
-        umma::tc_fence_before();
         BASED_TC_TRACE(1, it);
-        umma::mbar_arrive(bar_sread);
       }
       if (!umma::mbar_wait(bar_o, it & 1)) { fail(); break; }
       BASED_TC_TRACE(2, it);
       umma::tc_fence_after();
-      if constexpr (Lay::kTm) {
-        float o[64], den;
-        umma::tmem_ld64_1(tmem + Lay::kTmO + tm_lane, tmem + Lay::kTmO + tm_lane + DV, o, &den);
-        // O is in registers: #2 of the next chunk may overwrite it
-        umma::tc_fence_before();
-        if (c + 1 < c_end) {
-          umma::mbar_arrive(bar_ss);
-          ++kk;
-        }
-        BASED_TC_TRACE(3, it);
-        // y row t into the swizzled staging tile; one TMA store per chunk
-        uint8_t* ybuf = sm + Lay::kY;
-        if (t == 0) {  // the store of chunk c-1 has finished reading ybuf
-          umma::bulk_wait_read<0>();
-          umma::mbar_arrive(bar_yfree);
-        }
-        if (!umma::mbar_wait(bar_yfree, it & 1)) { fail(); break; }
-        const float inv = 1.0f / (den + p.eps * sc);
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint32_t pk[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            pk[e] = as_u32(__floats2bfloat162_rn(o[ch * 8 + 2 * e] * inv, o[ch * 8 + 2 * e + 1] * inv));
-          *reinterpret_cast<uint4*>(ybuf + t * 128 + ((ch ^ (t & 7)) << 4)) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        }
-      } else {
-        const float den = umma::tmem_ld1(tmem + Lay::kTmO + tm_lane + DV);
-        const float inv = 1.0f / (den + p.eps * sc);
-#pragma unroll
-        for (int g = 0; g < DV / 64; ++g) {
-          float o[64];
-          umma::tmem_ld64(tmem + Lay::kTmO + tm_lane + g * 64, o);
-          if (t < n) {
-            uint4* dst = reinterpret_cast<uint4*>(out + (size_t)(t0 + t) * DV + g * 64);
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-              uint32_t pk[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                pk[e] = as_u32(__floats2bfloat162_rn(o[ch * 8 + 2 * e] * inv, o[ch * 8 + 2 * e + 1] * inv));
-              dst[ch] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            }
-          }
-        }
-      }
-      if (!Lay::kTm && c + 1 < c_end) copy_state(tc_chunk_scale((long long)t0 + 2 * kTcChunk));
-      umma::fence_async_smem();
+      float o[64], den;
+      umma::tmem_ld64_1(tmem + Lay::kTmO + tm_lane, tmem + Lay::kTmO + tm_lane + DV, o, &den);
+      // O and the state are in registers and the copy is written: #5 and #2 of
+      // the next chunk may go
       umma::tc_fence_before();
-      if (!Lay::kTm && c + 1 < c_end) {  // O and the state read
-        umma::mbar_arrive(bar_ss);
+      if (c + 1 < c_end) {
+        umma::mbar_arrive(bar_go);
         ++kk;
       }
-      if constexpr (Lay::kTm) {
-        BASED_TC_TRACE(4, it);
-        umma::mbar_arrive(bar_yfull);
-        if (t == 0) {
-          if (!umma::mbar_wait(bar_yfull, it & 1)) { fail(); break; }
-          umma::tma_store_3d(&ymap, sm + Lay::kY, col0, t0, bh_seq);
-          umma::bulk_commit();
-        }
+      BASED_TC_TRACE(3, it);
+      // every MMA of chunk c is done: its V stage takes chunk c + kVBuf
+      if (t == 0 && c + Lay::kVBuf < c_end) {
+        const int cn = c + Lay::kVBuf;
+        const uint32_t par = static_cast<uint32_t>((cn - c_begin) / Lay::kVBuf) & 1u;
+        v_issued |= issue_v(cn, vstage) << vstage;
+        v_par = (v_par & ~(1u << vstage)) | (par << vstage);
+      }
+      vstage = vstage == Lay::kVBuf - 1 ? 0 : vstage + 1;
+      // y row t into the swizzled staging tile; one TMA store per chunk
+      uint8_t* ybuf = sm + Lay::kY;
+      if (t == 0) {  // the store of chunk c-1 has finished reading ybuf
+        umma::bulk_wait_read<0>();
+        umma::mbar_arrive(bar_yfree);
+      }
+      if (!umma::mbar_wait(bar_yfree, it & 1)) { fail(); break; }
+      const float inv = 1.0f / (den + p.eps * sc);
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          pk[e] = as_u32(__floats2bfloat162_rn(o[ch * 8 + 2 * e] * inv, o[ch * 8 + 2 * e + 1] * inv));
+        *reinterpret_cast<uint4*>(ybuf + t * 128 + ((ch ^ (t & 7)) << 4)) =
+            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      umma::fence_async_smem();
+      BASED_TC_TRACE(4, it);
+      umma::mbar_arrive(bar_yfull);
+      if (t == 0) {
+        if (!umma::mbar_wait(bar_yfull, it & 1)) { fail(); break; }
+        umma::tma_store_3d(&ymap, sm + Lay::kY, col0, t0, bh_seq);
+        umma::bulk_commit();
       }
     }
     BASED_TC_TRACE(5, 0);
     // the last output store has read its staging tile (its global writes
-    // complete with the grid)
-    if (Lay::kTm && t == 0) umma::bulk_wait_read<0>();
+    // complete with the grid), and an aborted run's V loads have landed (bounded)
+    if (t == 0) {
+      umma::bulk_wait_read<0>();
+      for (int sidx = 0; sidx < Lay::kVBuf; ++sidx)
+        if ((v_issued >> sidx) & 1u) umma::mbar_wait(bar_tma + sidx, (v_par >> sidx) & 1u);
+    }
     BASED_TC_TRACE(6, 0);
   }
 
@@ -1133,53 +936,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (!*abort_flag && warp >= 8 && warp < 12) {
     // ---- state out of TMEM (group E lanes): segment partials or the final export ----
     const int t = tid - 2 * kTcGroup;
-    if constexpr (Lay::kSt) {
-      // the main pass exported from group P already (right after its last #5)
-      if (kStateOnly || c_begin == c_end) export_kst(t);
-    }
-    for (int tile = 0; tile < 2 && !Lay::kSt; ++tile) {
-      if (tile == 1 && quad > 1) break;
-      const int f = tile == 0 ? t : 128 + quad * 16 + (lane & 15);
-      const bool mine = tile == 0 || lane < 16;
-      const uint32_t base = tmem + (tile == 0 ? Lay::kTmS0 : Lay::kTmS1) + tm_lane;
-      const bool any = has_init || c_begin < c_end;
-      int r0 = -1, r1 = -1;
-      float scale = 1.0f;
-      const int nrows = (mine && f < kSymFP && !kStateOnly) ? tc_feature_rows(f, &r0, &r1, &scale) : 0;
-#pragma unroll
-      for (int g = 0; g < NG; ++g) {
-        float s[32];
-        umma::tmem_ld32(base + g * 32, s);
-        if (!any) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) s[i] = 0.0f;
-        }
-        if (!mine) continue;
-        if (kStateOnly) {
-          float* row = p.partial + (((size_t)bh * (p.n_seg - 1) + seg) * kSymFP + f) * NA + g * 32;
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (g * 32 + i < NA) row[i] = s[i];
-        } else if (seg == p.n_seg - 1) {
-          float* skv = p.state_kv ? p.state_kv + (size_t)bh_seq * kF * DV : nullptr;
-          float* sk = p.state_k ? p.state_k + (size_t)bh_seq * kF : nullptr;
-          for (int r = 0; r < nrows; ++r) {
-            const int row = r == 0 ? r0 : r1;
-            if (skv) {
-#pragma unroll
-              for (int i4 = 0; i4 < 8; ++i4) {
-                const int j = g * 32 + 4 * i4;
-                if (j < DV)
-                  *reinterpret_cast<float4*>(skv + (size_t)row * DV + j) =
-                      make_float4(s[4 * i4] * scale, s[4 * i4 + 1] * scale,
-                                  s[4 * i4 + 2] * scale, s[4 * i4 + 3] * scale);
-              }
-            }
-            if (sk && DV / 32 == g) sk[row] = s[0] * scale;
-          }
-        }
-      }
-    }
+    // the main pass exported from groups P and F already (right after its last #5)
+    if (kStateOnly || c_begin == c_end) export_kst(t);
   }
   umma::tc_fence_before();
   __syncthreads();
