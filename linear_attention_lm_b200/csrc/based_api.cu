@@ -7,6 +7,7 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 #include <stdint.h>
+#include <string.h>
 
 #include "based.h"
 #include "common.cuh"
@@ -145,6 +146,25 @@ bool make_rows_map(CUtensorMap* m, const void* base, int cols, int L, int BH, in
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Output map of one per-head projection: y as [B*H][L][D] bf16, boxes of 128
+// rows x min(D, 64) columns, swizzled by the box row's width (16 bytes: none).
+bool make_head_out_map(CUtensorMap* m, void* y, int D, int L, int BH) {
+  auto enc = encode_tiled();
+  if (!enc) return false;
+  const int bw = D < 64 ? D : 64;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)L, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)D * 2 * (cuuint64_t)L};
+  cuuint32_t box[3] = {(cuuint32_t)bw, (cuuint32_t)kPjM, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUtensorMapSwizzle sw = bw == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : bw == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                : bw == 16 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                           : CU_TENSOR_MAP_SWIZZLE_NONE;
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, y, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int device_sm_count() {
@@ -327,6 +347,15 @@ based_status_t launch_proj(const void* x, const void* w, ProjParams p, cudaStrea
   } else {
     hm = xm;  // unused
   }
+  // per-head outputs whose heads tile a 128-column half leave by TMA stores
+  ProjYMaps ym;
+  memset(&ym, 0, sizeof(ym));
+  if (Mode == kProjHeads) {
+    for (int g = 0; g < p.n_out; ++g)
+      if (kPjNHalf % p.D[g] == 0 &&
+          !make_head_out_map(&ym.m[g], p.y[g], p.D[g], p.L, (p.M / p.L) * p.H))
+        return BASED_ERR_CUDA;
+  }
   auto kern = proj_tc_kernel<Mode>;
   if (!set_smem(kern, PjLayout<Mode>::kSmem)) return BASED_ERR_CUDA;
   p.n_tiles_n = p.N / kPjN;
@@ -354,7 +383,7 @@ based_status_t launch_proj(const void* x, const void* w, ProjParams p, cudaStrea
   const long long pairs = tiles < max_clusters ? tiles : max_clusters;
   cfg.gridDim = dim3(2 * (unsigned)pairs, 1, 1);
   cfg.numAttrs = 2;
-  if (cudaLaunchKernelEx(&cfg, kern, xm, wm, hm, p) != cudaSuccess) return BASED_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, xm, wm, hm, ym, p) != cudaSuccess) return BASED_ERR_CUDA;
   return launch_status();
 }
 

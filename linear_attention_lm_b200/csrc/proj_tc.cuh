@@ -27,7 +27,13 @@
 // CTA (one thread) issues four M=256/N=256/K=16 MMAs per block into one of two
 // TMEM accumulators, so the epilogue of tile k overlaps the main loop of tile
 // k+1; warps 2-9 run the epilogue on the CTA's own 128 rows (warps w and w+4
-// share TMEM lane quadrant w mod 4 and take one half of the 256 columns each).  For BaseConv the producer also loads the CTA's input rows
+// share TMEM lane quadrant w mod 4 and take one half of the 256 columns each).
+// Per-head outputs leave by TMA: a head's 128 rows of one sequence are one box
+// of its [B*H, L, D] output, so each half writes its 128 columns into a
+// swizzled staging tile in shared memory and one thread stores them, a box per
+// head (or per 64 columns of a head); a tile whose rows cross a sequence end,
+// or a head width that does not divide 128, falls back to 16-byte stores from
+// every thread.  For BaseConv the producer also loads the CTA's input rows
 // [m0-8, m0+128) x [n0, n0+256) (the convolution's reach) into shared memory,
 // once the previous tile's epilogue has released them.
 #pragma once
@@ -52,7 +58,7 @@ enum ProjMode { kProjHeads = 0, kBaseConv = 1 };
 
 template <int Mode>
 struct PjLayout {
-  static constexpr int kStages = Mode == kBaseConv ? 4 : 6;
+  static constexpr int kStages = Mode == kBaseConv ? 4 : 5;
   static constexpr int kStageA = kPjM * kPjK * 2;                 // 16 KiB
   static constexpr int kStageB = kPjNHalf * kPjK * 2;             // 16 KiB
   static constexpr uint32_t kTxPair = 2u * (kStageA + kStageB);   // both CTAs' bytes
@@ -62,14 +68,25 @@ struct PjLayout {
   static constexpr int kHaloBlock = kPjHaloRows * 128;
   static constexpr int kHaloBytes = Mode == kBaseConv ? 4 * kHaloBlock : 0;
   // BaseConv: the tile's taps, transposed to [tap][column], and its bias
-  static constexpr int kTaps = kHalo + kHaloBytes;
+  // per-head outputs: one staging tile per half, [boxes][128 rows][box width]
+  static constexpr int kStg = kHalo + kHaloBytes;
+  static constexpr int kStgHalf = kPjM * kPjNHalf * 2;                       // 32 KiB
+  static constexpr int kStgBytes = Mode == kProjHeads ? 2 * kStgHalf : 0;
+  static constexpr int kTaps = kStg + kStgBytes;
   static constexpr int kBias = kTaps + (Mode == kBaseConv ? kPjMaxTaps * kPjN * 4 : 0);
   static constexpr int kBar = kBias + (Mode == kBaseConv ? kPjN * 4 : 0);
   static constexpr int kBytes = kBar + 256;
   static constexpr size_t kSmem = kBytes + 1024;
-  static_assert(kB % 1024 == 0 && kHalo % 1024 == 0 && kHaloBlock % 1024 == 0,
+  static_assert(kB % 1024 == 0 && kHalo % 1024 == 0 && kHaloBlock % 1024 == 0 &&
+                    kStg % 1024 == 0,
                 "swizzled tiles are 1024-byte aligned");
   static_assert(kSmem <= 232448, "shared memory budget");
+};
+
+// Output tensor maps of the per-head projections: y_g as [B*H][L][D] with
+// boxes of 128 rows x min(D, 64) columns, swizzled by the box row's width.
+struct ProjYMaps {
+  CUtensorMap m[kPjMaxOut];
 };
 
 struct ProjParams {
@@ -92,7 +109,8 @@ template <int Mode>
 __global__ void __launch_bounds__(kPjThreads, 1)
     proj_tc_kernel(const __grid_constant__ CUtensorMap xmap,
                    const __grid_constant__ CUtensorMap wmap,
-                   const __grid_constant__ CUtensorMap hmap, const ProjParams p) {
+                   const __grid_constant__ CUtensorMap hmap,
+                   const __grid_constant__ ProjYMaps ymaps, const ProjParams p) {
   using Lay = PjLayout<Mode>;
   constexpr int S = Lay::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -245,11 +263,23 @@ __global__ void __launch_bounds__(kPjThreads, 1)
     const int half = (warp - 2) >> 2;        // columns [128 half, 128 half + 128)
     const int et = (warp - 2) * 32 + lane;   // index among the epilogue threads
     const uint32_t aempty0 = umma::cluster_addr(bar_aempty, 0);
+    // the thread that stores this half's staging tile
+    const bool issuer = (et & (kPjEpiThreads / 2 - 1)) == 0;
+    uint8_t* stg = sm + Lay::kStg + half * Lay::kStgHalf;
     for (int k = 0; k < n_mine && !*abort_flag; ++k) {
       const int a = k & 1;
       int m0, n0;
       tile_at(k, &m0, &n0);
-      if (!umma::mbar_wait(bar_afull + a, (k >> 1) & 1)) { fail(); break; }
+      const bool ok_a = umma::mbar_wait(bar_afull + a, (k >> 1) & 1);
+      if (Mode == kProjHeads) {
+        // the half decides together (a named barrier must see all 128 threads),
+        // once the previous tile's stores have read the staging tile
+        if (issuer) umma::bulk_wait_read<0>();
+        if (!umma::named_sync_all(1 + half, kPjEpiThreads / 2, ok_a)) { fail(); break; }
+      } else if (!ok_a) {
+        fail();
+        break;
+      }
       if (Mode == kBaseConv && !umma::mbar_wait(bar_hfull, k & 1)) { fail(); break; }
       umma::tc_fence_after();
       float* tapsT = reinterpret_cast<float*>(sm + Lay::kTaps);
@@ -274,6 +304,15 @@ __global__ void __launch_bounds__(kPjThreads, 1)
       const int nb = n0 - p.col_begin[og];
       const int m = m0 + r;
       const int b = m / p.L, t = m - (m / p.L) * p.L;
+      // TMA stores: the CTA's 128 rows lie in one sequence and heads tile the half
+      const int t_first = m0 % p.L;
+      const bool tma_out = Mode == kProjHeads && m0 < p.M && t_first + kPjM <= p.L &&
+                           kPjNHalf % Dg == 0;
+      // staging tile: boxes of bw columns; row r of a box is rb bytes, its 16-byte
+      // chunk c at position c ^ ((r >> sh) & (rb / 16 - 1)) (the tensor map's swizzle)
+      const int bw = Dg < 64 ? Dg : 64, rb = 2 * bw;
+      const int sh = rb == 128 ? 0 : (rb == 64 ? 1 : 2);
+      const int cmask = rb / 16 - 1;
 #pragma unroll 1
       for (int c32 = 4 * half; c32 < 4 * half + 4; ++c32) {
         float acc[32];
@@ -325,19 +364,46 @@ __global__ void __launch_bounds__(kPjThreads, 1)
             const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
             pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
           }
-          *reinterpret_cast<uint4*>(yo + dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          if (tma_out) {
+            const int ch = cl - half * kPjNHalf;  // column within the half
+            const int bx = ch / bw, c = (ch - bx * bw) >> 3;
+            *reinterpret_cast<uint4*>(stg + bx * (rb * kPjM) + r * rb +
+                                      ((c ^ ((r >> sh) & cmask)) << 4)) =
+                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          } else {
+            *reinterpret_cast<uint4*>(yo + dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
         }
       }
       // accumulator a is read: one arrival per warp on the even CTA's barrier
       umma::tc_fence_before();
       __syncwarp();
       if (lane == 0) umma::mbar_arrive_cluster(aempty0 + 8u * a);
+      if (tma_out) {
+        // the staging tile is written: one thread stores a box per head (or per
+        // 64 columns of a head), [d0, d0 + bw) x rows [t_first, t_first + 128)
+        umma::fence_async_smem();
+        umma::named_sync(1 + half, kPjEpiThreads / 2);
+        if (issuer) {
+          const int b0 = m0 / p.L;
+          for (int bx = 0; bx < kPjNHalf / bw; ++bx) {
+            const int col = nb + half * kPjNHalf + bx * bw;  // column within the projection
+            const int hh = col / Dg;
+            umma::tma_store_3d(&ymaps.m[og], stg + bx * (rb * kPjM), col - hh * Dg, t_first,
+                               b0 * p.H + hh);
+          }
+          umma::bulk_commit();
+        }
+      }
       if (Mode == kBaseConv) {
         umma::mbar_arrive(bar_hempty);
         umma::mbar_arrive(bar_tfree);
       }
     }
   }
+  // the last stores have read their staging tiles
+  if (Mode == kProjHeads && warp >= 2 && ((tid - 64) & (kPjEpiThreads / 2 - 1)) == 0)
+    umma::bulk_wait_read<0>();
   umma::tc_fence_before();
   __syncthreads();
   // every MMA of the pair has completed before either CTA releases its TMEM

@@ -84,6 +84,9 @@ def test_proj_heads_full_size_sampled():
     (1, 100, 256, 16, (16, 16, 64, 64, 64, 64)),  # one pair tile, the odd CTA's rows all past M
     (3, 257, 192, 32, (8, 64)),                    # ragged M over several pair tiles
     (2, 300, 1024, 16, (64, 16, 64, 16)),          # projections of different widths interleaved
+    (2, 384, 256, 32, (8, 32, 128)),               # rows in whole 128-row blocks of a sequence
+                                                   # leave by TMA: boxes 16, 64 and 2 x 128
+                                                   # bytes wide (no swizzle, 64B, 128B)
 ])
 def test_proj_heads_multi_matches_oracle(B, L, d_model, H, Ds):
     """Every output of one multi-projection launch against the oracle's
