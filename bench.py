@@ -78,8 +78,9 @@ def replica_rate(units_per_rank: float, ms: float, world: int) -> float:
 # since the capture
 # ---------------------------------------------------------------------------
 
-_KERNEL_SOURCES = {"linattn_prefill": "linattn_tc.cuh", "window_attn": "window_tcp.cuh",
-                   "decode_step": "decode.cuh"}
+_KERNEL_SOURCES = {"linattn_prefill": ("linattn_tc.cuh",),
+                   "window_attn": ("window_tcp.cuh", "window_softmax.cuh"),
+                   "decode_step": ("decode.cuh",)}
 
 
 def measured_traffic(kernel, workload):
@@ -93,7 +94,7 @@ def measured_traffic(kernel, workload):
         if entry["workload"] != workload:
             return None
         h = hashlib.sha256()
-        for name in (_KERNEL_SOURCES[kernel], "umma.cuh", "common.cuh"):
+        for name in (*_KERNEL_SOURCES[kernel], "umma.cuh", "common.cuh"):
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(f.read())
         if h.hexdigest() != entry["sources_sha256"]:

@@ -24,6 +24,7 @@
 
 #include "common.cuh"
 #include "umma.cuh"
+#include "window_softmax.cuh"
 
 namespace based {
 
@@ -154,30 +155,11 @@ __global__ void __launch_bounds__(kWtThreads, 1)
     umma::tmem_ld64_32(tmem + Lay::kTmS + tm_lane + cb, tmem + Lay::kTmS + tm_lane + cb + 64, sv);
     // staged column c holds key s = t0 - 64 + c; row t sees s in [max(0, t-W+1), t]
     const int lo = max(max(r + 1, 64 - t0), t - W + 1 - (t0 - 64)) - cb;
-    const int hi = lane + 64;
     const float scale = rsqrtf((float)DH) * 1.4426950408889634f;  // 1/sqrt(dh) * log2(e)
-    // four interleaved partial maxima / sums keep the dependent chains short
-    float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-    for (int i = 0; i < 96; ++i)
-      if (i >= lo && (i < 64 || i <= hi)) mp[i & 3] = fmaxf(mp[i & 3], sv[i]);
-    const float ms = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])) * scale;
-    float lp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-    for (int i = 0; i < 96; ++i) {
-      const float e = ex2_approx(fmaf(sv[i], scale, -ms));
-      sv[i] = (i >= lo && (i < 64 || i <= hi)) ? e : 0.0f;
-      lp[i & 3] += sv[i];
-    }
-    l_row = (lp[0] + lp[1]) + (lp[2] + lp[3]);  // >= 1: the row maximum contributes exp2(0)
     // P (bf16 pairs, column j = keys 2j, 2j+1) replaces S in this lane: the band
     // of quadrant w lands in columns [16w, 16w + 48), the rest of [0, 96) is zero
     uint32_t pk[48], zero[32];
-#pragma unroll
-    for (int j = 0; j < 48; ++j) {
-      const __nv_bfloat162 b2 = __floats2bfloat162_rn(sv[2 * j], sv[2 * j + 1]);
-      pk[j] = *reinterpret_cast<const uint32_t*>(&b2);
-    }
+    l_row = window_band_softmax(sv, lane, lo, W == 64 && t0 >= 64, scale, pk);
 #pragma unroll
     for (int j = 0; j < 32; ++j) zero[j] = 0u;
     const uint32_t prow = tmem + Lay::kTmS + tm_lane;

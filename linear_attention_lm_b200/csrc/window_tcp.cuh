@@ -16,6 +16,7 @@
 
 #include "common.cuh"
 #include "umma.cuh"
+#include "window_softmax.cuh"
 
 // Optional per-tile event stamps for performance analysis (a build may define
 // BASED_WP_TRACE(event, tile); by default the marks compile to nothing).
@@ -207,26 +208,8 @@ __global__ void __launch_bounds__(kWpThreads, 1)
         umma::tmem_ld64_32(sbase + cb, sbase + cb + 64, sv);
         // staged column c holds key t0 - 64 + c; row t sees [max(0, t - W + 1), t]
         const int lo = max(max(r + 1, 64 - t0), t - W + 1 - (t0 - 64)) - cb;
-        const int hi = lane + 64;
-        float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int i = 0; i < 96; ++i)
-          if (i >= lo && (i < 64 || i <= hi)) mp[i & 3] = fmaxf(mp[i & 3], sv[i]);
-        const float ms = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])) * scale;
-        float lp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-        for (int i = 0; i < 96; ++i) {
-          const float e = ex2_approx(fmaf(sv[i], scale, -ms));
-          sv[i] = (i >= lo && (i < 64 || i <= hi)) ? e : 0.0f;
-          lp[i & 3] += sv[i];
-        }
-        l_row = (lp[0] + lp[1]) + (lp[2] + lp[3]);
         uint32_t pk[48], zero[32];
-#pragma unroll
-        for (int e = 0; e < 48; ++e) {
-          const __nv_bfloat162 b2 = __floats2bfloat162_rn(sv[2 * e], sv[2 * e + 1]);
-          pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
-        }
+        l_row = window_band_softmax(sv, lane, lo, W == 64 && t0 >= 64, scale, pk);
 #pragma unroll
         for (int e = 0; e < 32; ++e) zero[e] = 0u;
         if (quad == 0) {
