@@ -207,16 +207,29 @@ __global__ void __launch_bounds__(kWgThreads, 1)
     const float scale = rsqrtf((float)DH) * 1.4426950408889634f;  // 1/sqrt(dh) * log2(e)
     float pv[96];
     umma::tmem_ld64_32(tmem + Lay::kTmS + tm_lane + cb, tmem + Lay::kTmS + tm_lane + cb + 64, pv);
+    // scores outside the window become -inf once, so the max and the
+    // exponentials need no mask (exp2(-inf) = 0); when every row sees a whole
+    // window of 64 keys (lo = lane + 1) only the two ragged ends are tested
+    if (W == 64 && t0 >= 64) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (i <= lane) pv[i] = -INFINITY;
+#pragma unroll
+      for (int i = 65; i < 96; ++i)
+        if (i > hi) pv[i] = -INFINITY;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 96; ++i)
+        if (i < lo || i > hi) pv[i] = -INFINITY;
+    }
     float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-    for (int i = 0; i < 96; ++i)
-      if (i >= lo && i <= hi) mp[i & 3] = fmaxf(mp[i & 3], pv[i]);
+    for (int i = 0; i < 96; ++i) mp[i & 3] = fmaxf(mp[i & 3], pv[i]);
     const float ms = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])) * scale;
     float lp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
     for (int i = 0; i < 96; ++i) {
-      const float e = ex2_approx(fmaf(pv[i], scale, -ms));
-      pv[i] = (i >= lo && i <= hi) ? e : 0.0f;
+      pv[i] = ex2_approx(fmaf(pv[i], scale, -ms));
       lp[i & 3] += pv[i];
     }
     const float l = (lp[0] + lp[1]) + (lp[2] + lp[3]);  // >= 1 (the maximum contributes 1)
@@ -375,11 +388,24 @@ __global__ void __launch_bounds__(kWgThreads, 1)
     const float scale = rsqrtf((float)DH) * 1.4426950408889634f;
     float pv[96];
     umma::tmem_ld64_32(tmem + Lay::kTmS + tm_lane + cb, tmem + Lay::kTmS + tm_lane + cb + 64, pv);
+    // pairs outside the window become -inf once (exp2(-inf) = 0, and every
+    // staged statistic is finite); with W = 64 and all 192 staged queries inside
+    // the sequence, hi = lane + 63 and only the two ragged ends are tested
+    if (W == 64 && s0 + kWgN <= L) {
 #pragma unroll
-    for (int i = 0; i < 96; ++i) {
-      const float e = ex2_approx(fmaf(pv[i], scale, -st_m[cb + i])) * st_l[cb + i];
-      pv[i] = (i >= lo && i <= hi) ? e : 0.0f;
+      for (int i = 0; i < 32; ++i)
+        if (i < lane) pv[i] = -INFINITY;
+#pragma unroll
+      for (int i = 64; i < 96; ++i)
+        if (i > lane + 63) pv[i] = -INFINITY;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 96; ++i)
+        if (i < lo || i > hi) pv[i] = -INFINITY;
     }
+#pragma unroll
+    for (int i = 0; i < 96; ++i)
+      pv[i] = ex2_approx(fmaf(pv[i], scale, -st_m[cb + i])) * st_l[cb + i];
     float dp[96];
     umma::tmem_ld64_32(tmem + Lay::kTmP + tm_lane + cb, tmem + Lay::kTmP + tm_lane + cb + 64, dp);
     uint32_t pk[48], dk[48];
