@@ -280,24 +280,43 @@ def make_sets(w, dev, min_sets=2):
 
 def time_prefill(lab, w, sets, steps, warmup, warm, dev, world):
     """Time `steps` prefill steps (linear attention with state export, then
-    window attention), with per-kernel event pairs; returns (total ms,
-    per-step linear ms, per-step window ms, launches per step)."""
+    window attention); returns (total ms, linear ms and window ms per launch
+    from event pairs inside the step, launches per step, the same two per-launch
+    times with each kernel launched back to back on its own)."""
     ws_bytes = lab.based_linattn_workspace_bytes(w.B, w.H, w.L, w.d, w.dv,
                                                  lab.BASED_BF16 if w.dtype == "bf16" else lab.BASED_F32)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     n_sets = len(sets)
 
-    def step(i, ev=None):
+    def lin(i):
         x, o = sets[i % n_sets]
-        if ev is not None:
-            ev[0].record()
         lab.based_linattn_fwd(x["q"], x["k"], x["v"], o["y"], w.eps, o["S"], o["z"],
                               workspace=ws[:ws_bytes] if ws_bytes else None)
+
+    def win(i):
+        x, o = sets[i % n_sets]
+        lab.based_window_attn_fwd(x["wq"], x["wk"], x["wv"], o["yw"], w.window)
+
+    def step(i, ev=None):
+        if ev is not None:
+            ev[0].record()
+        lin(i)
         if ev is not None:
             ev[1].record()
-        lab.based_window_attn_fwd(x["wq"], x["wk"], x["wv"], o["yw"], w.window)
+        win(i)
         if ev is not None:
             ev[2].record()
+
+    def chained(fn):
+        # K launches of one kernel back to back, each a dependent launch of the
+        # previous one as inside the step; one event pair around all of them
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for i in range(steps):
+            fn(i)
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps
 
     warm()
     for i in range(warmup):
@@ -314,8 +333,11 @@ def time_prefill(lab, w, sets, steps, warmup, warm, dev, world):
         step(i)
     stop.record()
     torch.cuda.synchronize()
-    # the per-kernel times: the same K steps again, with an event pair around
-    # each kernel (an event between two kernels ends that overlap)
+    # the per-kernel times: the same K steps again with an event pair around
+    # each kernel (an event between two kernels ends their launch overlap, so
+    # each time includes its kernel's launch latency); and, for context, each
+    # kernel's K launches back to back on their own (launches overlapped, but
+    # each kernel's output write-back now competes with its next launch)
     for i in range(steps):
         step(i, evs[i])
     torch.cuda.synchronize()
@@ -323,11 +345,13 @@ def time_prefill(lab, w, sets, steps, warmup, warm, dev, world):
         torch.distributed.barrier()
     t_lin = sum(e[0].elapsed_time(e[1]) for e in evs) / steps
     t_win = sum(e[1].elapsed_time(e[2]) for e in evs) / steps
+    t_lin_chain = chained(lin)
+    t_win_chain = chained(win)
     # the split path adds a state-only pass, and with more than two segments a
     # running sum over their partials (160 x 80 fp32 per 64-column slice)
     n_part = ws_bytes // (w.B * w.H * (w.dv // 64) * 160 * 80 * 4) if ws_bytes else 0
     launches = 2 + (1 if n_part >= 1 else 0) + (1 if n_part >= 2 else 0)
-    return start.elapsed_time(stop), t_lin, t_win, launches
+    return start.elapsed_time(stop), t_lin, t_win, launches, t_lin_chain, t_win_chain
 
 
 def run_ours(args, rank, world, dev):
@@ -350,8 +374,8 @@ def run_ours(args, rank, world, dev):
         # steps as well: a timed region of a few ms holds at most one sample
         clk.mark("t_start")
         warm()
-        elapsed_ms, t_lin, t_win, launches = time_prefill(lab, w, sets, args.steps, args.warmup,
-                                                          lambda: warm(30.0), dev, world)
+        elapsed_ms, t_lin, t_win, launches, t_lin_p, t_win_p = time_prefill(
+            lab, w, sets, args.steps, args.warmup, lambda: warm(30.0), dev, world)
         clk.mark("t_stop")
     assert lab.based_get_device_error() == 0
     elapsed_max = max_over_ranks(elapsed_ms, dev, world)
@@ -362,11 +386,18 @@ def run_ours(args, rank, world, dev):
     dom = max(kern, key=lambda k: kern[k][1])
     b, t_ms = kern[dom]
     roofline = hbm_roofline(dom, b, t_ms, peaks, workload=w.name)
+    chain = {"linattn_prefill": t_lin_p, "window_attn": t_win_p}
     roofline["per_kernel_ms"] = {k: round(v[1], 5) for k, v in kern.items()}
-    roofline["per_kernel_timing"] = ("CUDA event pairs around each kernel, over a second pass "
-                                     "of the same K steps right after the timed one")
+    roofline["per_kernel_timing"] = (
+        "CUDA event pairs around each kernel, over a second pass of the same K steps right "
+        "after the timed one (each pair includes its kernel's launch latency, which the "
+        "step itself overlaps with the previous kernel); per_kernel_ms_chained: each "
+        "kernel's K launches back to back on their own, on the same inputs")
     roofline["per_kernel_frac"] = {k: round(v[0] / (v[1] / 1e3) / 1e9 / peaks["hbm_gbs"], 4)
                                    for k, v in kern.items()}
+    roofline["per_kernel_ms_chained"] = {k: round(v, 5) for k, v in chain.items()}
+    roofline["per_kernel_frac_chained"] = {
+        k: round(kern[k][0] / (v / 1e3) / 1e9 / peaks["hbm_gbs"], 4) for k, v in chain.items()}
     roofline["linattn_prefill_tensor"] = tensor_side(w, t_lin, peaks)
     del sets
 
@@ -416,7 +447,8 @@ def run_other_prefill(args, lab, w, dev, world, peaks, warm):
     per kernel over rotating input sets; tokens/s = B L / (K1 + K2)."""
     sets, _ = make_sets(w, dev)
     n = max(10, min(args.steps, 200))
-    total_ms, t_lin, t_win, launches = time_prefill(lab, w, sets, n, args.warmup, warm, dev, world)
+    total_ms, t_lin, t_win, launches, t_lin_p, t_win_p = time_prefill(lab, w, sets, n, args.warmup,
+                                                                        warm, dev, world)
     assert lab.based_get_device_error() == 0
     del sets
     ms = max_over_ranks(total_ms / n, dev, world)
@@ -424,6 +456,8 @@ def run_other_prefill(args, lab, w, dev, world, peaks, warm):
                        tensor_side(w, t_lin, peaks) if w.dtype == "bf16" else None,
                        workload=w.name)
     win = hbm_roofline("window_attn", window_bytes(w), t_win, peaks, workload=w.name)
+    lin["ms_chained"] = round(t_lin_p, 5)
+    win["ms_chained"] = round(t_win_p, 5)
     out = {"workload": prefill_config(w, world)["workload"],
            "tokens_per_s": round(world * w.B * w.L / (ms / 1e3), 1),
            "ms_per_step": round(ms, 5), "steps": n, "launches_per_step": launches,
