@@ -63,6 +63,13 @@ inline bool set_smem(K kernel, size_t bytes) {
 // Launch as a programmatic dependent of the previous kernel in the stream: the
 // kernel's CTAs may start (and run their set-up) while that kernel finishes;
 // the kernel waits for it (griddepcontrol.wait) before touching global memory.
+// TMEM: a kernel that allocates TMEM before that wait (the prefill, the
+// persistent window kernel, the projections) must never share an SM with a CTA
+// of the previous kernel that has yet to allocate, which would wait for columns
+// held by a CTA waiting for it.  Those kernels take more than half of an SM's
+// shared memory, so no other kernel's CTA runs beside them; the kernels whose
+// CTAs share SMs (the backward kernels, the d_h = 128 window kernel) wait first
+// and allocate after.
 template <typename... KArgs, typename... Args>
 bool launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
                       cudaStream_t st, Args... args) {

@@ -22,10 +22,10 @@
 //     pass 2, key tiles j = 0..i:  U = Q_i K_j^T, G = dN_i V_j^T (K = d_v)
 //                                  E = mask((G + dD)(1 + u'))
 //                                  dQ += E K_j           (N = 16)
-//   kernel KV (one CTA per 128-key tile j), query tiles i = j..last:
-//                                  U^T = K_j Q_i^T, G^T = V_j dN_i^T
+//   kernel KV (one CTA per 128-key tile j), query tiles i = j..last, at d_v = 64
+//   in two blocks of 64 queries h: U^T = K_j Q_ih^T, G^T = V_j dN_ih^T
 //                                  W^T, E^T as above (dD_t from the workspace)
-//                                  dV += W^T dN_i, dK += E^T Q_i
+//                                  dV += W^T dN_ih, dK += E^T Q_ih
 //
 // Operand precision: q, k, v, dy are the bf16 inputs; W, E and dN are rounded
 // to bf16 for the MMAs; D, dD, the accumulators and the outputs are fp32.
@@ -69,6 +69,13 @@ struct BtLayout {
   // and each pass-2 step's dQ contribution lands in U's columns [64, 80) (free
   // once E is packed into [0, 64)) and is added up in registers
   static constexpr int kQCols = 256, kQTmN = 128, kQTmDq = 64;
+  // kernel KV at d_v = 64 takes each query tile in two blocks of kKvQ = 64
+  // queries: U^T, G^T of a block (64 columns each), the d_v accumulator and the
+  // 16-wide one make 208 columns, so two of its CTAs share an SM; at d_v = 128
+  // the accumulator alone is 128 columns and one CTA per SM takes whole tiles
+  static constexpr int kKvQ = DV == 64 ? 64 : 128;
+  static constexpr int kKvTmU = 0, kKvTmG = kKvQ, kKvTmAcc = 2 * kKvQ, kKvTmAcc16 = 2 * kKvQ + DV;
+  static constexpr int kKvCols = kKvTmAcc16 + 16 <= 256 ? 256 : 512;
   static_assert(kV % 1024 == 0 && kDN % 1024 == 0 && kVk % 1024 == 0 && kDNk % 1024 == 0,
                 "swizzled tiles need 1024-byte alignment");
 };
@@ -390,7 +397,7 @@ __global__ void __launch_bounds__(kBtThreads, DV == 64 ? 2 : 1)
 // kernel KV: dk, dv from the workspace (dN bf16, dD fp32)
 // ---------------------------------------------------------------------------
 template <int DV>
-__global__ void __launch_bounds__(kBtThreads, 1)
+__global__ void __launch_bounds__(kBtThreads, DV == 64 ? 2 : 1)
     linattn_bwd_tc_kv_kernel(const __grid_constant__ CUtensorMap vmap,
                              const __grid_constant__ CUtensorMap dnmap, const BtParams p) {
   using Lay = BtLayout<DV>;
@@ -427,7 +434,7 @@ __global__ void __launch_bounds__(kBtThreads, 1)
     umma::fence_mbar_init();
   }
   if (warp == 0) {
-    umma::tmem_alloc(tmem_slot, 512);
+    umma::tmem_alloc(tmem_slot, Lay::kKvCols);
     umma::tmem_relinquish();
   }
   if (!issuer) {  // K_j rows
@@ -488,84 +495,100 @@ __global__ void __launch_bounds__(kBtThreads, 1)
       if (step + 1 < n_steps) load_q(ti + 1);
     }
     if (__syncthreads_or(failed)) break;
-    if (issuer && lane == 0) {
-      if (!umma::mbar_wait(bar_dn + b, (step >> 1) & 1)) {
-        fail();
-      } else {
-        --inflight;
-        umma::tc_fence_after();
-        const uint32_t sQ = umma::smem_u32(sm + Lay::kQk + b * 4096);
-        const uint32_t sD = umma::smem_u32(sm + Lay::kDNk + b * Lay::kVTile);
-        umma::mma_bf16(tmem + Lay::kTmU, umma::desc_kmajor_none(sK, 0, 16),
-                       umma::desc_kmajor_none(sQ, 0, 16), umma::idesc_bf16(128, 128, false, false), 0);
+    const uint32_t sQ = umma::smem_u32(sm + Lay::kQk + b * 4096);
+    const uint32_t sQm = umma::smem_u32(sm + Lay::kQm + b * 4096);
+    const uint32_t sD = umma::smem_u32(sm + Lay::kDNk + b * Lay::kVTile);
+    // the blocks of kKvQ queries (m1, m2 complete once per block: phase
+    // kNQ step + h); a failure stops every thread at the same barrier, in both loops
+    constexpr int QW = Lay::kKvQ, kNQ = kBtT / QW;
+    bool stop = false;
+    for (int h = 0; h < kNQ; ++h) {
+      const uint32_t ph = static_cast<uint32_t>(kNQ * step + h) & 1u;
+      if (issuer && lane == 0) {
+        if (h == 0 && !umma::mbar_wait(bar_dn + b, (step >> 1) & 1)) {
+          fail();
+        } else {
+          if (h == 0) --inflight;
+          umma::tc_fence_after();
+          // U^T = K_j Q_ih^T: block h's rows of the K-major Q tile start QW h / 8
+          // core matrix rows (256 B each) in; G^T = V_j dN_ih^T: they start QW h
+          // rows (128 B each) into each 64-column block of dN
+          umma::mma_bf16(tmem + Lay::kKvTmU, umma::desc_kmajor_none(sK, 0, 16),
+                         umma::desc_kmajor_none(sQ + 32u * QW * h, 0, 16),
+                         umma::idesc_bf16(128, QW, false, false), 0);
 #pragma unroll
-        for (int k0 = 0; k0 < DV; k0 += 16)  // G^T = V_j dN_i^T
-          umma::mma_bf16(tmem + Lay::kTmG, umma::desc_kmajor_sw128(sV, k0, kBtT),
-                         umma::desc_kmajor_sw128(sD, k0, kBtT),
-                         umma::idesc_bf16(128, 128, false, false), k0 > 0);
-        umma::mma_commit(bar_m1);
-        // the next step's dN tile goes to the other buffer (the previous step's
-        // MMAs are complete)
-        if (step + 1 < n_steps) {
-          issue_dn(step + 1);
-          ++inflight;
-        }
-      }
-    }
-    if (!issuer) {
-      if (!__all_sync(0xffffffffu, umma::mbar_wait(bar_m1, step & 1))) {
-        fail();
-      } else {
-        umma::tc_fence_after();
-        const float* dd = reinterpret_cast<const float*>(sm + Lay::kDD + b * 512);
-        const int lo_c = diag ? row : 0;  // queries ti*128 + c with c < lo_c come before key s
-#pragma unroll 1
-        for (int c32 = 0; c32 < 4; ++c32) {
-          float u[32], g[32];
-          umma::tmem_ld32(tmem + Lay::kTmU + tm_lane + 32 * c32, u);
-          umma::tmem_ld32(tmem + Lay::kTmG + tm_lane + 32 * c32, g);
-          uint32_t pw[16], pe[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            float w2[2], e2[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int c = 32 * c32 + 2 * e + h;
-              const float up = 0.25f * u[2 * e + h];
-              const bool live = c >= lo_c;
-              w2[h] = live ? fmaf(0.5f * up, up, 1.0f + up) : 0.0f;
-              e2[h] = live ? (g[2 * e + h] + dd[c]) * (1.0f + up) : 0.0f;
-            }
-            pw[e] = bt_pack(w2[0], w2[1]);
-            pe[e] = bt_pack(e2[0], e2[1]);
+          for (int k0 = 0; k0 < DV; k0 += 16)
+            umma::mma_bf16(tmem + Lay::kKvTmG, umma::desc_kmajor_sw128(sV, k0, kBtT),
+                           umma::desc_kmajor_sw128(sD + 128u * QW * h, k0, kBtT),
+                           umma::idesc_bf16(128, QW, false, false), k0 > 0);
+          umma::mma_commit(bar_m1);
+          // the next step's dN tile goes to the other buffer (the previous step's
+          // MMAs are complete)
+          if (h == 0 && step + 1 < n_steps) {
+            issue_dn(step + 1);
+            ++inflight;
           }
-          // W^T pairs over U^T's columns [16 c32, +16), E^T pairs over G^T's
-          umma::tmem_st16_nowait(tmem + Lay::kTmU + tm_lane + 16 * c32, pw);
-          umma::tmem_st16_nowait(tmem + Lay::kTmG + tm_lane + 16 * c32, pe);
         }
-        umma::tmem_wait_st();
       }
-      umma::tc_fence_before();
-    }
-    if (__syncthreads_or(failed)) break;
-    if (issuer && lane == 0) {
-      umma::tc_fence_after();
-      const uint32_t sD = umma::smem_u32(sm + Lay::kDNk + b * Lay::kVTile);
-      const uint32_t sQm = umma::smem_u32(sm + Lay::kQm + b * 4096);
+      if (!issuer) {
+        if (!__all_sync(0xffffffffu, umma::mbar_wait(bar_m1, ph))) {
+          fail();
+        } else {
+          umma::tc_fence_after();
+          const float* dd = reinterpret_cast<const float*>(sm + Lay::kDD + b * 512) + QW * h;
+          // queries ti*128 + QW h + c with c < lo_c come before key s
+          const int lo_c = diag ? row - QW * h : 0;
+#pragma unroll 1
+          for (int c32 = 0; c32 < QW / 32; ++c32) {
+            float u[32], g[32];
+            umma::tmem_ld32(tmem + Lay::kKvTmU + tm_lane + 32 * c32, u);
+            umma::tmem_ld32(tmem + Lay::kKvTmG + tm_lane + 32 * c32, g);
+            uint32_t pw[16], pe[16];
 #pragma unroll
-      for (int ks = 0; ks < kBtT / 16; ++ks) {
-        const uint32_t acc = (step > 0 || ks > 0) ? 1u : 0u;
-        umma::mma_ts(tmem + Lay::kTmAcc, tmem + Lay::kTmU + ks * 8,
-                     umma::desc_mnmajor_sw128(sD, ks * 16, kBtT),
-                     umma::idesc_bf16(128, DV, false, true), acc);  // dV += W^T dN_i
-        umma::mma_ts(tmem + Lay::kTmAcc16, tmem + Lay::kTmG + ks * 8,
-                     umma::desc_mnmajor_none(sQm, ks * 16, kBtT),
-                     umma::idesc_bf16(128, 16, false, true), acc);  // dK += E^T Q_i
+            for (int e = 0; e < 16; ++e) {
+              float w2[2], e2[2];
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                const int c = 32 * c32 + 2 * e + hh;
+                const float up = 0.25f * u[2 * e + hh];
+                const bool live = c >= lo_c;
+                w2[hh] = live ? fmaf(0.5f * up, up, 1.0f + up) : 0.0f;
+                e2[hh] = live ? (g[2 * e + hh] + dd[c]) * (1.0f + up) : 0.0f;
+              }
+              pw[e] = bt_pack(w2[0], w2[1]);
+              pe[e] = bt_pack(e2[0], e2[1]);
+            }
+            // W^T pairs over U^T's columns [16 c32, +16), E^T pairs over G^T's
+            umma::tmem_st16_nowait(tmem + Lay::kKvTmU + tm_lane + 16 * c32, pw);
+            umma::tmem_st16_nowait(tmem + Lay::kKvTmG + tm_lane + 16 * c32, pe);
+          }
+          umma::tmem_wait_st();
+        }
+        umma::tc_fence_before();
       }
-      umma::mma_commit(bar_m2);
+      if (__syncthreads_or(failed)) {
+        stop = true;
+        break;
+      }
+      if (issuer && lane == 0) {
+        umma::tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < QW / 16; ++ks) {
+          const uint32_t acc = (step > 0 || h > 0 || ks > 0) ? 1u : 0u;
+          const int kq = QW * h + 16 * ks;  // query (K) index within the tile
+          umma::mma_ts(tmem + Lay::kKvTmAcc, tmem + Lay::kKvTmU + ks * 8,
+                       umma::desc_mnmajor_sw128(sD, kq, kBtT),
+                       umma::idesc_bf16(128, DV, false, true), acc);  // dV += W^T dN_ih
+          umma::mma_ts(tmem + Lay::kKvTmAcc16, tmem + Lay::kKvTmG + ks * 8,
+                       umma::desc_mnmajor_none(sQm, kq, kBtT),
+                       umma::idesc_bf16(128, 16, false, true), acc);  // dK += E^T Q_ih
+        }
+        umma::mma_commit(bar_m2);
+      }
+      if (!umma::mbar_wait(bar_m2, ph)) fail();
+      umma::tc_fence_after();
     }
-    if (!umma::mbar_wait(bar_m2, step & 1)) fail();
-    umma::tc_fence_after();
+    if (stop) break;
   }
   const bool any_failed = __syncthreads_or(failed);
   // ---- dk, dv of this lane's key (TMEM loads by whole warps, stores by live rows) ----
@@ -576,7 +599,7 @@ __global__ void __launch_bounds__(kBtThreads, 1)
 #pragma unroll
     for (int blk = 0; blk < DV / 64; ++blk) {
       float a[64];
-      umma::tmem_ld64(tmem + Lay::kTmAcc + tm_lane + 64 * blk, a);
+      umma::tmem_ld64(tmem + Lay::kKvTmAcc + tm_lane + 64 * blk, a);
       if (live) {
 #pragma unroll
         for (int c4 = 0; c4 < 16; ++c4)
@@ -584,7 +607,7 @@ __global__ void __launch_bounds__(kBtThreads, 1)
       }
     }
     float g[32];
-    umma::tmem_ld32(tmem + Lay::kTmAcc16 + tm_lane, g);
+    umma::tmem_ld32(tmem + Lay::kKvTmAcc16 + tm_lane, g);
     if (live) {
       float4* dkd = reinterpret_cast<float4*>(p.dk + (bh * L + s) * kD);
 #pragma unroll
@@ -601,7 +624,7 @@ __global__ void __launch_bounds__(kBtThreads, 1)
     umma::mbar_wait(bar_v, 0);
   }
   __syncthreads();
-  if (warp == 0) umma::tmem_dealloc(tmem, 512);
+  if (warp == 0) umma::tmem_dealloc(tmem, Lay::kKvCols);
 }
 
 }  // namespace based
