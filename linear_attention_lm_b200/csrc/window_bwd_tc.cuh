@@ -98,6 +98,32 @@ __device__ __forceinline__ uint32_t wg_pack(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// Packed pairs of fp32 (each lane of an f32x2 operation rounds like its scalar
+// form, so these give the scalar results, two at a time).
+__device__ __forceinline__ uint64_t wg_f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void wg_unf2(uint64_t v, float* lo, float* hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(*lo), "=f"(*hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t wg_fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t wg_mul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t wg_add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 // Row r of an fp32 accumulator [128 x DH] in TMEM, times `scale`, to row `row`
 // of a [L, DH] fp32 tensor (skipped past L).
 template <int DH>
@@ -226,27 +252,46 @@ __global__ void __launch_bounds__(kWgThreads, 1)
 #pragma unroll
     for (int i = 0; i < 96; ++i) mp[i & 3] = fmaxf(mp[i & 3], pv[i]);
     const float ms = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])) * scale;
-    float lp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    // weights, row sum, delta = sum P dP and dS = P (dP - delta), in packed pairs
+    // (pair j feeds partial sums 2 (j & 1) + {0, 1}, as a scalar loop over i & 3)
+    const uint64_t sc2 = wg_f2(scale, scale), nm2 = wg_f2(-ms, -ms);
+    uint64_t lp2[2] = {wg_f2(0.0f, 0.0f), wg_f2(0.0f, 0.0f)};
 #pragma unroll
-    for (int i = 0; i < 96; ++i) {
-      pv[i] = ex2_approx(fmaf(pv[i], scale, -ms));
-      lp[i & 3] += pv[i];
+    for (int j = 0; j < 48; ++j) {
+      float a, b;
+      wg_unf2(wg_fma2(wg_f2(pv[2 * j], pv[2 * j + 1]), sc2, nm2), &a, &b);
+      pv[2 * j] = ex2_approx(a);
+      pv[2 * j + 1] = ex2_approx(b);
+      lp2[j & 1] = wg_add2(lp2[j & 1], wg_f2(pv[2 * j], pv[2 * j + 1]));
     }
-    const float l = (lp[0] + lp[1]) + (lp[2] + lp[3]);  // >= 1 (the maximum contributes 1)
+    float lq[4];
+    wg_unf2(lp2[0], &lq[0], &lq[1]);
+    wg_unf2(lp2[1], &lq[2], &lq[3]);
+    const float l = (lq[0] + lq[1]) + (lq[2] + lq[3]);  // >= 1 (the maximum contributes 1)
     const float inv_l = 1.0f / l;
     float dp[96];
     umma::tmem_ld64_32(tmem + Lay::kTmP + tm_lane + cb, tmem + Lay::kTmP + tm_lane + cb + 64, dp);
-    float dl[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    const uint64_t il2 = wg_f2(inv_l, inv_l);
+    uint64_t dl2[2] = {wg_f2(0.0f, 0.0f), wg_f2(0.0f, 0.0f)};
 #pragma unroll
-    for (int i = 0; i < 96; ++i) {
-      pv[i] *= inv_l;
-      dl[i & 3] = fmaf(pv[i], dp[i], dl[i & 3]);
+    for (int j = 0; j < 48; ++j) {
+      const uint64_t p2 = wg_mul2(wg_f2(pv[2 * j], pv[2 * j + 1]), il2);
+      wg_unf2(p2, &pv[2 * j], &pv[2 * j + 1]);
+      dl2[j & 1] = wg_fma2(p2, wg_f2(dp[2 * j], dp[2 * j + 1]), dl2[j & 1]);
     }
-    const float delta = (dl[0] + dl[1]) + (dl[2] + dl[3]);
+    float dq4[4];
+    wg_unf2(dl2[0], &dq4[0], &dq4[1]);
+    wg_unf2(dl2[1], &dq4[2], &dq4[3]);
+    const float delta = (dq4[0] + dq4[1]) + (dq4[2] + dq4[3]);
+    const uint64_t nd2 = wg_f2(-delta, -delta);
     uint32_t pk[48];
 #pragma unroll
-    for (int j = 0; j < 48; ++j)
-      pk[j] = wg_pack(pv[2 * j] * (dp[2 * j] - delta), pv[2 * j + 1] * (dp[2 * j + 1] - delta));
+    for (int j = 0; j < 48; ++j) {
+      float a, b;
+      wg_unf2(wg_mul2(wg_f2(pv[2 * j], pv[2 * j + 1]),
+                      wg_add2(wg_f2(dp[2 * j], dp[2 * j + 1]), nd2)), &a, &b);
+      pk[j] = wg_pack(a, b);
+    }
     wg_store_band(tmem + Lay::kTmS + tm_lane, warp, pk);
     umma::tmem_wait_st();
     if (live) {
