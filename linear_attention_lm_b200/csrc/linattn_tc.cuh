@@ -601,22 +601,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         else umma::tmem_ld32(tmem + Lay::kTmU + tm_lane + 32 * b, u);
         const int lim = row - 32 * b;  // keys 32b + j with j > lim lie in the future
         uint32_t pk[32];
-        if (b + 1 >= quad) {  // the pair holds the diagonal block: causal mask
+        // the causal mask is a no-op below the diagonal (lim >= 63 there): one
+        // loop body for every pair keeps this group's code small
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            float w0, w1;
-            poly2(u[2 * e], u[2 * e + 1], c0x2, c1x2, c2x2, &w0, &w1);
-            if (2 * e > lim) w0 = 0.0f;
-            if (2 * e + 1 > lim) w1 = 0.0f;
-            pk[e] = as_u32(__floats2bfloat162_rn(w0, w1));
-          }
-        } else {  // entirely below the diagonal
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            float w0, w1;
-            poly2(u[2 * e], u[2 * e + 1], c0x2, c1x2, c2x2, &w0, &w1);
-            pk[e] = as_u32(__floats2bfloat162_rn(w0, w1));
-          }
+        for (int e = 0; e < 32; ++e) {
+          float w0, w1;
+          poly2(u[2 * e], u[2 * e + 1], c0x2, c1x2, c2x2, &w0, &w1);
+          if (2 * e > lim) w0 = 0.0f;
+          if (2 * e + 1 > lim) w1 = 0.0f;
+          pk[e] = as_u32(__floats2bfloat162_rn(w0, w1));
         }
         if (two) umma::tmem_st32_nowait(tmem + Lay::kTmU + tm_lane + 16 * b, pk);
         else umma::tmem_st16_nowait(tmem + Lay::kTmU + tm_lane + 16 * b, pk);
