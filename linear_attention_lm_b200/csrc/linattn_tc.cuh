@@ -141,6 +141,12 @@ struct TcParams {
   int ld_v;
 };
 
+// A bounded wait gave up: record the timeout and tell the other groups to stop.
+__device__ __noinline__ void tc_fail(volatile int* abort_flag) {
+  record_device_error(BASED_ERR_TIMEOUT);
+  *abort_flag = 1;
+}
+
 // Power-of-two scale applied to the fp16 state copy (and to P) for the chunk
 // ending at t_end, keeping every state entry (|z_0| <= t) below 2^15.
 __device__ __forceinline__ float tc_chunk_scale(long long t_end) {
@@ -338,10 +344,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tm_lane = static_cast<uint32_t>(quad * 32) << 16;
   BASED_TC_TRACE(15, 0);
-  auto fail = [&]() {
-    record_device_error(BASED_ERR_TIMEOUT);
-    *abort_flag = 1;
-  };
+  // (the failure path is a call, so that its code stays out of the hot loops,
+  // which share the instruction cache with three other warps per sub-partition)
+  auto fail = [&]() { tc_fail(abort_flag); };
   // Export of [S|z]^T in two steps.  export_stage: TMEM -> shared memory as
   // [feature][value column | z] (stride DV + 4) and the map from the 273 output
   // rows to features; run by the 128 threads of one warp group (t = index in
