@@ -725,10 +725,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int m = 0; m < 8; ++m) XK[m] = __hmul2(k2[m], halfk);
 #pragma unroll
         for (int m = 0; m < 8; ++m) YK[m] = H2Ops::shift(XK[m], XK[(m + 1) & 7]);
+        // rows past the end of the sequence were loaded as zeros, so all their
+        // features but the constant one (chunk 0) are zero already
 #pragma unroll
         for (int ch = 0; ch < 20; ++ch)
           *reinterpret_cast<uint4*>(phik + (ch * 16 + (t >> 3)) * 128 + (t & 7) * 16) =
-              live ? tc_feature_chunk(XK, YK, k2, ch) : make_uint4(0, 0, 0, 0);
+              (ch > 0 || live) ? tc_feature_chunk(XK, YK, k2, ch) : make_uint4(0, 0, 0, 0);
 
         if (!kStateOnly) {
           uint8_t* qrow = sm + Lay::kQ + ((t >> 3) * 2) * 128 + (t & 7) * 16;
