@@ -6,10 +6,14 @@
 //   num_t  = phi(q_t)^T S + sum_s A_ts v_s,  den_t = phi(q_t).z + sum_s A_ts
 //   y_t    = num_t / (den_t + eps)
 //   S     += phi(K_c)^T V_c,  z += sum_s phi(k_s)                (state update)
-// with S (273 x 64 fp32) and z resident in shared memory for the whole
-// sequence.  One CTA per (b, h, 64-column slice of d_v).  The feature rows use
-// a pitch of 273 floats (odd), so a warp reading one feature of 32 different
-// tokens touches 32 distinct banks.
+// with S (273 x 16 fp32) and z resident in shared memory for the whole
+// sequence.  One CTA per (b, h, 16-column slice of d_v): the slices of one
+// sequence share nothing but the scores, which are cheap, so a short sequence
+// still spreads over several SMs.  A uses the closed form phi(q).phi(k) =
+// 1 + u/4 + u^2/32 with u = q.k (an identity of the map above, 16 terms instead
+// of 273); the read-out and the state use all 273 features.  The feature rows
+// use a pitch of 273 floats (odd), so a warp reading one feature of 32
+// different tokens touches 32 distinct banks.
 #pragma once
 
 #include "common.cuh"
@@ -17,13 +21,15 @@
 namespace based {
 
 constexpr int kSimtChunk = 32;
-constexpr int kSimtCols = 64;
+constexpr int kSimtCols = 16;
 constexpr int kSimtThreads = 256;
+constexpr int kSimtXP = kD + 1;  // pitch of the staged q, k rows (odd: the score loop's
+                                 // 32 lanes read 32 different rows without bank conflicts)
 
 __host__ __device__ constexpr size_t linattn_simt_smem_bytes() {
   return sizeof(float) * (size_t)(kF * kSimtCols + 276 + 2 * kSimtChunk * kF +
                                   kSimtChunk * kSimtCols + kSimtChunk * 33 + kSimtChunk +
-                                  2 * kSimtChunk * kD);
+                                  2 * kSimtChunk * kSimtXP);
 }
 
 template <typename T>
@@ -43,8 +49,8 @@ __global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
   float* vs = fk + C * kF;         // [32][64]
   float* A = vs + C * NC;          // [32][33]
   float* den = A + C * 33;         // [32]
-  float* xq = den + C;             // [32][16]
-  float* xk = xq + C * kD;         // [32][16]
+  float* xq = den + C;             // [32][17]
+  float* xk = xq + C * kSimtXP;    // [32][17]
 
   const int tid = threadIdx.x;
   const int bh = blockIdx.x, col0 = blockIdx.y * NC;
@@ -61,9 +67,9 @@ __global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
     const int n = min(C, L - t0);
     __syncthreads();  // previous chunk's state update is complete
     for (int i = tid; i < C * kD; i += NT) {
-      const int r = i / kD;
-      xq[i] = r < n ? to_f32(q[(size_t)t0 * kD + i]) : 0.0f;
-      xk[i] = r < n ? to_f32(k[(size_t)t0 * kD + i]) : 0.0f;
+      const int r = i / kD, c = i - r * kD;
+      xq[r * kSimtXP + c] = r < n ? to_f32(q[(size_t)t0 * kD + i]) : 0.0f;
+      xk[r * kSimtXP + c] = r < n ? to_f32(k[(size_t)t0 * kD + i]) : 0.0f;
     }
     for (int i = tid; i < C * NC; i += NT) {
       const int r = i / NC, c = i - r * NC;
@@ -72,25 +78,22 @@ __global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
     __syncthreads();
     for (int i = tid; i < C * kF; i += NT) {
       const int r = i / kF, f = i - r * kF;
-      fq[i] = phi_feature(xq + r * kD, f);
-      fk[i] = phi_feature(xk + r * kD, f);
+      fq[i] = phi_feature(xq + r * kSimtXP, f);
+      fk[i] = phi_feature(xk + r * kSimtXP, f);
     }
     __syncthreads();
-    // intra-chunk scores, causal mask s <= t (four partial sums: the loop is
-    // latency-bound on one chain)
+    // intra-chunk scores, causal mask s <= t, in closed form from u = q_t . k_s
     for (int i = tid; i < C * C; i += NT) {
       const int t = i / C, s = i - t * C;
       float a = 0.0f;
       if (s <= t) {
-        const float* a_row = fq + t * kF;
-        const float* b_row = fk + s * kF;
-        float a4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll 4
-        for (int f = 0; f < kF - 1; f += 4) {
+        const float* qr = xq + t * kSimtXP;
+        const float* kr = xk + s * kSimtXP;
+        float u2[2] = {0.0f, 0.0f};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) a4[e] = fmaf(a_row[f + e], b_row[f + e], a4[e]);
-        }
-        a = fmaf(a_row[kF - 1], b_row[kF - 1], (a4[0] + a4[1]) + (a4[2] + a4[3]));
+        for (int d = 0; d < kD; ++d) u2[d & 1] = fmaf(qr[d], kr[d], u2[d & 1]);
+        const float u = u2[0] + u2[1];
+        a = fmaf(u, fmaf(u, 0.03125f, 0.25f), 1.0f);
       }
       A[t * 33 + s] = a;
     }
