@@ -315,8 +315,8 @@ based_status_t launch_window_simt(const void* q, const void* k, const void* v, v
   const long long nblk = (L + kWinQ - 1) / kWinQ;
   if (nblk > 0x7fffffffLL || BH > 65535) return BASED_ERR_UNSUPPORTED;
   dim3 grid((unsigned)nblk, (unsigned)BH);
-  kern<<<grid, kWinQ, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
-                                  static_cast<const T*>(v), static_cast<T*>(out), L, dh, W);
+  kern<<<grid, kWinThreads, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
+                                        static_cast<const T*>(v), static_cast<T*>(out), L, dh, W);
   return launch_status();
 }
 

@@ -4,66 +4,78 @@
 // sliding window (size 64) for local token interactions.  For query t the keys
 // are s in [max(0, t-W+1), t], scores q_t.k_s / sqrt(d_head).
 //
-// This is the fp32 path (fp32 inputs, fp32 arithmetic): one CTA of 64 threads
-// per block of 64 queries; the 127 key/value rows the block can touch
-// ([t0-63, t0+63]) and its 64 query rows are staged once in shared memory with
-// a row pitch of d_head+4 floats, so the float4 reads of 8 consecutive threads
-// (consecutive rows) fall in distinct banks.
+// This is the fp32 path (fp32 inputs, fp32 arithmetic): one CTA of 256 threads
+// per block of 64 queries, four threads per query.  The 127 key/value rows the
+// block can touch ([t0-63, t0+63]) and its 64 query rows are staged once in
+// shared memory with a row pitch of d_head+4 floats, so the float4 reads of 8
+// consecutive rows fall in distinct banks.  Thread `sub` of a query scores keys
+// sub, sub+4, ... (16 of the 64), the four combine max and sum by shuffles, the
+// weights go to shared memory, and each thread then forms a quarter of the
+// output columns over all 64 keys: a quarter of the serial work of one thread
+// per query.
 #pragma once
 
 #include "common.cuh"
 
 namespace based {
 
-constexpr int kWinQ = 64;          // queries per CTA
+constexpr int kWinQ = 64;                // queries per CTA
+constexpr int kWinSub = 4;               // threads per query
+constexpr int kWinThreads = kWinQ * kWinSub;
 constexpr int kWinRows = 2 * kWinQ - 1;  // key/value rows staged per CTA
+constexpr int kWinPP = kWinQ + 1;        // pitch of the weight rows (odd: no bank conflicts)
 
 __host__ __device__ constexpr size_t window_simt_smem_bytes(int dh) {
-  return sizeof(float) * (size_t)(2 * kWinRows + kWinQ) * (size_t)(dh + 4);
+  return sizeof(float) * ((size_t)(2 * kWinRows + kWinQ) * (size_t)(dh + 4) +
+                          (size_t)kWinQ * kWinPP);
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kWinQ) window_simt_kernel(const T* __restrict__ q,
-                                                            const T* __restrict__ k,
-                                                            const T* __restrict__ v,
-                                                            T* __restrict__ out, int L, int dh,
-                                                            int W) {
+__global__ void __launch_bounds__(kWinThreads) window_simt_kernel(const T* __restrict__ q,
+                                                                  const T* __restrict__ k,
+                                                                  const T* __restrict__ v,
+                                                                  T* __restrict__ out, int L,
+                                                                  int dh, int W) {
   extern __shared__ __align__(16) float smem[];
   const int ld = dh + 4;
   float* ks = smem;
   float* vs = ks + kWinRows * ld;
   float* qs = vs + kWinRows * ld;
+  float* ps = qs + kWinQ * ld;  // [64][65] weights of each query over its 64 staged keys
   const int tid = threadIdx.x;
   const int t0 = blockIdx.x * kWinQ;
   const size_t base = (size_t)blockIdx.y * L * dh;
   q += base; k += base; v += base; out += base;
 
-  for (int idx = tid; idx < kWinRows * dh; idx += kWinQ) {
+  for (int idx = tid; idx < kWinRows * dh; idx += kWinThreads) {
     const int r = idx / dh, c = idx - r * dh;
     const int g = t0 - (kWinQ - 1) + r;
     const bool ok = g >= 0 && g < L;
     ks[r * ld + c] = ok ? to_f32(k[(size_t)g * dh + c]) : 0.0f;
     vs[r * ld + c] = ok ? to_f32(v[(size_t)g * dh + c]) : 0.0f;
   }
-  for (int idx = tid; idx < kWinQ * dh; idx += kWinQ) {
+  for (int idx = tid; idx < kWinQ * dh; idx += kWinThreads) {
     const int r = idx / dh, c = idx - r * dh;
     const int g = t0 + r;
     qs[r * ld + c] = g < L ? to_f32(q[(size_t)g * dh + c]) : 0.0f;
   }
   __syncthreads();
-  const int t = t0 + tid;
-  if (t >= L) return;
+  const int qi = tid / kWinSub, sub = tid % kWinSub;  // query of the block, key / column share
+  const int t = t0 + qi;
   const int lo = max(0, t - W + 1);
   const float scale = rsqrtf((float)dh);
-  const float4* q4 = reinterpret_cast<const float4*>(qs + tid * ld);
-  float sc[kWinQ];
+  const float4* q4 = reinterpret_cast<const float4*>(qs + qi * ld);
+  // scores of keys j = sub + 4 jj: key s = t - 63 + j, staged row qi + j
+  constexpr int kPer = kWinQ / kWinSub;
+  float sc[kPer];
   float m = -INFINITY;
 #pragma unroll
-  for (int j = 0; j < kWinQ; ++j) {
-    const int s = t - (kWinQ - 1) + j;  // key index; its staged row is tid + j
+  for (int jj = 0; jj < kPer; ++jj) {
+    const int j = sub + kWinSub * jj;
+    const int s = t - (kWinQ - 1) + j;
     float a = -INFINITY;
     if (s >= lo) {
-      const float4* k4 = reinterpret_cast<const float4*>(ks + (tid + j) * ld);
+      const float4* k4 = reinterpret_cast<const float4*>(ks + (qi + j) * ld);
       // four independent chains: the loop is latency-bound on one
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int c = 0; c < dh / 4; ++c) {
@@ -75,28 +87,39 @@ __global__ void __launch_bounds__(kWinQ) window_simt_kernel(const T* __restrict_
       }
       a = ((acc.x + acc.y) + (acc.z + acc.w)) * scale;
     }
-    sc[j] = a;
+    sc[jj] = a;
     m = fmaxf(m, a);
   }
+  // the four threads of a query are consecutive lanes of one warp
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
   float sum = 0.0f;
 #pragma unroll
-  for (int j = 0; j < kWinQ; ++j) {
-    const float e = (t - (kWinQ - 1) + j >= lo) ? expf(sc[j] - m) : 0.0f;
-    sc[j] = e;
+  for (int jj = 0; jj < kPer; ++jj) {
+    const int j = sub + kWinSub * jj;
+    const float e = (t - (kWinQ - 1) + j >= lo) ? expf(sc[jj] - m) : 0.0f;
+    ps[qi * kWinPP + j] = e;
     sum += e;
   }
+  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+  sum += __shfl_xor_sync(0xffffffffu, sum, 2);
   const float inv = 1.0f / sum;
-  for (int c = 0; c < dh / 4; ++c) {
+  __syncwarp();  // the query's four threads have written its 64 weights
+  if (t >= L) return;
+  // output columns [4 c4, 4 c4 + 4) for c4 = sub, sub + 4, ... over all 64 keys
+  const float* pr = ps + qi * kWinPP;
+  for (int c4 = sub; c4 < dh / 4; c4 += kWinSub) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
+#pragma unroll 8
     for (int j = 0; j < kWinQ; ++j) {
-      const float4 y = reinterpret_cast<const float4*>(vs + (tid + j) * ld)[c];
-      acc.x = fmaf(sc[j], y.x, acc.x);
-      acc.y = fmaf(sc[j], y.y, acc.y);
-      acc.z = fmaf(sc[j], y.z, acc.z);
-      acc.w = fmaf(sc[j], y.w, acc.w);
+      const float p = pr[j];
+      const float4 y = reinterpret_cast<const float4*>(vs + (qi + j) * ld)[c4];
+      acc.x = fmaf(p, y.x, acc.x);
+      acc.y = fmaf(p, y.y, acc.y);
+      acc.z = fmaf(p, y.z, acc.z);
+      acc.w = fmaf(p, y.w, acc.w);
     }
-    T* o = out + (size_t)t * dh + 4 * c;
+    T* o = out + (size_t)t * dh + 4 * c4;
     o[0] = from_f32<T>(acc.x * inv);
     o[1] = from_f32<T>(acc.y * inv);
     o[2] = from_f32<T>(acc.z * inv);
