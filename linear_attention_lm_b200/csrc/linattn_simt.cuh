@@ -6,14 +6,25 @@
 //   num_t  = phi(q_t)^T S + sum_s A_ts v_s,  den_t = phi(q_t).z + sum_s A_ts
 //   y_t    = num_t / (den_t + eps)
 //   S     += phi(K_c)^T V_c,  z += sum_s phi(k_s)                (state update)
-// with S (273 x 8 fp32) and z resident in shared memory for the whole
-// sequence.  One CTA per (b, h, 8-column slice of d_v): the slices of one
-// sequence share nothing but the scores, which are cheap, so a short sequence
-// still spreads over several SMs.  A uses the closed form phi(q).phi(k) =
-// 1 + u/4 + u^2/32 with u = q.k (an identity of the map above, 16 terms instead
-// of 273); the read-out and the state use all 273 features.  The feature rows
-// use a pitch of 273 floats (odd), so a warp reading one feature of 32
-// different tokens touches 32 distinct banks.
+// One CTA per (b, h, 8-column slice of d_v): the slices of one sequence share
+// nothing but the scores, which are cheap, so a short sequence still spreads
+// over several SMs.
+//
+// Two exact identities of the feature map shrink the work:
+//  - A uses the closed form phi(q).phi(k) = 1 + u/4 + u^2/32 with u = q.k
+//    (16 terms instead of 273);
+//  - the quadratic features x_i x_j and x_j x_i are equal, so rows (i, j) and
+//    (j, i) of S and z are equal too.  The CTA keeps 153 rows (constant,
+//    16 linear, the 136 pairs i <= j) and weights an off-diagonal pair twice on
+//    the query side, which gives phi(q)^T S exactly; the export writes every
+//    pair row to both of its places in the 273-row state.
+// Every feature is a product x[a] * x[b] * scale over the staged row extended
+// by a 1 (column 16): (16, 16) is the constant, (i, 16) the linear features.
+//
+// Per chunk two barriers: (1) the features of q and k and the scores, (2) the
+// read-out of every row and the state update, which read the state of the
+// previous chunk and write the other of two state buffers, while the next
+// chunk's inputs (loaded into registers one chunk ahead) are staged.
 #pragma once
 
 #include "common.cuh"
@@ -23,13 +34,39 @@ namespace based {
 constexpr int kSimtChunk = 32;
 constexpr int kSimtCols = 8;
 constexpr int kSimtThreads = 256;
-constexpr int kSimtXP = kD + 1;  // pitch of the staged q, k rows (odd: the score loop's
-                                 // 32 lanes read 32 different rows without bank conflicts)
+constexpr int kSimtFc = 1 + kD + kD * (kD + 1) / 2;  // 153 distinct feature rows
+constexpr int kSimtFcPad = 160;                      // rows of a state buffer (zeros past 153)
+constexpr int kSimtXP = kD + 1;  // staged q, k row: 16 values and the 1 (odd pitch: the
+                                 // score loop's 32 lanes read 32 different rows conflict-free)
+constexpr int kSimtFP = 168;     // pitch of the feature rows: 4 rows x 4 feature lanes of a
+                                 // read-out warp fall in 16 different banks
+constexpr int kSimtAP = 36;      // pitch of the score rows (same reason)
+
+// Shared-memory carve-up, in floats.
+constexpr int kSimtSBuf = kSimtFcPad * kSimtCols;
+constexpr int kSimtOffZ = 2 * kSimtSBuf;
+constexpr int kSimtOffFq = kSimtOffZ + 2 * kSimtFcPad;
+constexpr int kSimtOffFk = kSimtOffFq + kSimtChunk * kSimtFP;
+constexpr int kSimtOffV = kSimtOffFk + kSimtChunk * kSimtFP;
+constexpr int kSimtOffA = kSimtOffV + 2 * kSimtChunk * kSimtCols;
+constexpr int kSimtOffXq = kSimtOffA + kSimtChunk * kSimtAP;
+constexpr int kSimtOffXk = kSimtOffXq + kSimtChunk * kSimtXP;
+constexpr int kSimtOffTab = kSimtOffXk + kSimtChunk * kSimtXP;
+constexpr int kSimtFloats = kSimtOffTab + 3 * kSimtFcPad;
+static_assert(kSimtOffV % 4 == 0, "float4 alignment of the value tiles");
 
 __host__ __device__ constexpr size_t linattn_simt_smem_bytes() {
-  return sizeof(float) * (size_t)(kF * kSimtCols + 276 + 2 * kSimtChunk * kF +
-                                  kSimtChunk * kSimtCols + kSimtChunk * 33 + kSimtChunk +
-                                  2 * kSimtChunk * kSimtXP);
+  return sizeof(float) * (size_t)kSimtFloats;
+}
+
+// Row of the 153-row state that holds feature f of the 273-row map: f itself
+// for the constant and linear features; for the quadratic feature (i, j) the
+// pair (a, b) = (min, max) in row-major order over a <= b.
+__device__ __forceinline__ int simt_state_row(int f) {
+  if (f <= kD) return f;
+  const int i = (f - kD - 1) >> 4, j = (f - kD - 1) & 15;
+  const int a = min(i, j), b = max(i, j);
+  return kD + 1 + a * kD - (a * (a - 1)) / 2 + (b - a);
 }
 
 template <typename T>
@@ -37,20 +74,22 @@ __global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
     T* __restrict__ out, float* __restrict__ state_kv, float* __restrict__ state_k, int L,
     int DV, float eps) {
-  constexpr int C = kSimtChunk, NC = kSimtCols, NT = kSimtThreads;
-  constexpr int G = NT / NC;   // row groups
-  constexpr int RPT = C / G;   // rows per thread in the numerator
-  static_assert(NT % NC == 0 && C % G == 0, "thread layout");
+  constexpr int C = kSimtChunk, NC = kSimtCols, NT = kSimtThreads, FC = kSimtFc;
+  constexpr int kQK = C * kD / NT, kVV = C * NC / NT;  // staged values per thread
+  static_assert(NT == C * (NC / 4) * 4, "read-out layout: row x 4-column group x 4 lanes");
+  static_assert(C * kD % NT == 0 && C * NC % NT == 0, "staging layout");
   extern __shared__ __align__(16) float smem[];
-  float* S = smem;                 // [273][kSimtCols]
-  float* z = S + kF * NC;          // [273] (+pad)
-  float* fq = z + 276;             // [32][273]
-  float* fk = fq + C * kF;         // [32][273]
-  float* vs = fk + C * kF;         // [32][kSimtCols]
-  float* A = vs + C * NC;          // [32][33]
-  float* den = A + C * 33;         // [32]
-  float* xq = den + C;             // [32][17]
-  float* xk = xq + C * kSimtXP;    // [32][17]
+  float* S2 = smem;                 // 2 x [160][8]  (state: rows of the 153-row map)
+  float* z2 = smem + kSimtOffZ;     // 2 x [160]
+  float* fq = smem + kSimtOffFq;    // [32][168]     phi(q) (off-diagonal pairs doubled)
+  float* fk = smem + kSimtOffFk;    // [32][168]     phi(k), zero rows past the end
+  float* vs2 = smem + kSimtOffV;    // 2 x [32][8]
+  float* A = smem + kSimtOffA;      // [32][36]
+  float* xq = smem + kSimtOffXq;    // [32][17]
+  float* xk = smem + kSimtOffXk;    // [32][17]
+  int* tab = reinterpret_cast<int*>(smem + kSimtOffTab);  // [160] a | b << 8
+  float* scq = smem + kSimtOffTab + kSimtFcPad;           // [160] query-side scale
+  float* sck = scq + kSimtFcPad;                          // [160] key-side scale
 
   const int tid = threadIdx.x;
   const int bh = blockIdx.x, col0 = blockIdx.y * NC;
@@ -59,35 +98,93 @@ __global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
   v += (size_t)bh * L * DV + col0;
   out += (size_t)bh * L * DV + col0;
 
-  for (int i = tid; i < kF * NC; i += NT) S[i] = 0.0f;
-  for (int i = tid; i < 276; i += NT) z[i] = 0.0f;
+  for (int i = tid; i < kSimtOffV; i += NT) smem[i] = 0.0f;  // states, z, feature tiles
+  for (int r = tid; r < C; r += NT) xq[r * kSimtXP + kD] = xk[r * kSimtXP + kD] = 1.0f;
+  for (int f = tid; f < kF; f += NT) {
+    int a = kD, b = kD;
+    float sq = 1.0f, sk = 1.0f;
+    bool own = true;
+    if (f > 0 && f <= kD) {
+      a = f - 1;
+      sq = sk = kLinScale;
+    } else if (f > kD) {
+      const int i = (f - kD - 1) >> 4, j = (f - kD - 1) & 15;
+      own = i <= j;
+      a = i;
+      b = j;
+      sk = kQuadScale;
+      sq = i == j ? kQuadScale : 2.0f * kQuadScale;
+    }
+    if (own) {
+      const int r = simt_state_row(f);
+      tab[r] = a | (b << 8);
+      scq[r] = sq;
+      sck[r] = sk;
+    }
+  }
 
-  const int j = tid % NC, grp = tid / NC;  // output column, row group (0..G-1)
-  for (int t0 = 0; t0 < L; t0 += C) {
-    const int n = min(C, L - t0);
-    __syncthreads();  // previous chunk's state update is complete
-    for (int i = tid; i < C * kD; i += NT) {
-      const int r = i / kD, c = i - r * kD;
-      xq[r * kSimtXP + c] = r < n ? to_f32(q[(size_t)t0 * kD + i]) : 0.0f;
-      xk[r * kSimtXP + c] = r < n ? to_f32(k[(size_t)t0 * kD + i]) : 0.0f;
+  float rq[kQK], rk[kQK], rv[kVV];
+  auto fetch = [&](int t0) {
+#pragma unroll
+    for (int m = 0; m < kQK; ++m) {
+      const int i = tid + m * NT;
+      const bool ok = t0 + i / kD < L;
+      rq[m] = ok ? to_f32(q[(size_t)t0 * kD + i]) : 0.0f;
+      rk[m] = ok ? to_f32(k[(size_t)t0 * kD + i]) : 0.0f;
     }
-    for (int i = tid; i < C * NC; i += NT) {
-      const int r = i / NC, c = i - r * NC;
-      vs[i] = r < n ? to_f32(v[(size_t)(t0 + r) * DV + c]) : 0.0f;
+#pragma unroll
+    for (int m = 0; m < kVV; ++m) {
+      const int i = tid + m * NT, r = i / NC, c = i - r * NC;
+      rv[m] = t0 + r < L ? to_f32(v[(size_t)(t0 + r) * DV + c]) : 0.0f;
     }
-    __syncthreads();
-    for (int i = tid; i < C * kF; i += NT) {
-      const int r = i / kF, f = i - r * kF;
-      fq[i] = phi_feature(xq + r * kSimtXP, f);
-      fk[i] = phi_feature(xk + r * kSimtXP, f);
+  };
+  auto stage = [&](int buf) {
+#pragma unroll
+    for (int m = 0; m < kQK; ++m) {
+      const int i = tid + m * NT, r = i / kD, c = i - r * kD;
+      xq[r * kSimtXP + c] = rq[m];
+      xk[r * kSimtXP + c] = rk[m];
     }
-    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < kVV; ++m) vs2[buf * C * NC + tid + m * NT] = rv[m];
+  };
+
+  if (L > 0) {
+    fetch(0);
+    stage(0);
+    if (C < L) fetch(C);
+  }
+
+  // read-out layout: row t, columns 4*cg .. 4*cg+3, features fl, fl+4, ...
+  const int fl = tid & 3, cg = (tid >> 2) & 1, t = tid >> 3;
+  int nchunks = 0;
+  for (int t0 = 0; t0 < L; t0 += C, ++nchunks) {
+    const int n = min(C, L - t0), cur = nchunks & 1;
+    __syncthreads();  // chunk inputs staged; the previous read-out and update are done
+
+    // features: items (q or k, feature row, half of the chunk's rows)
+    for (int it = tid; it < 4 * FC; it += NT) {
+      const bool key = it >= 2 * FC;
+      const int rem = key ? it - 2 * FC : it;
+      const int half = rem >= FC;
+      const int f = rem - half * FC;
+      const int e = tab[f], a = e & 0xff, b = e >> 8;
+      const float sc = key ? sck[f] : scq[f];
+      const float* xr = (key ? xk : xq) + half * (C / 2) * kSimtXP;
+      float* dst = (key ? fk : fq) + half * (C / 2) * kSimtFP + f;
+      const int live = key ? n - half * (C / 2) : C;  // key rows past the end stay zero
+#pragma unroll
+      for (int r = 0; r < C / 2; ++r) {
+        const float val = (xr[r * kSimtXP + a] * xr[r * kSimtXP + b]) * sc;
+        dst[r * kSimtFP] = r < live ? val : 0.0f;
+      }
+    }
     // intra-chunk scores, causal mask s <= t, in closed form from u = q_t . k_s
     for (int i = tid; i < C * C; i += NT) {
-      const int t = i / C, s = i - t * C;
+      const int tt = i / C, s = i - tt * C;
       float a = 0.0f;
-      if (s <= t) {
-        const float* qr = xq + t * kSimtXP;
+      if (s <= tt) {
+        const float* qr = xq + tt * kSimtXP;
         const float* kr = xk + s * kSimtXP;
         float u2[2] = {0.0f, 0.0f};
 #pragma unroll
@@ -95,62 +192,89 @@ __global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
         const float u = u2[0] + u2[1];
         a = fmaf(u, fmaf(u, 0.03125f, 0.25f), 1.0f);
       }
-      A[t * 33 + s] = a;
+      A[tt * kSimtAP + s] = a;
     }
     __syncthreads();
-    // denominators: inter (phi(q).z) + intra (row sum of A)
-    if (tid < C) {
-      float d = 0.0f;
-      const float* a_row = fq + tid * kF;
-      for (int f = 0; f < kF; ++f) d = fmaf(a_row[f], z[f], d);
-      for (int s = 0; s < C; ++s) d += A[tid * 33 + s];
-      den[tid] = d;
+
+    const float* Sc = S2 + cur * kSimtSBuf;
+    const float* zc = z2 + cur * kSimtFcPad;
+    const float* vc = vs2 + cur * C * NC;
+    // read-out: four lanes split the feature rows (rows 153..159 are zero)
+    {
+      float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      float den = 0.0f;
+      const float* fr = fq + t * kSimtFP;
+#pragma unroll 4
+      for (int f = fl; f < kSimtFcPad; f += 4) {
+        const float a = fr[f];
+        const float4 s4 = *reinterpret_cast<const float4*>(Sc + f * NC + 4 * cg);
+        acc.x = fmaf(a, s4.x, acc.x);
+        acc.y = fmaf(a, s4.y, acc.y);
+        acc.z = fmaf(a, s4.z, acc.z);
+        acc.w = fmaf(a, s4.w, acc.w);
+        den = fmaf(a, zc[f], den);
+      }
+      const float* ar = A + t * kSimtAP;
+#pragma unroll
+      for (int s = fl; s < C; s += 4) {
+        const float a = ar[s];
+        const float4 v4 = *reinterpret_cast<const float4*>(vc + s * NC + 4 * cg);
+        acc.x = fmaf(a, v4.x, acc.x);
+        acc.y = fmaf(a, v4.y, acc.y);
+        acc.z = fmaf(a, v4.z, acc.z);
+        acc.w = fmaf(a, v4.w, acc.w);
+        den += a;
+      }
+#pragma unroll
+      for (int o = 1; o < 4; o <<= 1) {
+        acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
+        acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
+        acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
+        acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
+        den += __shfl_xor_sync(0xffffffffu, den, o);
+      }
+      const float num = fl == 0 ? acc.x : fl == 1 ? acc.y : fl == 2 ? acc.z : acc.w;
+      if (t < n) out[(size_t)(t0 + t) * DV + 4 * cg + fl] = from_f32<T>(num / (den + eps));
     }
-    // numerators for rows grp, grp+G, ..., column j
-    float acc[RPT];
+    // state update into the other buffer: items (feature row, 4-column group)
+    {
+      float* Sn = S2 + (cur ^ 1) * kSimtSBuf;
+      float* zn = z2 + (cur ^ 1) * kSimtFcPad;
+      for (int it = tid; it < 2 * FC; it += NT) {
+        const int f = it >> 1, c4 = (it & 1) * 4;
+        float4 s4 = *reinterpret_cast<const float4*>(Sc + f * NC + c4);
+        float zs = 0.0f;
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) acc[i] = 0.0f;
-    for (int f = 0; f < kF; ++f) {
-      const float sf = S[f * NC + j];
-#pragma unroll
-      for (int i = 0; i < RPT; ++i) acc[i] = fmaf(fq[(grp + G * i) * kF + f], sf, acc[i]);
+        for (int s = 0; s < C; ++s) {
+          const float a = fk[s * kSimtFP + f];
+          const float4 v4 = *reinterpret_cast<const float4*>(vc + s * NC + c4);
+          s4.x = fmaf(a, v4.x, s4.x);
+          s4.y = fmaf(a, v4.y, s4.y);
+          s4.z = fmaf(a, v4.z, s4.z);
+          s4.w = fmaf(a, v4.w, s4.w);
+          zs += a;
+        }
+        *reinterpret_cast<float4*>(Sn + f * NC + c4) = s4;
+        if (c4 == 0) zn[f] = zc[f] + zs;
+      }
     }
-    for (int s = 0; s < C; ++s) {
-      const float vj = vs[s * NC + j];
-#pragma unroll
-      for (int i = 0; i < RPT; ++i) acc[i] = fmaf(A[(grp + G * i) * 33 + s], vj, acc[i]);
-    }
-    __syncthreads();  // den ready; all reads of S and z for this chunk done
-#pragma unroll
-    for (int i = 0; i < RPT; ++i) {
-      const int t = grp + G * i;
-      if (t < n) out[(size_t)(t0 + t) * DV + j] = from_f32<T>(acc[i] / (den[t] + eps));
-    }
-    // state update over the chunk's 32 rows (rows past the end have v = 0;
-    // z skips them), four partial sums per entry
-    for (int f = grp; f < kF; f += G) {
-      float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-      for (int s = 0; s < C; ++s) s4[s & 3] = fmaf(fk[s * kF + f], vs[s * NC + j], s4[s & 3]);
-      S[f * NC + j] += (s4[0] + s4[1]) + (s4[2] + s4[3]);
-    }
-    for (int f = tid; f < kF; f += NT) {
-      float z4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-      for (int s = 0; s < C; ++s) z4[s & 3] += s < n ? fk[s * kF + f] : 0.0f;
-      z[f] += (z4[0] + z4[1]) + (z4[2] + z4[3]);
+    if (t0 + C < L) {  // stage the next chunk (its q, k are read only after the next barrier)
+      stage(cur ^ 1);
+      if (t0 + 2 * C < L) fetch(t0 + 2 * C);
     }
   }
   __syncthreads();
+  const float* Sf = S2 + (nchunks & 1) * kSimtSBuf;
+  const float* zf = z2 + (nchunks & 1) * kSimtFcPad;
   if (state_kv) {
     float* dst = state_kv + (size_t)bh * kF * DV + col0;
     for (int i = tid; i < kF * NC; i += NT) {
       const int f = i / NC, c = i - f * NC;
-      dst[(size_t)f * DV + c] = S[i];
+      dst[(size_t)f * DV + c] = Sf[simt_state_row(f) * NC + c];
     }
   }
   if (state_k && blockIdx.y == 0) {
-    for (int f = tid; f < kF; f += NT) state_k[(size_t)bh * kF + f] = z[f];
+    for (int f = tid; f < kF; f += NT) state_k[(size_t)bh * kF + f] = zf[simt_state_row(f)];
   }
 }
 
