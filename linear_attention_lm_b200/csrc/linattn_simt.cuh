@@ -33,14 +33,14 @@ namespace based {
 
 constexpr int kSimtChunk = 32;
 constexpr int kSimtCols = 8;
-constexpr int kSimtThreads = 256;
+constexpr int kSimtThreads = 512;
 constexpr int kSimtFc = 1 + kD + kD * (kD + 1) / 2;  // 153 distinct feature rows
 constexpr int kSimtFcPad = 160;                      // rows of a state buffer (zeros past 153)
 constexpr int kSimtXP = kD + 1;  // staged q, k row: 16 values and the 1 (odd pitch: the
                                  // score loop's 32 lanes read 32 different rows conflict-free)
-constexpr int kSimtFP = 168;     // pitch of the feature rows: 4 rows x 4 feature lanes of a
-                                 // read-out warp fall in 16 different banks
-constexpr int kSimtAP = 36;      // pitch of the score rows (same reason)
+constexpr int kSimtFP = 168;     // pitch of the feature rows and (below) of the score rows:
+constexpr int kSimtAP = 40;      // 8 banks apart, so the rows and feature lanes of a read-out
+                                 // warp fall in different banks
 
 // Shared-memory carve-up, in floats.
 constexpr int kSimtSBuf = kSimtFcPad * kSimtCols;
@@ -75,16 +75,16 @@ __global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
     T* __restrict__ out, float* __restrict__ state_kv, float* __restrict__ state_k, int L,
     int DV, float eps) {
   constexpr int C = kSimtChunk, NC = kSimtCols, NT = kSimtThreads, FC = kSimtFc;
-  constexpr int kQK = C * kD / NT, kVV = C * NC / NT;  // staged values per thread
-  static_assert(NT == C * (NC / 4) * 4, "read-out layout: row x 4-column group x 4 lanes");
-  static_assert(C * kD % NT == 0 && C * NC % NT == 0, "staging layout");
+  constexpr int kQK = (C * kD + NT - 1) / NT, kVV = (C * NC + NT - 1) / NT;  // staged per thread
+  constexpr int FL = NT / (C * (NC / 4));  // feature lanes per output row and column group
+  static_assert(FL == 4 || FL == 8, "read-out layout: row x 4-column group x 4 or 8 lanes");
   extern __shared__ __align__(16) float smem[];
   float* S2 = smem;                 // 2 x [160][8]  (state: rows of the 153-row map)
   float* z2 = smem + kSimtOffZ;     // 2 x [160]
   float* fq = smem + kSimtOffFq;    // [32][168]     phi(q) (off-diagonal pairs doubled)
   float* fk = smem + kSimtOffFk;    // [32][168]     phi(k), zero rows past the end
   float* vs2 = smem + kSimtOffV;    // 2 x [32][8]
-  float* A = smem + kSimtOffA;      // [32][36]
+  float* A = smem + kSimtOffA;      // [32][40]
   float* xq = smem + kSimtOffXq;    // [32][17]
   float* xk = smem + kSimtOffXk;    // [32][17]
   int* tab = reinterpret_cast<int*>(smem + kSimtOffTab);  // [160] a | b << 8
@@ -128,25 +128,28 @@ __global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
 #pragma unroll
     for (int m = 0; m < kQK; ++m) {
       const int i = tid + m * NT;
-      const bool ok = t0 + i / kD < L;
+      const bool ok = i < C * kD && t0 + i / kD < L;
       rq[m] = ok ? to_f32(q[(size_t)t0 * kD + i]) : 0.0f;
       rk[m] = ok ? to_f32(k[(size_t)t0 * kD + i]) : 0.0f;
     }
 #pragma unroll
     for (int m = 0; m < kVV; ++m) {
       const int i = tid + m * NT, r = i / NC, c = i - r * NC;
-      rv[m] = t0 + r < L ? to_f32(v[(size_t)(t0 + r) * DV + c]) : 0.0f;
+      rv[m] = i < C * NC && t0 + r < L ? to_f32(v[(size_t)(t0 + r) * DV + c]) : 0.0f;
     }
   };
   auto stage = [&](int buf) {
 #pragma unroll
     for (int m = 0; m < kQK; ++m) {
       const int i = tid + m * NT, r = i / kD, c = i - r * kD;
-      xq[r * kSimtXP + c] = rq[m];
-      xk[r * kSimtXP + c] = rk[m];
+      if (i < C * kD) {
+        xq[r * kSimtXP + c] = rq[m];
+        xk[r * kSimtXP + c] = rk[m];
+      }
     }
 #pragma unroll
-    for (int m = 0; m < kVV; ++m) vs2[buf * C * NC + tid + m * NT] = rv[m];
+    for (int m = 0; m < kVV; ++m)
+      if (tid + m * NT < C * NC) vs2[buf * C * NC + tid + m * NT] = rv[m];
   };
 
   if (L > 0) {
@@ -155,8 +158,10 @@ __global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
     if (C < L) fetch(C);
   }
 
-  // read-out layout: row t, columns 4*cg .. 4*cg+3, features fl, fl+4, ...
-  const int fl = tid & 3, cg = (tid >> 2) & 1, t = tid >> 3;
+  // read-out layout: row t, columns 4*cg .. 4*cg+3, feature rows fl, fl+FL, ...; lane bits
+  // (fl0, fl1, cg, fl2): the 8 lanes of a float4 phase read 8 different 16-byte words
+  const int fl = (tid & 3) | (FL == 8 ? ((tid >> 3) & 1) << 2 : 0);
+  const int cg = (tid >> 2) & 1, t = FL == 8 ? tid >> 4 : tid >> 3;
   int nchunks = 0;
   for (int t0 = 0; t0 < L; t0 += C, ++nchunks) {
     const int n = min(C, L - t0), cur = nchunks & 1;
@@ -199,13 +204,13 @@ __global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
     const float* Sc = S2 + cur * kSimtSBuf;
     const float* zc = z2 + cur * kSimtFcPad;
     const float* vc = vs2 + cur * C * NC;
-    // read-out: four lanes split the feature rows (rows 153..159 are zero)
+    // read-out: FL lanes split the feature rows (rows 153..159 are zero)
     {
       float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
       float den = 0.0f;
       const float* fr = fq + t * kSimtFP;
 #pragma unroll 4
-      for (int f = fl; f < kSimtFcPad; f += 4) {
+      for (int f = fl; f < kSimtFcPad; f += FL) {
         const float a = fr[f];
         const float4 s4 = *reinterpret_cast<const float4*>(Sc + f * NC + 4 * cg);
         acc.x = fmaf(a, s4.x, acc.x);
@@ -216,7 +221,7 @@ __global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
       }
       const float* ar = A + t * kSimtAP;
 #pragma unroll
-      for (int s = fl; s < C; s += 4) {
+      for (int s = fl; s < C; s += FL) {
         const float a = ar[s];
         const float4 v4 = *reinterpret_cast<const float4*>(vc + s * NC + 4 * cg);
         acc.x = fmaf(a, v4.x, acc.x);
@@ -226,15 +231,17 @@ __global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
         den += a;
       }
 #pragma unroll
-      for (int o = 1; o < 4; o <<= 1) {
+      for (int o = 1; o < 2 * FL; o <<= 1) {
+        if (o == 4) continue;  // lane bit 2 is the column group
         acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
         acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
         acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
         acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
         den += __shfl_xor_sync(0xffffffffu, den, o);
       }
-      const float num = fl == 0 ? acc.x : fl == 1 ? acc.y : fl == 2 ? acc.z : acc.w;
-      if (t < n) out[(size_t)(t0 + t) * DV + 4 * cg + fl] = from_f32<T>(num / (den + eps));
+      const int c = fl & 3;
+      const float num = c == 0 ? acc.x : c == 1 ? acc.y : c == 2 ? acc.z : acc.w;
+      if (t < n && fl < 4) out[(size_t)(t0 + t) * DV + 4 * cg + c] = from_f32<T>(num / (den + eps));
     }
     // state update into the other buffer: items (feature row, 4-column group)
     {
