@@ -306,18 +306,28 @@ based_status_t launch_window_tcp(const void* q, const void* k, const void* v, vo
   return launch_status();
 }
 
+template <typename T, int Q, int SUB>
+based_status_t launch_window_simt_q(const void* q, const void* k, const void* v, void* out,
+                                    int BH, int L, int dh, int W, cudaStream_t st) {
+  auto kern = window_simt_kernel<T, Q, SUB>;
+  const size_t smem = window_simt_smem_bytes<Q>(dh);
+  if (!set_smem(kern, smem)) return BASED_ERR_CUDA;
+  const long long nblk = (L + Q - 1) / Q;
+  if (nblk > 0x7fffffffLL || BH > 65535) return BASED_ERR_UNSUPPORTED;
+  dim3 grid((unsigned)nblk, (unsigned)BH);
+  kern<<<grid, Q * SUB, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
+                                    static_cast<const T*>(v), static_cast<T*>(out), L, dh, W);
+  return launch_status();
+}
+
+// 64-query blocks once they give every SM two CTAs; 16-query blocks below that.
 template <typename T>
 based_status_t launch_window_simt(const void* q, const void* k, const void* v, void* out,
                                   int BH, int L, int dh, int W, cudaStream_t st) {
-  auto kern = window_simt_kernel<T>;
-  const size_t smem = window_simt_smem_bytes(dh);
-  if (!set_smem(kern, smem)) return BASED_ERR_CUDA;
-  const long long nblk = (L + kWinQ - 1) / kWinQ;
-  if (nblk > 0x7fffffffLL || BH > 65535) return BASED_ERR_UNSUPPORTED;
-  dim3 grid((unsigned)nblk, (unsigned)BH);
-  kern<<<grid, kWinThreads, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
-                                        static_cast<const T*>(v), static_cast<T*>(out), L, dh, W);
-  return launch_status();
+  const long long blocks64 = (long long)BH * ((L + 63) / 64);
+  if (blocks64 >= 2LL * device_sm_count())
+    return launch_window_simt_q<T, 64, 4>(q, k, v, out, BH, L, dh, W, st);
+  return launch_window_simt_q<T, 16, 16>(q, k, v, out, BH, L, dh, W, st);
 }
 
 template <typename T, int DV>
@@ -608,7 +618,7 @@ based_status_t based_window_attn_fwd(const void* q, const void* k, const void* v
   if (B < 0 || H < 0 || L < 0) return BASED_ERR_INVALID_ARG;
   if (dt != BASED_F32 && dt != BASED_BF16) return BASED_ERR_INVALID_ARG;
   if (window < 1) return BASED_ERR_INVALID_ARG;
-  if (window > kWinQ) return BASED_ERR_UNSUPPORTED;
+  if (window > kWinK) return BASED_ERR_UNSUPPORTED;
   if (d_head != 64 && d_head != 128) return BASED_ERR_UNSUPPORTED;
   const bool empty = (long long)B * H * L == 0;
   based_status_t s;
@@ -629,7 +639,7 @@ based_status_t based_window_ring_fill(const void* k, const void* v, int B, int H
                                       based_dtype_t dt, based_stream_t stream) {
   if (B < 0 || H < 0 || L < 0 || window < 1) return BASED_ERR_INVALID_ARG;
   if (dt != BASED_F32 && dt != BASED_BF16) return BASED_ERR_INVALID_ARG;
-  if (window > kWinQ) return BASED_ERR_UNSUPPORTED;
+  if (window > kWinK) return BASED_ERR_UNSUPPORTED;
   if (d_head != 64 && d_head != 128) return BASED_ERR_UNSUPPORTED;
   const long long BH = (long long)B * H;
   if (BH > 0x7fffffffLL) return BASED_ERR_UNSUPPORTED;
@@ -683,7 +693,7 @@ based_status_t decode_step_impl(const void* q, const void* k, const void* v, flo
         !aligned16(v_ring) || !aligned16(wout))
       return BASED_ERR_INVALID_ARG;
     if (window < 1) return BASED_ERR_INVALID_ARG;
-    if (window > kWinQ) return BASED_ERR_UNSUPPORTED;
+    if (window > kWinK) return BASED_ERR_UNSUPPORTED;
     if (d_head != 64 && d_head != 128) return BASED_ERR_UNSUPPORTED;
   }
   const long long n_lin = lin ? (long long)B * H : 0, n_win = win ? (long long)B * H_w : 0;

@@ -160,6 +160,15 @@ def test_window_head_dims(dh):
     run_window(w)
 
 
+@pytest.mark.parametrize("dh", [64, 128])
+def test_window_fp32_large_blocks(dh):
+    """fp32 window on a problem with two 64-query blocks per SM (the small
+    fp32 cases above run 16-query blocks); ragged last block."""
+    w = WORKLOADS["layer_1b3"].with_(B=2, Hw=16, L=1000, dh=dh, dtype="f32",
+                                     name=f"winf32_{dh}")
+    run_window(w)
+
+
 @pytest.mark.parametrize("name", ["layer_360m", "layer_1b3", "long_16k"])
 def test_window_full_workloads(name):
     run_window(WORKLOADS[name])
