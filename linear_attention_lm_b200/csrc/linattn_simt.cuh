@@ -18,13 +18,20 @@
 //    16 linear, the 136 pairs i <= j) and weights an off-diagonal pair twice on
 //    the query side, which gives phi(q)^T S exactly; the export writes every
 //    pair row to both of its places in the 273-row state.
-// Every feature is a product x[a] * x[b] * scale over the staged row extended
-// by a 1 (column 16): (16, 16) is the constant, (i, 16) the linear features.
+// Every feature is a product x[a] * x[b] * scale over the row extended by a 1
+// (index 16): (16, 16) is the constant, (i, 16) the linear features.
 //
-// Per chunk two barriers: (1) the features of q and k and the scores, (2) the
-// read-out of every row and the state update, which read the state of the
-// previous chunk and write the other of two state buffers, while the next
-// chunk's inputs (loaded into registers one chunk ahead) are staged.
+// The kernel is bound by shared-memory accesses, so each phase is laid out to
+// make one access feed many FMAs.  Per chunk two barriers:
+//  (1) features: one warp per (q or k, eighth of the feature rows), one lane
+//      per token row, the row in registers and the feature indices fixed at
+//      compile time; scores: float4 loads, two query rows per thread;
+//  (2) read-out on warps 0-7: one lane per row, warp w over feature rows
+//      w, w+8, ... and keys w, w+8, ..., reading each state row at one address
+//      for the whole warp; the eight partial sums meet in shared memory.
+//      State update on warps 8-12: one thread per state row, all eight
+//      columns and z, into the other of two state buffers.  Meanwhile the
+//      next chunk's inputs, loaded into registers one chunk ahead, are staged.
 #pragma once
 
 #include "common.cuh"
@@ -35,25 +42,28 @@ constexpr int kSimtChunk = 32;
 constexpr int kSimtCols = 8;
 constexpr int kSimtThreads = 512;
 constexpr int kSimtFc = 1 + kD + kD * (kD + 1) / 2;  // 153 distinct feature rows
-constexpr int kSimtFcPad = 160;                      // rows of a state buffer (zeros past 153)
-constexpr int kSimtXP = kD + 1;  // staged q, k row: 16 values and the 1 (odd pitch: the
-                                 // score loop's 32 lanes read 32 different rows conflict-free)
-constexpr int kSimtFP = 168;     // pitch of the feature rows and (below) of the score rows:
-constexpr int kSimtAP = 40;      // 8 banks apart, so the rows and feature lanes of a read-out
-                                 // warp fall in different banks
+constexpr int kSimtFcPad = 160;                      // feature rows read (zeros past 153)
+constexpr int kSimtSZ = 12;      // state row: S (8 columns), z, 3 zeros (48 bytes: the float4
+                                 // reads of 8 consecutive rows fall in distinct banks)
+constexpr int kSimtXP = 20;      // staged q, k rows: 16 values, float4-aligned, 8 rows of a
+                                 // float4 phase in distinct banks
+constexpr int kSimtFP = 169;     // feature rows (odd: 32 token rows in 32 banks)
+constexpr int kSimtAP = 33;      // score rows (same reason)
+constexpr int kSimtRO = 8;       // read-out warps
 
 // Shared-memory carve-up, in floats.
-constexpr int kSimtSBuf = kSimtFcPad * kSimtCols;
-constexpr int kSimtOffZ = 2 * kSimtSBuf;
-constexpr int kSimtOffFq = kSimtOffZ + 2 * kSimtFcPad;
+constexpr int kSimtSBuf = kSimtFcPad * kSimtSZ;
+constexpr int kSimtOffFq = 2 * kSimtSBuf;
 constexpr int kSimtOffFk = kSimtOffFq + kSimtChunk * kSimtFP;
-constexpr int kSimtOffV = kSimtOffFk + kSimtChunk * kSimtFP;
+constexpr int kSimtOffRed = kSimtOffFk + kSimtChunk * kSimtFP;
+constexpr int kSimtOffRedD = kSimtOffRed + kSimtRO * kSimtChunk * kSimtCols;
+constexpr int kSimtOffV = kSimtOffRedD + kSimtRO * kSimtChunk;
 constexpr int kSimtOffA = kSimtOffV + 2 * kSimtChunk * kSimtCols;
 constexpr int kSimtOffXq = kSimtOffA + kSimtChunk * kSimtAP;
 constexpr int kSimtOffXk = kSimtOffXq + kSimtChunk * kSimtXP;
-constexpr int kSimtOffTab = kSimtOffXk + kSimtChunk * kSimtXP;
-constexpr int kSimtFloats = kSimtOffTab + 3 * kSimtFcPad;
-static_assert(kSimtOffV % 4 == 0, "float4 alignment of the value tiles");
+constexpr int kSimtFloats = kSimtOffXk + kSimtChunk * kSimtXP;
+static_assert(kSimtOffRed % 4 == 0 && kSimtOffV % 4 == 0 && kSimtOffXq % 4 == 0 &&
+                  kSimtOffXk % 4 == 0, "float4 alignment");
 
 __host__ __device__ constexpr size_t linattn_simt_smem_bytes() {
   return sizeof(float) * (size_t)kSimtFloats;
@@ -69,66 +79,73 @@ __device__ __forceinline__ int simt_state_row(int f) {
   return kD + 1 + a * kD - (a * (a - 1)) / 2 + (b - a);
 }
 
+// The factors (a, b) of state row r (inverse of the map above; index 16 is the 1).
+__host__ __device__ constexpr int simt_row_a(int r) {
+  if (r == 0) return kD;
+  if (r <= kD) return r - 1;
+  int p = r - kD - 1, a = 0;
+  while (p >= kD - a) p -= kD - a++;
+  return a;
+}
+__host__ __device__ constexpr int simt_row_b(int r) {
+  if (r <= kD) return kD;
+  int p = r - kD - 1, a = 0;
+  while (p >= kD - a) p -= kD - a++;
+  return a + p;
+}
+
+// Feature rows P, P+8, ... of one token row x (x[16] = 1, or 0 for a key row
+// past the end), with the indices fixed at compile time.
+template <int P, int M = 0>
+__device__ __forceinline__ void simt_features(const float (&x)[kD + 1], float* dst, bool key) {
+  if constexpr (P + 8 * M < kSimtFc) {
+    constexpr int r = P + 8 * M, a = simt_row_a(r), b = simt_row_b(r);
+    constexpr float sk = r == 0 ? 1.0f : r <= kD ? kLinScale : kQuadScale;
+    constexpr float sq = r > kD && a != b ? 2.0f * kQuadScale : sk;
+    dst[r] = (x[a] * x[b]) * (key ? sk : sq);
+    simt_features<P, M + 1>(x, dst, key);
+  }
+}
+
+__device__ __forceinline__ float simt_score(float u) {
+  return fmaf(u, fmaf(u, 0.03125f, 0.25f), 1.0f);  // phi(q).phi(k) from u = q.k
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
     T* __restrict__ out, float* __restrict__ state_kv, float* __restrict__ state_k, int L,
     int DV, float eps) {
   constexpr int C = kSimtChunk, NC = kSimtCols, NT = kSimtThreads, FC = kSimtFc;
-  constexpr int kQK = (C * kD + NT - 1) / NT, kVV = (C * NC + NT - 1) / NT;  // staged per thread
-  constexpr int FL = NT / (C * (NC / 4));  // feature lanes per output row and column group
-  static_assert(FL == 4 || FL == 8, "read-out layout: row x 4-column group x 4 or 8 lanes");
+  constexpr int kQK = C * kD / NT, kVV = (C * NC + NT - 1) / NT;  // staged per thread
+  static_assert(C == 32 && NC == 8 && NT == 512 && C * kD == NT, "thread layout");
+  static_assert(FC <= 5 * 32, "state update: one thread per row on warps 8-12");
   extern __shared__ __align__(16) float smem[];
-  float* S2 = smem;                 // 2 x [160][8]  (state: rows of the 153-row map)
-  float* z2 = smem + kSimtOffZ;     // 2 x [160]
-  float* fq = smem + kSimtOffFq;    // [32][168]     phi(q) (off-diagonal pairs doubled)
-  float* fk = smem + kSimtOffFk;    // [32][168]     phi(k), zero rows past the end
-  float* vs2 = smem + kSimtOffV;    // 2 x [32][8]
-  float* A = smem + kSimtOffA;      // [32][40]
-  float* xq = smem + kSimtOffXq;    // [32][17]
-  float* xk = smem + kSimtOffXk;    // [32][17]
-  int* tab = reinterpret_cast<int*>(smem + kSimtOffTab);  // [160] a | b << 8
-  float* scq = smem + kSimtOffTab + kSimtFcPad;           // [160] query-side scale
-  float* sck = scq + kSimtFcPad;                          // [160] key-side scale
+  float* SZ2 = smem;                  // 2 x [160][12]  state rows: S, z
+  float* fq = smem + kSimtOffFq;      // [32][169]      phi(q) (off-diagonal pairs doubled)
+  float* fk = smem + kSimtOffFk;      // [32][169]      phi(k), zero rows past the end
+  float* red = smem + kSimtOffRed;    // [8][32][8]     read-out partial numerators
+  float* redd = smem + kSimtOffRedD;  // [8][32]        read-out partial denominators
+  float* vs2 = smem + kSimtOffV;      // 2 x [32][8]
+  float* A = smem + kSimtOffA;        // [32][33]
+  float* xq = smem + kSimtOffXq;      // [32][20]
+  float* xk = smem + kSimtOffXk;      // [32][20]
 
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bh = blockIdx.x, col0 = blockIdx.y * NC;
   q += (size_t)bh * L * kD;
   k += (size_t)bh * L * kD;
   v += (size_t)bh * L * DV + col0;
   out += (size_t)bh * L * DV + col0;
 
-  for (int i = tid; i < kSimtOffV; i += NT) smem[i] = 0.0f;  // states, z, feature tiles
-  for (int r = tid; r < C; r += NT) xq[r * kSimtXP + kD] = xk[r * kSimtXP + kD] = 1.0f;
-  for (int f = tid; f < kF; f += NT) {
-    int a = kD, b = kD;
-    float sq = 1.0f, sk = 1.0f;
-    bool own = true;
-    if (f > 0 && f <= kD) {
-      a = f - 1;
-      sq = sk = kLinScale;
-    } else if (f > kD) {
-      const int i = (f - kD - 1) >> 4, j = (f - kD - 1) & 15;
-      own = i <= j;
-      a = i;
-      b = j;
-      sk = kQuadScale;
-      sq = i == j ? kQuadScale : 2.0f * kQuadScale;
-    }
-    if (own) {
-      const int r = simt_state_row(f);
-      tab[r] = a | (b << 8);
-      scq[r] = sq;
-      sck[r] = sk;
-    }
-  }
+  for (int i = tid; i < kSimtOffRed; i += NT) smem[i] = 0.0f;  // states, feature tiles
 
   float rq[kQK], rk[kQK], rv[kVV];
   auto fetch = [&](int t0) {
 #pragma unroll
     for (int m = 0; m < kQK; ++m) {
       const int i = tid + m * NT;
-      const bool ok = i < C * kD && t0 + i / kD < L;
+      const bool ok = t0 + i / kD < L;
       rq[m] = ok ? to_f32(q[(size_t)t0 * kD + i]) : 0.0f;
       rk[m] = ok ? to_f32(k[(size_t)t0 * kD + i]) : 0.0f;
     }
@@ -142,10 +159,8 @@ __global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
 #pragma unroll
     for (int m = 0; m < kQK; ++m) {
       const int i = tid + m * NT, r = i / kD, c = i - r * kD;
-      if (i < C * kD) {
-        xq[r * kSimtXP + c] = rq[m];
-        xk[r * kSimtXP + c] = rk[m];
-      }
+      xq[r * kSimtXP + c] = rq[m];
+      xk[r * kSimtXP + c] = rk[m];
     }
 #pragma unroll
     for (int m = 0; m < kVV; ++m)
@@ -158,111 +173,137 @@ __global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
     if (C < L) fetch(C);
   }
 
-  // read-out layout: row t, columns 4*cg .. 4*cg+3, feature rows fl, fl+FL, ...; lane bits
-  // (fl0, fl1, cg, fl2): the 8 lanes of a float4 phase read 8 different 16-byte words
-  const int fl = (tid & 3) | (FL == 8 ? ((tid >> 3) & 1) << 2 : 0);
-  const int cg = (tid >> 2) & 1, t = FL == 8 ? tid >> 4 : tid >> 3;
   int nchunks = 0;
   for (int t0 = 0; t0 < L; t0 += C, ++nchunks) {
     const int n = min(C, L - t0), cur = nchunks & 1;
     __syncthreads();  // chunk inputs staged; the previous read-out and update are done
 
-    // features: items (q or k, feature row, half of the chunk's rows)
-    for (int it = tid; it < 4 * FC; it += NT) {
-      const bool key = it >= 2 * FC;
-      const int rem = key ? it - 2 * FC : it;
-      const int half = rem >= FC;
-      const int f = rem - half * FC;
-      const int e = tab[f], a = e & 0xff, b = e >> 8;
-      const float sc = key ? sck[f] : scq[f];
-      const float* xr = (key ? xk : xq) + half * (C / 2) * kSimtXP;
-      float* dst = (key ? fk : fq) + half * (C / 2) * kSimtFP + f;
-      const int live = key ? n - half * (C / 2) : C;  // key rows past the end stay zero
+    {  // features of token row `lane`: warps 0-7 the query, 8-15 the key
+      const bool key = warp >= 8;
+      const float4* xr = reinterpret_cast<const float4*>((key ? xk : xq) + lane * kSimtXP);
+      float x[kD + 1];
 #pragma unroll
-      for (int r = 0; r < C / 2; ++r) {
-        const float val = (xr[r * kSimtXP + a] * xr[r * kSimtXP + b]) * sc;
-        dst[r * kSimtFP] = r < live ? val : 0.0f;
+      for (int c = 0; c < kD / 4; ++c) {
+        const float4 t4 = xr[c];
+        x[4 * c] = t4.x;
+        x[4 * c + 1] = t4.y;
+        x[4 * c + 2] = t4.z;
+        x[4 * c + 3] = t4.w;
+      }
+      x[kD] = key && lane >= n ? 0.0f : 1.0f;  // key rows past the end: all features zero
+      float* dst = (key ? fk : fq) + lane * kSimtFP;
+      switch (warp & 7) {
+        case 0: simt_features<0>(x, dst, key); break;
+        case 1: simt_features<1>(x, dst, key); break;
+        case 2: simt_features<2>(x, dst, key); break;
+        case 3: simt_features<3>(x, dst, key); break;
+        case 4: simt_features<4>(x, dst, key); break;
+        case 5: simt_features<5>(x, dst, key); break;
+        case 6: simt_features<6>(x, dst, key); break;
+        default: simt_features<7>(x, dst, key); break;
       }
     }
-    // intra-chunk scores, causal mask s <= t, in closed form from u = q_t . k_s
-    for (int i = tid; i < C * C; i += NT) {
-      const int tt = i / C, s = i - tt * C;
-      float a = 0.0f;
-      if (s <= tt) {
-        const float* qr = xq + tt * kSimtXP;
-        const float* kr = xk + s * kSimtXP;
-        float u2[2] = {0.0f, 0.0f};
+    {  // intra-chunk scores of query rows `warp` and `warp`+16 with key `lane`
+      const float4* k4 = reinterpret_cast<const float4*>(xk + lane * kSimtXP);
+      const float4* qa = reinterpret_cast<const float4*>(xq + warp * kSimtXP);
+      const float4* qb = reinterpret_cast<const float4*>(xq + (warp + 16) * kSimtXP);
+      float ua = 0.0f, ub = 0.0f, ua2 = 0.0f, ub2 = 0.0f;
 #pragma unroll
-        for (int d = 0; d < kD; ++d) u2[d & 1] = fmaf(qr[d], kr[d], u2[d & 1]);
-        const float u = u2[0] + u2[1];
-        a = fmaf(u, fmaf(u, 0.03125f, 0.25f), 1.0f);
+      for (int c = 0; c < kD / 4; ++c) {
+        const float4 y = k4[c], a4 = qa[c], b4 = qb[c];
+        ua = fmaf(a4.x, y.x, ua);
+        ua2 = fmaf(a4.y, y.y, ua2);
+        ua = fmaf(a4.z, y.z, ua);
+        ua2 = fmaf(a4.w, y.w, ua2);
+        ub = fmaf(b4.x, y.x, ub);
+        ub2 = fmaf(b4.y, y.y, ub2);
+        ub = fmaf(b4.z, y.z, ub);
+        ub2 = fmaf(b4.w, y.w, ub2);
       }
-      A[tt * kSimtAP + s] = a;
+      A[warp * kSimtAP + lane] = lane <= warp ? simt_score(ua + ua2) : 0.0f;
+      A[(warp + 16) * kSimtAP + lane] = lane <= warp + 16 ? simt_score(ub + ub2) : 0.0f;
     }
     __syncthreads();
 
-    const float* Sc = S2 + cur * kSimtSBuf;
-    const float* zc = z2 + cur * kSimtFcPad;
+    const float* SZc = SZ2 + cur * kSimtSBuf;
     const float* vc = vs2 + cur * C * NC;
-    // read-out: FL lanes split the feature rows (rows 153..159 are zero)
-    {
-      float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-      float den = 0.0f;
-      const float* fr = fq + t * kSimtFP;
-#pragma unroll 4
-      for (int f = fl; f < kSimtFcPad; f += FL) {
-        const float a = fr[f];
-        const float4 s4 = *reinterpret_cast<const float4*>(Sc + f * NC + 4 * cg);
-        acc.x = fmaf(a, s4.x, acc.x);
-        acc.y = fmaf(a, s4.y, acc.y);
-        acc.z = fmaf(a, s4.z, acc.z);
-        acc.w = fmaf(a, s4.w, acc.w);
-        den = fmaf(a, zc[f], den);
-      }
-      const float* ar = A + t * kSimtAP;
+    if (warp < kSimtRO) {
+      // read-out of row `lane`: this warp's share of the feature rows and keys
+      float acc[NC], den = 0.0f;
 #pragma unroll
-      for (int s = fl; s < C; s += FL) {
-        const float a = ar[s];
-        const float4 v4 = *reinterpret_cast<const float4*>(vc + s * NC + 4 * cg);
-        acc.x = fmaf(a, v4.x, acc.x);
-        acc.y = fmaf(a, v4.y, acc.y);
-        acc.z = fmaf(a, v4.z, acc.z);
-        acc.w = fmaf(a, v4.w, acc.w);
+      for (int c = 0; c < NC; ++c) acc[c] = 0.0f;
+      const float* fr = fq + lane * kSimtFP;
+#pragma unroll 4
+      for (int f = warp; f < kSimtFcPad; f += kSimtRO) {  // rows 153..159 are zero
+        const float a = fr[f];
+        const float* sr = SZc + f * kSimtSZ;
+        const float4 s0 = *reinterpret_cast<const float4*>(sr);
+        const float4 s1 = *reinterpret_cast<const float4*>(sr + 4);
+        acc[0] = fmaf(a, s0.x, acc[0]);
+        acc[1] = fmaf(a, s0.y, acc[1]);
+        acc[2] = fmaf(a, s0.z, acc[2]);
+        acc[3] = fmaf(a, s0.w, acc[3]);
+        acc[4] = fmaf(a, s1.x, acc[4]);
+        acc[5] = fmaf(a, s1.y, acc[5]);
+        acc[6] = fmaf(a, s1.z, acc[6]);
+        acc[7] = fmaf(a, s1.w, acc[7]);
+        den = fmaf(a, sr[NC], den);
+      }
+#pragma unroll
+      for (int s = warp; s < C; s += kSimtRO) {
+        const float a = A[lane * kSimtAP + s];
+        const float4 v0 = *reinterpret_cast<const float4*>(vc + s * NC);
+        const float4 v1 = *reinterpret_cast<const float4*>(vc + s * NC + 4);
+        acc[0] = fmaf(a, v0.x, acc[0]);
+        acc[1] = fmaf(a, v0.y, acc[1]);
+        acc[2] = fmaf(a, v0.z, acc[2]);
+        acc[3] = fmaf(a, v0.w, acc[3]);
+        acc[4] = fmaf(a, v1.x, acc[4]);
+        acc[5] = fmaf(a, v1.y, acc[5]);
+        acc[6] = fmaf(a, v1.z, acc[6]);
+        acc[7] = fmaf(a, v1.w, acc[7]);
         den += a;
       }
+      float4* rp = reinterpret_cast<float4*>(red + (warp * C + lane) * NC);
+      rp[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      rp[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      redd[warp * C + lane] = den;
+      asm volatile("bar.sync 1, %0;" ::"n"(kSimtRO * 32) : "memory");  // read-out warps only
+      const int ot = tid >> 3, oc = tid & 7;  // output row, column
+      float num = 0.0f, dd = 0.0f;
 #pragma unroll
-      for (int o = 1; o < 2 * FL; o <<= 1) {
-        if (o == 4) continue;  // lane bit 2 is the column group
-        acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
-        acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
-        acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
-        acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
-        den += __shfl_xor_sync(0xffffffffu, den, o);
+      for (int w = 0; w < kSimtRO; ++w) {
+        num += red[(w * C + ot) * NC + oc];
+        dd += redd[w * C + ot];
       }
-      const int c = fl & 3;
-      const float num = c == 0 ? acc.x : c == 1 ? acc.y : c == 2 ? acc.z : acc.w;
-      if (t < n && fl < 4) out[(size_t)(t0 + t) * DV + 4 * cg + c] = from_f32<T>(num / (den + eps));
-    }
-    // state update into the other buffer: items (feature row, 4-column group)
-    {
-      float* Sn = S2 + (cur ^ 1) * kSimtSBuf;
-      float* zn = z2 + (cur ^ 1) * kSimtFcPad;
-      for (int it = tid; it < 2 * FC; it += NT) {
-        const int f = it >> 1, c4 = (it & 1) * 4;
-        float4 s4 = *reinterpret_cast<const float4*>(Sc + f * NC + c4);
+      if (ot < n) out[(size_t)(t0 + ot) * DV + oc] = from_f32<T>(num / (dd + eps));
+    } else {
+      // state update of row f into the other buffer
+      const int f = tid - kSimtRO * 32;
+      if (f < FC) {
+        const float* sr = SZc + f * kSimtSZ;
+        float4 s0 = *reinterpret_cast<const float4*>(sr);
+        float4 s1 = *reinterpret_cast<const float4*>(sr + 4);
         float zs = 0.0f;
 #pragma unroll
         for (int s = 0; s < C; ++s) {
           const float a = fk[s * kSimtFP + f];
-          const float4 v4 = *reinterpret_cast<const float4*>(vc + s * NC + c4);
-          s4.x = fmaf(a, v4.x, s4.x);
-          s4.y = fmaf(a, v4.y, s4.y);
-          s4.z = fmaf(a, v4.z, s4.z);
-          s4.w = fmaf(a, v4.w, s4.w);
+          const float4 v0 = *reinterpret_cast<const float4*>(vc + s * NC);
+          const float4 v1 = *reinterpret_cast<const float4*>(vc + s * NC + 4);
+          s0.x = fmaf(a, v0.x, s0.x);
+          s0.y = fmaf(a, v0.y, s0.y);
+          s0.z = fmaf(a, v0.z, s0.z);
+          s0.w = fmaf(a, v0.w, s0.w);
+          s1.x = fmaf(a, v1.x, s1.x);
+          s1.y = fmaf(a, v1.y, s1.y);
+          s1.z = fmaf(a, v1.z, s1.z);
+          s1.w = fmaf(a, v1.w, s1.w);
           zs += a;
         }
-        *reinterpret_cast<float4*>(Sn + f * NC + c4) = s4;
-        if (c4 == 0) zn[f] = zc[f] + zs;
+        float* sn = SZ2 + (cur ^ 1) * kSimtSBuf + f * kSimtSZ;
+        *reinterpret_cast<float4*>(sn) = s0;
+        *reinterpret_cast<float4*>(sn + 4) = s1;
+        sn[NC] = sr[NC] + zs;
       }
     }
     if (t0 + C < L) {  // stage the next chunk (its q, k are read only after the next barrier)
@@ -271,17 +312,17 @@ __global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
     }
   }
   __syncthreads();
-  const float* Sf = S2 + (nchunks & 1) * kSimtSBuf;
-  const float* zf = z2 + (nchunks & 1) * kSimtFcPad;
+  const float* SZf = SZ2 + (nchunks & 1) * kSimtSBuf;
   if (state_kv) {
     float* dst = state_kv + (size_t)bh * kF * DV + col0;
     for (int i = tid; i < kF * NC; i += NT) {
       const int f = i / NC, c = i - f * NC;
-      dst[(size_t)f * DV + c] = Sf[simt_state_row(f) * NC + c];
+      dst[(size_t)f * DV + c] = SZf[simt_state_row(f) * kSimtSZ + c];
     }
   }
   if (state_k && blockIdx.y == 0) {
-    for (int f = tid; f < kF; f += NT) state_k[(size_t)bh * kF + f] = zf[simt_state_row(f)];
+    for (int f = tid; f < kF; f += NT)
+      state_k[(size_t)bh * kF + f] = SZf[simt_state_row(f) * kSimtSZ + NC];
   }
 }
 
