@@ -69,7 +69,7 @@ inline bool set_smem(K kernel, size_t bytes) {
 // held by a CTA waiting for it.  Those kernels take more than half of an SM's
 // shared memory, so no other kernel's CTA runs beside them; the kernels whose
 // CTAs share SMs (the backward kernels, the d_h = 128 window kernel) wait first
-// and allocate after.
+// and allocate after; the fp32 kernels hold no TMEM.
 template <typename... KArgs, typename... Args>
 bool launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
                       cudaStream_t st, Args... args) {
@@ -121,9 +121,10 @@ based_status_t launch_linattn_simt(const void* q, const void* k, const void* v, 
   const size_t smem = linattn_simt_smem_bytes();
   if (!set_smem(kern, smem)) return BASED_ERR_CUDA;
   dim3 grid((unsigned)BH, (unsigned)(d_v / kSimtCols));
-  kern<<<grid, kSimtThreads, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
-                                         static_cast<const T*>(v), static_cast<T*>(out),
-                                         state_kv, state_k, L, d_v, eps);
+  if (!launch_dependent(kern, grid, dim3(kSimtThreads), smem, st, static_cast<const T*>(q),
+                        static_cast<const T*>(k), static_cast<const T*>(v), static_cast<T*>(out),
+                        state_kv, state_k, L, d_v, eps))
+    return BASED_ERR_CUDA;
   return launch_status();
 }
 
@@ -315,8 +316,10 @@ based_status_t launch_window_simt_q(const void* q, const void* k, const void* v,
   const long long nblk = (L + Q - 1) / Q;
   if (nblk > 0x7fffffffLL || BH > 65535) return BASED_ERR_UNSUPPORTED;
   dim3 grid((unsigned)nblk, (unsigned)BH);
-  kern<<<grid, Q * SUB, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
-                                    static_cast<const T*>(v), static_cast<T*>(out), L, dh, W);
+  if (!launch_dependent(kern, grid, dim3(Q * SUB), smem, st, static_cast<const T*>(q),
+                        static_cast<const T*>(k), static_cast<const T*>(v), static_cast<T*>(out),
+                        L, dh, W))
+    return BASED_ERR_CUDA;
   return launch_status();
 }
 

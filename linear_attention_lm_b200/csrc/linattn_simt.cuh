@@ -35,6 +35,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "umma.cuh"
 
 namespace based {
 
@@ -139,6 +140,9 @@ __global__ void __launch_bounds__(kSimtThreads) linattn_simt_kernel(
   out += (size_t)bh * L * DV + col0;
 
   for (int i = tid; i < kSimtOffRed; i += NT) smem[i] = 0.0f;  // states, feature tiles
+  // the set-up above touched no global memory: it overlaps the previous kernel
+  umma::grid_dep_wait();
+  umma::grid_dep_launch();
 
   float rq[kQK], rk[kQK], rv[kVV];
   auto fetch = [&](int t0) {

@@ -52,6 +52,8 @@ __global__ void __launch_bounds__(Q * SUB) window_simt_kernel(const T* __restric
   const size_t base = (size_t)blockIdx.y * L * dh;
   q += base; k += base; v += base; out += base;
 
+  umma::grid_dep_wait();  // the previous kernel in the stream has finished
+  umma::grid_dep_launch();
   const int d4 = dh / 4;  // 16-byte pieces per row
   for (int idx = tid; idx < kWinRows * d4; idx += kWinThreads) {
     const int r = idx / d4, c = 4 * (idx - r * d4);
