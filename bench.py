@@ -307,54 +307,54 @@ def time_prefill(lab, w, sets, steps, warmup, warm, dev, world):
         if ev is not None:
             ev[2].record()
 
+    def replayed(body, before=None, after=None):
+        # body() captured once as a CUDA graph on a side stream, replayed once
+        # untimed (the first launch uploads the graph) and once between the
+        # optional events
+        cap = torch.cuda.Stream(device=dev)
+        cap.wait_stream(torch.cuda.current_stream(dev))
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cap):
+            body()
+        graph.replay()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        if before is not None:
+            before.record()
+        graph.replay()
+        if after is not None:
+            after.record()
+        torch.cuda.synchronize()
+        del graph
+
     def chained(fn):
         # K launches of one kernel back to back, each a dependent launch of the
         # previous one as inside the step; one event pair around all of them
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for i in range(steps):
-            fn(i)
-        b.record()
-        torch.cuda.synchronize()
+        replayed(lambda: [fn(i) for i in range(steps)], a, b)
         return a.elapsed_time(b) / steps
 
     warm()
     for i in range(warmup):
         step(i)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    # event-record nodes inside a graph (the per-kernel pass) need external events
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+           for _ in range(steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        torch.distributed.barrier()
     # the step time: the K steps captured once as a CUDA graph (the same C-ABI
     # calls, nothing between the kernels, each kernel a programmatic dependent
     # launch of the previous one, so its set-up overlaps the previous one) and
     # replayed once, so that the host's cost per call does not pace short steps
-    cap = torch.cuda.Stream(device=dev)
-    cap.wait_stream(torch.cuda.current_stream(dev))
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=cap):
-        for i in range(steps):
-            step(i)
-    graph.replay()  # untimed: the first launch of a graph uploads it
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    start.record()
-    graph.replay()
-    stop.record()
-    torch.cuda.synchronize()
-    del graph
-    # the per-kernel times: the same K steps again with an event pair around
-    # each kernel (an event between two kernels ends their launch overlap, so
-    # each time includes its kernel's launch latency); and, for context, each
-    # kernel's K launches back to back on their own (launches overlapped, but
-    # each kernel's output write-back now competes with its next launch)
-    for i in range(steps):
-        step(i, evs[i])
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
+    replayed(lambda: [step(i) for i in range(steps)], start, stop)
+    # the per-kernel times: the same K steps again, replayed the same way, with
+    # an event pair around each kernel (an event between two kernels ends their
+    # launch overlap, so each time includes its kernel's launch latency); and,
+    # for context, each kernel's K launches back to back on their own
+    # (launches overlapped, but each kernel's output write-back now competes
+    # with its next launch)
+    replayed(lambda: [step(i, evs[i]) for i in range(steps)])
     t_lin = sum(e[0].elapsed_time(e[1]) for e in evs) / steps
     t_win = sum(e[1].elapsed_time(e[2]) for e in evs) / steps
     t_lin_chain = chained(lin)
@@ -444,8 +444,8 @@ def run_ours(args, rank, world, dev):
         "projections": projections,
         "gpu_launches": launches * args.steps,
         "step_timing": "CUDA events around one replay of a CUDA graph of the K steps, captured "
-                       "from the same C-ABI calls (per-kernel times: the same steps launched "
-                       "one by one)",
+                       "from the same C-ABI calls; per-kernel times from event pairs around each "
+                       "kernel in a second graph of the same steps",
         "clocks": clocks,
     }
     if rank == 0 and world == 1:
