@@ -41,6 +41,7 @@ __global__ void __launch_bounds__(Q * SUB) window_simt_kernel(const T* __restric
   constexpr int kWinQ = Q, kWinSub = SUB, kWinThreads = Q * SUB;
   constexpr int kWinRows = Q + kWinK - 1;  // key/value rows staged per CTA
   static_assert(kWinK % SUB == 0 && 32 % SUB == 0, "threads of a query in one warp");
+  static_assert(sizeof(T) == sizeof(float), "the cp.async staging copies fp32 rows");
   extern __shared__ __align__(16) float smem[];
   const int ld = dh + 4;
   float* ks = smem;
